@@ -1,0 +1,165 @@
+"""Pins of the oracle's RAC steps: selection, special cases, products, and the
+accuracy claim of the pages."""
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+from oracle import scalar
+from oracle.nvfp4 import F32
+from precision_rl_rollout_nvfp4_b200 import synthetic as S
+
+
+@pytest.mark.parametrize("k,K,want", [(0, 2048, 0), (100, 2048, 2048), (50, 2048, 1024),
+                                      (25, 2048, 512), (50, 11008, 5504), (12.5, 11008, 1376),
+                                      (33.3, 1000, 332), (0.1, 1000, 1), (99.99, 64, 63)])
+def test_n_selected(k, K, want):
+    # 33.3 and 99.99 are not exact in fp32: floor of the exact value of the float
+    assert oracle.n_selected(k, K) == want
+
+
+def test_select_matches_rank_definition():
+    """j is selected iff fewer than n_sel channels outrank it (higher score, or
+    equal score and lower index) -- brute force O(K^2) on tiny K with ties."""
+    rng = np.random.default_rng(7)
+    for trial in range(40):
+        K = int(rng.integers(1, 48))
+        score = rng.integers(0, 6, K).astype(np.float64) * 0.25     # many ties
+        n_sel = int(rng.integers(0, K + 1))
+        sel, mask = oracle.select_channels(score, n_sel)
+        for j in range(K):
+            outrank = sum(1 for i in range(K) if score[i] > score[j] or (score[i] == score[j] and i < j))
+            assert mask[j] == (outrank < n_sel)
+        assert len(sel) == n_sel and np.all(np.diff(sel) > 0)
+        assert np.array_equal(np.nonzero(mask)[0], sel)
+
+
+def test_identical_channels_tie_to_lower_index():
+    x = S.activations(40, 64, seed=2)
+    xb = S.bf16_bits(x).copy()
+    xb[:, 48:64] = xb[:, 0:16]       # block 3 repeats block 0: equal residuals
+    qa = oracle.quantize_activations(xb)
+    assert np.array_equal(qa["score"][48:64], qa["score"][0:16])
+    order = np.lexsort((np.arange(64), -qa["score"]))
+    pos10 = int(np.nonzero(order == 10)[0][0])
+    assert order[pos10 + 1] == 58     # the twin comes right after, by index
+    # choose n_sel so that exactly one of the pair fits
+    sel, mask = oracle.select_channels(qa["score"], pos10 + 1)
+    assert mask[10] == 1 and mask[58] == 0
+
+
+def test_score_order_and_bound():
+    x = S.activations(300, 32, seed=3)
+    qa = oracle.quantize_activations(S.bf16_bits(x))
+    a = np.abs(qa["dx"]).astype(np.float64)
+    exact = np.array([math.fsum(a[:, j]) for j in range(32)])
+    assert np.all(np.abs(qa["score"] - exact) <= 300 * 2.0 ** -52 * exact)
+    assert np.array_equal(qa["res_colamax"], np.abs(qa["dx"]).max(axis=0))
+
+
+def test_k0_is_plain_w4a4_and_k100_is_full_residual():
+    x = S.activations(64, 128, seed=4)
+    w = S.weights(96, 128, seed=4)
+    xb, wb = S.bf16_bits(x), S.bf16_bits(w)
+    r0 = oracle.rac_linear(xb, wb, 0.0)
+    assert r0["n_sel"] == 0 and not r0["mask"].any()
+    assert np.array_equal(r0["y"], r0["y_plain"])
+    r100 = oracle.rac_linear(xb, wb, 100.0)
+    assert np.array_equal(r100["sel"], np.arange(128))
+    # W_sel == W, so its second-pass quantization equals Q(W) bit for bit
+    assert np.array_equal(r100["ws_codes"], r100["wq"]["codes"])
+    assert np.array_equal(r100["ws_scales"], r100["wq"]["scales"])
+    assert r100["ws_st"] == r100["wq"]["s_t"]
+    # dX_sel == dX, so Q(dX_sel) equals Q(dX) with dX's own tensor scale
+    c, s, st = oracle.quantize_tensor(r100["dx"])
+    assert np.array_equal(r100["r_codes"], c) and np.array_equal(r100["r_scales"], s)
+    assert r100["r_st"] == st
+
+
+def test_gemm_fp64_matches_plain_loop():
+    rng = np.random.default_rng(9)
+    M, N, K = 5, 7, 64
+    ac = rng.integers(0, 16, (M, K)).astype(np.uint8)
+    bc = rng.integers(0, 16, (N, K)).astype(np.uint8)
+    asc = rng.integers(0, 0x7F, (M, K // 16)).astype(np.uint8)
+    bsc = rng.integers(0, 0x7F, (N, K // 16)).astype(np.uint8)
+    y = oracle.gemm_fp64(ac, asc, F32(0.75), bc, bsc, F32(1.5))
+    for i in range(M):
+        for j in range(N):
+            acc = 0.0
+            for k in range(K):
+                acc += (oracle.e2m1_decode(ac[i, k]) * oracle.e4m3_decode(asc[i, k // 16])
+                        * oracle.e2m1_decode(bc[j, k]) * oracle.e4m3_decode(bsc[j, k // 16]))
+            assert abs(y[i, j] - 0.75 * 1.5 * acc) <= 1e-12 * max(1.0, abs(acc))
+
+
+@pytest.mark.parametrize("M,K,N,k", [(5, 64, 3, 50.0), (9, 32, 4, 25.0), (130, 48, 2, 50.0),
+                                     (3, 80, 2, 100.0), (4, 64, 2, 0.0)])
+def test_scalar_restatement_agrees(M, K, N, k):
+    x = S.activations(M, K, seed=M + K)
+    w = S.weights(N, K, seed=N)
+    xb, wb = S.bf16_bits(x), S.bf16_bits(w)
+    r = oracle.rac_linear(xb, wb, k)
+    s = scalar.rac_linear(xb.tolist(), wb.tolist(), k)
+    assert np.array_equal(r["codes"], np.array(s["codes"], np.uint8))
+    assert np.array_equal(r["scales"], np.array(s["scales"], np.uint8))
+    assert np.array_equal(r["dx"], np.array(s["dx"], np.float32))
+    assert np.array_equal(r["score"], np.array(s["score"]))
+    assert r["sel"].tolist() == s["sel"]
+    if r["n_sel"]:
+        assert np.array_equal(r["r_codes"], np.array(s["r_codes"], np.uint8))
+        assert np.array_equal(r["r_scales"], np.array(s["r_scales"], np.uint8))
+        assert np.array_equal(r["ws_codes"], np.array(s["ws_codes"], np.uint8))
+        assert r["r_st"] == s["r_st"] and r["ws_st"] == s["ws_st"]
+    assert np.allclose(r["y"], np.array(s["y"]), rtol=1e-12, atol=1e-14)
+
+
+@pytest.mark.parametrize("M,K,N,seed", [(64, 512, 512, 0), (128, 256, 64, 1), (256, 1024, 128, 2)])
+def test_rac_reduces_error_against_bf16_product(M, K, N, seed):
+    """RAC brings the output closer to the BF16 reference (QUADS technical
+    summary, section 2.2 B, "Doel"); removing it leaves an accuracy gap
+    (section 4, ablation)."""
+    x = S.activations(M, K, seed=seed)
+    w = S.weights(N, K, seed=seed)
+    xb, wb = S.bf16_bits(x), S.bf16_bits(w)
+    ref = oracle.bf16_to_f32(xb).astype(np.float64) @ oracle.bf16_to_f32(wb).astype(np.float64).T
+    wq = oracle.weight_qdq(wb)
+    errs = {}
+    for k in (0.0, 25.0, 50.0, 100.0):
+        r = oracle.rac_linear(xb, wb, k, wq=wq)
+        errs[k] = np.linalg.norm(r["y"] - ref)
+    assert errs[50.0] <= errs[0.0]
+    assert errs[100.0] <= errs[0.0]
+
+
+def test_weight_qdq_on_grid_and_colamax():
+    w = S.weights(64, 256, seed=5)
+    wb = S.bf16_bits(w)
+    q = oracle.weight_qdq(wb)
+    dq = oracle.dequantize(q["codes"], q["scales"], q["s_t"])
+    assert np.array_equal(q["w_out"], oracle.f32_to_bf16(dq))
+    wf = oracle.bf16_to_f32(wb)
+    assert np.array_equal(q["colamax"], np.abs(wf).max(axis=0))
+    # fake quantization moves every weight by at most one grid half-gap
+    s_dec = np.repeat(oracle.e4m3_decode(q["scales"]) * float(q["s_t"]), 16, axis=1)
+    assert np.all(np.abs(oracle.bf16_to_f32(q["w_out"]) - wf) <= s_dec * 1.01 + 1e-30)
+
+
+def test_moe_groups_are_independent_linears():
+    rng = np.random.default_rng(1)
+    E, N, K = 4, 32, 64
+    counts = [70, 0, 130, 5]
+    off = np.concatenate([[0], np.cumsum(counts)])
+    x = S.activations(int(off[-1]), K, seed=6)
+    w = S.weights(N, K, seed=6, batch=E)
+    xb = S.bf16_bits(x)
+    wb = S.bf16_bits(w).reshape(E, N, K)
+    y, masks, per = oracle.moe_rac(xb, off, wb, 50.0)
+    for e in range(E):
+        if counts[e] == 0:
+            assert masks[e].tolist() == [1] * 32 + [0] * 32
+            continue
+        r = oracle.rac_linear(xb[off[e]:off[e + 1]], wb[e], 50.0)
+        assert np.array_equal(y[off[e]:off[e + 1]], r["y"])
+        assert np.array_equal(masks[e], r["mask"])
