@@ -1,0 +1,403 @@
+// Block-scaled FP4 (NVFP4) GEMM on the 5th-generation tensor cores of sm_100a
+// with the RAC residual folded in as a second K segment:
+//
+//     Y = s_tA s_tB (A B^T) + s_tR s_tWs (R Ws^T)
+//
+// A / R: quantized activations / gathered residual [M, K] / [M, width],
+// B / Ws: quantized weights / gathered weight columns [N, K] / [N, width],
+// all K-major packed E2M1 with E4M3 scales per 16 elements (MMA-tiled layout).
+// QUADS technical summary (gist.science): native W4A4 GEMM on Blackwell
+// (section 1), the residual correction added to the quantized output while the
+// bulk keeps native W4A4 throughput (section 2.2 B).
+//
+// Design (one CTA per SM, persistent over 128 x 128 output tiles):
+//   warp 0      TMA producer: per 256-element K step, two 2-D tensor copies
+//               (A and B tiles, 128 B rows, 128 B swizzle) and two bulk
+//               copies of the matching 128 x 16 scale atoms into a 5-stage
+//               shared-memory ring guarded by full / empty mbarriers.
+//   warp 1      MMA issuer: copies each stage's scales into TMEM
+//               (tcgen05.cp 32x128b.warpx4), then issues four
+//               tcgen05.mma kind::mxf4nvf4 (128 x 128 x 64, ue4m3 scales per
+//               16 elements) into accumulator 0 for the plain K segment and
+//               accumulator 1 for the residual segment; tcgen05.commit frees
+//               the stage and, after the last step, signals the epilogue.
+//   warps 2..5  epilogue: tcgen05.ld of both accumulators (TMEM lane = output
+//               row), Y = alpha0 acc0 + alpha1 acc1, stores fp32 or bf16.
+// The two tensor scales differ, so the segments accumulate separately.  No
+// TMA multicast is used.  Every mbarrier wait is bounded (see common.cuh).
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "kernels.h"
+
+namespace nvfp4 {
+namespace {
+
+constexpr int BM = 128, BN = 128;
+constexpr int BK_BYTES = 128;                    // 256 FP4 elements per K step
+constexpr int STAGES = 5;
+constexpr int A_STAGE = BM * BK_BYTES;           // 16 KB
+constexpr int B_STAGE = BN * BK_BYTES;           // 16 KB
+constexpr int SF_ATOM = 512;                     // 128 rows x 4 scales
+constexpr int SF_STAGE = 4 * SF_ATOM;            // 4 MMA K blocks per step
+constexpr int SMEM_BYTES = 1024 + STAGES * (A_STAGE + B_STAGE + 2 * SF_STAGE) + 256;
+constexpr int THREADS = 192;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t ACC0_COL = 0, ACC1_COL = 128;   // two 128-column fp32 accumulators
+constexpr uint32_t SFA_COL = 256, SFB_COL = 272;
+
+// kind::mxf4nvf4 instruction descriptor: E2M1 x E2M1, ue4m3 scales, both
+// K-major, N = 128, M = 128.
+constexpr uint32_t IDESC = (1u << 7) | (1u << 10) | (uint32_t(BN >> 3) << 17) | (uint32_t(BM >> 4) << 24);
+
+struct KParams {
+  RowGroups g;
+  int64_t N;
+  int64_t m_tiles_dense;
+  int n_tiles;
+  int kt[2], kb_last[2];
+  const uint8_t* sfa[2];
+  const uint8_t* sfb[2];
+  int64_t sfa_rb[2], sfb_rb[2];   // bytes per 128-row block of the scale buffers
+  const float* sta[2];
+  const float* stb[2];
+  void* y;
+  int y_dtype;
+  int64_t ldy, M;
+  unsigned* err;
+};
+
+// ---- PTX wrappers ---------------------------------------------------------
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* tm, int x, int y,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+      :: "r"(dst), "l"(reinterpret_cast<uint64_t>(tm)), "r"(x), "r"(y), "r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+               :: "r"(dst), "l"(src), "r"(bytes), "r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor, K-major, 128-byte swizzle: 8-row groups
+// 1024 bytes apart (stride byte offset), leading byte offset unused (1).
+__device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr) {
+  return static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4) | (1ull << 16) |
+         (static_cast<uint64_t>(1024 >> 4) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// Descriptor of a 512-byte scale atom (32 rows x 16 bytes, no swizzle):
+// 8-row core matrices 128 bytes apart.
+__device__ __forceinline__ uint64_t desc_sf(uint32_t saddr) {
+  return static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4) | (static_cast<uint64_t>(128 >> 4) << 32) |
+         (1ull << 46);
+}
+
+__device__ __forceinline__ void utccp_sf(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" :: "r"(taddr), "l"(sdesc) : "memory");
+}
+
+__device__ __forceinline__ void mma_fp4(uint32_t d, uint64_t a, uint64_t b, uint32_t sfa, uint32_t sfb,
+                                        uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+      :: "r"(d), "l"(a), "l"(b), "r"(IDESC), "r"(accumulate), "r"(sfa), "r"(sfb) : "memory");
+}
+
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+               :: "r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void tmem_ld_wait() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// ---- the kernel -----------------------------------------------------------
+__global__ void __launch_bounds__(THREADS, 1)
+w4a4_rac_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
+                     const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
+                     const KParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  // 128-byte swizzled tiles need 1024-byte aligned shared addresses
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint8_t* sA = smem;
+  uint8_t* sB = sA + STAGES * A_STAGE;
+  uint8_t* sSFA = sB + STAGES * B_STAGE;
+  uint8_t* sSFB = sSFA + STAGES * SF_STAGE;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sSFB + STAGES * SF_STAGE);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tmem_full = empty + STAGES;
+  uint64_t* tmem_empty = tmem_full + 1;
+  uint64_t* drain = tmem_empty + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    mbar_init(tmem_full, 1);
+    mbar_init(tmem_empty, 128);
+    mbar_init(drain, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                 :: "r"(smem_u32(tmem_slot)), "r"(TMEM_COLS) : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  const int64_t m_tiles = p.g.off ? p.g.tile_start[p.g.E] : p.m_tiles_dense;
+  const int64_t total = m_tiles * p.n_tiles;
+  const int nseg = p.kt[1] > 0 ? 2 : 1;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------ producer
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t armed = 0, armed_phase = 0;     // per-stage: filled at least once / its parity
+      bool ok = true;
+      for (int64_t tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        const int64_t mt = tile / p.n_tiles, nt = tile % p.n_tiles;
+        const TileInfo ti = tile_info(p.g, mt);
+        const int64_t b_row = static_cast<int64_t>(ti.e) * p.N + nt * BN;
+        for (int seg = 0; seg < nseg && ok; ++seg) {
+          const CUtensorMap* tA = seg ? &tmA1 : &tmA0;
+          const CUtensorMap* tB = seg ? &tmB1 : &tmB0;
+          for (int kt = 0; kt < p.kt[seg]; ++kt) {
+            if (!mbar_wait(&empty[stage], phase ^ 1, p.err)) { ok = false; break; }
+            const int nkb = kt == p.kt[seg] - 1 ? p.kb_last[seg] : 4;
+            const uint32_t sf_bytes = nkb * SF_ATOM;
+            const uint32_t fb = smem_u32(&full[stage]);
+            mbar_arrive_expect_tx(&full[stage], A_STAGE + B_STAGE + 2 * sf_bytes);
+            tma_load_2d(smem_u32(sA + stage * A_STAGE), tA, kt * BK_BYTES, static_cast<int>(mt * BM), fb);
+            tma_load_2d(smem_u32(sB + stage * B_STAGE), tB, kt * BK_BYTES, static_cast<int>(b_row), fb);
+            bulk_load(smem_u32(sSFA + stage * SF_STAGE), p.sfa[seg] + mt * p.sfa_rb[seg] + kt * SF_STAGE,
+                      sf_bytes, fb);
+            bulk_load(smem_u32(sSFB + stage * SF_STAGE),
+                      p.sfb[seg] + (b_row / BN) * p.sfb_rb[seg] + kt * SF_STAGE, sf_bytes, fb);
+            armed |= 1u << stage;
+            armed_phase = (armed_phase & ~(1u << stage)) | (phase << stage);
+            if (++stage == STAGES) { stage = 0; phase ^= 1; }
+          }
+        }
+      }
+      // let every copy in flight land before the CTA can exit
+      for (int s = 0; s < STAGES; ++s)
+        if (armed & (1u << s)) mbar_wait(&full[s], (armed_phase >> s) & 1u, p.err);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------ MMA issuer
+      int stage = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      bool ok = true;
+      for (int64_t tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        if (!mbar_wait(tmem_empty, acc_phase ^ 1, p.err)) break;
+        tc_fence_after();
+        for (int seg = 0; seg < nseg && ok; ++seg) {
+          const uint32_t d = tmem + (seg ? ACC1_COL : ACC0_COL);
+          for (int kt = 0; kt < p.kt[seg]; ++kt) {
+            if (!mbar_wait(&full[stage], phase, p.err)) { ok = false; break; }
+            tc_fence_after();
+            const int nkb = kt == p.kt[seg] - 1 ? p.kb_last[seg] : 4;
+            const uint32_t a0 = smem_u32(sA + stage * A_STAGE), b0 = smem_u32(sB + stage * B_STAGE);
+            const uint32_t fa = smem_u32(sSFA + stage * SF_STAGE), fb = smem_u32(sSFB + stage * SF_STAGE);
+            for (int j = 0; j < nkb; ++j) {
+              utccp_sf(tmem + SFA_COL + 4 * j, desc_sf(fa + j * SF_ATOM));
+              utccp_sf(tmem + SFB_COL + 4 * j, desc_sf(fb + j * SF_ATOM));
+            }
+            for (int j = 0; j < nkb; ++j)
+              mma_fp4(d, desc_sw128(a0 + 32 * j), desc_sw128(b0 + 32 * j), tmem + SFA_COL + 4 * j,
+                      tmem + SFB_COL + 4 * j, (kt > 0 || j > 0) ? 1u : 0u);
+            umma_commit(&empty[stage]);
+            if (++stage == STAGES) { stage = 0; phase ^= 1; }
+          }
+        }
+        umma_commit(tmem_full);
+        acc_phase ^= 1;
+      }
+      umma_commit(drain);                 // all issued tensor-core work done
+      mbar_wait(drain, 0, p.err);
+    }
+  } else {
+    // ------------------------------ epilogue (warps 2..5)
+    const int q = warp & 3;                        // TMEM lane quadrant of this warp
+    const uint32_t trow = tmem + (static_cast<uint32_t>(32 * q) << 16);
+    uint32_t acc_phase = 0;
+    for (int64_t tile = blockIdx.x; tile < total; tile += gridDim.x) {
+      bool ok = true;
+      if (lane == 0) ok = mbar_wait(tmem_full, acc_phase, p.err);
+      ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+      if (!ok) break;
+      tc_fence_after();
+      const int64_t mt = tile / p.n_tiles, nt = tile % p.n_tiles;
+      const TileInfo ti = tile_info(p.g, mt);
+      const float al0 = __fmul_rn(p.sta[0][ti.e], p.stb[0][ti.e]);
+      const float al1 = nseg > 1 ? __fmul_rn(p.sta[1][ti.e], p.stb[1][ti.e]) : 0.0f;
+      const int64_t row = ti.row0 + 32 * q + lane;
+      const bool row_ok = ti.valid && row < ti.row_end;
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        float v[32], u[32];
+        tmem_ld32(trow + ACC0_COL + 32 * c, v);
+        if (nseg > 1) tmem_ld32(trow + ACC1_COL + 32 * c, u);
+        tmem_ld_wait();
+        if (nseg > 1) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = __fadd_rn(__fmul_rn(al0, v[i]), __fmul_rn(al1, u[i]));
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(al0, v[i]);
+        }
+        const int64_t col = nt * BN + 32 * c;
+        if (!row_ok || col >= p.N) continue;
+        if (p.y_dtype == 0) {
+          float* yr = static_cast<float*>(p.y) + row * p.ldy + col;
+          if (col + 32 <= p.N) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 4)
+              *reinterpret_cast<float4*>(yr + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+          } else {
+            for (int i = 0; i < 32 && col + i < p.N; ++i) yr[i] = v[i];
+          }
+        } else {
+          uint16_t* yr = static_cast<uint16_t*>(p.y) + row * p.ldy + col;
+          uint32_t w[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            w[i] = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(v[2 * i]))) |
+                   (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(v[2 * i + 1]))) << 16);
+          if (col + 32 <= p.N) {
+#pragma unroll
+            for (int i = 0; i < 16; i += 4)
+              *reinterpret_cast<uint4*>(yr + 2 * i) = make_uint4(w[i], w[i + 1], w[i + 2], w[i + 3]);
+          } else {
+            for (int i = 0; i < 32 && col + i < p.N; ++i)
+              yr[i] = static_cast<uint16_t>(w[i >> 1] >> (16 * (i & 1)));
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(tmem_empty);
+      acc_phase ^= 1;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(tmem), "r"(TMEM_COLS) : "memory");
+  }
+}
+
+// ---- host side -------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (fn == nullptr) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+// 2-D map over packed FP4 codes [rows, cols/2] bytes, box 128 B x box_rows.
+bool make_code_map(CUtensorMap* tm, const uint8_t* codes, int64_t rows, int64_t cols, int box_rows) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols / 2), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols / 2)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(BK_BYTES), static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(codes), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int sm_count() {
+  int dev = 0, n = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+}  // namespace
+
+cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s) {
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(w4a4_rac_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  KParams p{};
+  p.g = a.g;
+  p.N = a.N;
+  p.m_tiles_dense = (a.M + BM - 1) / BM;
+  p.n_tiles = static_cast<int>((a.N + BN - 1) / BN);
+  p.M = a.M;
+  const GemmOperand* A[2] = {&a.a0, &a.a1};
+  const GemmOperand* B[2] = {&a.b0, &a.b1};
+  CUtensorMap maps[4];
+  const int nseg = a.a1.codes ? 2 : 1;
+  for (int seg = 0; seg < 2; ++seg) {
+    const int sg = seg < nseg ? seg : 0;      // unused segment: harmless copy of segment 0
+    const int64_t cols = A[sg]->cols;
+    p.kt[seg] = seg < nseg ? static_cast<int>((cols + 255) / 256) : 0;
+    p.kb_last[seg] = static_cast<int>(((cols + 63) / 64 - 1) % 4 + 1);
+    p.sfa[seg] = A[sg]->scales;
+    p.sfb[seg] = B[sg]->scales;
+    p.sfa_rb[seg] = (cols + 63) / 64 * SF_ATOM;
+    p.sfb_rb[seg] = (B[sg]->cols + 63) / 64 * SF_ATOM;
+    p.sta[seg] = A[sg]->st;
+    p.stb[seg] = B[sg]->st;
+    if (!make_code_map(&maps[2 * seg], A[sg]->codes, A[sg]->rows, cols, BM)) return cudaErrorInvalidValue;
+    if (!make_code_map(&maps[2 * seg + 1], B[sg]->codes, B[sg]->rows, B[sg]->cols, BN))
+      return cudaErrorInvalidValue;
+  }
+  p.y = a.y;
+  p.y_dtype = a.y_dtype;
+  p.ldy = a.ldy;
+  p.err = a.err;
+  const int64_t tiles_bound = a.m_tiles * p.n_tiles;
+  if (tiles_bound == 0) return cudaSuccess;
+  const int grid = static_cast<int>(tiles_bound < sm_count() ? tiles_bound : sm_count());
+  w4a4_rac_gemm_kernel<<<grid, THREADS, SMEM_BYTES, s>>>(maps[0], maps[1], maps[2], maps[3], p);
+  return cudaGetLastError();
+}
+
+}  // namespace nvfp4

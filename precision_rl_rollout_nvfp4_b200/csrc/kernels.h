@@ -1,0 +1,100 @@
+// Host-side launchers of the NVFP4 W4A4 + RAC kernels.  Internal to the
+// library: the C ABI in api.cu validates arguments and calls these.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace nvfp4 {
+
+// Upper bound of the number of 128-row tiles of `g` (exact for dense).
+inline int64_t max_tiles(const RowGroups& g, int64_t rows) {
+  return g.off ? (rows + kTileRows - 1) / kTileRows + g.E : (g.M + kTileRows - 1) / kTileRows;
+}
+
+// amax_bits[e] |= max |x| over group e (as fp32 bits); amax_bits zeroed by caller.
+// With batch > 1, blockIdx.z walks `batch` dense matrices mat_stride elements
+// apart and writes amax_bits[b].
+cudaError_t launch_amax(const uint16_t* x, int64_t rows, int64_t K, int64_t ldx,
+                        const RowGroups& g, unsigned* amax_bits, cudaStream_t s,
+                        int32_t batch = 1, int64_t mat_stride = 0);
+
+// MoE only: tile_start[e] = sum_{e' < e} ceil(m_e' / 128), e = 0..E.
+cudaError_t launch_group_tiles(const int64_t* off, int32_t E, int32_t* tile_start, cudaStream_t s);
+
+// Q(X) plus score partials.  amax: fp32 per group.  codes [codes_rows, K/2]
+// on padded rows; scales in `layout`; tensor_scale[e] written for non-empty
+// groups; part_sum / part_max [tiles, K] (may be null).
+cudaError_t launch_quant_score(const uint16_t* x, int64_t rows, int64_t K, int64_t ldx,
+                               const RowGroups& g, const float* amax, int64_t codes_rows,
+                               uint8_t* codes, uint8_t* scales, int layout, float* tensor_scale,
+                               double* part_sum, float* part_max, cudaStream_t s);
+
+// score[e, j] = sum over the group's tiles of part_sum in tile order;
+// colamax[e, j] = max of part_max.  For empty groups (MoE) also writes
+// tensor_scale[e] = 0 and zero scores.
+cudaError_t launch_score_reduce(const double* part_sum, const float* part_max, int64_t K,
+                                const RowGroups& g, int64_t tiles, double* score, float* colamax,
+                                float* tensor_scale_empty, cudaStream_t s);
+
+// Per group: top-n_sel mask, ascending sel, s_tR = RN(max_sel colamax / 2688).
+cudaError_t launch_topk(const double* score, const float* colamax, int64_t K, int32_t E,
+                        int64_t n_sel, uint8_t* mask, int32_t* sel, float* s_t_out,
+                        cudaStream_t s);
+
+// Q(dX_sel) on padded rows (width = n_sel rounded to 64, zero padded).
+cudaError_t launch_residual_gather(const uint16_t* x, int64_t rows, int64_t K, int64_t ldx,
+                                   const RowGroups& g, int64_t prows,
+                                   const uint8_t* qx_codes, const uint8_t* qx_scales, int qx_layout,
+                                   const float* qx_st, const int32_t* sel, int64_t n_sel,
+                                   int64_t width, const float* r_st, uint8_t* r_codes,
+                                   uint8_t* r_scales, int r_layout, cudaStream_t s);
+
+// s_t[e] = RN(max_{j < n_sel} colamax[e*K + sel[e*n_sel + j]] / 2688).
+cudaError_t launch_sel_tensor_scale(const float* colamax, int64_t K, const int32_t* sel,
+                                    int64_t n_sel, int32_t E, float* s_t, cudaStream_t s);
+
+// Q(W_sel) for E stacked weights [E, N, K] (row stride ldw, matrix stride
+// N*ldw): out rows E*N, width columns.
+cudaError_t launch_weight_gather(const uint16_t* w, int64_t N, int64_t K, int64_t ldw, int32_t E,
+                                 const int32_t* sel, int64_t n_sel, int64_t width,
+                                 const float* s_t, uint8_t* codes, uint8_t* scales, int layout,
+                                 cudaStream_t s);
+
+// W' = bf16(DQ(Q(W))) for `batch` matrices; optional Q(W) and colamax
+// (colamax_bits zeroed by the caller, written as fp32 bits).
+cudaError_t launch_weight_qdq(const uint16_t* w, int64_t N, int64_t K, int64_t ldw, int32_t batch,
+                              const unsigned* amax_bits, uint16_t* w_out, uint8_t* codes,
+                              uint8_t* scales, int layout, float* tensor_scale,
+                              unsigned* colamax_bits, cudaStream_t s);
+
+cudaError_t launch_encode(const float* in, uint8_t* out, int64_t n, int which, cudaStream_t s);
+
+cudaError_t launch_wait_probe(uint64_t limit_ns, unsigned* err, cudaStream_t s);
+
+// Block-scaled FP4 GEMM with an optional second (residual) K segment.
+struct GemmOperand {
+  const uint8_t* codes;   // [rows, cols/2]
+  const uint8_t* scales;  // MMA-tiled
+  const float* st;        // tensor scale(s), indexed by group
+  int64_t rows, cols;
+};
+
+struct GemmArgs {
+  GemmOperand a0, b0;     // plain segment: A [M(padded), K], B [E*N, K]
+  GemmOperand a1, b1;     // residual segment (a1.codes == null: none)
+  RowGroups g;            // rows of A / Y
+  int64_t M;              // dense rows (or T for MoE)
+  int64_t N;              // out-features per group
+  int64_t m_tiles;        // dense: ceil(M/128); MoE: upper bound
+  void* y;
+  int32_t y_dtype;        // 0 fp32, 1 bf16
+  int64_t ldy;
+  unsigned* err;
+};
+
+cudaError_t launch_gemm(const GemmArgs& args, cudaStream_t s);
+
+}  // namespace nvfp4

@@ -1,0 +1,70 @@
+"""The C ABI library loads and exports every symbol the header declares; pure
+host-side behaviour (sizes, n_sel, argument checks) needs no GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from precision_rl_rollout_nvfp4_b200 import build_lib
+    build_lib.build()
+    return ctypes.CDLL(build_lib.LIB)
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "nvfp4rac.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b([a-z0-9_]+)\s*\(", text)) - {"defined", "sizeof"})
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert len(names) >= 16
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_binding_matches_header():
+    from precision_rl_rollout_nvfp4_b200 import binding
+    assert sorted(binding.EXPORTS) == declared_functions()
+
+
+def test_nsel_and_width(lib):
+    import oracle
+    f = lib.nvfp4_rac_nsel
+    f.restype, f.argtypes = ctypes.c_int64, [ctypes.c_float, ctypes.c_int64]
+    for k in (0.0, 12.5, 25.0, 33.3, 50.0, 99.99, 100.0, 0.1):
+        for K in (64, 1000, 2048, 11008):
+            assert f(k, K) == oracle.n_selected(k, K)
+    assert f(-1.0, 64) == -1 and f(100.5, 64) == -1
+    w = lib.nvfp4_rac_width
+    w.restype, w.argtypes = ctypes.c_int64, [ctypes.c_int64]
+    assert [w(n) for n in (0, 1, 64, 65, 5504)] == [0, 64, 64, 128, 5504]
+
+
+def test_scale_bytes_and_workspace(lib):
+    f = lib.nvfp4_scale_bytes
+    f.restype, f.argtypes = ctypes.c_size_t, [ctypes.c_int64, ctypes.c_int64, ctypes.c_int32]
+    assert f(64, 512, 0) == 64 * 32
+    assert f(64, 512, 1) == 128 * 32
+    assert f(300, 192, 1) == 384 * 4 * 3
+    ws = lib.nvfp4_workspace_size
+    ws.restype = ctypes.c_size_t
+    ws.argtypes = [ctypes.c_int32, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int32]
+    assert ws(0, 4096, 0, 2048, 1) >= 32 * 2048 * 12
+    assert ws(9, 1, 1, 64, 1) == 0
+
+
+def test_argument_errors_without_gpu(lib):
+    q = lib.nvfp4_quantize
+    q.restype = ctypes.c_int32
+    # null input -> NVFP4_ERR_INVALID_ARG before any CUDA call
+    assert q(None, 64, 64, 64, None, None, None, None, None, 0, None) == 1
+    s = lib.nvfp4_status_string
+    s.restype, s.argtypes = ctypes.c_char_p, [ctypes.c_int32]
+    assert s(6) == b"device-side wait timed out"
