@@ -166,6 +166,23 @@ def profiled_traffic(kernel, workload):
     return None
 
 
+# ---------------------------------------------------------------- ranks
+def max_over_ranks(values, world, device="cpu"):
+    """Element-wise max of per-rank timings (every rank gets the result)."""
+    if world <= 1:
+        return [float(v) for v in values]
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.cpu()]
+
+
+def replica_seed(rank):
+    """Each data-parallel replica quantizes its own batch."""
+    return rank
+
+
 # ---------------------------------------------------------------- ours
 def run_ours(args, rank, world, local_rank):
     import torch
@@ -178,7 +195,7 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(dev)
     M, K, N, k = WORKLOADS[args.workload]
     k = args.k if args.k is not None else k
-    seed = rank                                   # each replica its own batch
+    seed = replica_seed(rank)
     x_host = S.activations(M, K, seed=seed).pin_memory()
     w_host = S.weights(N, K, seed=seed).pin_memory()
     x = x_host.to(dev)
@@ -298,12 +315,7 @@ def run_ours(args, rank, world, local_rank):
     if B.stream_status() != 0:
         raise RuntimeError("device error word set during timing")
 
-    if world > 1:
-        t = torch.tensor([total_ms, sum(e2e_ms)], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms, e2e_total = float(t[0]), float(t[1])
-    else:
-        e2e_total = sum(e2e_ms)
+    total_ms, e2e_total = max_over_ranks([total_ms, sum(e2e_ms)], world, dev)
 
     n_sel, width = plan.n_sel, plan.width
     flops_step = 2.0 * M * N * (K + n_sel)

@@ -93,7 +93,7 @@ struct QuantWs {
 QuantWs carve_quant(Carver& c, int64_t M, int64_t K, bool scores) {
   QuantWs w{};
   const int64_t tiles = ceil_div(M, kTileRows);
-  w.amax = c.take<unsigned>(1);
+  w.amax = c.take<unsigned>(1 + K / 64);      // amax, then one counter per 64-column strip
   if (scores) {
     w.part_sum = c.take<double>(tiles * K);
     w.part_max = c.take<float>(tiles * K);
@@ -216,16 +216,14 @@ nvfp4_status nvfp4_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ldx
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const RowGroups g = dense_groups(M);
   const float* amax = amax_or_null;
+  NV_TRY(cudaMemsetAsync(w.amax, 0, sizeof(unsigned) * (1 + K / 64), s));
   if (amax == nullptr) {
-    NV_TRY(cudaMemsetAsync(w.amax, 0, sizeof(unsigned), s));
     NV_TRY(launch_amax(x, M, K, ldx, g, w.amax, s));
     amax = reinterpret_cast<const float*>(w.amax);
   }
   NV_TRY(launch_quant_score(x, M, K, ldx, g, amax, M, qx->codes, qx->scales, qx->scale_layout,
-                            qx->tensor_scale, w.part_sum, w.part_max, s));
-  if (scores)
-    NV_TRY(launch_score_reduce(w.part_sum, w.part_max, K, g, ceil_div(M, kTileRows), score_or_null,
-                               res_colamax_or_null, nullptr, s));
+                            qx->tensor_scale, w.part_sum, w.part_max, scores ? w.amax + 1 : nullptr,
+                            score_or_null, res_colamax_or_null, s));
   return NVFP4_OK;
 }
 
@@ -272,11 +270,10 @@ nvfp4_status rac_weight_quant(const uint16_t* w, int64_t N, int64_t K, int64_t l
   const nvfp4_status d = device_ok();
   if (d != NVFP4_OK) return d;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  NV_TRY(launch_sel_tensor_scale(w_colamax, K, sel, n_sel, 1, q_wsel->tensor_scale, s));
   if (q_wsel->scale_layout == 1 && N % 128 != 0)
     NV_TRY(cudaMemsetAsync(q_wsel->scales, 0, scale_bytes(N, width, 1), s));
-  NV_TRY(launch_weight_gather(w, N, K, ldw, 1, sel, n_sel, width, q_wsel->tensor_scale, q_wsel->codes,
-                              q_wsel->scales, q_wsel->scale_layout, s));
+  NV_TRY(launch_weight_gather(w, N, K, ldw, 1, sel, n_sel, width, w_colamax, q_wsel->tensor_scale,
+                              q_wsel->codes, q_wsel->scales, q_wsel->scale_layout, s));
   return NVFP4_OK;
 }
 
@@ -381,7 +378,8 @@ nvfp4_status moe_grouped_w4a4_rac_gemm(const uint16_t* x_perm, int64_t T, int64_
   NV_TRY(cudaMemsetAsync(m.amax, 0, sizeof(unsigned) * E, s));
   NV_TRY(launch_amax(x_perm, T, K, K, g, m.amax, s));
   NV_TRY(launch_quant_score(x_perm, T, K, K, g, reinterpret_cast<const float*>(m.amax), prows,
-                            m.qx_codes, m.qx_scales, 1, m.qx_st, m.part_sum, m.part_max, s));
+                            m.qx_codes, m.qx_scales, 1, m.qx_st, m.part_sum, m.part_max, nullptr,
+                            nullptr, nullptr, s));
   NV_TRY(launch_score_reduce(m.part_sum, m.part_max, K, g, tiles, m.score, m.colamax, m.qx_st, s));
   NV_TRY(launch_topk(m.score, m.colamax, K, E, n_sel, mask, m.sel, m.r_st, s));
   GemmArgs a{};
@@ -390,8 +388,8 @@ nvfp4_status moe_grouped_w4a4_rac_gemm(const uint16_t* x_perm, int64_t T, int64_
   if (n_sel > 0) {
     NV_TRY(launch_residual_gather(x_perm, T, K, K, g, prows, m.qx_codes, m.qx_scales, 1, m.qx_st, m.sel,
                                   n_sel, width, m.r_st, m.r_codes, m.r_scales, 1, s));
-    NV_TRY(launch_sel_tensor_scale(w_colamax, K, m.sel, n_sel, E, m.ws_st, s));
-    NV_TRY(launch_weight_gather(w, N, K, K, E, m.sel, n_sel, width, m.ws_st, m.ws_codes, m.ws_scales, 1, s));
+    NV_TRY(launch_weight_gather(w, N, K, K, E, m.sel, n_sel, width, w_colamax, m.ws_st, m.ws_codes,
+                                m.ws_scales, 1, s));
     a.a1 = {m.r_codes, m.r_scales, m.r_st, prows, width};
     a.b1 = {m.ws_codes, m.ws_scales, m.ws_st, static_cast<int64_t>(E) * N, width};
   }

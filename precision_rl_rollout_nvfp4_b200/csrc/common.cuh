@@ -9,6 +9,7 @@
 
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <stdint.h>
 
 namespace nvfp4 {
@@ -94,18 +95,143 @@ __device__ __forceinline__ BlockScale block_scale(float amax_b, float s_t) {
   return r;
 }
 
-// RN(x / s_dec), or the signed zero of x when s_dec == 0.
-__device__ __forceinline__ float scaled(float x, float s_dec) {
-  return s_dec > 0.0f ? __fdiv_rn(x, s_dec) : __uint_as_float(__float_as_uint(x) & 0x80000000u);
+// RN(x / b) for a whole block that shares the divisor b = s_dec > 0, with
+// y = RN(1/b) computed once per block (__frcp_rn).  Markstein's correction
+// (P. Markstein, IBM J. Res. Dev. 1990; Muller et al., Handbook of
+// Floating-Point Arithmetic, division with an FMA): q = RN(x y) is within one
+// ulp of x/b, the remainder r = x - b q is exact with an FMA, and
+// RN(q + r y) = RN(x / b) when y is within half an ulp of 1/b and nothing
+// under- or overflows.  Blocks whose divisor is below 2^-100 use the full
+// division instead.  The sign of the result is that of x (x = -0 gives -0).
+struct BlockDivisor {
+  float b, y;
+  bool fast;
+};
+
+__device__ __forceinline__ BlockDivisor block_divisor(float s_dec) {
+  BlockDivisor d;
+  d.b = s_dec;
+  d.fast = s_dec >= 7.888609052210118e-31f;   // 2^-100
+  d.y = d.fast ? __frcp_rn(s_dec) : 0.0f;
+  return d;
+}
+
+__device__ __forceinline__ float div_block(float x, const BlockDivisor& d) {
+  float q;
+  if (d.b <= 0.0f) {
+    q = 0.0f;
+  } else if (d.fast) {
+    const float q0 = __fmul_rn(x, d.y);
+    const float r = __fmaf_rn(-q0, d.b, x);
+    q = __fmaf_rn(r, d.y, q0);
+  } else {
+    q = __fdiv_rn(x, d.b);
+  }
+  return __uint_as_float((__float_as_uint(q) & 0x7FFFFFFFu) | (__float_as_uint(x) & 0x80000000u));
 }
 
 // Codes of 8 consecutive elements (one half of a block) -> 4 bytes, element
 // 2j in the low nibble of byte j.
-__device__ __forceinline__ uint32_t encode8(const float* v, float s_dec) {
+__device__ __forceinline__ uint32_t encode8(const float* v, const BlockDivisor& d) {
   float q[8];
 #pragma unroll
-  for (int j = 0; j < 8; ++j) q[j] = scaled(v[j], s_dec);
+  for (int j = 0; j < 8; ++j) q[j] = div_block(v[j], d);
   return e2m1x8(q);
+}
+
+// Per-tensor-scale lookup of everything a block needs, built once per CTA
+// (and per tensor scale): for every non-negative E4M3 code sb,
+//   sbv[sb]  = E4M3dec(sb)                 (exact),
+//   sdec[sb] = RN(sbv[sb] * s_t)           (the block decode scale),
+//   rcp[sb]  = RN(1 / sdec[sb])            (0 when sdec < 2^-64: full division),
+// plus d = RN(6 s_t) and its reciprocal for the block-scale quotient.  The
+// quotients then cost one multiply and two FMAs (Markstein's correction, see
+// div_block) instead of a full IEEE division per block and per element.
+struct ScaleTable {
+  float sbv[128], sdec[128], rcp[128];
+  float s_t, d, rcp_d;
+};
+
+// Threads [0, nthreads) fill the table; the caller synchronizes afterwards.
+__device__ __forceinline__ void build_scale_table(ScaleTable& T, float s_t, int tid) {
+  if (tid < 128) {
+    const float v = tid < 127 ? e4m3_to_f32(static_cast<uint32_t>(tid)) : 0.0f;
+    const float sd = __fmul_rn(v, s_t);
+    T.sbv[tid] = v;
+    T.sdec[tid] = sd;
+    T.rcp[tid] = sd >= 5.421010862427522e-20f ? __frcp_rn(sd) : 0.0f;   // 2^-64
+  }
+  if (tid == 0) {
+    const float d = __fmul_rn(6.0f, s_t);
+    T.s_t = s_t;
+    T.d = d;
+    T.rcp_d = d >= 5.421010862427522e-20f ? __frcp_rn(d) : 0.0f;
+  }
+}
+
+static __device__ __noinline__ float div_slow(float a, float b) { return __fdiv_rn(a, b); }
+
+// RN(a / b) for a >= 0, b > 0, with y = RN(1/b) (or y == 0: full division).
+// With b >= 2^-64 the remainder a - b q0 is exact for every quotient that can
+// change an E2M1 or E4M3 code (>= 2^-10), so Markstein's correction holds.
+__device__ __forceinline__ float div_rn_pos(float a, float b, float y) {
+  if (y == 0.0f) return div_slow(a, b);
+  const float q0 = __fmul_rn(a, y);
+  const float r = __fmaf_rn(-q0, b, a);
+  return __fmaf_rn(r, y, q0);
+}
+
+// Block parameters from the table: sb = E4M3(RN(amax_b / d)).
+struct BlockQ {
+  uint32_t sb;
+  float sbv, sdec, rcp;
+};
+
+__device__ __forceinline__ BlockQ block_q(float amax_b, const ScaleTable& T) {
+  BlockQ q;
+  q.sb = T.d > 0.0f ? f32_to_e4m3(div_rn_pos(amax_b, T.d, T.rcp_d)) : 0u;
+  q.sbv = T.sbv[q.sb];
+  q.sdec = T.sdec[q.sb];
+  q.rcp = T.rcp[q.sb];
+  return q;
+}
+
+// E2M1 codes of 8 values with block parameters q: magnitudes of RN(|v|/sdec)
+// through the hardware conversion, sign bits from v (so -0 keeps code 0x8).
+__device__ __forceinline__ uint32_t encode8_q(const float* v, const BlockQ& q) {
+  float a[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) a[j] = q.sdec > 0.0f ? div_rn_pos(fabsf(v[j]), q.sdec, q.rcp) : 0.0f;
+  uint32_t mags;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(mags)
+      : "f"(a[0]), "f"(a[1]), "f"(a[2]), "f"(a[3]), "f"(a[4]), "f"(a[5]), "f"(a[6]), "f"(a[7]));
+  uint32_t signs = 0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) signs |= (__float_as_uint(v[j]) >> 31) << (4 * j + 3);
+  return mags | signs;
+}
+
+// Exact E4M3 value of a non-negative code through the hardware e4m3 -> f16
+// conversion (every E4M3 value is an f16 value).
+__device__ __forceinline__ float e4m3_to_f32_hw(uint32_t code) {
+  uint32_t h2;
+  asm("{\n\t.reg .b16 t;\n\tcvt.u16.u32 t, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, t;\n\t}" : "=r"(h2) : "r"(code & 0xFFu));
+  return __half2float(__ushort_as_half(static_cast<unsigned short>(h2 & 0xFFFFu)));
+}
+
+// Exact E2M1 values of the two codes of a packed byte (low nibble first),
+// through the hardware e2m1x2 -> f16x2 conversion.
+__device__ __forceinline__ void e2m1x2_to_f32(uint32_t byte, float& lo, float& hi) {
+  uint32_t h2;
+  asm("{\n\t.reg .b8 t;\n\tcvt.u8.u32 t, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, t;\n\t}" : "=r"(h2) : "r"(byte));
+  lo = __half2float(__ushort_as_half(static_cast<unsigned short>(h2 & 0xFFFFu)));
+  hi = __half2float(__ushort_as_half(static_cast<unsigned short>(h2 >> 16)));
 }
 
 // DQ = RN(RN(E2M1dec(code) * E4M3dec(sb)) * s_t).
@@ -195,12 +321,14 @@ __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" :: "r"(smem_u32(bar)), "r"(count));
 }
 
+// One poll; the thread may be parked by the hardware until the phase
+// completes or the suspend-time hint (10 ms) expires, whichever is first.
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile("{\n\t.reg .pred p;\n\t"
-               "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+               "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
                "selp.u32 %0, 1, 0, p;\n\t}"
-               : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+               : "=r"(ok) : "r"(bar), "r"(parity), "r"(10000000u) : "memory");
   return ok != 0;
 }
 

@@ -13,7 +13,7 @@
 // Design (one CTA per SM, persistent over 128 x 128 output tiles):
 //   warp 0      TMA producer: per 256-element K step, two 2-D tensor copies
 //               (A and B tiles, 128 B rows, 128 B swizzle) and two bulk
-//               copies of the matching 128 x 16 scale atoms into a 5-stage
+//               copies of the matching 128 x 16 scale atoms into a 4/5-stage
 //               shared-memory ring guarded by full / empty mbarriers.
 //   warp 1      MMA issuer: copies each stage's scales into TMEM
 //               (tcgen05.cp 32x128b.warpx4), then issues four
@@ -22,7 +22,8 @@
 //               accumulator 1 for the residual segment; tcgen05.commit frees
 //               the stage and, after the last step, signals the epilogue.
 //   warps 2..5  epilogue: tcgen05.ld of both accumulators (TMEM lane = output
-//               row), Y = alpha0 acc0 + alpha1 acc1, stores fp32 or bf16.
+//               row), Y = alpha0 acc0 + alpha1 acc1 into a shared staging tile,
+//               TMEM released, then coalesced fp32 / bf16 row stores.
 // The two tensor scales differ, so the segments accumulate separately.  No
 // TMA multicast is used.  Every mbarrier wait is bounded (see common.cuh).
 #include <cuda.h>
@@ -35,13 +36,22 @@ namespace {
 
 constexpr int BM = 128, BN = 128;
 constexpr int BK_BYTES = 128;                    // 256 FP4 elements per K step
-constexpr int STAGES = 5;
 constexpr int A_STAGE = BM * BK_BYTES;           // 16 KB
 constexpr int B_STAGE = BN * BK_BYTES;           // 16 KB
 constexpr int SF_ATOM = 512;                     // 128 rows x 4 scales
 constexpr int SF_STAGE = 4 * SF_ATOM;            // 4 MMA K blocks per step
-constexpr int SMEM_BYTES = 1024 + STAGES * (A_STAGE + B_STAGE + 2 * SF_STAGE) + 256;
 constexpr int THREADS = 192;
+
+// Per output type: pipeline depth and the epilogue staging tile (128 rows,
+// row stride padded by 16 bytes so 16-byte shared stores of 8 consecutive
+// rows hit distinct banks).
+template <int YBYTES>
+struct Cfg {
+  static constexpr int STAGES = YBYTES == 2 ? 5 : 4;
+  static constexpr int STG_STRIDE = BN * YBYTES + 16;
+  static constexpr int STG_BYTES = BM * STG_STRIDE;
+  static constexpr int SMEM_BYTES = 1024 + STAGES * (A_STAGE + B_STAGE + 2 * SF_STAGE) + STG_BYTES + 256;
+};
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC0_COL = 0, ACC1_COL = 128;   // two 128-column fp32 accumulators
 constexpr uint32_t SFA_COL = 256, SFB_COL = 272;
@@ -139,10 +149,13 @@ __device__ __forceinline__ void tmem_ld_wait() {
 }
 
 // ---- the kernel -----------------------------------------------------------
+template <int YBYTES>
 __global__ void __launch_bounds__(THREADS, 1)
 w4a4_rac_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
                      const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
                      const KParams p) {
+  constexpr int STAGES = Cfg<YBYTES>::STAGES;
+  constexpr int STG_STRIDE = Cfg<YBYTES>::STG_STRIDE;
   extern __shared__ uint8_t smem_raw[];
   // 128-byte swizzled tiles need 1024-byte aligned shared addresses
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -150,7 +163,8 @@ w4a4_rac_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_cons
   uint8_t* sB = sA + STAGES * A_STAGE;
   uint8_t* sSFA = sB + STAGES * B_STAGE;
   uint8_t* sSFB = sSFA + STAGES * SF_STAGE;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sSFB + STAGES * SF_STAGE);
+  uint8_t* sOut = sSFB + STAGES * SF_STAGE;                     // epilogue staging
+  uint64_t* full = reinterpret_cast<uint64_t*>(sOut + Cfg<YBYTES>::STG_BYTES);
   uint64_t* empty = full + STAGES;
   uint64_t* tmem_full = empty + STAGES;
   uint64_t* tmem_empty = tmem_full + 1;
@@ -252,8 +266,13 @@ w4a4_rac_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_cons
     }
   } else {
     // ------------------------------ epilogue (warps 2..5)
+    // TMEM -> registers -> Y = a0 acc0 + a1 acc1 -> shared staging (this
+    // warp's 32 rows); TMEM is released before the global stores so the next
+    // tile's MMAs overlap them; rows then leave as coalesced 256/512 B stores.
     const int q = warp & 3;                        // TMEM lane quadrant of this warp
     const uint32_t trow = tmem + (static_cast<uint32_t>(32 * q) << 16);
+    uint8_t* stg_warp = sOut + (32 * q) * STG_STRIDE;
+    uint8_t* stg_row = stg_warp + lane * STG_STRIDE;
     uint32_t acc_phase = 0;
     for (int64_t tile = blockIdx.x; tile < total; tile += gridDim.x) {
       bool ok = true;
@@ -265,9 +284,7 @@ w4a4_rac_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_cons
       const TileInfo ti = tile_info(p.g, mt);
       const float al0 = __fmul_rn(p.sta[0][ti.e], p.stb[0][ti.e]);
       const float al1 = nseg > 1 ? __fmul_rn(p.sta[1][ti.e], p.stb[1][ti.e]) : 0.0f;
-      const int64_t row = ti.row0 + 32 * q + lane;
-      const bool row_ok = ti.valid && row < ti.row_end;
-#pragma unroll 1
+#pragma unroll
       for (int c = 0; c < BN / 32; ++c) {
         float v[32], u[32];
         tmem_ld32(trow + ACC0_COL + 32 * c, v);
@@ -280,36 +297,37 @@ w4a4_rac_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_cons
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(al0, v[i]);
         }
-        const int64_t col = nt * BN + 32 * c;
-        if (!row_ok || col >= p.N) continue;
-        if (p.y_dtype == 0) {
-          float* yr = static_cast<float*>(p.y) + row * p.ldy + col;
-          if (col + 32 <= p.N) {
+        if (YBYTES == 4) {
 #pragma unroll
-            for (int i = 0; i < 32; i += 4)
-              *reinterpret_cast<float4*>(yr + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
-          } else {
-            for (int i = 0; i < 32 && col + i < p.N; ++i) yr[i] = v[i];
-          }
+          for (int i = 0; i < 32; i += 4)
+            *reinterpret_cast<float4*>(stg_row + (32 * c + i) * 4) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
         } else {
-          uint16_t* yr = static_cast<uint16_t*>(p.y) + row * p.ldy + col;
           uint32_t w[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i)
             w[i] = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(v[2 * i]))) |
                    (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(v[2 * i + 1]))) << 16);
-          if (col + 32 <= p.N) {
 #pragma unroll
-            for (int i = 0; i < 16; i += 4)
-              *reinterpret_cast<uint4*>(yr + 2 * i) = make_uint4(w[i], w[i + 1], w[i + 2], w[i + 3]);
-          } else {
-            for (int i = 0; i < 32 && col + i < p.N; ++i)
-              yr[i] = static_cast<uint16_t>(w[i >> 1] >> (16 * (i & 1)));
-          }
+          for (int i = 0; i < 16; i += 4)
+            *reinterpret_cast<uint4*>(stg_row + (32 * c + 2 * i) * 2) = make_uint4(w[i], w[i + 1], w[i + 2], w[i + 3]);
         }
       }
       tc_fence_before();
-      mbar_arrive(tmem_empty);
+      mbar_arrive(tmem_empty);                     // accumulators free for the next tile
+      __syncwarp();
+      const int64_t col = nt * BN + 4 * lane;      // this lane's 4 columns of every row
+      const bool col_ok = col + 4 <= p.N;
+#pragma unroll 4
+      for (int r = 0; r < 32; ++r) {
+        const int64_t row = ti.row0 + 32 * q + r;
+        if (!ti.valid || row >= ti.row_end || !col_ok) continue;
+        const uint8_t* src = stg_warp + r * STG_STRIDE + lane * 4 * YBYTES;
+        if (YBYTES == 4)
+          *reinterpret_cast<float4*>(static_cast<float*>(p.y) + row * p.ldy + col) = *reinterpret_cast<const float4*>(src);
+        else
+          *reinterpret_cast<uint2*>(static_cast<uint16_t*>(p.y) + row * p.ldy + col) = *reinterpret_cast<const uint2*>(src);
+      }
+      __syncwarp();
       acc_phase ^= 1;
     }
   }
@@ -354,16 +372,23 @@ int sm_count() {
   return n > 0 ? n : 148;
 }
 
-}  // namespace
-
-cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s) {
+template <int YBYTES>
+cudaError_t prepare_kernel() {
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(w4a4_rac_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         SMEM_BYTES);
+    cudaError_t e = cudaFuncSetAttribute(w4a4_rac_gemm_kernel<YBYTES>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<YBYTES>::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
+  return cudaSuccess;
+}
+
+}  // namespace
+
+cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s) {
+  cudaError_t e = a.y_dtype == 0 ? prepare_kernel<4>() : prepare_kernel<2>();
+  if (e != cudaSuccess) return e;
   KParams p{};
   p.g = a.g;
   p.N = a.N;
@@ -396,7 +421,10 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s) {
   const int64_t tiles_bound = a.m_tiles * p.n_tiles;
   if (tiles_bound == 0) return cudaSuccess;
   const int grid = static_cast<int>(tiles_bound < sm_count() ? tiles_bound : sm_count());
-  w4a4_rac_gemm_kernel<<<grid, THREADS, SMEM_BYTES, s>>>(maps[0], maps[1], maps[2], maps[3], p);
+  if (a.y_dtype == 0)
+    w4a4_rac_gemm_kernel<4><<<grid, THREADS, Cfg<4>::SMEM_BYTES, s>>>(maps[0], maps[1], maps[2], maps[3], p);
+  else
+    w4a4_rac_gemm_kernel<2><<<grid, THREADS, Cfg<2>::SMEM_BYTES, s>>>(maps[0], maps[1], maps[2], maps[3], p);
   return cudaGetLastError();
 }
 

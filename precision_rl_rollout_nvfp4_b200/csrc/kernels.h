@@ -26,11 +26,14 @@ cudaError_t launch_group_tiles(const int64_t* off, int32_t E, int32_t* tile_star
 
 // Q(X) plus score partials.  amax: fp32 per group.  codes [codes_rows, K/2]
 // on padded rows; scales in `layout`; tensor_scale[e] written for non-empty
-// groups; part_sum / part_max [tiles, K] (may be null).
+// groups; part_sum / part_max [tiles, K] (may be null).  With strip_count
+// (E x K/64 counters, zero on entry and left zero) the last CTA of every
+// column strip of a group also writes score[e, :] and colamax[e, :].
 cudaError_t launch_quant_score(const uint16_t* x, int64_t rows, int64_t K, int64_t ldx,
                                const RowGroups& g, const float* amax, int64_t codes_rows,
                                uint8_t* codes, uint8_t* scales, int layout, float* tensor_scale,
-                               double* part_sum, float* part_max, cudaStream_t s);
+                               double* part_sum, float* part_max, unsigned* strip_count,
+                               double* score, float* colamax, cudaStream_t s);
 
 // score[e, j] = sum over the group's tiles of part_sum in tile order;
 // colamax[e, j] = max of part_max.  For empty groups (MoE) also writes
@@ -57,11 +60,12 @@ cudaError_t launch_sel_tensor_scale(const float* colamax, int64_t K, const int32
                                     int64_t n_sel, int32_t E, float* s_t, cudaStream_t s);
 
 // Q(W_sel) for E stacked weights [E, N, K] (row stride ldw, matrix stride
-// N*ldw): out rows E*N, width columns.
+// N*ldw): out rows E*N, width columns.  Also writes the W_sel tensor scales
+// s_t[e] = RN(max_{j in sel_e} colamax[e*K + j] / 2688).
 cudaError_t launch_weight_gather(const uint16_t* w, int64_t N, int64_t K, int64_t ldw, int32_t E,
                                  const int32_t* sel, int64_t n_sel, int64_t width,
-                                 const float* s_t, uint8_t* codes, uint8_t* scales, int layout,
-                                 cudaStream_t s);
+                                 const float* colamax, float* s_t, uint8_t* codes, uint8_t* scales,
+                                 int layout, cudaStream_t s);
 
 // W' = bf16(DQ(Q(W))) for `batch` matrices; optional Q(W) and colamax
 // (colamax_bits zeroed by the caller, written as fp32 bits).

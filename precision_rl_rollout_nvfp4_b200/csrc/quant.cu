@@ -73,58 +73,72 @@ __global__ void group_tiles_kernel(const int64_t* __restrict__ off, int32_t E,
 }
 
 // ---------------------------------------------------------------------------
-// quantize + residual + score partials
+// quantize + residual + score partials (+ the ordered reduction of the
+// partials by the last CTA of each 64-column strip of a row group)
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(kQThreads)
+__global__ void __launch_bounds__(kQThreads, 5)
 quant_score_kernel(const uint16_t* __restrict__ x, int64_t K, int64_t ldx, RowGroups g,
                    const float* __restrict__ amax, int64_t codes_rows,
                    uint8_t* __restrict__ codes, uint8_t* __restrict__ scales, int layout,
                    float* __restrict__ tensor_scale, double* __restrict__ part_sum,
-                   float* __restrict__ part_max) {
+                   float* __restrict__ part_max, unsigned* __restrict__ strip_count,
+                   double* __restrict__ score, float* __restrict__ colamax) {
   const int64_t tile = blockIdx.y;
   const TileInfo ti = tile_info(g, tile);
   if (!ti.valid) return;
-  __shared__ float dxs[kTileRows][kDxStride];
+  // |dX| of the tile; reused by the strip's last CTA to stage partials
+  __shared__ __align__(16) float dxs[kTileRows][kDxStride];
+  __shared__ bool s_last;
   const int t = threadIdx.x, cg = t & 7, rr = t >> 3;
   const int64_t col0 = static_cast<int64_t>(blockIdx.x) * kQCols;
   const int64_t col = col0 + 8 * cg;
   const float s_t = __fdiv_rn(amax[ti.e], kTensorScaleDiv);
   if (blockIdx.x == 0 && t == 0 && (g.off == nullptr ? tile == 0 : tile == g.tile_start[ti.e]))
     tensor_scale[ti.e] = s_t;
+  __shared__ ScaleTable T;
+  build_scale_table(T, s_t, t);
 
+  uint4 raw[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int64_t row = ti.row0 + rr + 32 * i;
+    raw[i] = row < ti.row_end ? ld_nc_v4(x + row * ldx + col) : make_uint4(0, 0, 0, 0);
+  }
+  __syncthreads();                               // table ready
+  uint8_t* code_base = codes + tile * kTileRows * (K / 2) + col / 2;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int r = rr + 32 * i;
-    const int64_t row = ti.row0 + r;
     const int64_t prow = tile * kTileRows + r;
     float f[8];
-    if (row < ti.row_end) {
-      unpack_bf16x8(ld_nc_v4(x + row * ldx + col), f);
-    } else {
-#pragma unroll
-      for (int j = 0; j < 8; ++j) f[j] = 0.0f;
-    }
+    unpack_bf16x8(raw[i], f);
     float am = 0.0f;
 #pragma unroll
     for (int j = 0; j < 8; ++j) am = fmaxf(am, fabsf(f[j]));
     am = fmaxf(am, __shfl_xor_sync(0xFFFFFFFFu, am, 1));
-    const BlockScale bs = block_scale(am, s_t);
-    const uint32_t q = encode8(f, bs.s_dec);
+    const BlockQ bq = block_q(am, T);
+    const uint32_t packed = encode8_q(f, bq);
+    float d[8];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const float dq = dequant((q >> (4 * j)) & 15u, bs.sbv, s_t);
-      dxs[r][8 * cg + j] = fabsf(__fsub_rn(f[j], dq));
+    for (int j = 0; j < 4; ++j) {
+      float lo, hi;
+      e2m1x2_to_f32((packed >> (8 * j)) & 0xFFu, lo, hi);
+      d[2 * j] = fabsf(__fsub_rn(f[2 * j], __fmul_rn(__fmul_rn(lo, bq.sbv), s_t)));
+      d[2 * j + 1] = fabsf(__fsub_rn(f[2 * j + 1], __fmul_rn(__fmul_rn(hi, bq.sbv), s_t)));
     }
+    *reinterpret_cast<float4*>(&dxs[r][8 * cg]) = make_float4(d[0], d[1], d[2], d[3]);
+    *reinterpret_cast<float4*>(&dxs[r][8 * cg + 4]) = make_float4(d[4], d[5], d[6], d[7]);
     if (prow < codes_rows)
-      *reinterpret_cast<uint32_t*>(codes + prow * (K / 2) + col / 2) = q;
+      *reinterpret_cast<uint32_t*>(code_base + static_cast<uint32_t>(r) * static_cast<uint32_t>(K / 2)) = packed;
     if ((cg & 1) == 0 && (layout == 1 || prow < codes_rows))
-      scales[scale_offset(prow, col / kBlock, K, layout)] = static_cast<uint8_t>(bs.sb);
+      scales[scale_offset(prow, col / kBlock, K, layout)] = static_cast<uint8_t>(bq.sb);
   }
   if (part_sum == nullptr) return;
   __syncthreads();
   if (t < kQCols) {
     double acc = 0.0;
     float mx = 0.0f;
+#pragma unroll 8
     for (int r = 0; r < kTileRows; ++r) {       // row order within the chunk
       const float v = dxs[r][t];
       acc += static_cast<double>(v);
@@ -133,6 +147,50 @@ quant_score_kernel(const uint16_t* __restrict__ x, int64_t K, int64_t ldx, RowGr
     part_sum[tile * K + col0 + t] = acc;
     part_max[tile * K + col0 + t] = mx;
   }
+  if (strip_count == nullptr) return;
+  // The last CTA of this group's column strip sums the group's partials in
+  // tile order (so the result does not depend on which CTA finishes last).
+  __threadfence();
+  __syncthreads();
+  const int64_t t0 = g.off == nullptr ? 0 : g.tile_start[ti.e];
+  const int64_t t1 = g.off == nullptr ? (g.M + kTileRows - 1) / kTileRows : g.tile_start[ti.e + 1];
+  unsigned* counter = strip_count + static_cast<int64_t>(ti.e) * gridDim.x + blockIdx.x;
+  if (t == 0) {
+    const unsigned prev = atomicAdd(counter, 1u);
+    s_last = prev == static_cast<unsigned>(t1 - t0 - 1);
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  // stage up to 32 tiles' partials of this strip in shared memory (all 256
+  // threads load; 24 KB fits in the |dX| buffer), then 64 threads add them
+  // in tile order
+  constexpr int kStage = 32;
+  double* ps = reinterpret_cast<double*>(&dxs[0][0]);            // [32 tiles][64 cols]
+  float* pm = reinterpret_cast<float*>(ps + kStage * kQCols);     // [32 tiles][64 cols]
+  double acc = 0.0;
+  float mx = 0.0f;
+  for (int64_t c0 = t0; c0 < t1; c0 += kStage) {
+    const int nt = static_cast<int>(t1 - c0 < kStage ? t1 - c0 : kStage);
+    __syncthreads();
+    for (int k = t; k < nt * kQCols; k += kQThreads) {
+      const int tt = k / kQCols, cc = k % kQCols;
+      ps[k] = __ldcg(part_sum + (c0 + tt) * K + col0 + cc);
+      pm[k] = __ldcg(part_max + (c0 + tt) * K + col0 + cc);
+    }
+    __syncthreads();
+    if (t < kQCols) {
+      for (int tt = 0; tt < nt; ++tt) {          // chunk order
+        acc += ps[tt * kQCols + t];
+        mx = fmaxf(mx, pm[tt * kQCols + t]);
+      }
+    }
+  }
+  if (t < kQCols) {
+    score[static_cast<int64_t>(ti.e) * K + col0 + t] = acc;
+    colamax[static_cast<int64_t>(ti.e) * K + col0 + t] = mx;
+  }
+  if (t == 0) *counter = 0;                      // ready for the next call
 }
 
 __global__ void score_reduce_kernel(const double* __restrict__ part_sum,
@@ -158,52 +216,154 @@ __global__ void score_reduce_kernel(const double* __restrict__ part_sum,
 // ---------------------------------------------------------------------------
 // second-pass gather + quantize
 // ---------------------------------------------------------------------------
-constexpr int kGThreads = 128;
+constexpr int kGThreads = 256;
 
-// One thread per (padded row, 16-block of the gathered width).  grid.x = rows,
-// grid.y = ceil(width/16 / 128).
+// Second-pass gather + quantize, shared by the residual and the weight side.
+// A CTA (256 threads) takes tiles of 16 rows x 256 gathered channels:
+//   phase 1: sel[j0 .. j0+255] into shared memory; every thread gathers 16
+//            values (rows r, channels j0 + lane + 32 u): a warp's loads cover
+//            32 consecutive gathered channels, and all 16 are in flight;
+//            the residual side recomputes dX = x - DQ(Q(x)) from X, Q(X) and
+//            its scales; values go to shared memory;
+//   phase 2: thread = one 16-block (row, block): block scale, codes, stores.
+// Tiles are visited grid-stride; with fuse_scale (one weight) every CTA first
+// reduces the W_sel tensor scale from colamax and sel, CTA 0 publishes it.
+constexpr int kGRows = 16, kGCols = 256;
+
+template <bool RESIDUAL>
 __global__ void __launch_bounds__(kGThreads)
-residual_gather_kernel(const uint16_t* __restrict__ x, int64_t K, int64_t ldx, RowGroups g,
-                       const uint8_t* __restrict__ qx_codes, const uint8_t* __restrict__ qx_scales,
-                       int qx_layout, const float* __restrict__ qx_st,
-                       const int32_t* __restrict__ sel, int64_t n_sel, int64_t width,
-                       const float* __restrict__ r_st, uint8_t* __restrict__ r_codes,
-                       uint8_t* __restrict__ r_scales, int r_layout, int64_t r_rows) {
-  const int64_t prow = blockIdx.x;
-  const int64_t blk = static_cast<int64_t>(blockIdx.y) * kGThreads + threadIdx.x;
-  if (blk * kBlock >= width) return;
-  const TileInfo ti = tile_info(g, prow / kTileRows);
-  const int64_t row = ti.row0 + (prow % kTileRows);
-  const bool live = ti.valid && row < ti.row_end;
-  const int e = ti.e;
-  const float st_x = live ? qx_st[e] : 0.0f;
-  const float st_r = live ? r_st[e] : 0.0f;
-  const int32_t* s = sel + static_cast<int64_t>(e) * n_sel;
-  float v[16];
+gather_quant_kernel(const uint16_t* __restrict__ src, int64_t K, int64_t ld, RowGroups g,
+                    int64_t N_per_group, const uint8_t* __restrict__ qx_codes,
+                    const uint8_t* __restrict__ qx_scales, int qx_layout, const float* __restrict__ qx_st,
+                    const int32_t* __restrict__ sel, int64_t n_sel, int64_t width,
+                    const float* __restrict__ colamax, int fuse_scale, float* __restrict__ out_st,
+                    uint8_t* __restrict__ out_codes, uint8_t* __restrict__ out_scales, int out_layout,
+                    int64_t out_rows, int64_t grid_rows) {
+  __shared__ int32_t s_sel[kGCols];
+  __shared__ __align__(16) float s_val[kGRows][kGCols + 4];
+  __shared__ float s_fused;
+  __shared__ ScaleTable T;
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  if (!RESIDUAL && fuse_scale) {
+    float m = 0.0f;
+    for (int64_t j = t; j < n_sel; j += kGThreads) {
+      const int64_t c = __ldg(sel + j);
+      if (c >= 0 && c < K) m = fmaxf(m, __ldg(colamax + c));
+    }
+    m = __uint_as_float(__reduce_max_sync(0xFFFFFFFFu, __float_as_uint(m)));
+    __shared__ float wm[kGThreads / 32];
+    if (lane == 0) wm[warp] = m;
+    __syncthreads();
+    if (t == 0) {
+      float r = 0.0f;
+      for (int k = 0; k < kGThreads / 32; ++k) r = fmaxf(r, wm[k]);
+      s_fused = __fdiv_rn(r, kTensorScaleDiv);
+      if (blockIdx.x == 0) out_st[0] = s_fused;
+    }
+    __syncthreads();
+  }
+  const int64_t row_tiles = (grid_rows + kGRows - 1) / kGRows;
+  const int64_t col_tiles = (width + kGCols - 1) / kGCols;
+  for (int64_t tile = blockIdx.x; tile < row_tiles * col_tiles; tile += gridDim.x) {
+    const int64_t r0 = (tile / col_tiles) * kGRows, j0 = (tile % col_tiles) * kGCols;
+    // rows of this tile belong to one group: 16 divides 128 and N % 16 == 0
+    int e;
+    int64_t row_base, row_end;     // source row of r0, end of the group's rows
+    bool valid;
+    if (RESIDUAL) {
+      const TileInfo ti = tile_info(g, r0 / kTileRows);
+      e = ti.e;
+      valid = ti.valid;
+      row_base = ti.row0 + (r0 % kTileRows);
+      row_end = ti.row_end;
+    } else {
+      e = static_cast<int>(r0 / N_per_group);
+      valid = true;
+      row_base = r0;                               // stacked weight row e*N + n
+      row_end = static_cast<int64_t>(e + 1) * N_per_group;
+    }
+    __syncthreads();                               // previous tile done with shared memory
+    {
+      const int64_t j = j0 + t;
+      s_sel[t] = (valid && j < n_sel) ? __ldg(sel + static_cast<int64_t>(e) * n_sel + j) : -1;
+    }
+    __syncthreads();
+    const float st_x = (RESIDUAL && valid) ? qx_st[e] : 0.0f;
+    float st = 0.0f;
+    if (valid) st = RESIDUAL ? out_st[e] : (fuse_scale ? s_fused : out_st[e]);
+    build_scale_table(T, st, t);
+    // scale bytes of Q(X) for this row: row part of the tiled / canonical offset
+    const int64_t k4 = (K + 63) / 64;
+    // phase 1: warp w gathers rows 2w, 2w+1; lane takes channels lane + 32 u
 #pragma unroll
-  for (int u = 0; u < 16; ++u) {
-    const int64_t j = blk * kBlock + u;
-    v[u] = 0.0f;
-    if (live && j < n_sel) {
-      const int64_t c = s[j];
-      if (c < 0 || c >= K) continue;            // never taken for a valid sel list
-      const float xv = bf16_bits_to_f32(x[row * ldx + c]);
-      const uint32_t code = (qx_codes[prow * (K / 2) + (c >> 1)] >> (4 * (c & 1))) & 15u;
-      const uint32_t sb = qx_scales[scale_offset(prow, c / kBlock, K, qx_layout)];
-      v[u] = __fsub_rn(xv, dequant(code, e4m3_to_f32(sb), st_x));
+    for (int rr = 0; rr < 2; ++rr) {
+      const int r = 2 * warp + rr;
+      const int64_t srow = row_base + r;
+      const int64_t prow = r0 + r;
+      const bool live = valid && srow < row_end;
+      const uint16_t* xrow = src + srow * ld;
+      const uint8_t* crow = RESIDUAL ? qx_codes + prow * (K / 2) : nullptr;
+      const uint8_t* srow_sc = nullptr;
+      if (RESIDUAL)
+        srow_sc = qx_layout == 1
+                      ? qx_scales + ((prow >> 7) * k4) * 512 + (prow & 31) * 16 + ((prow & 127) >> 5) * 4
+                      : qx_scales + prow * (K / kBlock);
+      uint32_t xb[8], cb[8], sb[8];
+      int32_t c[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        c[u] = live ? s_sel[lane + 32 * u] : -1;
+        const bool ok = static_cast<uint32_t>(c[u]) < static_cast<uint32_t>(K);   // never false for a valid sel list
+        const uint32_t cc = ok ? static_cast<uint32_t>(c[u]) : 0u;
+        xb[u] = ok ? __ldg(xrow + cc) : 0u;
+        if (RESIDUAL) {
+          cb[u] = ok ? __ldg(crow + (cc >> 1)) : 0u;
+          const uint32_t so = qx_layout == 1 ? (cc >> 6) * 512u + ((cc >> 4) & 3u) : (cc >> 4);
+          sb[u] = ok ? __ldg(srow_sc + so) : 0u;
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        float v = 0.0f;
+        if (static_cast<uint32_t>(c[u]) < static_cast<uint32_t>(K)) {
+          v = bf16_bits_to_f32(xb[u]);
+          if (RESIDUAL) {
+            float lo, hi;
+            e2m1x2_to_f32((cb[u] >> (4 * (c[u] & 1))) & 15u, lo, hi);
+            v = __fsub_rn(v, __fmul_rn(__fmul_rn(lo, e4m3_to_f32_hw(sb[u])), st_x));
+          }
+        }
+        s_val[r][lane + 32 * u] = v;
+      }
+    }
+    __syncthreads();
+    // phase 2: thread = (row t/16, block t%16)
+    {
+      const int r = t >> 4, b = t & 15;
+      const int64_t prow = r0 + r;
+      const int64_t blk = j0 / kBlock + b;
+      const bool in_rows = prow < out_rows;
+      if (blk * kBlock < width && prow < grid_rows && (in_rows || out_layout == 1)) {
+        float v[16];
+        const float4* vp = reinterpret_cast<const float4*>(&s_val[r][16 * b]);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float4 f = vp[q];
+          v[4 * q] = f.x; v[4 * q + 1] = f.y; v[4 * q + 2] = f.z; v[4 * q + 3] = f.w;
+        }
+        float am = 0.0f;
+#pragma unroll
+        for (int u = 0; u < 16; ++u) am = fmaxf(am, fabsf(v[u]));
+        const BlockQ bq = block_q(am, T);
+        const uint32_t lo = encode8_q(v, bq), hi = encode8_q(v + 8, bq);
+        if (in_rows) *reinterpret_cast<uint2*>(out_codes + prow * (width / 2) + blk * 8) = make_uint2(lo, hi);
+        out_scales[scale_offset(prow, blk, width, out_layout)] = static_cast<uint8_t>(bq.sb);
+      }
     }
   }
-  float am = 0.0f;
-#pragma unroll
-  for (int u = 0; u < 16; ++u) am = fmaxf(am, fabsf(v[u]));
-  const BlockScale bs = block_scale(am, st_r);
-  const uint32_t lo = encode8(v, bs.s_dec), hi = encode8(v + 8, bs.s_dec);
-  if (prow < r_rows)
-    *reinterpret_cast<uint2*>(r_codes + prow * (width / 2) + blk * 8) = make_uint2(lo, hi);
-  if (r_layout == 1 || prow < r_rows)
-    r_scales[scale_offset(prow, blk, width, r_layout)] = static_cast<uint8_t>(bs.sb);
 }
 
+// s_t[e] = RN(max_{j < n_sel} colamax[e*K + sel[e*n_sel + j]] / 2688), one CTA per group.
 __global__ void sel_tensor_scale_kernel(const float* __restrict__ colamax, int64_t K,
                                         const int32_t* __restrict__ sel, int64_t n_sel,
                                         float* __restrict__ s_t) {
@@ -224,40 +384,12 @@ __global__ void sel_tensor_scale_kernel(const float* __restrict__ colamax, int64
   }
 }
 
-// One thread per (weight row, 16-block of the gathered width).
-// grid.x = E*N rows, grid.y = ceil(width/16 / 128).
-__global__ void __launch_bounds__(kGThreads)
-weight_gather_kernel(const uint16_t* __restrict__ w, int64_t N, int64_t K, int64_t ldw,
-                     const int32_t* __restrict__ sel, int64_t n_sel, int64_t width,
-                     const float* __restrict__ s_t, uint8_t* __restrict__ codes,
-                     uint8_t* __restrict__ scales, int layout) {
-  const int64_t row = blockIdx.x;                 // e * N + n
-  const int64_t blk = static_cast<int64_t>(blockIdx.y) * kGThreads + threadIdx.x;
-  if (blk * kBlock >= width) return;
-  const int64_t e = row / N;
-  const int32_t* s = sel + e * n_sel;
-  const uint16_t* wr = w + e * N * ldw + (row - e * N) * ldw;
-  float v[16];
-#pragma unroll
-  for (int u = 0; u < 16; ++u) {
-    const int64_t j = blk * kBlock + u;
-    const int64_t c = j < n_sel ? s[j] : -1;
-    v[u] = (c >= 0 && c < K) ? bf16_bits_to_f32(wr[c]) : 0.0f;
-  }
-  float am = 0.0f;
-#pragma unroll
-  for (int u = 0; u < 16; ++u) am = fmaxf(am, fabsf(v[u]));
-  const BlockScale bs = block_scale(am, s_t[e]);
-  const uint32_t lo = encode8(v, bs.s_dec), hi = encode8(v + 8, bs.s_dec);
-  *reinterpret_cast<uint2*>(codes + row * (width / 2) + blk * 8) = make_uint2(lo, hi);
-  scales[scale_offset(row, blk, width, layout)] = static_cast<uint8_t>(bs.sb);
-}
-
 // ---------------------------------------------------------------------------
 // weight fake quantization (W4A16 trainer side)
 // ---------------------------------------------------------------------------
-// CTA: 64 rows x 64 columns of one matrix; thread t: columns 8 (t & 7), rows
-// t/8 and t/8 + 32.  grid = (K/64, ceil(N/64), batch).
+// CTA: 128 rows x 64 columns of one matrix; thread t: columns 8 (t & 7), rows
+// t/8 + 32 i, i = 0..3 (all four 16-byte loads issued first).
+// grid = (K/64, ceil(N/128), batch).
 __global__ void __launch_bounds__(kQThreads)
 weight_qdq_kernel(const uint16_t* w, int64_t N, int64_t K, int64_t ldw,
                   const unsigned* __restrict__ amax_bits, uint16_t* w_out,   // w_out may alias w
@@ -268,19 +400,24 @@ weight_qdq_kernel(const uint16_t* w, int64_t N, int64_t K, int64_t ldw,
   const int64_t col = static_cast<int64_t>(blockIdx.x) * 64 + 8 * cg;
   const float s_t = __fdiv_rn(__uint_as_float(amax_bits[b]), kTensorScaleDiv);
   if (tensor_scale && blockIdx.x == 0 && blockIdx.y == 0 && t == 0) tensor_scale[b] = s_t;
+  __shared__ ScaleTable T;
+  build_scale_table(T, s_t, t);
   uint32_t cmax[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  uint4 raw[4];
 #pragma unroll
-  for (int i = 0; i < 2; ++i) {
-    const int64_t n = static_cast<int64_t>(blockIdx.y) * 64 + rr + 32 * i;
+  for (int i = 0; i < 4; ++i) {
+    const int64_t n = static_cast<int64_t>(blockIdx.y) * 128 + rr + 32 * i;
+    // coherent load: w may alias w_out
+    raw[i] = n < N ? *reinterpret_cast<const uint4*>(w + (b * N + n) * ldw + col) : make_uint4(0, 0, 0, 0);
+  }
+  __syncthreads();                               // table ready
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int64_t n = static_cast<int64_t>(blockIdx.y) * 128 + rr + 32 * i;
     const bool live = n < N;
     const int64_t off = (b * N + n) * ldw + col;
     float f[8];
-    if (live) {
-      unpack_bf16x8(*reinterpret_cast<const uint4*>(w + off), f);   // coherent load: w may alias w_out
-    } else {
-#pragma unroll
-      for (int j = 0; j < 8; ++j) f[j] = 0.0f;
-    }
+    unpack_bf16x8(raw[i], f);
     float am = 0.0f;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
@@ -288,15 +425,17 @@ weight_qdq_kernel(const uint16_t* w, int64_t N, int64_t K, int64_t ldw,
       cmax[j] = max(cmax[j], __float_as_uint(fabsf(f[j])));
     }
     am = fmaxf(am, __shfl_xor_sync(0xFFFFFFFFu, am, 1));
-    const BlockScale bs = block_scale(am, s_t);
-    const uint32_t q = encode8(f, bs.s_dec);
+    const BlockQ bs = block_q(am, T);
+    const uint32_t q = encode8_q(f, bs);
     const int64_t qrow = b * N + n;
     if (live) {
       uint32_t o[4];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const float d0 = dequant((q >> (8 * j)) & 15u, bs.sbv, s_t);
-        const float d1 = dequant((q >> (8 * j + 4)) & 15u, bs.sbv, s_t);
+        float lo, hi;
+        e2m1x2_to_f32((q >> (8 * j)) & 0xFFu, lo, hi);
+        const float d0 = __fmul_rn(__fmul_rn(lo, bs.sbv), s_t);
+        const float d1 = __fmul_rn(__fmul_rn(hi, bs.sbv), s_t);
         const uint32_t b0 = __bfloat16_as_ushort(__float2bfloat16_rn(d0));
         const uint32_t b1 = __bfloat16_as_ushort(__float2bfloat16_rn(d1));
         o[j] = b0 | (b1 << 16);
@@ -368,12 +507,14 @@ cudaError_t launch_group_tiles(const int64_t* off, int32_t E, int32_t* tile_star
 cudaError_t launch_quant_score(const uint16_t* x, int64_t rows, int64_t K, int64_t ldx,
                                const RowGroups& g, const float* amax, int64_t codes_rows,
                                uint8_t* codes, uint8_t* scales, int layout, float* tensor_scale,
-                               double* part_sum, float* part_max, cudaStream_t s) {
+                               double* part_sum, float* part_max, unsigned* strip_count,
+                               double* score, float* colamax, cudaStream_t s) {
   const int64_t tiles = max_tiles(g, rows);
   if (tiles == 0) return cudaSuccess;
   dim3 grid(static_cast<unsigned>(K / kQCols), static_cast<unsigned>(tiles));
   quant_score_kernel<<<grid, kQThreads, 0, s>>>(x, K, ldx, g, amax, codes_rows, codes, scales,
-                                                layout, tensor_scale, part_sum, part_max);
+                                                layout, tensor_scale, part_sum, part_max, strip_count,
+                                                score, colamax);
   return cudaGetLastError();
 }
 
@@ -386,6 +527,11 @@ cudaError_t launch_score_reduce(const double* part_sum, const float* part_max, i
   return cudaGetLastError();
 }
 
+int gather_grid(int64_t rows, int64_t width) {
+  const int64_t tiles = (rows + kGRows - 1) / kGRows * ((width + kGCols - 1) / kGCols);
+  return static_cast<int>(tiles < 8 * 148 ? tiles : 8 * 148);
+}
+
 cudaError_t launch_residual_gather(const uint16_t* x, int64_t rows, int64_t K, int64_t ldx,
                                    const RowGroups& g, int64_t prows,
                                    const uint8_t* qx_codes, const uint8_t* qx_scales, int qx_layout,
@@ -394,13 +540,11 @@ cudaError_t launch_residual_gather(const uint16_t* x, int64_t rows, int64_t K, i
                                    uint8_t* r_scales, int r_layout, cudaStream_t s) {
   (void)rows;
   if (width == 0 || prows == 0) return cudaSuccess;
-  const int64_t nblk = width / kBlock;
   // rows of the scale buffer are padded to 128 for the tiled layout
   const int64_t grid_rows = r_layout == 1 ? (prows + kTileRows - 1) / kTileRows * kTileRows : prows;
-  dim3 grid(static_cast<unsigned>(grid_rows), static_cast<unsigned>((nblk + kGThreads - 1) / kGThreads));
-  residual_gather_kernel<<<grid, kGThreads, 0, s>>>(x, K, ldx, g, qx_codes, qx_scales, qx_layout,
-                                                    qx_st, sel, n_sel, width, r_st, r_codes,
-                                                    r_scales, r_layout, prows);
+  gather_quant_kernel<true><<<gather_grid(grid_rows, width), kGThreads, 0, s>>>(
+      x, K, ldx, g, 0, qx_codes, qx_scales, qx_layout, qx_st, sel, n_sel, width, nullptr, 0,
+      const_cast<float*>(r_st), r_codes, r_scales, r_layout, prows, grid_rows);
   return cudaGetLastError();
 }
 
@@ -412,13 +556,19 @@ cudaError_t launch_sel_tensor_scale(const float* colamax, int64_t K, const int32
 
 cudaError_t launch_weight_gather(const uint16_t* w, int64_t N, int64_t K, int64_t ldw, int32_t E,
                                  const int32_t* sel, int64_t n_sel, int64_t width,
-                                 const float* s_t, uint8_t* codes, uint8_t* scales, int layout,
-                                 cudaStream_t s) {
+                                 const float* colamax, float* s_t, uint8_t* codes, uint8_t* scales,
+                                 int layout, cudaStream_t s) {
   if (width == 0) return cudaSuccess;
-  const int64_t nblk = width / kBlock;
-  dim3 grid(static_cast<unsigned>(E * N), static_cast<unsigned>((nblk + kGThreads - 1) / kGThreads));
-  weight_gather_kernel<<<grid, kGThreads, 0, s>>>(w, N, K, ldw, sel, n_sel, width, s_t, codes,
-                                                  scales, layout);
+  const int fuse = E == 1 ? 1 : 0;
+  if (!fuse) {
+    cudaError_t e = launch_sel_tensor_scale(colamax, K, sel, n_sel, E, s_t, s);
+    if (e != cudaSuccess) return e;
+  }
+  const int64_t rows = static_cast<int64_t>(E) * N;
+  RowGroups none{};
+  gather_quant_kernel<false><<<gather_grid(rows, width), kGThreads, 0, s>>>(
+      w, K, ldw, none, N, nullptr, nullptr, 0, nullptr, sel, n_sel, width, colamax, fuse, s_t, codes,
+      scales, layout, rows, rows);
   return cudaGetLastError();
 }
 
@@ -426,7 +576,7 @@ cudaError_t launch_weight_qdq(const uint16_t* w, int64_t N, int64_t K, int64_t l
                               const unsigned* amax_bits, uint16_t* w_out, uint8_t* codes,
                               uint8_t* scales, int layout, float* tensor_scale,
                               unsigned* colamax_bits, cudaStream_t s) {
-  dim3 grid(static_cast<unsigned>(K / 64), static_cast<unsigned>((N + 63) / 64),
+  dim3 grid(static_cast<unsigned>(K / 64), static_cast<unsigned>((N + 127) / 128),
             static_cast<unsigned>(batch));
   weight_qdq_kernel<<<grid, kQThreads, 0, s>>>(w, N, K, ldw, amax_bits, w_out, codes, scales,
                                                layout, tensor_scale, colamax_bits);

@@ -62,3 +62,38 @@ def test_quantize_edge_values():
     _check_quant(b, t, 1)
     _check_quant(b, S.to_bf16(np.zeros((70, 64), np.float32)), 1)
     _check_quant(b, S.to_bf16(-np.zeros((3, 64), np.float32)), 0)
+
+
+def _boundary_tensor(s_t_target, seed):
+    """Blocks whose elements sit within a few bf16 ulps of every E2M1 rounding
+    midpoint (times the block's decode scale), for all 126 positive E4M3
+    block scales; the first block carries the tensor amax 2688 * s_t."""
+    import torch as _t
+    from oracle import formats as F
+    rng = np.random.default_rng(seed)
+    mids = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0])
+    blocks = [np.r_[2688.0 * s_t_target, np.zeros(15)]]
+    for sb in range(1, 0x7F):
+        sdec = F.E4M3_POSITIVE[sb] * s_t_target
+        bmax = 6.0 * sdec
+        cands = []
+        for m in mids:
+            c = np.float32(m * sdec)
+            b = _t.tensor([c]).to(_t.bfloat16).view(_t.int16).item() & 0xFFFF
+            cands += [np.uint16(b + d).view(np.int16) for d in range(-3, 4)]
+        vals = S.bf16_bits(_t.tensor(np.array(cands, np.int16)).view(_t.bfloat16)).astype(np.uint32)
+        vals = (vals << 16).view(np.float32)
+        vals = vals[np.abs(vals) <= bmax]
+        vals = vals * rng.choice([-1.0, 1.0], vals.size)
+        for i in range(0, len(vals), 15):
+            chunk = vals[i:i + 15]
+            blocks.append(np.r_[bmax, chunk, np.zeros(15 - len(chunk))])
+    x = np.concatenate(blocks)
+    pad = (-len(x)) % 256
+    return S.to_bf16(np.r_[x, np.zeros(pad)].astype(np.float32).reshape(-1, 256))
+
+
+@pytest.mark.parametrize("s_t,seed", [(1.0, 0), (2.0 ** -7, 1), (0.0123456, 2), (3.7e-5, 3)])
+def test_quantize_rounding_boundaries(s_t, seed):
+    b = need_gpu()
+    _check_quant(b, _boundary_tensor(s_t, seed), 1)
