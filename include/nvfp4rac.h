@@ -213,6 +213,31 @@ nvfp4_status weight_qdq(const uint16_t* w, int64_t N, int64_t K, int64_t ldw, in
                         void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * nvfp4_quantize_static_ws -- nvfp4_quantize with the same arguments minus
+ * the workspace, for callers that cannot allocate device memory (plugin hooks
+ * whose interface passes only inputs and outputs, processes whose device
+ * memory is entirely reserved by another runtime's allocator).  The pages
+ * have no counterpart: this is a property of the library, not of the method.
+ *   Scratch lives in one file-scope device array of 4 MiB that every GPU
+ *   loading the library keeps until the process exits; shapes needing more
+ *   (nvfp4_workspace_size(NVFP4_OP_QUANTIZE, M, 0, K, 1) > 4 MiB with scores,
+ *   e.g. M * K above ~44.7 million elements) are refused with
+ *   NVFP4_ERR_WORKSPACE before anything is queued.  The call allocates
+ *   nothing and calls no allocating routine.
+ *   The first call on a device looks up the array's device address
+ *   (cudaGetSymbolAddress with that device current); make that first call
+ *   before any stream capture.
+ *   All calls share the one array: calls whose work overlaps on the GPU
+ *   (different streams, no ordering between them) race on it and give wrong
+ *   results.  Calls ordered on one stream are safe; the words that must
+ *   start at zero are cleared on the stream by every call.
+ */
+nvfp4_status nvfp4_quantize_static_ws(const uint16_t* x, int64_t M, int64_t K, int64_t ldx,
+                                      const float* amax_or_null, nvfp4_tensor* qx,
+                                      double* score_or_null, float* res_colamax_or_null,
+                                      void* stream);
+
+/*
  * Element converters used by the kernels, exposed for checking them:
  * nvfp4_encode_e2m1 writes one E2M1 code (0..15) per fp32 input,
  * nvfp4_encode_e4m3 one E4M3 code per fp32 input >= 0 (RN, saturating).

@@ -29,7 +29,7 @@ EXPORTS = ["nvfp4_scale_bytes", "nvfp4_workspace_size", "nvfp4_quantize", "rac_s
            "nvfp4_rac_nsel", "nvfp4_rac_width", "rac_weight_quant", "w4a4_rac_gemm",
            "w4a4_gemm_quantized", "moe_grouped_w4a4_rac_gemm", "weight_qdq",
            "nvfp4_encode_e2m1", "nvfp4_encode_e4m3", "nvfp4_stream_status",
-           "nvfp4_check_bounded_wait", "nvfp4_status_string"]
+           "nvfp4_check_bounded_wait", "nvfp4_status_string", "nvfp4_quantize_static_ws"]
 
 
 class _Tensor(ctypes.Structure):
@@ -44,6 +44,7 @@ _sig = {
     "nvfp4_scale_bytes": (SZ, [I64, I64, I32]),
     "nvfp4_workspace_size": (SZ, [I32, I64, I64, I64, I32]),
     "nvfp4_quantize": (I32, [P, I64, I64, I64, P, TP, P, P, P, SZ, P]),
+    "nvfp4_quantize_static_ws": (I32, [P, I64, I64, I64, P, TP, P, P, P]),
     "rac_select": (I32, [P, I64, I64, I64, TP, P, P, F32, P, P, ctypes.POINTER(I64), TP, P, SZ, P]),
     "nvfp4_rac_nsel": (I64, [F32, I64]),
     "nvfp4_rac_width": (I64, [I64]),
@@ -164,6 +165,21 @@ def quantize(x, amax=None, layout=1, scores=True, out=None, stream=None):
     _check(_lib.nvfp4_quantize(_ptr(x), M, K, x.stride(0), _ptr(amax), ctypes.byref(st),
                                _ptr(score), _ptr(colamax), _ptr(ws), ws.numel(), _stream(stream)),
            "nvfp4_quantize")
+    return qx, score, colamax
+
+
+def quantize_static_ws(x, amax=None, layout=1, scores=True, out=None, stream=None):
+    """Same as quantize() but through nvfp4_quantize_static_ws: no workspace
+    is passed; the library uses its own fixed 4 MiB device scratch array."""
+    x = _bits(x)
+    M, K = x.shape
+    qx = out if out is not None else NvFP4Tensor.empty(M, K, layout, device=x.device)
+    score = torch.empty(K, dtype=torch.float64, device=x.device) if scores else None
+    colamax = torch.empty(K, dtype=torch.float32, device=x.device) if scores else None
+    st = qx.c()
+    _check(_lib.nvfp4_quantize_static_ws(_ptr(x), M, K, x.stride(0), _ptr(amax), ctypes.byref(st),
+                                         _ptr(score), _ptr(colamax), _stream(stream)),
+           "nvfp4_quantize_static_ws")
     return qx, score, colamax
 
 

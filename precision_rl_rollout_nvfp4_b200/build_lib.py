@@ -8,7 +8,7 @@ import subprocess
 
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
-SOURCES = ["api.cu", "quant.cu", "select.cu", "gemm.cu"]
+SOURCES = ["api.cu", "quant.cu", "select.cu", "gemm.cu", "noalloc.cu"]
 LIB = os.path.join(PKG, "libnvfp4rac.so")
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-gencode", "arch=compute_100a,code=sm_100a",
          "-Xcompiler", "-fPIC", "-shared", "-Xptxas", "-warn-spills"]
