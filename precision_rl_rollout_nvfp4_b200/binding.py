@@ -344,6 +344,11 @@ class RacLinearPlan:
         sizes = [workspace_size(OP_QUANTIZE, M, 0, K), workspace_size(OP_RAC_SELECT, M, 0, K),
                  workspace_size(OP_WEIGHT_QDQ, 0, N, K, 1)]
         self.ws = torch.empty(max(sizes), dtype=torch.uint8, device=dev)
+        # weight preparation may run concurrently on a side stream: own workspace
+        self.ws_w = torch.empty(workspace_size(OP_WEIGHT_QDQ, 0, N, K, 1), dtype=torch.uint8, device=dev)
+        self.side = torch.cuda.Stream(device=dev)
+        self._fork = torch.cuda.Event()
+        self._join = torch.cuda.Event()
         self._qw, self._qx = self.qw.c(), self.qx.c()
         self._qr = self.q_res.c() if self.q_res is not None else None
         self._qs = self.q_wsel.c() if self.q_wsel is not None else None
@@ -359,8 +364,8 @@ class RacLinearPlan:
 
     def prepare_weight(self, stream=None):
         _check(_lib.weight_qdq(_ptr(self.w), self.N, self.K, self.w.stride(0), 1, _ptr(self.w_out),
-                               ctypes.byref(self._qw), _ptr(self.w_colamax), _ptr(self.ws), self.ws.numel(),
-                               _stream(stream)), "weight_qdq")
+                               ctypes.byref(self._qw), _ptr(self.w_colamax), _ptr(self.ws_w),
+                               self.ws_w.numel(), _stream(stream)), "weight_qdq")
 
     def quantize(self, stream=None, scores=True):
         _check(_lib.nvfp4_quantize(_ptr(self.x), self.M, self.K, self.x.stride(0), None, ctypes.byref(self._qx),
@@ -395,6 +400,21 @@ class RacLinearPlan:
         self.select(stream)
         self.weight_select(stream)
         self.gemm(stream)
+
+    def full_step(self):
+        """Weight preparation and the rollout linear, with the weight
+        preparation (independent of X) on a side stream that forks from and
+        joins back into the current stream, so the two overlap on the GPU."""
+        main = torch.cuda.current_stream()
+        self._fork.record(main)
+        self.side.wait_event(self._fork)
+        self.prepare_weight(stream=self.side)
+        self._join.record(self.side)
+        self.quantize()
+        self.select()
+        main.wait_event(self._join)
+        self.weight_select()
+        self.gemm()
 
     def plain_step(self, stream=None):
         """Plain NVFP4 W4A4 (no RAC): Q(X) without scores, one-segment GEMM."""

@@ -20,7 +20,6 @@ namespace {
 
 constexpr int kQThreads = 256;
 constexpr int kQCols = 64;
-constexpr int kDxStride = kQCols + 4;
 
 // ---------------------------------------------------------------------------
 // amax
@@ -75,8 +74,15 @@ __global__ void group_tiles_kernel(const int64_t* __restrict__ off, int32_t E,
 // ---------------------------------------------------------------------------
 // quantize + residual + score partials (+ the ordered reduction of the
 // partials by the last CTA of each 64-column strip of a row group)
+//
+// Thread t of the 256 owns 8 consecutive columns (one 16-byte load) of the 4
+// consecutive rows 4 (t/8) .. 4 (t/8) + 3 of the tile; the two halves of a
+// 16-element block sit in threads t and t^1.  The score order (4-row groups
+// summed in row order, group sums in group order, chunk sums in chunk order)
+// lets every thread sum its own group in fp64 registers; 64 threads then add
+// the tile's 32 group sums in order from shared memory.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(kQThreads, 5)
+__global__ void __launch_bounds__(kQThreads)
 quant_score_kernel(const uint16_t* __restrict__ x, int64_t K, int64_t ldx, RowGroups g,
                    const float* __restrict__ amax, int64_t codes_rows,
                    uint8_t* __restrict__ codes, uint8_t* __restrict__ scales, int layout,
@@ -86,29 +92,34 @@ quant_score_kernel(const uint16_t* __restrict__ x, int64_t K, int64_t ldx, RowGr
   const int64_t tile = blockIdx.y;
   const TileInfo ti = tile_info(g, tile);
   if (!ti.valid) return;
-  // |dX| of the tile; reused by the strip's last CTA to stage partials
-  __shared__ __align__(16) float dxs[kTileRows][kDxStride];
+  constexpr int kGroups = kTileRows / 4;                          // 32 groups of 4 rows
+  __shared__ __align__(16) double gsum[kGroups][kQCols];          // also tail staging
+  __shared__ __align__(16) float gmax[kGroups][kQCols];
   __shared__ bool s_last;
-  const int t = threadIdx.x, cg = t & 7, rr = t >> 3;
+  __shared__ ScaleTable T;
+  const int t = threadIdx.x, cg = t & 7, grp = t >> 3;
   const int64_t col0 = static_cast<int64_t>(blockIdx.x) * kQCols;
   const int64_t col = col0 + 8 * cg;
   const float s_t = __fdiv_rn(amax[ti.e], kTensorScaleDiv);
   if (blockIdx.x == 0 && t == 0 && (g.off == nullptr ? tile == 0 : tile == g.tile_start[ti.e]))
     tensor_scale[ti.e] = s_t;
-  __shared__ ScaleTable T;
   build_scale_table(T, s_t, t);
 
   uint4 raw[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const int64_t row = ti.row0 + rr + 32 * i;
+    const int64_t row = ti.row0 + 4 * grp + i;
     raw[i] = row < ti.row_end ? ld_nc_v4(x + row * ldx + col) : make_uint4(0, 0, 0, 0);
   }
   __syncthreads();                               // table ready
   uint8_t* code_base = codes + tile * kTileRows * (K / 2) + col / 2;
+  double acc[8];
+  float mx[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) { acc[j] = 0.0; mx[j] = 0.0f; }
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const int r = rr + 32 * i;
+    const int r = 4 * grp + i;
     const int64_t prow = tile * kTileRows + r;
     float f[8];
     unpack_bf16x8(raw[i], f);
@@ -118,34 +129,39 @@ quant_score_kernel(const uint16_t* __restrict__ x, int64_t K, int64_t ldx, RowGr
     am = fmaxf(am, __shfl_xor_sync(0xFFFFFFFFu, am, 1));
     const BlockQ bq = block_q(am, T);
     const uint32_t packed = encode8_q(f, bq);
-    float d[8];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       float lo, hi;
       e2m1x2_to_f32((packed >> (8 * j)) & 0xFFu, lo, hi);
-      d[2 * j] = fabsf(__fsub_rn(f[2 * j], __fmul_rn(__fmul_rn(lo, bq.sbv), s_t)));
-      d[2 * j + 1] = fabsf(__fsub_rn(f[2 * j + 1], __fmul_rn(__fmul_rn(hi, bq.sbv), s_t)));
+      const float d0 = fabsf(__fsub_rn(f[2 * j], __fmul_rn(__fmul_rn(lo, bq.sbv), s_t)));
+      const float d1 = fabsf(__fsub_rn(f[2 * j + 1], __fmul_rn(__fmul_rn(hi, bq.sbv), s_t)));
+      acc[2 * j] += static_cast<double>(d0);       // rows of the group in order
+      acc[2 * j + 1] += static_cast<double>(d1);
+      mx[2 * j] = fmaxf(mx[2 * j], d0);
+      mx[2 * j + 1] = fmaxf(mx[2 * j + 1], d1);
     }
-    *reinterpret_cast<float4*>(&dxs[r][8 * cg]) = make_float4(d[0], d[1], d[2], d[3]);
-    *reinterpret_cast<float4*>(&dxs[r][8 * cg + 4]) = make_float4(d[4], d[5], d[6], d[7]);
     if (prow < codes_rows)
       *reinterpret_cast<uint32_t*>(code_base + static_cast<uint32_t>(r) * static_cast<uint32_t>(K / 2)) = packed;
     if ((cg & 1) == 0 && (layout == 1 || prow < codes_rows))
       scales[scale_offset(prow, col / kBlock, K, layout)] = static_cast<uint8_t>(bq.sb);
   }
   if (part_sum == nullptr) return;
+#pragma unroll
+  for (int j = 0; j < 8; j += 2)
+    *reinterpret_cast<double2*>(&gsum[grp][8 * cg + j]) = make_double2(acc[j], acc[j + 1]);
+  *reinterpret_cast<float4*>(&gmax[grp][8 * cg]) = make_float4(mx[0], mx[1], mx[2], mx[3]);
+  *reinterpret_cast<float4*>(&gmax[grp][8 * cg + 4]) = make_float4(mx[4], mx[5], mx[6], mx[7]);
   __syncthreads();
   if (t < kQCols) {
-    double acc = 0.0;
-    float mx = 0.0f;
+    double part = 0.0;
+    float m = 0.0f;
 #pragma unroll 8
-    for (int r = 0; r < kTileRows; ++r) {       // row order within the chunk
-      const float v = dxs[r][t];
-      acc += static_cast<double>(v);
-      mx = fmaxf(mx, v);
+    for (int q = 0; q < kGroups; ++q) {          // group order within the chunk
+      part += gsum[q][t];
+      m = fmaxf(m, gmax[q][t]);
     }
-    part_sum[tile * K + col0 + t] = acc;
-    part_max[tile * K + col0 + t] = mx;
+    part_sum[tile * K + col0 + t] = part;
+    part_max[tile * K + col0 + t] = m;
   }
   if (strip_count == nullptr) return;
   // The last CTA of this group's column strip sums the group's partials in
@@ -163,15 +179,13 @@ quant_score_kernel(const uint16_t* __restrict__ x, int64_t K, int64_t ldx, RowGr
   if (!s_last) return;
   __threadfence();
   // stage up to 32 tiles' partials of this strip in shared memory (all 256
-  // threads load; 24 KB fits in the |dX| buffer), then 64 threads add them
-  // in tile order
-  constexpr int kStage = 32;
-  double* ps = reinterpret_cast<double*>(&dxs[0][0]);            // [32 tiles][64 cols]
-  float* pm = reinterpret_cast<float*>(ps + kStage * kQCols);     // [32 tiles][64 cols]
-  double acc = 0.0;
-  float mx = 0.0f;
-  for (int64_t c0 = t0; c0 < t1; c0 += kStage) {
-    const int nt = static_cast<int>(t1 - c0 < kStage ? t1 - c0 : kStage);
+  // threads load), then 64 threads add them in tile order
+  double* ps = &gsum[0][0];                      // [32 tiles][64 cols]
+  float* pm = &gmax[0][0];
+  double total = 0.0;
+  float tmax = 0.0f;
+  for (int64_t c0 = t0; c0 < t1; c0 += kGroups) {
+    const int nt = static_cast<int>(t1 - c0 < kGroups ? t1 - c0 : kGroups);
     __syncthreads();
     for (int k = t; k < nt * kQCols; k += kQThreads) {
       const int tt = k / kQCols, cc = k % kQCols;
@@ -181,14 +195,14 @@ quant_score_kernel(const uint16_t* __restrict__ x, int64_t K, int64_t ldx, RowGr
     __syncthreads();
     if (t < kQCols) {
       for (int tt = 0; tt < nt; ++tt) {          // chunk order
-        acc += ps[tt * kQCols + t];
-        mx = fmaxf(mx, pm[tt * kQCols + t]);
+        total += ps[tt * kQCols + t];
+        tmax = fmaxf(tmax, pm[tt * kQCols + t]);
       }
     }
   }
   if (t < kQCols) {
-    score[static_cast<int64_t>(ti.e) * K + col0 + t] = acc;
-    colamax[static_cast<int64_t>(ti.e) * K + col0 + t] = mx;
+    score[static_cast<int64_t>(ti.e) * K + col0 + t] = total;
+    colamax[static_cast<int64_t>(ti.e) * K + col0 + t] = tmax;
   }
   if (t == 0) *counter = 0;                      // ready for the next call
 }
