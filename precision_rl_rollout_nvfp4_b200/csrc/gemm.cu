@@ -24,10 +24,20 @@
 //   warps 2..5  epilogue: tcgen05.ld of both accumulators (TMEM lane = output
 //               row), Y = alpha0 acc0 + alpha1 acc1 into a shared staging tile,
 //               TMEM released, then coalesced fp32 / bf16 row stores.
-// The two tensor scales differ, so the segments accumulate separately.  No
-// TMA multicast is used.  Every mbarrier wait is bounded (see common.cuh).
+// The two tensor scales differ, so the segments accumulate separately.  Every
+// CTA loads its own tiles (no load is shared between CTAs).  Every mbarrier
+// wait is bounded (see common.cuh).
+//
+// For dense activations with at least 512 rows a second kernel runs the same
+// product on CTA pairs (tcgen05 cta_group::2): a pair computes a 256 x 256
+// tile, each CTA loading its own 128 rows of A and of B, so a pair fetches
+// half the operand bytes per FLOP of two 128 x 128 tiles.  Its TMEM holds one
+// 256-column accumulator; the residual segment is computed first and scaled
+// in place by s_R s_Ws / (s_X s_W) (tcgen05.ld, multiply, tcgen05.st), then
+// the plain segment accumulates on top and Y = s_X s_W acc.
 #include <cuda.h>
 #include <cudaTypedefs.h>
+#include <cstdlib>
 
 #include "kernels.h"
 
@@ -372,6 +382,17 @@ int sm_count() {
   return n > 0 ? n : 148;
 }
 
+// NVFP4_GEMM_SINGLE_CTA=1 in the environment keeps every GEMM on the
+// single-CTA kernel (used to compare the two kernels).
+bool gemm_force_single_cta() {
+  static int v = -1;
+  if (v < 0) {
+    const char* e = getenv("NVFP4_GEMM_SINGLE_CTA");
+    v = (e != nullptr && e[0] == '1') ? 1 : 0;
+  }
+  return v == 1;
+}
+
 template <int YBYTES>
 cudaError_t prepare_kernel() {
   static bool attr_set = false;
@@ -384,9 +405,408 @@ cudaError_t prepare_kernel() {
   return cudaSuccess;
 }
 
+// ===========================================================================
+// CTA-pair kernel (tcgen05 cta_group::2), dense activations.
+// ===========================================================================
+template <int YBYTES>
+struct Cfg2 {
+  static constexpr int STAGES = YBYTES == 2 ? 5 : 4;
+  static constexpr int A_ST = 128 * BK_BYTES;          // own 128 rows of A
+  static constexpr int B_ST = 128 * BK_BYTES;          // own 128 rows (N half) of B
+  static constexpr int SFA_ST = 4 * SF_ATOM;           // own 128 rows x 4 K blocks
+  static constexpr int SFB_ST = 8 * SF_ATOM;           // all 256 N rows x 4 K blocks
+  static constexpr int STAGE = A_ST + B_ST + SFA_ST + SFB_ST;
+  static constexpr int STG_STRIDE = 128 * YBYTES + 16; // staging: 128 columns per half tile
+  static constexpr int STG_BYTES = 128 * STG_STRIDE;
+  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE + STG_BYTES + 512;
+  static constexpr uint32_t TX = 2 * STAGE;            // bytes landing per stage (both CTAs)
+};
+
+constexpr uint32_t ACC2_COL = 0, SFA2_COL = 256, SFB2_COL = 272;
+// kind::mxf4nvf4, M = 256 (pair), N = 256, both K-major, ue4m3 scales.
+constexpr uint32_t IDESC2 = (1u << 7) | (1u << 10) | (uint32_t(256 >> 3) << 17) | (uint32_t(256 >> 4) << 24);
+
+struct KParams2 {
+  int64_t M, N;
+  int m_tiles, n_tiles;        // 256-row / 256-column tiles
+  int kt[2];                   // K steps of the residual (0) and plain (1) segments
+  const float* sta[2];
+  const float* stb[2];
+  void* y;
+  int64_t ldy;
+  unsigned* err;
+};
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Shared::cluster address of the same shared variable in CTA `rank`.
+__device__ __forceinline__ uint32_t peer_addr(const void* p, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+  return r;
+}
+
+// 2-D tensor load into this CTA's shared memory that completes its bytes on
+// an mbarrier of the CTA pair (here: the leader's).
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* tm, int x, int y,
+                                                 uint32_t bar_cluster) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+      :: "r"(dst), "l"(reinterpret_cast<uint64_t>(tm)), "r"(x), "r"(y), "r"(bar_cluster) : "memory");
+}
+
+__device__ __forceinline__ void utccp_sf_pair(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" :: "r"(taddr), "l"(sdesc) : "memory");
+}
+
+__device__ __forceinline__ void mma_fp4_pair(uint32_t d, uint64_t a, uint64_t b, uint32_t sfa, uint32_t sfb,
+                                             uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+      :: "r"(d), "l"(a), "l"(b), "r"(IDESC2), "r"(accumulate), "r"(sfa), "r"(sfb) : "memory");
+}
+
+// Completion of this thread's tcgen05 work arrives on the mbarrier at the
+// same shared offset in both CTAs of the pair.
+__device__ __forceinline__ void umma_commit_pair(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
+               :: "r"(smem_u32(bar)), "h"(static_cast<uint16_t>(3)) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" :: "r"(bar_cluster) : "memory");
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
+      "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};"
+      :: "r"(taddr), "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]),
+         "f"(v[7]), "f"(v[8]), "f"(v[9]), "f"(v[10]), "f"(v[11]), "f"(v[12]), "f"(v[13]), "f"(v[14]),
+         "f"(v[15]), "f"(v[16]), "f"(v[17]), "f"(v[18]), "f"(v[19]), "f"(v[20]), "f"(v[21]),
+         "f"(v[22]), "f"(v[23]), "f"(v[24]), "f"(v[25]), "f"(v[26]), "f"(v[27]), "f"(v[28]),
+         "f"(v[29]), "f"(v[30]), "f"(v[31])
+      : "memory");
+}
+
+template <int YBYTES>
+__global__ void __launch_bounds__(THREADS, 1)
+w4a4_rac_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
+                          const __grid_constant__ CUtensorMap tmSA0, const __grid_constant__ CUtensorMap tmSB0,
+                          const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
+                          const __grid_constant__ CUtensorMap tmSA1, const __grid_constant__ CUtensorMap tmSB1,
+                          const KParams2 p) {
+  using C = Cfg2<YBYTES>;
+  constexpr int STAGES = C::STAGES;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint8_t* sStage = smem;                                       // [STAGES][A | B | SFA | SFB]
+  uint8_t* sOut = smem + STAGES * C::STAGE;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sOut + C::STG_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tmem_full = empty + STAGES;
+  uint64_t* tmem_empty = tmem_full + 1;
+  uint64_t* res_full = tmem_empty + 1;
+  uint64_t* res_done = res_full + 1;
+  uint64_t* drain = res_done + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    mbar_init(tmem_full, 1);
+    mbar_init(tmem_empty, 8);          // one arrival per epilogue warp of both CTAs
+    mbar_init(res_full, 1);
+    mbar_init(res_done, 8);
+    mbar_init(drain, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  cluster_sync_all();                  // barriers of both CTAs initialised
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;"
+                 :: "r"(smem_u32(tmem_slot)), "r"(TMEM_COLS) : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  const int total = p.m_tiles * p.n_tiles;
+  const bool has_res = p.kt[0] > 0;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------ producer (both CTAs)
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t armed = 0, armed_phase = 0;
+      bool ok = true;
+      for (int tile = pair; tile < total && ok; tile += npairs) {
+        const int mt = tile / p.n_tiles, nt = tile % p.n_tiles;
+        const int a_row = mt * 256 + static_cast<int>(rank) * 128;
+        const int b_row = nt * 256 + static_cast<int>(rank) * 128;
+        for (int seg = has_res ? 0 : 1; seg < 2 && ok; ++seg) {
+          const CUtensorMap* tA = seg ? &tmA1 : &tmA0;
+          const CUtensorMap* tB = seg ? &tmB1 : &tmB0;
+          const CUtensorMap* tSA = seg ? &tmSA1 : &tmSA0;
+          const CUtensorMap* tSB = seg ? &tmSB1 : &tmSB0;
+          for (int kt = 0; kt < p.kt[seg]; ++kt) {
+            if (!mbar_wait(&empty[stage], phase ^ 1, p.err)) { ok = false; break; }
+            if (rank == 0) mbar_arrive_expect_tx(&full[stage], C::TX);
+            const uint32_t lead_full = peer_addr(&full[stage], 0);
+            uint8_t* st = sStage + stage * C::STAGE;
+            tma_load_2d_pair(smem_u32(st), tA, kt * BK_BYTES, a_row, lead_full);
+            tma_load_2d_pair(smem_u32(st + C::A_ST), tB, kt * BK_BYTES, b_row, lead_full);
+            tma_load_2d_pair(smem_u32(st + C::A_ST + C::B_ST), tSA, kt * 256, a_row / 128, lead_full);
+            tma_load_2d_pair(smem_u32(st + C::A_ST + C::B_ST + C::SFA_ST), tSB, kt * 256, nt * 2, lead_full);
+            armed |= 1u << stage;
+            armed_phase = (armed_phase & ~(1u << stage)) | (phase << stage);
+            if (++stage == STAGES) { stage = 0; phase ^= 1; }
+          }
+        }
+      }
+      // let this CTA's copies land before it can exit: the stages it filled
+      // are freed (empty) once the leader's MMAs consumed them
+      if (rank == 0) {
+        for (int s = 0; s < STAGES; ++s)
+          if (armed & (1u << s)) mbar_wait(&full[s], (armed_phase >> s) & 1u, p.err);
+      } else {
+        for (int s = 0; s < STAGES; ++s)
+          if (armed & (1u << s)) mbar_wait(&empty[s], (armed_phase >> s) & 1u, p.err);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && rank == 0) {
+      // ------------------------------ MMA issuer (leader CTA only)
+      int stage = 0;
+      uint32_t phase = 0, acc_phase = 0, res_phase = 0;
+      bool ok = true;
+      for (int tile = pair; tile < total && ok; tile += npairs) {
+        if (!mbar_wait(tmem_empty, acc_phase ^ 1, p.err)) break;
+        tc_fence_after();
+        for (int seg = has_res ? 0 : 1; seg < 2 && ok; ++seg) {
+          for (int kt = 0; kt < p.kt[seg]; ++kt) {
+            if (!mbar_wait(&full[stage], phase, p.err)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t st = smem_u32(sStage + stage * C::STAGE);
+            const uint32_t a0 = st, b0 = st + C::A_ST;
+            const uint32_t fa = st + C::A_ST + C::B_ST, fb = fa + C::SFA_ST;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              utccp_sf_pair(tmem + SFA2_COL + 4 * j, desc_sf(fa + j * SF_ATOM));
+              utccp_sf_pair(tmem + SFB2_COL + 8 * j, desc_sf(fb + j * SF_ATOM));
+              utccp_sf_pair(tmem + SFB2_COL + 8 * j + 4, desc_sf(fb + 4 * SF_ATOM + j * SF_ATOM));
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const uint32_t accum = (seg == 1 && has_res) ? 1u : ((kt > 0 || j > 0) ? 1u : 0u);
+              mma_fp4_pair(tmem + ACC2_COL, desc_sw128(a0 + 32 * j), desc_sw128(b0 + 32 * j),
+                           tmem + SFA2_COL + 4 * j, tmem + SFB2_COL + 8 * j, accum);
+            }
+            umma_commit_pair(&empty[stage]);
+            if (++stage == STAGES) { stage = 0; phase ^= 1; }
+          }
+          if (seg == 0 && ok) {
+            // residual product ready: let the epilogue scale it in place
+            umma_commit_pair(res_full);
+            if (!mbar_wait(res_done, res_phase, p.err)) { ok = false; break; }
+            tc_fence_after();
+            res_phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        umma_commit_pair(tmem_full);
+        acc_phase ^= 1;
+      }
+      asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                   :: "r"(smem_u32(drain)) : "memory");
+      mbar_wait(drain, 0, p.err);
+    }
+  } else {
+    // ------------------------------ epilogue (warps 2..5 of both CTAs)
+    const int q = warp & 3;
+    const uint32_t trow = tmem + (static_cast<uint32_t>(32 * q) << 16);
+    uint8_t* stg_warp = sOut + (32 * q) * C::STG_STRIDE;
+    uint8_t* stg_row = stg_warp + lane * C::STG_STRIDE;
+    const uint32_t lead_tmem_empty = peer_addr(tmem_empty, 0);
+    const uint32_t lead_res_done = peer_addr(res_done, 0);
+    uint32_t acc_phase = 0, res_phase = 0;
+    for (int tile = pair; tile < total; tile += npairs) {
+      const int mt = tile / p.n_tiles, nt = tile % p.n_tiles;
+      const float al0 = __fmul_rn(p.sta[1][0], p.stb[1][0]);
+      const float al1 = has_res ? __fmul_rn(p.sta[0][0], p.stb[0][0]) : 0.0f;
+      // the residual is scaled to the plain segment's units, then Y = al0 acc;
+      // with al0 == 0 the plain operands are all zero codes and Y = al1 acc
+      const float ratio = al0 != 0.0f ? __fdiv_rn(al1, al0) : 1.0f;
+      const float fin = (has_res && al0 == 0.0f) ? al1 : al0;
+      bool ok = true;
+      if (has_res) {
+        if (lane == 0) ok = mbar_wait(res_full, res_phase, p.err);
+        ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll 1
+        for (int c = 0; c < 8; ++c) {
+          float v[32];
+          tmem_ld32(trow + ACC2_COL + 32 * c, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(v[i], ratio);
+          tmem_st32(trow + ACC2_COL + 32 * c, v);
+        }
+        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(lead_res_done);
+        res_phase ^= 1;
+      }
+      if (lane == 0) ok = mbar_wait(tmem_full, acc_phase, p.err);
+      ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+      if (!ok) break;
+      tc_fence_after();
+      const int64_t row0 = static_cast<int64_t>(mt) * 256 + rank * 128 + 32 * q;
+#pragma unroll 1
+      for (int h = 0; h < 2; ++h) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          float v[32];
+          tmem_ld32(trow + ACC2_COL + 128 * h + 32 * c, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(fin, v[i]);
+          if (YBYTES == 4) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 4)
+              *reinterpret_cast<float4*>(stg_row + (32 * c + i) * 4) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+          } else {
+            uint32_t w[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              w[i] = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(v[2 * i]))) |
+                     (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(v[2 * i + 1]))) << 16);
+#pragma unroll
+            for (int i = 0; i < 16; i += 4)
+              *reinterpret_cast<uint4*>(stg_row + (32 * c + 2 * i) * 2) = make_uint4(w[i], w[i + 1], w[i + 2], w[i + 3]);
+          }
+        }
+        if (h == 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(lead_tmem_empty);   // accumulator free
+        }
+        __syncwarp();
+        const int64_t col = static_cast<int64_t>(nt) * 256 + 128 * h + 4 * lane;
+        const bool col_ok = col + 4 <= p.N;
+#pragma unroll 4
+        for (int r = 0; r < 32; ++r) {
+          const int64_t row = row0 + r;
+          if (row >= p.M || !col_ok) continue;
+          const uint8_t* src = stg_warp + r * C::STG_STRIDE + lane * 4 * YBYTES;
+          if (YBYTES == 4)
+            *reinterpret_cast<float4*>(static_cast<float*>(p.y) + row * p.ldy + col) = *reinterpret_cast<const float4*>(src);
+          else
+            *reinterpret_cast<uint2*>(static_cast<uint16_t*>(p.y) + row * p.ldy + col) = *reinterpret_cast<const uint2*>(src);
+        }
+        __syncwarp();
+      }
+      acc_phase ^= 1;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();                  // neither CTA leaves while its peer may still signal it
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" :: "r"(tmem), "r"(TMEM_COLS) : "memory");
+  }
+}
+
+// 2-D map over a tiled scale buffer seen as int64 elements: one row per
+// 128-row block (all its 512-byte atoms), box = 4 atoms x box_rows blocks.
+bool make_scale_map(CUtensorMap* tm, const uint8_t* scales, int64_t rows, int64_t cols, int box_rows) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  const int64_t atoms = (cols + 63) / 64;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(atoms * 64), static_cast<cuuint64_t>((rows + 127) / 128)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(atoms * 512)};
+  cuuint32_t box[2] = {256u, static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(tm, CU_TENSOR_MAP_DATA_TYPE_INT64, 2, const_cast<uint8_t*>(scales), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int YBYTES>
+cudaError_t launch_pair(const GemmArgs& a, cudaStream_t s) {
+  using C = Cfg2<YBYTES>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(w4a4_rac_gemm_pair_kernel<YBYTES>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  KParams2 p{};
+  p.M = a.M;
+  p.N = a.N;
+  p.m_tiles = static_cast<int>((a.M + 255) / 256);
+  p.n_tiles = static_cast<int>((a.N + 255) / 256);
+  const bool res = a.a1.codes != nullptr;
+  // segment 0: residual (may be absent), segment 1: plain
+  const GemmOperand* A[2] = {res ? &a.a1 : &a.a0, &a.a0};
+  const GemmOperand* B[2] = {res ? &a.b1 : &a.b0, &a.b0};
+  CUtensorMap maps[8];
+  for (int seg = 0; seg < 2; ++seg) {
+    p.kt[seg] = (seg == 0 && !res) ? 0 : static_cast<int>((A[seg]->cols + 255) / 256);
+    p.sta[seg] = A[seg]->st;
+    p.stb[seg] = B[seg]->st;
+    if (!make_code_map(&maps[4 * seg + 0], A[seg]->codes, A[seg]->rows, A[seg]->cols, 128) ||
+        !make_code_map(&maps[4 * seg + 1], B[seg]->codes, B[seg]->rows, B[seg]->cols, 128) ||
+        !make_scale_map(&maps[4 * seg + 2], A[seg]->scales, A[seg]->rows, A[seg]->cols, 1) ||
+        !make_scale_map(&maps[4 * seg + 3], B[seg]->scales, B[seg]->rows, B[seg]->cols, 2))
+      return cudaErrorInvalidValue;
+  }
+  p.y = a.y;
+  p.ldy = a.ldy;
+  p.err = a.err;
+  const int tiles = p.m_tiles * p.n_tiles;
+  const int pairs = tiles < sm_count() / 2 ? tiles : sm_count() / 2;
+  if (pairs == 0) return cudaSuccess;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
+  cfg.blockDim = dim3(THREADS);
+  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, w4a4_rac_gemm_pair_kernel<YBYTES>, maps[0], maps[1], maps[2], maps[3],
+                            maps[4], maps[5], maps[6], maps[7], p);
+}
+
 }  // namespace
 
 cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s) {
+  // dense activations with enough rows for 256-row tiles: the CTA-pair kernel
+  if (a.g.off == nullptr && a.M >= 512 && !gemm_force_single_cta())
+    return a.y_dtype == 0 ? launch_pair<4>(a, s) : launch_pair<2>(a, s);
   cudaError_t e = a.y_dtype == 0 ? prepare_kernel<4>() : prepare_kernel<2>();
   if (e != cudaSuccess) return e;
   KParams p{};

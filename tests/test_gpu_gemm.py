@@ -28,23 +28,28 @@ def _random_operand(b, rows, cols, rng, st):
 
 @pytest.mark.parametrize("M,N,K,W", [(128, 128, 256, 0), (128, 128, 64, 0), (256, 256, 512, 256),
                                      (300, 144, 320, 64), (1, 16, 64, 0), (130, 384, 1024, 192),
-                                     (512, 512, 2048, 1024)])
-def test_gemm_on_random_operands(M, N, K, W):
+                                     (512, 512, 2048, 1024),
+                                     # M >= 512: CTA-pair kernel (256 x 256 tiles), ragged edges
+                                     (600, 400, 320, 64), (1024, 2048, 4096, 0), (777, 272, 576, 448),
+                                     (512, 16, 64, 64)])
+@pytest.mark.parametrize("out", ["f32", "bf16"])
+def test_gemm_on_random_operands(M, N, K, W, out):
     b = need_gpu()
     rng = np.random.default_rng(M * 7 + N)
     a, ac, asc = _random_operand(b, M, K, rng, 0.5)
     w, wc, wsc = _random_operand(b, N, K, rng, 0.25)
     ref = oracle.gemm_fp64(ac, asc, np.float32(0.5), wc, wsc, np.float32(0.25))
+    r = s = None
     if W:
         r, rc, rsc = _random_operand(b, M, W, rng, 0.125)
         s, sc, ssc = _random_operand(b, N, W, rng, 2.0)
         ref = ref + oracle.gemm_fp64(rc, rsc, np.float32(0.125), sc, ssc, np.float32(2.0))
-        y = b.gemm_quantized(a, w, r, s)
-    else:
-        y = b.gemm_quantized(a, w)
+    dt = torch.float32 if out == "f32" else torch.bfloat16
+    y = b.gemm_quantized(a, w, r, s, out_dtype=dt) if W else b.gemm_quantized(a, w, out_dtype=dt)
     torch.cuda.synchronize()
     assert b.stream_status() == 0
-    assert rel_err(y.cpu().numpy(), ref) < REL_TOL
+    tol = REL_TOL if out == "f32" else REL_TOL + 2.0 ** -8
+    assert rel_err(y.float().cpu().numpy(), ref) < tol
 
 
 def _check_linear(b, M, K, N, k, seed=0, rows=None, out_dtype=torch.float32):
