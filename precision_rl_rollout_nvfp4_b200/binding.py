@@ -422,4 +422,4 @@ class RacLinearPlan:
         self.gemm(stream, plain=True)
 
     # kernels each call launches (for launch accounting)
-    LAUNCHES = dict(prepare_weight=2, quantize=3, quantize_plain=2, select=2, weight_select=2, gemm=1)
+    LAUNCHES = dict(prepare_weight=2, quantize=2, quantize_plain=2, select=2, weight_select=2, gemm=1)

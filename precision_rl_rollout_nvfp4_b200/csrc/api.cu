@@ -86,6 +86,7 @@ bool tensor_ok(const nvfp4_tensor* t) {
 
 // Workspace pieces of nvfp4_quantize.
 struct QuantWs {
+  unsigned* counters;
   unsigned* amax;
   double* part_sum;
   float* part_max;
@@ -93,7 +94,8 @@ struct QuantWs {
 QuantWs carve_quant(Carver& c, int64_t M, int64_t K, bool scores) {
   QuantWs w{};
   const int64_t tiles = ceil_div(M, kTileRows);
-  w.amax = c.take<unsigned>(1 + K / 64);      // amax, then one counter per 64-column strip
+  w.counters = c.take<unsigned>(K / 64);      // one counter per 64-column strip
+  w.amax = c.take<unsigned>(amax_parts_count(M, K));   // partial maxima
   if (scores) {
     w.part_sum = c.take<double>(tiles * K);
     w.part_max = c.take<float>(tiles * K);
@@ -193,7 +195,7 @@ size_t nvfp4_workspace_size(int32_t op, int64_t M, int64_t N, int64_t K, int32_t
     case NVFP4_OP_RAC_SELECT: c.take<float>(1); break;
     case NVFP4_OP_GEMM: carve_gemm(c, N, nvfp4_rac_width(K)); break;
     case NVFP4_OP_MOE: carve_moe(c, M, N, K, E, K, nvfp4_rac_width(K)); break;
-    case NVFP4_OP_WEIGHT_QDQ: c.take<unsigned>(E > 0 ? E : 1); break;
+    case NVFP4_OP_WEIGHT_QDQ: c.take<unsigned>(static_cast<size_t>(E > 0 ? E : 1) * amax_parts_count(N, K)); break;
     default: return 0;
   }
   return c.off + 256;
@@ -215,15 +217,19 @@ nvfp4_status nvfp4_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ldx
   if (d != NVFP4_OK) return d;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const RowGroups g = dense_groups(M);
-  const float* amax = amax_or_null;
-  NV_TRY(cudaMemsetAsync(w.amax, 0, sizeof(unsigned) * (1 + K / 64), s));
-  if (amax == nullptr) {
-    NV_TRY(launch_amax(x, M, K, ldx, g, w.amax, s));
-    amax = reinterpret_cast<const float*>(w.amax);
+  // the strip counters must start at zero: the amax pass clears them, or a
+  // memset does when the caller supplies amax
+  int n_parts = 0;
+  if (amax_or_null == nullptr) {
+    n_parts = amax_parts_count(M, K);
+    NV_TRY(launch_amax_partial(x, M, K, ldx, 1, 0, w.amax, n_parts, w.counters,
+                               scores ? static_cast<int>(K / 64) : 0, s));
+  } else if (scores) {
+    NV_TRY(cudaMemsetAsync(w.counters, 0, sizeof(unsigned) * (K / 64), s));
   }
-  NV_TRY(launch_quant_score(x, M, K, ldx, g, amax, M, qx->codes, qx->scales, qx->scale_layout,
-                            qx->tensor_scale, w.part_sum, w.part_max, scores ? w.amax + 1 : nullptr,
-                            score_or_null, res_colamax_or_null, s));
+  NV_TRY(launch_quant_score(x, M, K, ldx, g, amax_or_null, w.amax, n_parts, M, qx->codes, qx->scales,
+                            qx->scale_layout, qx->tensor_scale, w.part_sum, w.part_max,
+                            scores ? w.counters : nullptr, score_or_null, res_colamax_or_null, s));
   return NVFP4_OK;
 }
 
@@ -377,7 +383,7 @@ nvfp4_status moe_grouped_w4a4_rac_gemm(const uint16_t* x_perm, int64_t T, int64_
   NV_TRY(launch_group_tiles(offsets_dev, E, m.tile_start, s));
   NV_TRY(cudaMemsetAsync(m.amax, 0, sizeof(unsigned) * E, s));
   NV_TRY(launch_amax(x_perm, T, K, K, g, m.amax, s));
-  NV_TRY(launch_quant_score(x_perm, T, K, K, g, reinterpret_cast<const float*>(m.amax), prows,
+  NV_TRY(launch_quant_score(x_perm, T, K, K, g, reinterpret_cast<const float*>(m.amax), nullptr, 0, prows,
                             m.qx_codes, m.qx_scales, 1, m.qx_st, m.part_sum, m.part_max, nullptr,
                             nullptr, nullptr, s));
   NV_TRY(launch_score_reduce(m.part_sum, m.part_max, K, g, tiles, m.score, m.colamax, m.qx_st, s));
@@ -417,17 +423,19 @@ nvfp4_status weight_qdq(const uint16_t* w, int64_t N, int64_t K, int64_t ldw, in
              NVFP4_ERR_UNSUPPORTED_SHAPE);
   }
   Carver c(ws);
-  unsigned* amax = c.take<unsigned>(batch);
+  const int n_parts = amax_parts_count(N, K);
+  unsigned* amax = c.take<unsigned>(static_cast<size_t>(batch) * n_parts);
   NV_CHECK(ws != nullptr && ws_bytes >= c.off, NVFP4_ERR_WORKSPACE);
   const nvfp4_status d = device_ok();
   if (d != NVFP4_OK) return d;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  NV_TRY(cudaMemsetAsync(amax, 0, sizeof(unsigned) * batch, s));
-  if (colamax_or_null) NV_TRY(cudaMemsetAsync(colamax_or_null, 0, sizeof(float) * batch * K, s));
   if (qw_or_null && qw_or_null->scale_layout == 1 && (static_cast<int64_t>(batch) * N) % 128 != 0)
     NV_TRY(cudaMemsetAsync(qw_or_null->scales, 0, scale_bytes(static_cast<int64_t>(batch) * N, K, 1), s));
-  NV_TRY(launch_amax(w, N, K, ldw, dense_groups(N), amax, s, batch, N * ldw));
-  NV_TRY(launch_weight_qdq(w, N, K, ldw, batch, amax, w_out, qw_or_null ? qw_or_null->codes : nullptr,
+  // the amax pass also clears colamax (accumulated with atomic max)
+  NV_TRY(launch_amax_partial(w, N, K, ldw, batch, N * ldw, amax, n_parts,
+                             reinterpret_cast<unsigned*>(colamax_or_null),
+                             colamax_or_null ? static_cast<int>(batch * K) : 0, s));
+  NV_TRY(launch_weight_qdq(w, N, K, ldw, batch, amax, n_parts, w_out, qw_or_null ? qw_or_null->codes : nullptr,
                            qw_or_null ? qw_or_null->scales : nullptr,
                            qw_or_null ? qw_or_null->scale_layout : 0,
                            qw_or_null ? qw_or_null->tensor_scale : nullptr,

@@ -29,8 +29,18 @@ cudaError_t launch_group_tiles(const int64_t* off, int32_t E, int32_t* tile_star
 // groups; part_sum / part_max [tiles, K] (may be null).  With strip_count
 // (E x K/64 counters, zero on entry and left zero) the last CTA of every
 // column strip of a group also writes score[e, :] and colamax[e, :].
+// Dense activations without a caller amax: per-CTA partial maxima (see
+// amax_partial_kernel); n_parts from amax_parts_count.  zero_ptr[0 .. n_zero)
+// is cleared on the way (counters that must start at zero).
+int amax_parts_count(int64_t rows, int64_t K);
+cudaError_t launch_amax_partial(const uint16_t* x, int64_t rows, int64_t K, int64_t ldx, int32_t batch,
+                                int64_t mat_stride, unsigned* parts, int n_parts, unsigned* zero_ptr,
+                                int n_zero, cudaStream_t s);
+
+// amax: fp32 per group, or (n_parts > 0) the max of amax_parts[0 .. n_parts).
 cudaError_t launch_quant_score(const uint16_t* x, int64_t rows, int64_t K, int64_t ldx,
-                               const RowGroups& g, const float* amax, int64_t codes_rows,
+                               const RowGroups& g, const float* amax, const unsigned* amax_parts,
+                               int n_parts, int64_t codes_rows,
                                uint8_t* codes, uint8_t* scales, int layout, float* tensor_scale,
                                double* part_sum, float* part_max, unsigned* strip_count,
                                double* score, float* colamax, cudaStream_t s);
@@ -68,9 +78,10 @@ cudaError_t launch_weight_gather(const uint16_t* w, int64_t N, int64_t K, int64_
                                  int layout, cudaStream_t s);
 
 // W' = bf16(DQ(Q(W))) for `batch` matrices; optional Q(W) and colamax
-// (colamax_bits zeroed by the caller, written as fp32 bits).
+// (colamax_bits zeroed beforehand, written as fp32 bits).  amax of matrix b:
+// max of amax_parts[b * n_parts .. + n_parts).
 cudaError_t launch_weight_qdq(const uint16_t* w, int64_t N, int64_t K, int64_t ldw, int32_t batch,
-                              const unsigned* amax_bits, uint16_t* w_out, uint8_t* codes,
+                              const unsigned* amax_parts, int n_parts, uint16_t* w_out, uint8_t* codes,
                               uint8_t* scales, int layout, float* tensor_scale,
                               unsigned* colamax_bits, cudaStream_t s);
 

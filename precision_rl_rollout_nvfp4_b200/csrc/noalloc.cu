@@ -44,9 +44,9 @@ extern "C" nvfp4_status nvfp4_quantize_static_ws(const uint16_t* x, int64_t M, i
   void* ws = scratch_address();
   if (ws == nullptr) return NVFP4_ERR_CUDA;
   // nvfp4_quantize refuses (NVFP4_ERR_WORKSPACE, before anything is queued)
-  // any shape whose scratch exceeds the array, and clears the amax and
-  // counter words on the stream before use, so whatever an earlier call left
-  // in the array does not matter.
+  // any shape whose scratch exceeds the array, and writes every scratch word
+  // it reads (partial maxima, cleared counters) on the stream before use, so
+  // whatever an earlier call left in the array does not matter.
   return nvfp4_quantize(x, M, K, ldx, amax_or_null, qx, score_or_null, res_colamax_or_null, ws,
                         kStaticScratchBytes, stream);
 }

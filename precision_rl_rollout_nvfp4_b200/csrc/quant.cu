@@ -71,6 +71,68 @@ __global__ void group_tiles_kernel(const int64_t* __restrict__ off, int32_t E,
   tile_start[E] = acc;
 }
 
+// Per-CTA partial maxima of |x| for `batch` dense matrices (blockIdx.y), no
+// atomics and nothing to clear beforehand: CTA i of matrix b writes
+// parts[b * gridDim.x + i] (fp32 bits); the consumer takes the max of the
+// partials (exact in any order).  Grid-stride over 16-byte vectors with eight
+// loads in flight per thread.  The grid also clears zero_ptr[0 .. n_zero).
+__global__ void __launch_bounds__(kQThreads)
+amax_partial_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t K, int64_t ldx,
+                    int64_t mat_stride, unsigned* __restrict__ parts, unsigned* __restrict__ zero_ptr,
+                    int n_zero) {
+  x += blockIdx.y * mat_stride;
+  {
+    const int cta = blockIdx.y * gridDim.x + blockIdx.x;
+    const int nthreads = gridDim.x * gridDim.y * kQThreads;
+    for (int i = cta * kQThreads + threadIdx.x; i < n_zero; i += nthreads) zero_ptr[i] = 0u;
+  }
+  const int64_t kv = K / 8;                       // 16-byte vectors per row
+  const int64_t nvec = rows * kv;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * kQThreads;
+  const bool flat = ldx == K;
+  uint32_t m = 0;
+  for (int64_t v0 = static_cast<int64_t>(blockIdx.x) * kQThreads + threadIdx.x; v0 < nvec; v0 += 8 * stride) {
+    uint4 r[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int64_t v = v0 + u * stride;
+      r[u] = make_uint4(0, 0, 0, 0);
+      if (v < nvec) {
+        const int64_t off = flat ? v * 8 : (v / kv) * ldx + (v % kv) * 8;
+        r[u] = ld_nc_v4(x + off);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const uint32_t w[4] = {r[u].x, r[u].y, r[u].z, r[u].w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) m = max(m, max(w[j] & 0x7FFFu, (w[j] >> 16) & 0x7FFFu));
+    }
+  }
+  m = __reduce_max_sync(0xFFFFFFFFu, m);
+  __shared__ uint32_t wmax[kQThreads / 32];
+  if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    uint32_t r = 0;
+    for (int i = 0; i < kQThreads / 32; ++i) r = max(r, wmax[i]);
+    parts[blockIdx.y * gridDim.x + blockIdx.x] = r << 16;   // |bf16| bits order like their values
+  }
+}
+
+// Block-wide max of n partial maxima (fp32 bits); every thread gets it.
+__device__ __forceinline__ float reduce_parts(const unsigned* parts, int n, uint32_t* wscratch) {
+  uint32_t m = 0;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) m = max(m, __ldcg(parts + i));
+  m = __reduce_max_sync(0xFFFFFFFFu, m);
+  if ((threadIdx.x & 31) == 0) wscratch[threadIdx.x >> 5] = m;
+  __syncthreads();
+  uint32_t r = 0;
+  for (int i = 0; i < static_cast<int>(blockDim.x >> 5); ++i) r = max(r, wscratch[i]);
+  __syncthreads();
+  return __uint_as_float(r);
+}
+
 // ---------------------------------------------------------------------------
 // quantize + residual + score partials (+ the ordered reduction of the
 // partials by the last CTA of each 64-column strip of a row group)
@@ -84,7 +146,8 @@ __global__ void group_tiles_kernel(const int64_t* __restrict__ off, int32_t E,
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(kQThreads)
 quant_score_kernel(const uint16_t* __restrict__ x, int64_t K, int64_t ldx, RowGroups g,
-                   const float* __restrict__ amax, int64_t codes_rows,
+                   const float* __restrict__ amax, const unsigned* __restrict__ amax_parts,
+                   int n_parts, int64_t codes_rows,
                    uint8_t* __restrict__ codes, uint8_t* __restrict__ scales, int layout,
                    float* __restrict__ tensor_scale, double* __restrict__ part_sum,
                    float* __restrict__ part_max, unsigned* __restrict__ strip_count,
@@ -100,17 +163,18 @@ quant_score_kernel(const uint16_t* __restrict__ x, int64_t K, int64_t ldx, RowGr
   const int t = threadIdx.x, cg = t & 7, grp = t >> 3;
   const int64_t col0 = static_cast<int64_t>(blockIdx.x) * kQCols;
   const int64_t col = col0 + 8 * cg;
-  const float s_t = __fdiv_rn(amax[ti.e], kTensorScaleDiv);
-  if (blockIdx.x == 0 && t == 0 && (g.off == nullptr ? tile == 0 : tile == g.tile_start[ti.e]))
-    tensor_scale[ti.e] = s_t;
-  build_scale_table(T, s_t, t);
-
   uint4 raw[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int64_t row = ti.row0 + 4 * grp + i;
     raw[i] = row < ti.row_end ? ld_nc_v4(x + row * ldx + col) : make_uint4(0, 0, 0, 0);
   }
+  __shared__ uint32_t wscratch[kQThreads / 32];
+  const float a = n_parts > 0 ? reduce_parts(amax_parts, n_parts, wscratch) : amax[ti.e];
+  const float s_t = __fdiv_rn(a, kTensorScaleDiv);
+  if (blockIdx.x == 0 && t == 0 && (g.off == nullptr ? tile == 0 : tile == g.tile_start[ti.e]))
+    tensor_scale[ti.e] = s_t;
+  build_scale_table(T, s_t, t);
   __syncthreads();                               // table ready
   uint8_t* code_base = codes + tile * kTileRows * (K / 2) + col / 2;
   double acc[8];
@@ -406,16 +470,13 @@ __global__ void sel_tensor_scale_kernel(const float* __restrict__ colamax, int64
 // grid = (K/64, ceil(N/128), batch).
 __global__ void __launch_bounds__(kQThreads)
 weight_qdq_kernel(const uint16_t* w, int64_t N, int64_t K, int64_t ldw,
-                  const unsigned* __restrict__ amax_bits, uint16_t* w_out,   // w_out may alias w
+                  const unsigned* __restrict__ amax_parts, int n_parts,
+                  uint16_t* w_out,   // w_out may alias w
                   uint8_t* __restrict__ codes, uint8_t* __restrict__ scales, int layout,
                   float* __restrict__ tensor_scale, unsigned* __restrict__ colamax_bits) {
   const int64_t b = blockIdx.z;
   const int t = threadIdx.x, cg = t & 7, rr = t >> 3;
   const int64_t col = static_cast<int64_t>(blockIdx.x) * 64 + 8 * cg;
-  const float s_t = __fdiv_rn(__uint_as_float(amax_bits[b]), kTensorScaleDiv);
-  if (tensor_scale && blockIdx.x == 0 && blockIdx.y == 0 && t == 0) tensor_scale[b] = s_t;
-  __shared__ ScaleTable T;
-  build_scale_table(T, s_t, t);
   uint32_t cmax[8] = {0, 0, 0, 0, 0, 0, 0, 0};
   uint4 raw[4];
 #pragma unroll
@@ -424,6 +485,11 @@ weight_qdq_kernel(const uint16_t* w, int64_t N, int64_t K, int64_t ldw,
     // coherent load: w may alias w_out
     raw[i] = n < N ? *reinterpret_cast<const uint4*>(w + (b * N + n) * ldw + col) : make_uint4(0, 0, 0, 0);
   }
+  __shared__ uint32_t wscratch[kQThreads / 32];
+  const float s_t = __fdiv_rn(reduce_parts(amax_parts + b * n_parts, n_parts, wscratch), kTensorScaleDiv);
+  if (tensor_scale && blockIdx.x == 0 && blockIdx.y == 0 && t == 0) tensor_scale[b] = s_t;
+  __shared__ ScaleTable T;
+  build_scale_table(T, s_t, t);
   __syncthreads();                               // table ready
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
@@ -519,16 +585,31 @@ cudaError_t launch_group_tiles(const int64_t* off, int32_t E, int32_t* tile_star
 }
 
 cudaError_t launch_quant_score(const uint16_t* x, int64_t rows, int64_t K, int64_t ldx,
-                               const RowGroups& g, const float* amax, int64_t codes_rows,
+                               const RowGroups& g, const float* amax, const unsigned* amax_parts,
+                               int n_parts, int64_t codes_rows,
                                uint8_t* codes, uint8_t* scales, int layout, float* tensor_scale,
                                double* part_sum, float* part_max, unsigned* strip_count,
                                double* score, float* colamax, cudaStream_t s) {
   const int64_t tiles = max_tiles(g, rows);
   if (tiles == 0) return cudaSuccess;
   dim3 grid(static_cast<unsigned>(K / kQCols), static_cast<unsigned>(tiles));
-  quant_score_kernel<<<grid, kQThreads, 0, s>>>(x, K, ldx, g, amax, codes_rows, codes, scales,
-                                                layout, tensor_scale, part_sum, part_max, strip_count,
-                                                score, colamax);
+  quant_score_kernel<<<grid, kQThreads, 0, s>>>(x, K, ldx, g, amax, amax_parts, n_parts, codes_rows, codes,
+                                                scales, layout, tensor_scale, part_sum, part_max,
+                                                strip_count, score, colamax);
+  return cudaGetLastError();
+}
+
+int amax_parts_count(int64_t rows, int64_t K) {
+  const int64_t nvec = rows * (K / 8);
+  const int64_t want = (nvec + 8 * kQThreads - 1) / (8 * kQThreads);
+  return static_cast<int>(want < 4 * 148 ? (want > 0 ? want : 1) : 4 * 148);
+}
+
+cudaError_t launch_amax_partial(const uint16_t* x, int64_t rows, int64_t K, int64_t ldx, int32_t batch,
+                                int64_t mat_stride, unsigned* parts, int n_parts, unsigned* zero_ptr,
+                                int n_zero, cudaStream_t s) {
+  dim3 grid(static_cast<unsigned>(n_parts), static_cast<unsigned>(batch));
+  amax_partial_kernel<<<grid, kQThreads, 0, s>>>(x, rows, K, ldx, mat_stride, parts, zero_ptr, n_zero);
   return cudaGetLastError();
 }
 
@@ -587,12 +668,12 @@ cudaError_t launch_weight_gather(const uint16_t* w, int64_t N, int64_t K, int64_
 }
 
 cudaError_t launch_weight_qdq(const uint16_t* w, int64_t N, int64_t K, int64_t ldw, int32_t batch,
-                              const unsigned* amax_bits, uint16_t* w_out, uint8_t* codes,
+                              const unsigned* amax_parts, int n_parts, uint16_t* w_out, uint8_t* codes,
                               uint8_t* scales, int layout, float* tensor_scale,
                               unsigned* colamax_bits, cudaStream_t s) {
   dim3 grid(static_cast<unsigned>(K / 64), static_cast<unsigned>((N + 127) / 128),
             static_cast<unsigned>(batch));
-  weight_qdq_kernel<<<grid, kQThreads, 0, s>>>(w, N, K, ldw, amax_bits, w_out, codes, scales,
+  weight_qdq_kernel<<<grid, kQThreads, 0, s>>>(w, N, K, ldw, amax_parts, n_parts, w_out, codes, scales,
                                                layout, tensor_scale, colamax_bits);
   return cudaGetLastError();
 }
