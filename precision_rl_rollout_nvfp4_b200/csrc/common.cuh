@@ -53,90 +53,77 @@ __device__ __forceinline__ uint32_t f32_to_e4m3(float s) {
   return r & 0xFFu;
 }
 
-// E2M1 magnitude codes of |v[0..7]| packed 2 per byte, element 2j in the
-// low nibble of byte j (hardware conversion, round to nearest even,
-// saturating at 6).  The sign bits are added from the inputs' own sign bits,
-// so a negative value that rounds to zero keeps its sign (code 0x8).
+// E2M1 codes of v[0..7] packed 2 per byte, element 2j in the low nibble of
+// byte j (hardware conversion of the signed value: round to nearest even,
+// saturating at 6, the sign kept even when the value rounds to zero, so that
+// a negative input gives code 0x8 there).
 __device__ __forceinline__ uint32_t e2m1x8(const float* v) {
-  uint32_t mags;
+  uint32_t codes;
   asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
       "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
       "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
       "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
       "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
       "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
-      : "=r"(mags)
-      : "f"(fabsf(v[0])), "f"(fabsf(v[1])), "f"(fabsf(v[2])), "f"(fabsf(v[3])),
-        "f"(fabsf(v[4])), "f"(fabsf(v[5])), "f"(fabsf(v[6])), "f"(fabsf(v[7])));
-  uint32_t signs = 0;
-#pragma unroll
-  for (int j = 0; j < 8; ++j) signs |= (__float_as_uint(v[j]) >> 31) << (4 * j + 3);
-  return mags | signs;
+      : "=r"(codes)
+      : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
+  return codes;
 }
 
-// Per-block quantization parameters for a tensor with decode scale s_t:
-// sb = E4M3(RN(amax_b / RN(6 s_t))), s_dec = RN(E4M3dec(sb) s_t).
-struct BlockScale {
-  uint32_t sb;
-  float sbv;
-  float s_dec;
-};
+// ---- fp32 pairs ------------------------------------------------------------
+// sm_100a executes mul / fma (and add / sub) on two fp32 lanes in one
+// instruction (.f32x2, each lane rounded to nearest even like the scalar
+// form).  A pair lives in one 64-bit register: element 2j in the low half.
+// A packed product that feeds a packed sum or difference can be fused into
+// one rounding by the code generator, so only products whose result is
+// consumed by something other than an addition use the packed form.
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_abs(uint64_t a) { return a & 0x7FFFFFFF7FFFFFFFull; }
 
-__device__ __forceinline__ BlockScale block_scale(float amax_b, float s_t) {
-  BlockScale r;
-  const float d = __fmul_rn(6.0f, s_t);
-  if (d > 0.0f) {
-    r.sb = f32_to_e4m3(__fdiv_rn(amax_b, d));
-  } else {
-    r.sb = 0;
-  }
-  r.sbv = e4m3_to_f32(r.sb);
-  r.s_dec = __fmul_rn(r.sbv, s_t);
+// The two bf16 of a 32-bit word as an fp32 pair (exact).
+__device__ __forceinline__ uint64_t bf16x2_to_f2(uint32_t w) {
+  return f2_pack(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+}
+
+// Exact values of the two E2M1 codes of a byte (low nibble first) as an fp32
+// pair, through the hardware e2m1x2 -> f16x2 conversion.
+__device__ __forceinline__ uint64_t e2m1x2_to_f2(uint32_t byte) {
+  uint64_t r;
+  asm("{\n\t.reg .b8 t;\n\t.reg .b32 h;\n\t.reg .b16 l, u;\n\t.reg .f32 fl, fu;\n\t"
+      "cvt.u8.u32 t, %1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 h, t;\n\t"
+      "mov.b32 {l, u}, h;\n\t"
+      "cvt.f32.f16 fl, l;\n\t"
+      "cvt.f32.f16 fu, u;\n\t"
+      "mov.b64 %0, {fl, fu};\n\t}"
+      : "=l"(r) : "r"(byte));
   return r;
 }
 
-// RN(x / b) for a whole block that shares the divisor b = s_dec > 0, with
-// y = RN(1/b) computed once per block (__frcp_rn).  Markstein's correction
-// (P. Markstein, IBM J. Res. Dev. 1990; Muller et al., Handbook of
-// Floating-Point Arithmetic, division with an FMA): q = RN(x y) is within one
-// ulp of x/b, the remainder r = x - b q is exact with an FMA, and
-// RN(q + r y) = RN(x / b) when y is within half an ulp of 1/b and nothing
-// under- or overflows.  Blocks whose divisor is below 2^-100 use the full
-// division instead.  The sign of the result is that of x (x = -0 gives -0).
-struct BlockDivisor {
-  float b, y;
-  bool fast;
-};
-
-__device__ __forceinline__ BlockDivisor block_divisor(float s_dec) {
-  BlockDivisor d;
-  d.b = s_dec;
-  d.fast = s_dec >= 7.888609052210118e-31f;   // 2^-100
-  d.y = d.fast ? __frcp_rn(s_dec) : 0.0f;
-  return d;
-}
-
-__device__ __forceinline__ float div_block(float x, const BlockDivisor& d) {
-  float q;
-  if (d.b <= 0.0f) {
-    q = 0.0f;
-  } else if (d.fast) {
-    const float q0 = __fmul_rn(x, d.y);
-    const float r = __fmaf_rn(-q0, d.b, x);
-    q = __fmaf_rn(r, d.y, q0);
-  } else {
-    q = __fdiv_rn(x, d.b);
-  }
-  return __uint_as_float((__float_as_uint(q) & 0x7FFFFFFFu) | (__float_as_uint(x) & 0x80000000u));
-}
-
-// Codes of 8 consecutive elements (one half of a block) -> 4 bytes, element
-// 2j in the low nibble of byte j.
-__device__ __forceinline__ uint32_t encode8(const float* v, const BlockDivisor& d) {
-  float q[8];
+// E2M1 codes of four fp32 pairs (8 elements) -> 4 bytes, element 2j in the
+// low nibble of byte j.
+__device__ __forceinline__ uint32_t e2m1x8_f2(const uint64_t* p) {
+  float v[8];
 #pragma unroll
-  for (int j = 0; j < 8; ++j) q[j] = div_block(v[j], d);
-  return e2m1x8(q);
+  for (int j = 0; j < 4; ++j) f2_unpack(p[j], v[2 * j], v[2 * j + 1]);
+  return e2m1x8(v);
 }
 
 // Per-tensor-scale lookup of everything a block needs, built once per CTA
@@ -146,7 +133,7 @@ __device__ __forceinline__ uint32_t encode8(const float* v, const BlockDivisor& 
 //   rcp[sb]  = RN(1 / sdec[sb])            (0 when sdec < 2^-64: full division),
 // plus d = RN(6 s_t) and its reciprocal for the block-scale quotient.  The
 // quotients then cost one multiply and two FMAs (Markstein's correction, see
-// div_block) instead of a full IEEE division per block and per element.
+// div_rn_pos) instead of a full IEEE division per block and per element.
 struct ScaleTable {
   float sbv[128], sdec[128], rcp[128];
   float s_t, d, rcp_d;
@@ -171,9 +158,13 @@ __device__ __forceinline__ void build_scale_table(ScaleTable& T, float s_t, int 
 
 static __device__ __noinline__ float div_slow(float a, float b) { return __fdiv_rn(a, b); }
 
-// RN(a / b) for a >= 0, b > 0, with y = RN(1/b) (or y == 0: full division).
-// With b >= 2^-64 the remainder a - b q0 is exact for every quotient that can
-// change an E2M1 or E4M3 code (>= 2^-10), so Markstein's correction holds.
+// RN(a / b) for a >= 0, b > 0, with y = RN(1/b) (or y == 0: full division),
+// by Markstein's correction (P. Markstein, IBM J. Res. Dev. 1990; Muller et
+// al., Handbook of Floating-Point Arithmetic, division with an FMA):
+// q0 = RN(a y) is within one ulp of a/b, the remainder r = a - b q0 is exact
+// with an FMA, and RN(q0 + r y) = RN(a / b).  With b >= 2^-64 the remainder
+// is exact for every quotient that can change an E2M1 or E4M3 code
+// (>= 2^-10).
 __device__ __forceinline__ float div_rn_pos(float a, float b, float y) {
   if (y == 0.0f) return div_slow(a, b);
   const float q0 = __fmul_rn(a, y);
@@ -196,47 +187,40 @@ __device__ __forceinline__ BlockQ block_q(float amax_b, const ScaleTable& T) {
   return q;
 }
 
-// E2M1 codes of 8 values with block parameters q: magnitudes of RN(|v|/sdec)
-// through the hardware conversion, sign bits from v (so -0 keeps code 0x8).
+// Quotients of one block for four fp32 pairs: RN(|v| / sdec) with the sign
+// bit of v (signed zeros when sdec == 0), through div_rn_pos's steps on both
+// lanes at once.
+__device__ __forceinline__ void block_quotients(const uint64_t* x2, const BlockQ& q, uint64_t* out) {
+  constexpr uint64_t kSign = 0x8000000080000000ull;
+  if (q.sdec > 0.0f && q.rcp != 0.0f) {
+    const uint64_t y2 = f2_pack(q.rcp, q.rcp), nb2 = f2_pack(-q.sdec, -q.sdec);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint64_t a = f2_abs(x2[j]);
+      const uint64_t q0 = f2_mul(a, y2);
+      const uint64_t r = f2_fma(q0, nb2, a);          // a - q0 sdec, exact
+      out[j] = f2_fma(r, y2, q0) | (x2[j] & kSign);
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      float lo, hi;
+      f2_unpack(f2_abs(x2[j]), lo, hi);
+      const float ql = q.sdec > 0.0f ? div_slow(lo, q.sdec) : 0.0f;
+      const float qh = q.sdec > 0.0f ? div_slow(hi, q.sdec) : 0.0f;
+      out[j] = f2_pack(ql, qh) | (x2[j] & kSign);
+    }
+  }
+}
+
+// E2M1 codes of 8 values with block parameters q: the signed quotients of
+// block_quotients through the hardware conversion (so -0 keeps code 0x8).
 __device__ __forceinline__ uint32_t encode8_q(const float* v, const BlockQ& q) {
-  float a[8];
+  uint64_t x2[4], o[4];
 #pragma unroll
-  for (int j = 0; j < 8; ++j) a[j] = q.sdec > 0.0f ? div_rn_pos(fabsf(v[j]), q.sdec, q.rcp) : 0.0f;
-  uint32_t mags;
-  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
-      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
-      : "=r"(mags)
-      : "f"(a[0]), "f"(a[1]), "f"(a[2]), "f"(a[3]), "f"(a[4]), "f"(a[5]), "f"(a[6]), "f"(a[7]));
-  uint32_t signs = 0;
-#pragma unroll
-  for (int j = 0; j < 8; ++j) signs |= (__float_as_uint(v[j]) >> 31) << (4 * j + 3);
-  return mags | signs;
-}
-
-// Exact E4M3 value of a non-negative code through the hardware e4m3 -> f16
-// conversion (every E4M3 value is an f16 value).
-__device__ __forceinline__ float e4m3_to_f32_hw(uint32_t code) {
-  uint32_t h2;
-  asm("{\n\t.reg .b16 t;\n\tcvt.u16.u32 t, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, t;\n\t}" : "=r"(h2) : "r"(code & 0xFFu));
-  return __half2float(__ushort_as_half(static_cast<unsigned short>(h2 & 0xFFFFu)));
-}
-
-// Exact E2M1 values of the two codes of a packed byte (low nibble first),
-// through the hardware e2m1x2 -> f16x2 conversion.
-__device__ __forceinline__ void e2m1x2_to_f32(uint32_t byte, float& lo, float& hi) {
-  uint32_t h2;
-  asm("{\n\t.reg .b8 t;\n\tcvt.u8.u32 t, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, t;\n\t}" : "=r"(h2) : "r"(byte));
-  lo = __half2float(__ushort_as_half(static_cast<unsigned short>(h2 & 0xFFFFu)));
-  hi = __half2float(__ushort_as_half(static_cast<unsigned short>(h2 >> 16)));
-}
-
-// DQ = RN(RN(E2M1dec(code) * E4M3dec(sb)) * s_t).
-__device__ __forceinline__ float dequant(uint32_t code, float sbv, float s_t) {
-  return __fmul_rn(__fmul_rn(e2m1_to_f32(code), sbv), s_t);
+  for (int j = 0; j < 4; ++j) x2[j] = f2_pack(v[2 * j], v[2 * j + 1]);
+  block_quotients(x2, q, o);
+  return e2m1x8_f2(o);
 }
 
 // Byte offset of the scale of (row, block) in an NVFP4 scale buffer.
@@ -247,13 +231,15 @@ __device__ __host__ __forceinline__ int64_t scale_offset(int64_t row, int64_t bl
   return ((row >> 7) * k4 + (blk >> 2)) * 512 + (row & 31) * 16 + ((row & 127) >> 5) * 4 + (blk & 3);
 }
 
-__device__ __forceinline__ void unpack_bf16x8(const uint4& v, float* f) {
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    f[2 * j] = __uint_as_float(w[j] << 16);
-    f[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
-  }
+// Programmatic dependent launch (kernels started by launch_k): pdl_wait()
+// returns once the previous kernel of the stream has completed and its
+// writes are visible; every thread calls it before its first global memory
+// access.  pdl_launch_dependents() lets the next kernel of the stream be
+// scheduled (it then waits in its own pdl_wait()).  Both are no-ops for a
+// kernel launched without the attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 __device__ __forceinline__ uint4 ld_nc_v4(const void* p) {

@@ -199,6 +199,9 @@ w4a4_rac_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_cons
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // barriers and TMEM are set up: wait for the previous kernel's writes
+  pdl_wait();
+  pdl_launch_dependents();
 
   const int64_t m_tiles = p.g.off ? p.g.tile_start[p.g.E] : p.m_tiles_dense;
   const int64_t total = m_tiles * p.n_tiles;
@@ -543,6 +546,9 @@ w4a4_rac_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // barriers and TMEM are set up: wait for the previous kernel's writes
+  pdl_wait();
+  pdl_launch_dependents();
 
   const int total = p.m_tiles * p.n_tiles;
   const bool has_res = p.kt[0] > 0;
@@ -785,20 +791,14 @@ cudaError_t launch_pair(const GemmArgs& a, cudaStream_t s) {
   const int tiles = p.m_tiles * p.n_tiles;
   const int pairs = tiles < sm_count() / 2 ? tiles : sm_count() / 2;
   if (pairs == 0) return cudaSuccess;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
-  cfg.blockDim = dim3(THREADS);
-  cfg.dynamicSmemBytes = C::SMEM_BYTES;
-  cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, w4a4_rac_gemm_pair_kernel<YBYTES>, maps[0], maps[1], maps[2], maps[3],
-                            maps[4], maps[5], maps[6], maps[7], p);
+  return launch_k(w4a4_rac_gemm_pair_kernel<YBYTES>, dim3(static_cast<unsigned>(2 * pairs)), dim3(THREADS),
+                  C::SMEM_BYTES, s, attr, 1, maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], maps[6],
+                  maps[7], p);
 }
 
 }  // namespace
@@ -842,9 +842,17 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s) {
   if (tiles_bound == 0) return cudaSuccess;
   const int grid = static_cast<int>(tiles_bound < sm_count() ? tiles_bound : sm_count());
   if (a.y_dtype == 0)
-    w4a4_rac_gemm_kernel<4><<<grid, THREADS, Cfg<4>::SMEM_BYTES, s>>>(maps[0], maps[1], maps[2], maps[3], p);
+    {
+      const cudaError_t le = launch_k(w4a4_rac_gemm_kernel<4>, dim3(grid), dim3(THREADS), Cfg<4>::SMEM_BYTES, s, nullptr, 0,
+                                     maps[0], maps[1], maps[2], maps[3], p);
+      if (le != cudaSuccess) return le;
+    }
   else
-    w4a4_rac_gemm_kernel<2><<<grid, THREADS, Cfg<2>::SMEM_BYTES, s>>>(maps[0], maps[1], maps[2], maps[3], p);
+    {
+      const cudaError_t le = launch_k(w4a4_rac_gemm_kernel<2>, dim3(grid), dim3(THREADS), Cfg<2>::SMEM_BYTES, s, nullptr, 0,
+                                     maps[0], maps[1], maps[2], maps[3], p);
+      if (le != cudaSuccess) return le;
+    }
   return cudaGetLastError();
 }
 

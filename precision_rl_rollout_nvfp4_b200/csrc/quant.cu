@@ -27,6 +27,8 @@ constexpr int kQCols = 64;
 __global__ void __launch_bounds__(kQThreads)
 amax_kernel(const uint16_t* __restrict__ x, int64_t K, int64_t ldx, RowGroups g,
             int64_t mat_stride, unsigned* __restrict__ amax_bits) {
+  pdl_wait();
+  pdl_launch_dependents();
   // blockIdx.z: matrix of a stack of dense matrices (mat_stride elements apart)
   x += blockIdx.z * mat_stride;
   amax_bits += blockIdx.z;
@@ -61,6 +63,8 @@ amax_kernel(const uint16_t* __restrict__ x, int64_t K, int64_t ldx, RowGroups g,
 
 __global__ void group_tiles_kernel(const int64_t* __restrict__ off, int32_t E,
                                    int32_t* __restrict__ tile_start) {
+  pdl_wait();
+  pdl_launch_dependents();
   if (threadIdx.x != 0) return;
   int32_t acc = 0;
   for (int e = 0; e < E; ++e) {
@@ -80,6 +84,8 @@ __global__ void __launch_bounds__(kQThreads)
 amax_partial_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t K, int64_t ldx,
                     int64_t mat_stride, unsigned* __restrict__ parts, unsigned* __restrict__ zero_ptr,
                     int n_zero) {
+  pdl_wait();
+  pdl_launch_dependents();
   x += blockIdx.y * mat_stride;
   {
     const int cta = blockIdx.y * gridDim.x + blockIdx.x;
@@ -152,6 +158,8 @@ quant_score_kernel(const uint16_t* __restrict__ x, int64_t K, int64_t ldx, RowGr
                    float* __restrict__ tensor_scale, double* __restrict__ part_sum,
                    float* __restrict__ part_max, unsigned* __restrict__ strip_count,
                    double* __restrict__ score, float* __restrict__ colamax) {
+  pdl_wait();
+  pdl_launch_dependents();
   const int64_t tile = blockIdx.y;
   const TileInfo ti = tile_info(g, tile);
   if (!ti.valid) return;
@@ -185,20 +193,32 @@ quant_score_kernel(const uint16_t* __restrict__ x, int64_t K, int64_t ldx, RowGr
   for (int i = 0; i < 4; ++i) {
     const int r = 4 * grp + i;
     const int64_t prow = tile * kTileRows + r;
-    float f[8];
-    unpack_bf16x8(raw[i], f);
-    float am = 0.0f;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) am = fmaxf(am, fabsf(f[j]));
-    am = fmaxf(am, __shfl_xor_sync(0xFFFFFFFFu, am, 1));
-    const BlockQ bq = block_q(am, T);
-    const uint32_t packed = encode8_q(f, bq);
+    const uint32_t wv[4] = {raw[i].x, raw[i].y, raw[i].z, raw[i].w};
+    uint64_t x2[4];
+    uint32_t mbits = 0;                            // max |bf16| bits, two lanes
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      float lo, hi;
-      e2m1x2_to_f32((packed >> (8 * j)) & 0xFFu, lo, hi);
-      const float d0 = fabsf(__fsub_rn(f[2 * j], __fmul_rn(__fmul_rn(lo, bq.sbv), s_t)));
-      const float d1 = fabsf(__fsub_rn(f[2 * j + 1], __fmul_rn(__fmul_rn(hi, bq.sbv), s_t)));
+      x2[j] = bf16x2_to_f2(wv[j]);
+      mbits = __vmaxu2(mbits, wv[j] & 0x7FFF7FFFu);
+    }
+    float am = __uint_as_float(max(mbits & 0xFFFFu, mbits >> 16) << 16);
+    am = fmaxf(am, __shfl_xor_sync(0xFFFFFFFFu, am, 1));
+    const BlockQ bq = block_q(am, T);
+    uint64_t q2[4];
+    block_quotients(x2, bq, q2);
+    const uint32_t packed = e2m1x8_f2(q2);
+    const uint64_t sbv2 = f2_pack(bq.sbv, bq.sbv);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      // |dX| = |RN(x - RN(p * s_t))| with p = E2M1dec * E4M3dec (exact, both
+      // lanes at once).  The last product and the difference stay scalar:
+      // the packed forms of a product followed by a difference are fused
+      // into one rounding by the code generator, which changes dX.
+      float p0, p1, x0, x1;
+      f2_unpack(f2_mul(e2m1x2_to_f2((packed >> (8 * j)) & 0xFFu), sbv2), p0, p1);
+      f2_unpack(x2[j], x0, x1);
+      const float d0 = fabsf(__fsub_rn(x0, __fmul_rn(p0, s_t)));
+      const float d1 = fabsf(__fsub_rn(x1, __fmul_rn(p1, s_t)));
       acc[2 * j] += static_cast<double>(d0);       // rows of the group in order
       acc[2 * j + 1] += static_cast<double>(d1);
       mx[2 * j] = fmaxf(mx[2 * j], d0);
@@ -275,6 +295,8 @@ __global__ void score_reduce_kernel(const double* __restrict__ part_sum,
                                     const float* __restrict__ part_max, int64_t K, RowGroups g,
                                     int64_t tiles, double* __restrict__ score,
                                     float* __restrict__ colamax, float* __restrict__ st_empty) {
+  pdl_wait();
+  pdl_launch_dependents();
   const int e = blockIdx.y;
   int64_t t0 = 0, t1 = tiles;
   if (g.off != nullptr) { t0 = g.tile_start[e]; t1 = g.tile_start[e + 1]; }
@@ -298,14 +320,16 @@ constexpr int kGThreads = 256;
 
 // Second-pass gather + quantize, shared by the residual and the weight side.
 // A CTA (256 threads) takes tiles of 16 rows x 256 gathered channels:
-//   phase 1: sel[j0 .. j0+255] into shared memory; every thread gathers 16
-//            values (rows r, channels j0 + lane + 32 u): a warp's loads cover
-//            32 consecutive gathered channels, and all 16 are in flight;
-//            the residual side recomputes dX = x - DQ(Q(x)) from X, Q(X) and
-//            its scales; values go to shared memory;
+//   phase 1: every thread reads the 8 channels it gathers straight from
+//            sel[j0 + lane + 32 u] and then gathers 16 values (rows 2w and
+//            2w+1, those channels), all loads in flight at once; the residual
+//            side recomputes dX = x - DQ(Q(x)) from X, the code nibble and
+//            the block scale byte of Q(X) (decoded through small shared
+//            tables); values go to shared memory;
 //   phase 2: thread = one 16-block (row, block): block scale, codes, stores.
-// Tiles are visited grid-stride; with fuse_scale (one weight) every CTA first
-// reduces the W_sel tensor scale from colamax and sel, CTA 0 publishes it.
+// Tiles are visited grid-stride.  With fuse_scale (one weight) the W_sel
+// tensor scale max_{j in sel} colamax_j / 2688 is reduced during the first
+// tile, its loads issued beside that tile's gather loads; CTA 0 publishes it.
 constexpr int kGRows = 16, kGCols = 256;
 
 template <bool RESIDUAL>
@@ -317,29 +341,22 @@ gather_quant_kernel(const uint16_t* __restrict__ src, int64_t K, int64_t ld, Row
                     const float* __restrict__ colamax, int fuse_scale, float* __restrict__ out_st,
                     uint8_t* __restrict__ out_codes, uint8_t* __restrict__ out_scales, int out_layout,
                     int64_t out_rows, int64_t grid_rows) {
-  __shared__ int32_t s_sel[kGCols];
+  pdl_wait();
+  pdl_launch_dependents();
   __shared__ __align__(16) float s_val[kGRows][kGCols + 4];
-  __shared__ float s_fused;
+  __shared__ float s_e2m1[16];                     // E2M1 value of every code
+  __shared__ float s_e4m3[128];                    // E4M3 value of every scale byte
+  __shared__ float s_wm[kGThreads / 32];
   __shared__ ScaleTable T;
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-  if (!RESIDUAL && fuse_scale) {
-    float m = 0.0f;
-    for (int64_t j = t; j < n_sel; j += kGThreads) {
-      const int64_t c = __ldg(sel + j);
-      if (c >= 0 && c < K) m = fmaxf(m, __ldg(colamax + c));
-    }
-    m = __uint_as_float(__reduce_max_sync(0xFFFFFFFFu, __float_as_uint(m)));
-    __shared__ float wm[kGThreads / 32];
-    if (lane == 0) wm[warp] = m;
-    __syncthreads();
-    if (t == 0) {
-      float r = 0.0f;
-      for (int k = 0; k < kGThreads / 32; ++k) r = fmaxf(r, wm[k]);
-      s_fused = __fdiv_rn(r, kTensorScaleDiv);
-      if (blockIdx.x == 0) out_st[0] = s_fused;
-    }
-    __syncthreads();
+  if (RESIDUAL) {
+    if (t < 16) s_e2m1[t] = e2m1_to_f32(static_cast<uint32_t>(t));
+    if (t < 128) s_e4m3[t] = t < 127 ? e4m3_to_f32(static_cast<uint32_t>(t)) : 0.0f;
   }
+  const bool fuse = !RESIDUAL && fuse_scale != 0;
+  bool first = true;
+  float fused_st = 0.0f;
+  const uint32_t K32 = static_cast<uint32_t>(K);
   const int64_t row_tiles = (grid_rows + kGRows - 1) / kGRows;
   const int64_t col_tiles = (width + kGCols - 1) / kGCols;
   for (int64_t tile = blockIdx.x; tile < row_tiles * col_tiles; tile += gridDim.x) {
@@ -361,18 +378,24 @@ gather_quant_kernel(const uint16_t* __restrict__ src, int64_t K, int64_t ld, Row
       row_end = static_cast<int64_t>(e + 1) * N_per_group;
     }
     __syncthreads();                               // previous tile done with shared memory
-    {
-      const int64_t j = j0 + t;
-      s_sel[t] = (valid && j < n_sel) ? __ldg(sel + static_cast<int64_t>(e) * n_sel + j) : -1;
+    // level 1: the channels this thread gathers (and the fused scale's sel share)
+    const int32_t* sel_e = sel + static_cast<int64_t>(e) * n_sel;
+    int32_t c[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int64_t j = j0 + lane + 32 * u;
+      c[u] = (valid && j < n_sel) ? __ldg(sel_e + j) : -1;
     }
-    __syncthreads();
+    const bool do_fuse = fuse && first;
+    int32_t fc[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int64_t jf = t + kGThreads * u;
+      fc[u] = (do_fuse && jf < n_sel) ? __ldg(sel + jf) : -1;
+    }
+    // level 2: the values (and the fused scale's colamax share)
     const float st_x = (RESIDUAL && valid) ? qx_st[e] : 0.0f;
-    float st = 0.0f;
-    if (valid) st = RESIDUAL ? out_st[e] : (fuse_scale ? s_fused : out_st[e]);
-    build_scale_table(T, st, t);
-    // scale bytes of Q(X) for this row: row part of the tiled / canonical offset
     const int64_t k4 = (K + 63) / 64;
-    // phase 1: warp w gathers rows 2w, 2w+1; lane takes channels lane + 32 u
 #pragma unroll
     for (int rr = 0; rr < 2; ++rr) {
       const int r = 2 * warp + rr;
@@ -387,11 +410,9 @@ gather_quant_kernel(const uint16_t* __restrict__ src, int64_t K, int64_t ld, Row
                       ? qx_scales + ((prow >> 7) * k4) * 512 + (prow & 31) * 16 + ((prow & 127) >> 5) * 4
                       : qx_scales + prow * (K / kBlock);
       uint32_t xb[8], cb[8], sb[8];
-      int32_t c[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
-        c[u] = live ? s_sel[lane + 32 * u] : -1;
-        const bool ok = static_cast<uint32_t>(c[u]) < static_cast<uint32_t>(K);   // never false for a valid sel list
+        const bool ok = live && static_cast<uint32_t>(c[u]) < K32;   // never false for a valid sel list
         const uint32_t cc = ok ? static_cast<uint32_t>(c[u]) : 0u;
         xb[u] = ok ? __ldg(xrow + cc) : 0u;
         if (RESIDUAL) {
@@ -403,17 +424,45 @@ gather_quant_kernel(const uint16_t* __restrict__ src, int64_t K, int64_t ld, Row
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
         float v = 0.0f;
-        if (static_cast<uint32_t>(c[u]) < static_cast<uint32_t>(K)) {
+        if (live && static_cast<uint32_t>(c[u]) < K32) {
           v = bf16_bits_to_f32(xb[u]);
           if (RESIDUAL) {
-            float lo, hi;
-            e2m1x2_to_f32((cb[u] >> (4 * (c[u] & 1))) & 15u, lo, hi);
-            v = __fsub_rn(v, __fmul_rn(__fmul_rn(lo, e4m3_to_f32_hw(sb[u])), st_x));
+            const float q = s_e2m1[(cb[u] >> ((c[u] & 1) << 2)) & 15u];
+            v = __fsub_rn(v, __fmul_rn(__fmul_rn(q, s_e4m3[sb[u] & 127u]), st_x));
           }
         }
         s_val[r][lane + 32 * u] = v;
       }
     }
+    if (do_fuse) {
+      float fm = 0.0f;
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (static_cast<uint32_t>(fc[u]) < K32) fm = fmaxf(fm, __ldg(colamax + fc[u]));
+      for (int64_t base = t + 8 * kGThreads; base < n_sel; base += 8 * kGThreads) {   // n_sel > 2048
+        int32_t cf[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int64_t jf = base + kGThreads * u;
+          cf[u] = jf < n_sel ? __ldg(sel + jf) : -1;
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          if (static_cast<uint32_t>(cf[u]) < K32) fm = fmaxf(fm, __ldg(colamax + cf[u]));
+      }
+      fm = __uint_as_float(__reduce_max_sync(0xFFFFFFFFu, __float_as_uint(fm)));
+      if (lane == 0) s_wm[warp] = fm;
+      __syncthreads();
+      float r = 0.0f;
+#pragma unroll
+      for (int k = 0; k < kGThreads / 32; ++k) r = fmaxf(r, s_wm[k]);
+      fused_st = __fdiv_rn(r, kTensorScaleDiv);
+      if (blockIdx.x == 0 && t == 0) out_st[0] = fused_st;
+    }
+    first = false;
+    float st = 0.0f;
+    if (valid) st = RESIDUAL ? out_st[e] : (fuse ? fused_st : out_st[e]);
+    build_scale_table(T, st, t);
     __syncthreads();
     // phase 2: thread = (row t/16, block t%16)
     {
@@ -445,6 +494,8 @@ gather_quant_kernel(const uint16_t* __restrict__ src, int64_t K, int64_t ld, Row
 __global__ void sel_tensor_scale_kernel(const float* __restrict__ colamax, int64_t K,
                                         const int32_t* __restrict__ sel, int64_t n_sel,
                                         float* __restrict__ s_t) {
+  pdl_wait();
+  pdl_launch_dependents();
   const int e = blockIdx.x;
   float m = 0.0f;
   for (int64_t j = threadIdx.x; j < n_sel; j += blockDim.x) {
@@ -474,10 +525,12 @@ weight_qdq_kernel(const uint16_t* w, int64_t N, int64_t K, int64_t ldw,
                   uint16_t* w_out,   // w_out may alias w
                   uint8_t* __restrict__ codes, uint8_t* __restrict__ scales, int layout,
                   float* __restrict__ tensor_scale, unsigned* __restrict__ colamax_bits) {
+  pdl_wait();
+  pdl_launch_dependents();
   const int64_t b = blockIdx.z;
   const int t = threadIdx.x, cg = t & 7, rr = t >> 3;
   const int64_t col = static_cast<int64_t>(blockIdx.x) * 64 + 8 * cg;
-  uint32_t cmax[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  uint32_t cmax[4] = {0, 0, 0, 0};               // |bf16| bits of columns 2j, 2j+1
   uint4 raw[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
@@ -496,29 +549,31 @@ weight_qdq_kernel(const uint16_t* w, int64_t N, int64_t K, int64_t ldw,
     const int64_t n = static_cast<int64_t>(blockIdx.y) * 128 + rr + 32 * i;
     const bool live = n < N;
     const int64_t off = (b * N + n) * ldw + col;
-    float f[8];
-    unpack_bf16x8(raw[i], f);
-    float am = 0.0f;
+    const uint32_t wv[4] = {raw[i].x, raw[i].y, raw[i].z, raw[i].w};
+    uint64_t x2[4];
+    uint32_t mbits = 0;                          // max |bf16| bits, two lanes
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      am = fmaxf(am, fabsf(f[j]));
-      cmax[j] = max(cmax[j], __float_as_uint(fabsf(f[j])));
+    for (int j = 0; j < 4; ++j) {
+      x2[j] = bf16x2_to_f2(wv[j]);
+      const uint32_t a = wv[j] & 0x7FFF7FFFu;
+      mbits = __vmaxu2(mbits, a);
+      cmax[j] = __vmaxu2(cmax[j], a);            // columns 2j (low) and 2j+1 (high)
     }
+    float am = __uint_as_float(max(mbits & 0xFFFFu, mbits >> 16) << 16);
     am = fmaxf(am, __shfl_xor_sync(0xFFFFFFFFu, am, 1));
     const BlockQ bs = block_q(am, T);
-    const uint32_t q = encode8_q(f, bs);
+    uint64_t q2[4];
+    block_quotients(x2, bs, q2);
+    const uint32_t q = e2m1x8_f2(q2);
     const int64_t qrow = b * N + n;
     if (live) {
+      const uint64_t sbv2 = f2_pack(bs.sbv, bs.sbv), st2 = f2_pack(s_t, s_t);
       uint32_t o[4];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        float lo, hi;
-        e2m1x2_to_f32((q >> (8 * j)) & 0xFFu, lo, hi);
-        const float d0 = __fmul_rn(__fmul_rn(lo, bs.sbv), s_t);
-        const float d1 = __fmul_rn(__fmul_rn(hi, bs.sbv), s_t);
-        const uint32_t b0 = __bfloat16_as_ushort(__float2bfloat16_rn(d0));
-        const uint32_t b1 = __bfloat16_as_ushort(__float2bfloat16_rn(d1));
-        o[j] = b0 | (b1 << 16);
+        float d0, d1;
+        f2_unpack(f2_mul(f2_mul(e2m1x2_to_f2((q >> (8 * j)) & 0xFFu), sbv2), st2), d0, d1);
+        asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(o[j]) : "f"(d1), "f"(d0));   // d0 in the low half
       }
       *reinterpret_cast<uint4*>(w_out + off) = make_uint4(o[0], o[1], o[2], o[3]);
       if (codes) *reinterpret_cast<uint32_t*>(codes + qrow * (K / 2) + col / 2) = q;
@@ -531,7 +586,10 @@ weight_qdq_kernel(const uint16_t* w, int64_t N, int64_t K, int64_t ldw,
   if (colamax_bits == nullptr) return;
   __shared__ uint32_t cm[32][65];
 #pragma unroll
-  for (int j = 0; j < 8; ++j) cm[rr][8 * cg + j] = cmax[j];
+  for (int j = 0; j < 4; ++j) {                  // |bf16| bits -> fp32 bits
+    cm[rr][8 * cg + 2 * j] = (cmax[j] & 0xFFFFu) << 16;
+    cm[rr][8 * cg + 2 * j + 1] = cmax[j] & 0xFFFF0000u;
+  }
   __syncthreads();
   if (t < 64) {
     uint32_t m = 0;
@@ -575,12 +633,20 @@ cudaError_t launch_amax(const uint16_t* x, int64_t rows, int64_t K, int64_t ldx,
   const int64_t tiles = max_tiles(g, rows);
   if (tiles == 0) return cudaSuccess;
   dim3 grid(static_cast<unsigned>(K / kQCols), static_cast<unsigned>(tiles), static_cast<unsigned>(batch));
-  amax_kernel<<<grid, kQThreads, 0, s>>>(x, K, ldx, g, mat_stride, amax_bits);
+  {
+    const cudaError_t le = launch_k(amax_kernel, dim3(grid), dim3(kQThreads), 0, s, nullptr, 0,
+                                   x, K, ldx, g, mat_stride, amax_bits);
+    if (le != cudaSuccess) return le;
+  }
   return cudaGetLastError();
 }
 
 cudaError_t launch_group_tiles(const int64_t* off, int32_t E, int32_t* tile_start, cudaStream_t s) {
-  group_tiles_kernel<<<1, 32, 0, s>>>(off, E, tile_start);
+  {
+    const cudaError_t le = launch_k(group_tiles_kernel, dim3(1), dim3(32), 0, s, nullptr, 0,
+                                   off, E, tile_start);
+    if (le != cudaSuccess) return le;
+  }
   return cudaGetLastError();
 }
 
@@ -593,9 +659,12 @@ cudaError_t launch_quant_score(const uint16_t* x, int64_t rows, int64_t K, int64
   const int64_t tiles = max_tiles(g, rows);
   if (tiles == 0) return cudaSuccess;
   dim3 grid(static_cast<unsigned>(K / kQCols), static_cast<unsigned>(tiles));
-  quant_score_kernel<<<grid, kQThreads, 0, s>>>(x, K, ldx, g, amax, amax_parts, n_parts, codes_rows, codes,
-                                                scales, layout, tensor_scale, part_sum, part_max,
-                                                strip_count, score, colamax);
+  {
+    const cudaError_t le = launch_k(quant_score_kernel, dim3(grid), dim3(kQThreads), 0, s, nullptr, 0,
+                                   x, K, ldx, g, amax, amax_parts, n_parts, codes_rows, codes, scales,
+                                   layout, tensor_scale, part_sum, part_max, strip_count, score, colamax);
+    if (le != cudaSuccess) return le;
+  }
   return cudaGetLastError();
 }
 
@@ -609,7 +678,11 @@ cudaError_t launch_amax_partial(const uint16_t* x, int64_t rows, int64_t K, int6
                                 int64_t mat_stride, unsigned* parts, int n_parts, unsigned* zero_ptr,
                                 int n_zero, cudaStream_t s) {
   dim3 grid(static_cast<unsigned>(n_parts), static_cast<unsigned>(batch));
-  amax_partial_kernel<<<grid, kQThreads, 0, s>>>(x, rows, K, ldx, mat_stride, parts, zero_ptr, n_zero);
+  {
+    const cudaError_t le = launch_k(amax_partial_kernel, dim3(grid), dim3(kQThreads), 0, s, nullptr, 0,
+                                   x, rows, K, ldx, mat_stride, parts, zero_ptr, n_zero);
+    if (le != cudaSuccess) return le;
+  }
   return cudaGetLastError();
 }
 
@@ -617,8 +690,11 @@ cudaError_t launch_score_reduce(const double* part_sum, const float* part_max, i
                                 const RowGroups& g, int64_t tiles, double* score, float* colamax,
                                 float* tensor_scale_empty, cudaStream_t s) {
   dim3 grid(static_cast<unsigned>((K + 255) / 256), static_cast<unsigned>(g.E));
-  score_reduce_kernel<<<grid, 256, 0, s>>>(part_sum, part_max, K, g, tiles, score, colamax,
-                                           tensor_scale_empty);
+  {
+    const cudaError_t le = launch_k(score_reduce_kernel, dim3(grid), dim3(256), 0, s, nullptr, 0,
+                                   part_sum, part_max, K, g, tiles, score, colamax, tensor_scale_empty);
+    if (le != cudaSuccess) return le;
+  }
   return cudaGetLastError();
 }
 
@@ -637,15 +713,23 @@ cudaError_t launch_residual_gather(const uint16_t* x, int64_t rows, int64_t K, i
   if (width == 0 || prows == 0) return cudaSuccess;
   // rows of the scale buffer are padded to 128 for the tiled layout
   const int64_t grid_rows = r_layout == 1 ? (prows + kTileRows - 1) / kTileRows * kTileRows : prows;
-  gather_quant_kernel<true><<<gather_grid(grid_rows, width), kGThreads, 0, s>>>(
-      x, K, ldx, g, 0, qx_codes, qx_scales, qx_layout, qx_st, sel, n_sel, width, nullptr, 0,
-      const_cast<float*>(r_st), r_codes, r_scales, r_layout, prows, grid_rows);
+  {
+    const cudaError_t le = launch_k(gather_quant_kernel<true>, dim3(gather_grid(grid_rows, width)), dim3(kGThreads), 0, s, nullptr, 0,
+                                   x, K, ldx, g, 0, qx_codes, qx_scales, qx_layout, qx_st, sel, n_sel,
+                                   width, nullptr, 0, const_cast<float*>(r_st), r_codes, r_scales,
+                                   r_layout, prows, grid_rows);
+    if (le != cudaSuccess) return le;
+  }
   return cudaGetLastError();
 }
 
 cudaError_t launch_sel_tensor_scale(const float* colamax, int64_t K, const int32_t* sel,
                                     int64_t n_sel, int32_t E, float* s_t, cudaStream_t s) {
-  sel_tensor_scale_kernel<<<E, 512, 0, s>>>(colamax, K, sel, n_sel, s_t);
+  {
+    const cudaError_t le = launch_k(sel_tensor_scale_kernel, dim3(E), dim3(512), 0, s, nullptr, 0,
+                                   colamax, K, sel, n_sel, s_t);
+    if (le != cudaSuccess) return le;
+  }
   return cudaGetLastError();
 }
 
@@ -661,9 +745,12 @@ cudaError_t launch_weight_gather(const uint16_t* w, int64_t N, int64_t K, int64_
   }
   const int64_t rows = static_cast<int64_t>(E) * N;
   RowGroups none{};
-  gather_quant_kernel<false><<<gather_grid(rows, width), kGThreads, 0, s>>>(
-      w, K, ldw, none, N, nullptr, nullptr, 0, nullptr, sel, n_sel, width, colamax, fuse, s_t, codes,
-      scales, layout, rows, rows);
+  {
+    const cudaError_t le = launch_k(gather_quant_kernel<false>, dim3(gather_grid(rows, width)), dim3(kGThreads), 0, s, nullptr, 0,
+                                   w, K, ldw, none, N, nullptr, nullptr, 0, nullptr, sel, n_sel, width,
+                                   colamax, fuse, s_t, codes, scales, layout, rows, rows);
+    if (le != cudaSuccess) return le;
+  }
   return cudaGetLastError();
 }
 
@@ -673,8 +760,12 @@ cudaError_t launch_weight_qdq(const uint16_t* w, int64_t N, int64_t K, int64_t l
                               unsigned* colamax_bits, cudaStream_t s) {
   dim3 grid(static_cast<unsigned>(K / 64), static_cast<unsigned>((N + 127) / 128),
             static_cast<unsigned>(batch));
-  weight_qdq_kernel<<<grid, kQThreads, 0, s>>>(w, N, K, ldw, amax_parts, n_parts, w_out, codes, scales,
-                                               layout, tensor_scale, colamax_bits);
+  {
+    const cudaError_t le = launch_k(weight_qdq_kernel, dim3(grid), dim3(kQThreads), 0, s, nullptr, 0,
+                                   w, N, K, ldw, amax_parts, n_parts, w_out, codes, scales, layout,
+                                   tensor_scale, colamax_bits);
+    if (le != cudaSuccess) return le;
+  }
   return cudaGetLastError();
 }
 

@@ -35,7 +35,8 @@ def _check_select(b, x, k):
 
 
 @pytest.mark.parametrize("M,K,k", [(64, 512, 50.0), (300, 192, 25.0), (1, 64, 50.0), (130, 1024, 100.0),
-                                   (257, 2048, 0.0), (200, 11008 // 2, 50.0), (77, 448, 12.5)])
+                                   (257, 2048, 0.0), (200, 11008 // 2, 50.0), (77, 448, 12.5),
+                                   (40, 16384, 50.0), (9, 65536, 3.0)])
 def test_select_matches_oracle(M, K, k):
     b = need_gpu()
     _check_select(b, S.activations(M, K, seed=M), k)
