@@ -665,13 +665,18 @@ w4a4_rac_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid
         if (!ok) break;
         tc_fence_after();
 #pragma unroll 1
-        for (int c = 0; c < 8; ++c) {
-          float v[32];
+        for (int c = 0; c < 8; c += 2) {             // two loads in flight
+          float v[32], u[32];
           tmem_ld32(trow + ACC2_COL + 32 * c, v);
+          tmem_ld32(trow + ACC2_COL + 32 * (c + 1), u);
           tmem_ld_wait();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(v[i], ratio);
+          for (int i = 0; i < 32; ++i) {
+            v[i] = __fmul_rn(v[i], ratio);
+            u[i] = __fmul_rn(u[i], ratio);
+          }
           tmem_st32(trow + ACC2_COL + 32 * c, v);
+          tmem_st32(trow + ACC2_COL + 32 * (c + 1), u);
         }
         asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
         tc_fence_before();
@@ -684,36 +689,9 @@ w4a4_rac_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid
       if (!ok) break;
       tc_fence_after();
       const int64_t row0 = static_cast<int64_t>(mt) * 256 + rank * 128 + 32 * q;
-#pragma unroll 1
-      for (int h = 0; h < 2; ++h) {
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          float v[32];
-          tmem_ld32(trow + ACC2_COL + 128 * h + 32 * c, v);
-          tmem_ld_wait();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(fin, v[i]);
-          if (YBYTES == 4) {
-#pragma unroll
-            for (int i = 0; i < 32; i += 4)
-              *reinterpret_cast<float4*>(stg_row + (32 * c + i) * 4) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
-          } else {
-            uint32_t w[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i)
-              w[i] = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(v[2 * i]))) |
-                     (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(v[2 * i + 1]))) << 16);
-#pragma unroll
-            for (int i = 0; i < 16; i += 4)
-              *reinterpret_cast<uint4*>(stg_row + (32 * c + 2 * i) * 2) = make_uint4(w[i], w[i + 1], w[i + 2], w[i + 3]);
-          }
-        }
-        if (h == 1) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive_cluster(lead_tmem_empty);   // accumulator free
-        }
-        __syncwarp();
+      // rows of this warp (32 x 128 columns in the staging buffer) leave as
+      // coalesced row stores
+      auto store_rows = [&](int h) {
         const int64_t col = static_cast<int64_t>(nt) * 256 + 128 * h + 4 * lane;
         const bool col_ok = col + 4 <= p.N;
 #pragma unroll 4
@@ -726,7 +704,69 @@ w4a4_rac_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid
           else
             *reinterpret_cast<uint2*>(static_cast<uint16_t*>(p.y) + row * p.ldy + col) = *reinterpret_cast<const uint2*>(src);
         }
+      };
+      if constexpr (YBYTES == 2) {
+        // bf16: both halves leave TMEM first (the second one packed in
+        // registers), so the accumulator is released before any global store
+        // and the next tile's MMAs overlap the stores
+        uint32_t hold[64];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            float v[32];
+            tmem_ld32(trow + ACC2_COL + 128 * h + 32 * c, v);
+            tmem_ld_wait();
+            uint32_t w[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float lo = __fmul_rn(fin, v[2 * i]), hi = __fmul_rn(fin, v[2 * i + 1]);
+              asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(w[i]) : "f"(hi), "f"(lo));
+            }
+            if (h == 0) {
+#pragma unroll
+              for (int i = 0; i < 16; i += 4)
+                *reinterpret_cast<uint4*>(stg_row + (32 * c + 2 * i) * 2) = make_uint4(w[i], w[i + 1], w[i + 2], w[i + 3]);
+            } else {
+#pragma unroll
+              for (int i = 0; i < 16; ++i) hold[16 * c + i] = w[i];
+            }
+          }
+        }
+        tc_fence_before();
         __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(lead_tmem_empty);     // accumulator free
+        store_rows(0);
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < 64; i += 4)
+          *reinterpret_cast<uint4*>(stg_row + 4 * i) = make_uint4(hold[i], hold[i + 1], hold[i + 2], hold[i + 3]);
+        __syncwarp();
+        store_rows(1);
+        __syncwarp();
+      } else {
+#pragma unroll 1
+        for (int h = 0; h < 2; ++h) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            float v[32];
+            tmem_ld32(trow + ACC2_COL + 128 * h + 32 * c, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 32; i += 4)
+              *reinterpret_cast<float4*>(stg_row + (32 * c + i) * 4) =
+                  make_float4(__fmul_rn(fin, v[i]), __fmul_rn(fin, v[i + 1]), __fmul_rn(fin, v[i + 2]),
+                              __fmul_rn(fin, v[i + 3]));
+          }
+          if (h == 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(lead_tmem_empty);   // accumulator free
+          }
+          __syncwarp();
+          store_rows(h);
+          __syncwarp();
+        }
       }
       acc_phase ^= 1;
     }
