@@ -38,10 +38,14 @@ WORKLOADS = {
     # name: (M, K, N, k)
     "dense_rollout_projection": (4096, 2048, 2048, 50.0),
     "decode_step_up": (256, 4096, 11008, 50.0),
+    "decode_step_down": (256, 11008, 4096, 50.0),
     "single_linear": (64, 512, 512, 50.0),
     "large_prefill": (32768, 4096, 4096, 50.0),
 }
 DEFAULT_WORKLOAD = "dense_rollout_projection"
+# grouped MoE expert FFN (up 2048 -> 1024, down 1024 -> 2048 over 64 experts,
+# 8192 tokens routed top-8): its own step, see run_moe
+MOE_WORKLOAD = "moe_expert_ffn"
 FP4_OVER_BF16 = 4.0          # nominal dense FP4 / BF16 tensor ratio (9 / 2.25 PFLOP/s)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 ORACLE_SAMPLE_ROWS = 1024
@@ -54,7 +58,7 @@ def parse_args():
     p.add_argument("--steps", type=int, default=10)
     p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    p.add_argument("--workload", choices=sorted(WORKLOADS), default=DEFAULT_WORKLOAD)
+    p.add_argument("--workload", choices=sorted(WORKLOADS) + [MOE_WORKLOAD], default=DEFAULT_WORKLOAD)
     p.add_argument("--k", type=float, default=None, help="RAC k percent (default: workload's)")
     p.add_argument("--no-graph", action="store_true", help="issue calls directly, no CUDA graphs")
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -368,6 +372,179 @@ def run_ours(args, rank, world, local_rank):
     return line
 
 
+# ---------------------------------------------------------------- MoE expert FFN
+def moe_flops(offsets, K_up, N_up, K_dn, N_dn, k):
+    """Effective FLOPs of the up and down grouped RAC linears (every expert's
+    rows times N times K + n_sel)."""
+    from precision_rl_rollout_nvfp4_b200 import binding as B
+    T = int(offsets[-1])
+    return 2.0 * T * (N_up * (K_up + B.rac_nsel(k, K_up)) + N_dn * (K_dn + B.rac_nsel(k, K_dn)))
+
+
+def run_moe(args, rank, world, local_rank):
+    """Grouped MoE expert FFN: one step = the up (K 2048 -> N 1024) and the
+    down (K 1024 -> N 2048) grouped W4A4 + RAC linears over 64 experts, rows
+    expert-contiguous (8192 tokens routed top-8 with Zipf(1.1) loads).  Each
+    call runs, per expert, the quantizer, the channel selection, the W_sel
+    quantization and the grouped tensor-core GEMM.  Expert weights are
+    prepared once (weight_qdq over all experts, timed separately).  The
+    step's inputs (402 MB) exceed L2, so no flush is needed between steps."""
+    import torch
+    import torch.distributed as dist
+
+    from precision_rl_rollout_nvfp4_b200 import binding as B
+    from precision_rl_rollout_nvfp4_b200 import synthetic as S
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    cfg = S.MOE
+    k = args.k if args.k is not None else cfg["k"]
+    inp = S.moe_inputs(cfg["T"], cfg["hidden"], cfg["inter"], cfg["E"], cfg["topk"], seed=replica_seed(rank))
+    xu_host = inp["x_perm"].contiguous().pin_memory()
+    xd_host = inp["x_down"].contiguous().pin_memory()
+    xu, xd = xu_host.to(dev), xd_host.to(dev)
+    wu, wd = inp["w_up"].to(dev), inp["w_down"].to(dev)
+    off = torch.from_numpy(inp["offsets"]).to(dev)
+    E, N_up, K_up = wu.shape
+    _, N_dn, K_dn = wd.shape
+    T = xu.shape[0]
+    stream = torch.cuda.current_stream()
+
+    def ev():
+        e = torch.cuda.Event(enable_timing=True)
+        e.record(stream)
+        return e
+
+    # weight preparation (per weight sync): Q(W) and colamax of every expert
+    wu_out, wd_out = torch.empty_like(wu), torch.empty_like(wd)
+    prep = {}
+    for _ in range(3):              # the last pass reuses cached buffers
+        torch.cuda.synchronize()
+        a = ev()
+        _, qu, cu = B.weight_qdq(wu, out=wu_out)
+        b = ev()
+        _, qd, cd = B.weight_qdq(wd, out=wd_out)
+        c = ev()
+        torch.cuda.synchronize()
+        prep = {"weight_qdq_up": a.elapsed_time(b) * 1e3, "weight_qdq_down": b.elapsed_time(c) * 1e3}
+    yu = torch.empty(T, N_up, dtype=torch.bfloat16, device=dev)
+    yd = torch.empty(T, N_dn, dtype=torch.bfloat16, device=dev)
+
+    def up(kk=k):
+        B.moe_rac(xu, off, wu, qu, cu, kk, out_dtype=torch.bfloat16, masks=False, out=yu)
+
+    def down(kk=k):
+        B.moe_rac(xd, off, wd, qd, cd, kk, out_dtype=torch.bfloat16, masks=False, out=yd)
+
+    def step():
+        up()
+        down()
+
+    def plain():
+        up(0.0)
+        down(0.0)
+
+    for _ in range(max(args.warmup, 1)):
+        step()
+        plain()
+    torch.cuda.synchronize()
+    if B.stream_status() != 0:
+        raise RuntimeError("device error word set during warm-up")
+    graphs = {}
+    use_graph = not args.no_graph
+    if use_graph:
+        for name, fn in [("step", step), ("plain", plain), ("up", up), ("down", down)]:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                fn()
+            graphs[name] = g
+        torch.cuda.synchronize()
+    fns = {"step": step, "plain": plain, "up": up, "down": down}
+
+    def launch(name):
+        if use_graph:
+            graphs[name].replay()
+        else:
+            fns[name]()
+
+    for _ in range(args.warmup):
+        launch("step")
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clocks:
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        evs = []
+        for _ in range(args.steps):
+            a = ev()
+            launch("step")
+            evs.append((a, ev()))
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+    total_ms = sum(a.elapsed_time(b) for a, b in evs)
+    clock = clocks.summary()
+    per = {n: [] for n in ("up", "down", "plain")}
+    for _ in range(args.steps):
+        for n in per:
+            a = ev()
+            launch(n)
+            b = ev()
+            torch.cuda.synchronize()
+            per[n].append(a.elapsed_time(b))
+    # end to end: both inputs from pinned host memory, the step's output back
+    yd_host = torch.empty(T, N_dn, dtype=torch.bfloat16).pin_memory()
+    e2e = []
+    for i in range(args.warmup + args.steps):
+        a = ev()
+        xu.copy_(xu_host, non_blocking=True)
+        xd.copy_(xd_host, non_blocking=True)
+        step()
+        yd_host.copy_(yd, non_blocking=True)
+        b = ev()
+        torch.cuda.synchronize()
+        if i >= args.warmup:
+            e2e.append(a.elapsed_time(b))
+    if B.stream_status() != 0:
+        raise RuntimeError("device error word set during timing")
+    total_ms, e2e_total = max_over_ranks([total_ms, sum(e2e)], world, dev)
+
+    flops = moe_flops(inp["offsets"], K_up, N_up, K_dn, N_dn, k)
+    value = flops * world * args.steps / (total_ms * 1e-3) / 1e12
+    med = {n: statistics.median(v) for n, v in per.items()}
+    peaks, peak_kind = load_peaks()
+    fp4_peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]) * FP4_OVER_BF16
+    fl_up = 2.0 * T * N_up * (K_up + B.rac_nsel(k, K_up))
+    up_tf = fl_up / (med["up"] * 1e-3) / 1e12
+    step_ms = total_ms / args.steps
+    loads = [int(inp["offsets"][i + 1] - inp["offsets"][i]) for i in range(E)]
+    return {
+        "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s (effective 2MN(K+n_sel) per step)",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_ms, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4 (e2m1/ue4m3) x fp32 acc",
+        "data": "synthetic (seeded routing and activations; see DESIGN.md)",
+        "config": {"workload": MOE_WORKLOAD, "tokens": cfg["T"], "topk": cfg["topk"], "routed_rows": T, "experts": E,
+                   "up": [K_up, N_up], "down": [K_dn, N_dn], "k_percent": k, "expert_rows_max": max(loads),
+                   "expert_rows_min": min(loads), "y_dtype": "bf16", "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2 (402 MB per step)", "cuda_graph": use_graph},
+        "per_call_us": {"up": round(1e3 * med["up"], 2), "down": round(1e3 * med["down"], 2),
+                        **{n: round(v, 2) for n, v in prep.items()}},
+        "plain_w4a4_step_us": round(1e3 * med["plain"], 2),
+        "rac_overhead_pct": round(100 * (step_ms - med["plain"]) / med["plain"], 1),
+        "roofline": {"kernel": "moe_grouped_w4a4_rac_gemm (up call: quantizer, selection and GEMM)",
+                     "bound": "tensor", "achieved": round(up_tf, 1), "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
+                     "frac": round(up_tf / fp4_peak, 4), "traffic": None,
+                     "peak_source": f"{peak_kind}: bf16 sustained x {FP4_OVER_BF16:g} (FP4/BF16 nominal)"},
+        "e2e": {"value": round(flops * world * args.steps / (e2e_total * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+                "h2d_bytes_per_step": int(2 * (xu.numel() + xd.numel())), "d2h_bytes_per_step": int(2 * yd.numel()),
+                "ms_per_step": round(e2e_total / args.steps, 4)},
+        # per grouped call: group tiles, amax, quantize, score reduce, top-k,
+        # residual gather, W_sel scale, W_sel gather, GEMM (one memset too)
+        "gpu_launches": (9 if B.rac_nsel(k, K_up) else 6) * 2 * args.steps,
+        "clocks": clock,
+    }
+
+
 # ---------------------------------------------------------------- oracle (CPU)
 def oracle_step_time(M, K, N, k, rows, seed=0):
     import numpy as np
@@ -391,7 +568,42 @@ def blas_threads():
         return os.cpu_count() or 1
 
 
+_MOE_SAMPLE = {}
+
+
+def oracle_moe_time(k, n_experts=8, seed=0):
+    """Oracle up projection of the last n_experts experts (the smallest row
+    groups) of the MoE workload: every step of the grouped RAC linear on those
+    groups.  Returns (seconds, effective FLOPs, description)."""
+    import oracle
+    from precision_rl_rollout_nvfp4_b200 import synthetic as S
+    cfg = S.MOE
+    E = cfg["E"]
+    e0 = E - n_experts
+    if (n_experts, seed) not in _MOE_SAMPLE:
+        inp = S.moe_inputs(cfg["T"], cfg["hidden"], cfg["inter"], cfg["E"], cfg["topk"], seed=seed)
+        off = inp["offsets"]
+        r0, r1 = int(off[e0]), int(off[E])
+        _MOE_SAMPLE[(n_experts, seed)] = (S.bf16_bits(inp["x_perm"][r0:r1]), S.bf16_bits(inp["w_up"][e0:E]),
+                                          off[e0:] - r0, r0, r1)
+    x, w, sub_off, r0, r1 = _MOE_SAMPLE[(n_experts, seed)]
+    t0 = time.perf_counter()
+    oracle.moe_rac(x, sub_off, w, k)
+    dt = time.perf_counter() - t0
+    K, N = cfg["hidden"], cfg["inter"]
+    n_sel = oracle.n_selected(k, K)
+    return dt, 2.0 * (r1 - r0) * N * (K + n_sel), f"up projection of experts {e0}..{E - 1} ({r1 - r0} rows)"
+
+
 def cpu_baseline(args, budget_s=12.0):
+    if args.workload == MOE_WORKLOAD:
+        k = args.k if args.k is not None else 50.0
+        t, flops, n, desc = 0.0, 0.0, 0, ""
+        while (t < budget_s and n < 4) or n == 0:
+            dt, f, desc = oracle_moe_time(k)
+            t, flops, n = t + dt, flops + f, n + 1
+        return {"value": round(flops / t / 1e12, 6), "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+                "sample": f"{n} oracle run(s) of the grouped RAC linear: {desc} (numpy; fp64 product via BLAS)"}
     M, K, N, k = WORKLOADS[args.workload]
     k = args.k if args.k is not None else k
     rows = min(M, ORACLE_SAMPLE_ROWS)
@@ -409,6 +621,23 @@ def cpu_baseline(args, budget_s=12.0):
 
 
 def run_reference(args):
+    if args.workload == MOE_WORKLOAD:
+        k = args.k if args.k is not None else 50.0
+        for _ in range(args.warmup):
+            oracle_moe_time(k)
+        t, flops, desc = 0.0, 0.0, ""
+        for _ in range(args.steps):
+            dt, f, desc = oracle_moe_time(k)
+            t, flops = t + dt, flops + f
+        value = flops / t / 1e12
+        return {"impl": "reference", "metric": METRIC, "value": round(value, 6),
+                "unit": "TFLOP/s (effective 2MN(K+n_sel) per step)", "n_gpus": 1, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": round(1e3 * t / args.steps, 3), "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f32 quantizer steps, f64 product",
+                "data": "synthetic", "config": {"workload": MOE_WORKLOAD, "k_percent": k},
+                "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+                                 "sample": f"{desc} per step (numpy oracle; fp64 product via BLAS)"},
+                "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     M, K, N, k = WORKLOADS[args.workload]
     k = args.k if args.k is not None else k
     rows = min(M, ORACLE_SAMPLE_ROWS)
@@ -448,7 +677,7 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=torch.device("cuda", local_rank))
     try:
-        line = run_ours(args, rank, world, local_rank)
+        line = (run_moe if args.workload == MOE_WORKLOAD else run_ours)(args, rank, world, local_rank)
         if rank == 0:
             if not args.no_cpu_baseline:
                 line["cpu_baseline"] = cpu_baseline(args)

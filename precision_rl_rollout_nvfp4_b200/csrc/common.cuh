@@ -7,6 +7,7 @@
 // is built without fast-math and without flush-to-zero.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -338,6 +339,16 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsign
   }
   if (err) atomicOr(err, kErrTimeout);
   return false;
+}
+
+// 2-D tensor load (TMA) of one box into this CTA's shared memory; its bytes
+// complete on the mbarrier at shared address `bar`.  The innermost
+// coordinate times the element size must be a multiple of 16 bytes.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* tm, int x, int y,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+      :: "r"(dst), "l"(reinterpret_cast<uint64_t>(tm)), "r"(x), "r"(y), "r"(bar) : "memory");
 }
 
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {

@@ -2,6 +2,8 @@
 // library: the C ABI in api.cu validates arguments and calls these.
 #pragma once
 
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 #include <stdlib.h>
@@ -11,6 +13,11 @@
 #include "common.cuh"
 
 namespace nvfp4 {
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (null if
+// the driver does not provide it) and the current device's SM count.
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn();
+int sm_count();
 
 // Programmatic dependent launch is on unless NVFP4_NO_PDL=1.
 inline bool pdl_enabled() {
@@ -81,7 +88,7 @@ cudaError_t launch_quant_score(const uint16_t* x, int64_t rows, int64_t K, int64
                                int n_parts, int64_t codes_rows,
                                uint8_t* codes, uint8_t* scales, int layout, float* tensor_scale,
                                double* part_sum, float* part_max, unsigned* strip_count,
-                               double* score, float* colamax, cudaStream_t s);
+                               double* score, float* colamax, unsigned* err, cudaStream_t s);
 
 // score[e, j] = sum over the group's tiles of part_sum in tile order;
 // colamax[e, j] = max of part_max.  For empty groups (MoE) also writes

@@ -250,12 +250,14 @@ quant_score_kernel(const uint16_t* __restrict__ x, int64_t K, int64_t ldx, RowGr
   if (strip_count == nullptr) return;
   // The last CTA of this group's column strip sums the group's partials in
   // tile order (so the result does not depend on which CTA finishes last).
-  __threadfence();
+  // The barrier orders the 64 writers' partials before thread 0's fence, so
+  // the fence publishes them all (cumulativity) before the counter moves.
   __syncthreads();
   const int64_t t0 = g.off == nullptr ? 0 : g.tile_start[ti.e];
   const int64_t t1 = g.off == nullptr ? (g.M + kTileRows - 1) / kTileRows : g.tile_start[ti.e + 1];
   unsigned* counter = strip_count + static_cast<int64_t>(ti.e) * gridDim.x + blockIdx.x;
   if (t == 0) {
+    __threadfence();
     const unsigned prev = atomicAdd(counter, 1u);
     s_last = prev == static_cast<unsigned>(t1 - t0 - 1);
   }
@@ -655,7 +657,8 @@ cudaError_t launch_quant_score(const uint16_t* x, int64_t rows, int64_t K, int64
                                int n_parts, int64_t codes_rows,
                                uint8_t* codes, uint8_t* scales, int layout, float* tensor_scale,
                                double* part_sum, float* part_max, unsigned* strip_count,
-                               double* score, float* colamax, cudaStream_t s) {
+                               double* score, float* colamax, unsigned* err, cudaStream_t s) {
+  (void)err;                                       // no waits in this kernel
   const int64_t tiles = max_tiles(g, rows);
   if (tiles == 0) return cudaSuccess;
   dim3 grid(static_cast<unsigned>(K / kQCols), static_cast<unsigned>(tiles));
@@ -666,6 +669,25 @@ cudaError_t launch_quant_score(const uint16_t* x, int64_t rows, int64_t K, int64
     if (le != cudaSuccess) return le;
   }
   return cudaGetLastError();
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (fn == nullptr) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+int sm_count() {
+  int dev = 0, n = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
 }
 
 int amax_parts_count(int64_t rows, int64_t K) {
