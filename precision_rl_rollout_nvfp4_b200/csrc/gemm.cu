@@ -399,7 +399,13 @@ struct Cfg2 {
   static constexpr uint32_t TX = 2 * STAGE;            // bytes landing per stage (both CTAs)
 };
 
-constexpr uint32_t ACC2_COL = 0, SFA2_COL = 256, SFB2_COL = 272;
+// Warps of the pair kernel: 0 TMA producer, 1 MMA issuer, 2..5 epilogue,
+// 6 scale-factor copier (leader CTA).
+constexpr int THREADS2 = 224;
+// TMEM columns: the 256-column accumulator, then per pipeline stage 48
+// columns of block scales (16 for A, 32 for B), so the copies for later
+// stages run while the MMAs of earlier ones read theirs.
+constexpr uint32_t ACC2_COL = 0, SF2_COL = 256, SF2_STAGE_COLS = 48;
 // kind::mxf4nvf4, M = 256 (pair), N = 256, both K-major, ue4m3 scales.
 constexpr uint32_t IDESC2 = (1u << 7) | (1u << 10) | (uint32_t(256 >> 3) << 17) | (uint32_t(256 >> 4) << 24);
 
@@ -477,7 +483,7 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
 }
 
 template <int YBYTES>
-__global__ void __launch_bounds__(THREADS, 1)
+__global__ void __launch_bounds__(THREADS2, 1)
 w4a4_rac_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
                           const __grid_constant__ CUtensorMap tmSA0, const __grid_constant__ CUtensorMap tmSB0,
                           const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
@@ -491,23 +497,30 @@ w4a4_rac_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid
   uint8_t* sOut = smem + STAGES * C::STAGE;
   uint64_t* full = reinterpret_cast<uint64_t*>(sOut + C::STG_BYTES);
   uint64_t* empty = full + STAGES;
-  uint64_t* tmem_full = empty + STAGES;
+  uint64_t* sf_ready = empty + STAGES;   // the stage's scales are in TMEM
+  uint64_t* tmem_full = sf_ready + STAGES;
   uint64_t* tmem_empty = tmem_full + 1;
   uint64_t* res_full = tmem_empty + 1;
   uint64_t* res_done = res_full + 1;
   uint64_t* drain = res_done + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* drain_cp = drain + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_cp + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_rank();
   const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+      mbar_init(&sf_ready[s], 1);
+    }
     mbar_init(tmem_full, 1);
     mbar_init(tmem_empty, 8);          // one arrival per epilogue warp of both CTAs
     mbar_init(res_full, 1);
     mbar_init(res_done, 8);
     mbar_init(drain, 1);
+    mbar_init(drain_cp, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   cluster_sync_all();                  // barriers of both CTAs initialised
@@ -579,22 +592,19 @@ w4a4_rac_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid
         tc_fence_after();
         for (int seg = has_res ? 0 : 1; seg < 2 && ok; ++seg) {
           for (int kt = 0; kt < p.kt[seg]; ++kt) {
-            if (!mbar_wait(&full[stage], phase, p.err)) { ok = false; break; }
+            if (!mbar_wait(&full[stage], phase, p.err) || !mbar_wait(&sf_ready[stage], phase, p.err)) {
+              ok = false;
+              break;
+            }
             tc_fence_after();
             const uint32_t st = smem_u32(sStage + stage * C::STAGE);
             const uint32_t a0 = st, b0 = st + C::A_ST;
-            const uint32_t fa = st + C::A_ST + C::B_ST, fb = fa + C::SFA_ST;
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              utccp_sf_pair(tmem + SFA2_COL + 4 * j, desc_sf(fa + j * SF_ATOM));
-              utccp_sf_pair(tmem + SFB2_COL + 8 * j, desc_sf(fb + j * SF_ATOM));
-              utccp_sf_pair(tmem + SFB2_COL + 8 * j + 4, desc_sf(fb + 4 * SF_ATOM + j * SF_ATOM));
-            }
+            const uint32_t sfa = tmem + SF2_COL + SF2_STAGE_COLS * stage, sfb = sfa + 16;
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
               const uint32_t accum = (seg == 1 && has_res) ? 1u : ((kt > 0 || j > 0) ? 1u : 0u);
               mma_fp4_pair(tmem + ACC2_COL, desc_sw128(a0 + 32 * j), desc_sw128(b0 + 32 * j),
-                           tmem + SFA2_COL + 4 * j, tmem + SFB2_COL + 8 * j, accum);
+                           sfa + 4 * j, sfb + 8 * j, accum);
             }
             umma_commit_pair(&empty[stage]);
             if (++stage == STAGES) { stage = 0; phase ^= 1; }
@@ -614,6 +624,37 @@ w4a4_rac_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid
       asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];"
                    :: "r"(smem_u32(drain)) : "memory");
       mbar_wait(drain, 0, p.err);
+    }
+  } else if (warp == 6) {
+    if (lane == 0 && rank == 0) {
+      // ------------------------------ scale-factor copier (leader CTA only)
+      // smem -> TMEM copies of both CTAs' block scales for each stage; their
+      // completion arrives on sf_ready[stage], which the MMA issuer waits for
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int tile = pair; tile < total && ok; tile += npairs) {
+        for (int seg = has_res ? 0 : 1; seg < 2 && ok; ++seg) {
+          for (int kt = 0; kt < p.kt[seg]; ++kt) {
+            if (!mbar_wait(&full[stage], phase, p.err)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t fa = smem_u32(sStage + stage * C::STAGE) + C::A_ST + C::B_ST, fb = fa + C::SFA_ST;
+            const uint32_t sfa = tmem + SF2_COL + SF2_STAGE_COLS * stage, sfb = sfa + 16;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              utccp_sf_pair(sfa + 4 * j, desc_sf(fa + j * SF_ATOM));
+              utccp_sf_pair(sfb + 8 * j, desc_sf(fb + j * SF_ATOM));
+              utccp_sf_pair(sfb + 8 * j + 4, desc_sf(fb + 4 * SF_ATOM + j * SF_ATOM));
+            }
+            asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                         :: "r"(smem_u32(&sf_ready[stage])) : "memory");
+            if (++stage == STAGES) { stage = 0; phase ^= 1; }
+          }
+        }
+      }
+      asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                   :: "r"(smem_u32(drain_cp)) : "memory");
+      mbar_wait(drain_cp, 0, p.err);
     }
   } else {
     // ------------------------------ epilogue (warps 2..5 of both CTAs)
@@ -810,7 +851,7 @@ cudaError_t launch_pair(const GemmArgs& a, cudaStream_t s) {
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
-  return launch_k(w4a4_rac_gemm_pair_kernel<YBYTES>, dim3(static_cast<unsigned>(2 * pairs)), dim3(THREADS),
+  return launch_k(w4a4_rac_gemm_pair_kernel<YBYTES>, dim3(static_cast<unsigned>(2 * pairs)), dim3(THREADS2),
                   C::SMEM_BYTES, s, attr, 1, maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], maps[6],
                   maps[7], p);
 }
