@@ -15,8 +15,11 @@
 //               (A and B tiles, 128 B rows, 128 B swizzle) and two bulk
 //               copies of the matching 128 x 16 scale atoms into a 4/5-stage
 //               shared-memory ring guarded by full / empty mbarriers.
-//   warp 1      MMA issuer: copies each stage's scales into TMEM
-//               (tcgen05.cp 32x128b.warpx4), then issues four
+//   warp 6      scale copier: copies each stage's scales into that stage's
+//               own TMEM columns (tcgen05.cp 32x128b.warpx4) and commits
+//               them to a per-stage barrier.  The copies are issued by their
+//               own thread: from the MMA thread they throttled its issue.
+//   warp 1      MMA issuer: waits for the stage's data and scales, issues four
 //               tcgen05.mma kind::mxf4nvf4 (128 x 128 x 64, ue4m3 scales per
 //               16 elements) into accumulator 0 for the plain K segment and
 //               accumulator 1 for the residual segment; tcgen05.commit frees
@@ -31,7 +34,8 @@
 // For dense activations with at least 512 rows a second kernel runs the same
 // product on CTA pairs (tcgen05 cta_group::2): a pair computes a 256 x 256
 // tile, each CTA loading its own 128 rows of A and of B, so a pair fetches
-// half the operand bytes per FLOP of two 128 x 128 tiles.  Its TMEM holds one
+// half the operand bytes per FLOP of two 128 x 128 tiles; the leader's copier
+// warp copies both CTAs' scales (12 copies per K step).  Its TMEM holds one
 // 256-column accumulator; the residual segment is computed first and scaled
 // in place by s_R s_Ws / (s_X s_W) (tcgen05.ld, multiply, tcgen05.st), then
 // the plain segment accumulates on top and Y = s_X s_W acc.
@@ -50,7 +54,6 @@ constexpr int A_STAGE = BM * BK_BYTES;           // 16 KB
 constexpr int B_STAGE = BN * BK_BYTES;           // 16 KB
 constexpr int SF_ATOM = 512;                     // 128 rows x 4 scales
 constexpr int SF_STAGE = 4 * SF_ATOM;            // 4 MMA K blocks per step
-constexpr int THREADS = 192;
 
 // Per output type: pipeline depth and the epilogue staging tile (128 rows,
 // row stride padded by 16 bytes so 16-byte shared stores of 8 consecutive
@@ -64,7 +67,11 @@ struct Cfg {
 };
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC0_COL = 0, ACC1_COL = 128;   // two 128-column fp32 accumulators
-constexpr uint32_t SFA_COL = 256, SFB_COL = 272;
+// block scales: per pipeline stage 32 columns (16 for A, 16 for B)
+constexpr uint32_t SF1_COL = 256, SF1_STAGE_COLS = 32;
+// warps of the single-CTA kernel: 0 TMA producer, 1 MMA issuer, 2..5
+// epilogue, 6 scale-factor copier
+constexpr int THREADS1 = 224;
 
 // kind::mxf4nvf4 instruction descriptor: E2M1 x E2M1, ue4m3 scales, both
 // K-major, N = 128, M = 128.
@@ -153,7 +160,7 @@ __device__ __forceinline__ void tmem_ld_wait() {
 
 // ---- the kernel -----------------------------------------------------------
 template <int YBYTES>
-__global__ void __launch_bounds__(THREADS, 1)
+__global__ void __launch_bounds__(THREADS1, 1)
 w4a4_rac_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
                      const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
                      const KParams p) {
@@ -169,17 +176,24 @@ w4a4_rac_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_cons
   uint8_t* sOut = sSFB + STAGES * SF_STAGE;                     // epilogue staging
   uint64_t* full = reinterpret_cast<uint64_t*>(sOut + Cfg<YBYTES>::STG_BYTES);
   uint64_t* empty = full + STAGES;
-  uint64_t* tmem_full = empty + STAGES;
+  uint64_t* sf_ready = empty + STAGES;       // the stage's scales are in TMEM
+  uint64_t* tmem_full = sf_ready + STAGES;
   uint64_t* tmem_empty = tmem_full + 1;
   uint64_t* drain = tmem_empty + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* drain_cp = drain + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_cp + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+      mbar_init(&sf_ready[s], 1);
+    }
     mbar_init(tmem_full, 1);
     mbar_init(tmem_empty, 128);
     mbar_init(drain, 1);
+    mbar_init(drain_cp, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
@@ -248,18 +262,17 @@ w4a4_rac_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_cons
         for (int seg = 0; seg < nseg && ok; ++seg) {
           const uint32_t d = tmem + (seg ? ACC1_COL : ACC0_COL);
           for (int kt = 0; kt < p.kt[seg]; ++kt) {
-            if (!mbar_wait(&full[stage], phase, p.err)) { ok = false; break; }
+            if (!mbar_wait(&full[stage], phase, p.err) || !mbar_wait(&sf_ready[stage], phase, p.err)) {
+              ok = false;
+              break;
+            }
             tc_fence_after();
             const int nkb = kt == p.kt[seg] - 1 ? p.kb_last[seg] : 4;
             const uint32_t a0 = smem_u32(sA + stage * A_STAGE), b0 = smem_u32(sB + stage * B_STAGE);
-            const uint32_t fa = smem_u32(sSFA + stage * SF_STAGE), fb = smem_u32(sSFB + stage * SF_STAGE);
-            for (int j = 0; j < nkb; ++j) {
-              utccp_sf(tmem + SFA_COL + 4 * j, desc_sf(fa + j * SF_ATOM));
-              utccp_sf(tmem + SFB_COL + 4 * j, desc_sf(fb + j * SF_ATOM));
-            }
+            const uint32_t sfa = tmem + SF1_COL + SF1_STAGE_COLS * stage, sfb = sfa + 16;
             for (int j = 0; j < nkb; ++j)
-              mma_fp4(d, desc_sw128(a0 + 32 * j), desc_sw128(b0 + 32 * j), tmem + SFA_COL + 4 * j,
-                      tmem + SFB_COL + 4 * j, (kt > 0 || j > 0) ? 1u : 0u);
+              mma_fp4(d, desc_sw128(a0 + 32 * j), desc_sw128(b0 + 32 * j), sfa + 4 * j, sfb + 4 * j,
+                      (kt > 0 || j > 0) ? 1u : 0u);
             umma_commit(&empty[stage]);
             if (++stage == STAGES) { stage = 0; phase ^= 1; }
           }
@@ -269,6 +282,34 @@ w4a4_rac_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_cons
       }
       umma_commit(drain);                 // all issued tensor-core work done
       mbar_wait(drain, 0, p.err);
+    }
+  } else if (warp == 6) {
+    if (lane == 0) {
+      // ------------------------------ scale-factor copier: smem -> TMEM
+      // copies of the stage's block scales; completion arrives on
+      // sf_ready[stage], which the MMA issuer waits for
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int64_t tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        for (int seg = 0; seg < nseg && ok; ++seg) {
+          for (int kt = 0; kt < p.kt[seg]; ++kt) {
+            if (!mbar_wait(&full[stage], phase, p.err)) { ok = false; break; }
+            tc_fence_after();
+            const int nkb = kt == p.kt[seg] - 1 ? p.kb_last[seg] : 4;
+            const uint32_t fa = smem_u32(sSFA + stage * SF_STAGE), fb = smem_u32(sSFB + stage * SF_STAGE);
+            const uint32_t sfa = tmem + SF1_COL + SF1_STAGE_COLS * stage, sfb = sfa + 16;
+            for (int j = 0; j < nkb; ++j) {
+              utccp_sf(sfa + 4 * j, desc_sf(fa + j * SF_ATOM));
+              utccp_sf(sfb + 4 * j, desc_sf(fb + j * SF_ATOM));
+            }
+            umma_commit(&sf_ready[stage]);
+            if (++stage == STAGES) { stage = 0; phase ^= 1; }
+          }
+        }
+      }
+      umma_commit(drain_cp);
+      mbar_wait(drain_cp, 0, p.err);
     }
   } else {
     // ------------------------------ epilogue (warps 2..5)
@@ -898,13 +939,13 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s) {
   const int grid = static_cast<int>(tiles_bound < sm_count() ? tiles_bound : sm_count());
   if (a.y_dtype == 0)
     {
-      const cudaError_t le = launch_k(w4a4_rac_gemm_kernel<4>, dim3(grid), dim3(THREADS), Cfg<4>::SMEM_BYTES, s, nullptr, 0,
+      const cudaError_t le = launch_k(w4a4_rac_gemm_kernel<4>, dim3(grid), dim3(THREADS1), Cfg<4>::SMEM_BYTES, s, nullptr, 0,
                                      maps[0], maps[1], maps[2], maps[3], p);
       if (le != cudaSuccess) return le;
     }
   else
     {
-      const cudaError_t le = launch_k(w4a4_rac_gemm_kernel<2>, dim3(grid), dim3(THREADS), Cfg<2>::SMEM_BYTES, s, nullptr, 0,
+      const cudaError_t le = launch_k(w4a4_rac_gemm_kernel<2>, dim3(grid), dim3(THREADS1), Cfg<2>::SMEM_BYTES, s, nullptr, 0,
                                      maps[0], maps[1], maps[2], maps[3], p);
       if (le != cudaSuccess) return le;
     }
