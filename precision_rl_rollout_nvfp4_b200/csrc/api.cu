@@ -124,7 +124,7 @@ MoeWs carve_moe(Carver& c, int64_t T, int64_t N, int64_t K, int32_t E, int64_t n
   MoeWs w{};
   const int64_t tiles = ceil_div(T, kTileRows) + E;
   const int64_t prows = tiles * kTileRows;
-  w.tile_start = c.take<int32_t>(E + 1);
+  w.tile_start = c.take<int32_t>(2 * (E + 1));     // 128-row then 256-row tile prefixes
   w.amax = c.take<unsigned>(E);
   w.qx_codes = c.take<uint8_t>(prows * K / 2);
   w.qx_scales = c.take<uint8_t>(scale_bytes(prows, K, 1));
@@ -404,6 +404,7 @@ nvfp4_status moe_grouped_w4a4_rac_gemm(const uint16_t* x_perm, int64_t T, int64_
   a.M = T;
   a.N = N;
   a.m_tiles = tiles;
+  a.pair_start = m.tile_start + E + 1;
   a.y = y_perm;
   a.y_dtype = y_dtype;
   a.ldy = N;

@@ -452,14 +452,53 @@ constexpr uint32_t IDESC2 = (1u << 7) | (1u << 10) | (uint32_t(256 >> 3) << 17) 
 
 struct KParams2 {
   int64_t M, N;
-  int m_tiles, n_tiles;        // 256-row / 256-column tiles
+  int m_tiles, n_tiles;        // 256-row (dense) / 256-column tiles
   int kt[2];                   // K steps of the residual (0) and plain (1) segments
-  const float* sta[2];
+  const float* sta[2];         // tensor scales, one per group
   const float* stb[2];
+  RowGroups g;                 // row groups of A and Y (g.off null: dense)
+  const int32_t* pair_start;   // groups: prefix of each group's 256-row tiles
   void* y;
   int64_t ldy;
   unsigned* err;
 };
+
+// Rows of a 256-row pair tile.  Dense: tile mt covers rows 256 mt .. +255.
+// Groups: pair tile pt belongs to the group e with pair_start[e] <= pt <
+// pair_start[e + 1]; its two 128-row halves are the group's 128-row tiles
+// 2 lp and 2 lp + 1 (lp = pt - pair_start[e]) on the padded rows; a half past
+// the group's last tile computes rows that are never stored.
+struct PairRows {
+  int e;
+  int64_t a_tile;              // this CTA's 128-row tile (padded rows / 128)
+  int64_t local0;              // first row of this CTA's half within the group
+  int64_t out0;                // output row of local row 0 of the group
+  int64_t m;                   // rows of the group
+};
+
+__device__ __forceinline__ PairRows pair_rows(const KParams2& p, int64_t pt, uint32_t rank) {
+  PairRows r;
+  if (p.g.off == nullptr) {
+    r.e = 0;
+    r.a_tile = 2 * pt + rank;
+    r.local0 = r.a_tile * 128;
+    r.out0 = 0;
+    r.m = p.M;
+    return r;
+  }
+  int lo = 0, hi = p.g.E - 1;                      // last e with pair_start[e] <= pt
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (p.pair_start[mid] <= pt) lo = mid; else hi = mid - 1;
+  }
+  const int64_t local_tile = 2 * (pt - p.pair_start[lo]) + rank;
+  r.e = lo;
+  r.a_tile = p.g.tile_start[lo] + local_tile;
+  r.local0 = local_tile * 128;
+  r.out0 = p.g.off[lo];
+  r.m = p.g.off[lo + 1] - p.g.off[lo];
+  return r;
+}
 
 __device__ __forceinline__ uint32_t cluster_rank() {
   uint32_t r;
@@ -578,7 +617,7 @@ w4a4_rac_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid
   pdl_wait();
   pdl_launch_dependents();
 
-  const int total = p.m_tiles * p.n_tiles;
+  const int total = (p.g.off == nullptr ? p.m_tiles : p.pair_start[p.g.E]) * p.n_tiles;
   const bool has_res = p.kt[0] > 0;
 
   if (warp == 0) {
@@ -590,8 +629,10 @@ w4a4_rac_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid
       bool ok = true;
       for (int tile = pair; tile < total && ok; tile += npairs) {
         const int mt = tile / p.n_tiles, nt = tile % p.n_tiles;
-        const int a_row = mt * 256 + static_cast<int>(rank) * 128;
-        const int b_row = nt * 256 + static_cast<int>(rank) * 128;
+        const PairRows pr = pair_rows(p, mt, rank);
+        const int a_row = static_cast<int>(pr.a_tile * 128);
+        const int b_row0 = static_cast<int>(pr.e * p.N) + nt * 256;      // this group's B rows
+        const int b_row = b_row0 + static_cast<int>(rank) * 128;
         for (int seg = has_res ? 0 : 1; seg < 2 && ok; ++seg) {
           const CUtensorMap* tA = seg ? &tmA1 : &tmA0;
           const CUtensorMap* tB = seg ? &tmB1 : &tmB0;
@@ -605,7 +646,7 @@ w4a4_rac_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid
             tma_load_2d_pair(smem_u32(st), tA, kt * BK_BYTES, a_row, lead_full);
             tma_load_2d_pair(smem_u32(st + C::A_ST), tB, kt * BK_BYTES, b_row, lead_full);
             tma_load_2d_pair(smem_u32(st + C::A_ST + C::B_ST), tSA, kt * 256, a_row / 128, lead_full);
-            tma_load_2d_pair(smem_u32(st + C::A_ST + C::B_ST + C::SFA_ST), tSB, kt * 256, nt * 2, lead_full);
+            tma_load_2d_pair(smem_u32(st + C::A_ST + C::B_ST + C::SFA_ST), tSB, kt * 256, b_row0 / 128, lead_full);
             armed |= 1u << stage;
             armed_phase = (armed_phase & ~(1u << stage)) | (phase << stage);
             if (++stage == STAGES) { stage = 0; phase ^= 1; }
@@ -708,8 +749,9 @@ w4a4_rac_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid
     uint32_t acc_phase = 0, res_phase = 0;
     for (int tile = pair; tile < total; tile += npairs) {
       const int mt = tile / p.n_tiles, nt = tile % p.n_tiles;
-      const float al0 = __fmul_rn(p.sta[1][0], p.stb[1][0]);
-      const float al1 = has_res ? __fmul_rn(p.sta[0][0], p.stb[0][0]) : 0.0f;
+      const PairRows pr = pair_rows(p, mt, rank);
+      const float al0 = __fmul_rn(p.sta[1][pr.e], p.stb[1][pr.e]);
+      const float al1 = has_res ? __fmul_rn(p.sta[0][pr.e], p.stb[0][pr.e]) : 0.0f;
       // the residual is scaled to the plain segment's units, then Y = al0 acc;
       // with al0 == 0 the plain operands are all zero codes and Y = al1 acc
       const float ratio = al0 != 0.0f ? __fdiv_rn(al1, al0) : 1.0f;
@@ -744,7 +786,7 @@ w4a4_rac_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid
       ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
       if (!ok) break;
       tc_fence_after();
-      const int64_t row0 = static_cast<int64_t>(mt) * 256 + rank * 128 + 32 * q;
+      const int64_t lrow0 = pr.local0 + 32 * q;     // first row of this warp within the group
       // rows of this warp (32 x 128 columns in the staging buffer) leave as
       // coalesced row stores
       auto store_rows = [&](int h) {
@@ -752,8 +794,8 @@ w4a4_rac_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid
         const bool col_ok = col + 4 <= p.N;
 #pragma unroll 4
         for (int r = 0; r < 32; ++r) {
-          const int64_t row = row0 + r;
-          if (row >= p.M || !col_ok) continue;
+          if (lrow0 + r >= pr.m || !col_ok) continue;
+          const int64_t row = pr.out0 + lrow0 + r;
           const uint8_t* src = stg_warp + r * C::STG_STRIDE + lane * 4 * YBYTES;
           if (YBYTES == 4)
             *reinterpret_cast<float4*>(static_cast<float*>(p.y) + row * p.ldy + col) = *reinterpret_cast<const float4*>(src);
@@ -864,7 +906,11 @@ cudaError_t launch_pair(const GemmArgs& a, cudaStream_t s) {
   KParams2 p{};
   p.M = a.M;
   p.N = a.N;
-  p.m_tiles = static_cast<int>((a.M + 255) / 256);
+  p.g = a.g;
+  p.pair_start = a.pair_start;
+  // dense: 256-row tiles; groups: an upper bound of sum_e ceil(tiles_e / 2)
+  // (the kernel reads the exact count from pair_start)
+  p.m_tiles = static_cast<int>(a.g.off == nullptr ? (a.M + 255) / 256 : (a.m_tiles + a.g.E) / 2 + 1);
   p.n_tiles = static_cast<int>((a.N + 255) / 256);
   const bool res = a.a1.codes != nullptr;
   // segment 0: residual (may be absent), segment 1: plain
@@ -900,8 +946,10 @@ cudaError_t launch_pair(const GemmArgs& a, cudaStream_t s) {
 }  // namespace
 
 cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s) {
-  // dense activations with enough rows for 256-row tiles: the CTA-pair kernel
-  if (a.g.off == nullptr && a.M >= 512 && !gemm_force_single_cta())
+  // dense activations with enough rows for 256-row tiles, and row groups
+  // (256-row tiles per group): the CTA-pair kernel
+  const bool pair_ok = a.g.off == nullptr ? a.M >= 512 : a.pair_start != nullptr;
+  if (pair_ok && !gemm_force_single_cta())
     return a.y_dtype == 0 ? launch_pair<4>(a, s) : launch_pair<2>(a, s);
   cudaError_t e = a.y_dtype == 0 ? prepare_kernel<4>() : prepare_kernel<2>();
   if (e != cudaSuccess) return e;

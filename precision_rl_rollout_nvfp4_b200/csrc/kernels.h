@@ -66,7 +66,9 @@ cudaError_t launch_amax(const uint16_t* x, int64_t rows, int64_t K, int64_t ldx,
                         const RowGroups& g, unsigned* amax_bits, cudaStream_t s,
                         int32_t batch = 1, int64_t mat_stride = 0);
 
-// MoE only: tile_start[e] = sum_{e' < e} ceil(m_e' / 128), e = 0..E.
+// MoE only: tile_start[e] = sum_{e' < e} ceil(m_e' / 128), e = 0..E, and
+// (right after it, tile_start[E + 1 + e]) the prefix of ceil(tiles_e / 2),
+// the 256-row tiles of the CTA-pair GEMM.  tile_start holds 2 (E + 1) ints.
 cudaError_t launch_group_tiles(const int64_t* off, int32_t E, int32_t* tile_start, cudaStream_t s);
 
 // Q(X) plus score partials.  amax: fp32 per group.  codes [codes_rows, K/2]
@@ -149,6 +151,7 @@ struct GemmArgs {
   int64_t M;              // dense rows (or T for MoE)
   int64_t N;              // out-features per group
   int64_t m_tiles;        // dense: ceil(M/128); MoE: upper bound
+  const int32_t* pair_start;  // MoE: prefix of 256-row tiles per group (E + 1)
   void* y;
   int32_t y_dtype;        // 0 fp32, 1 bf16
   int64_t ldy;

@@ -66,13 +66,18 @@ __global__ void group_tiles_kernel(const int64_t* __restrict__ off, int32_t E,
   pdl_wait();
   pdl_launch_dependents();
   if (threadIdx.x != 0) return;
-  int32_t acc = 0;
+  int32_t acc = 0, pacc = 0;
+  int32_t* pair_start = tile_start + E + 1;
   for (int e = 0; e < E; ++e) {
     tile_start[e] = acc;
+    pair_start[e] = pacc;
     const int64_t m = off[e + 1] - off[e];
-    acc += static_cast<int32_t>((m + kTileRows - 1) / kTileRows);
+    const int32_t t = static_cast<int32_t>((m + kTileRows - 1) / kTileRows);
+    acc += t;
+    pacc += (t + 1) / 2;                           // 256-row tiles of the CTA-pair GEMM
   }
   tile_start[E] = acc;
+  pair_start[E] = pacc;
 }
 
 // Per-CTA partial maxima of |x| for `batch` dense matrices (blockIdx.y), no
