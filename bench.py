@@ -50,6 +50,7 @@ FP4_OVER_BF16 = 4.0          # nominal dense FP4 / BF16 tensor ratio (9 / 2.25 P
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 ORACLE_SAMPLE_ROWS = 1024
 L2_FLUSH_BYTES = 256 << 20
+PER_CALL_REPS = 10
 
 
 def parse_args():
@@ -329,17 +330,46 @@ def run_ours(args, rank, world, local_rank):
     total_ms = sum(a.elapsed_time(b) for a, b in step_ms)
     clock = clocks.summary()
 
-    # per-call breakdown inside the same sequence (same L2 state as a step)
+    # per-call breakdown: each call's average launch duration with L2
+    # flushed before every launch, from one graph of PER_CALL_REPS (flush,
+    # call) pairs minus a graph of the flushes alone (no replay gaps inside)
     per_call = {c: [] for c in calls}
-    for _ in range(args.steps):
-        flush.zero_()
-        evs = [ev()]
-        for c in calls:
-            launch(c)
-            evs.append(ev())
+
+    def reps_graph(fn):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for _ in range(PER_CALL_REPS):
+                flush.zero_()
+                fn()
+        return g
+
+    def time_graph(g):
+        g.replay()
+        a = ev()
+        g.replay()
+        b = ev()
         torch.cuda.synchronize()
-        for i, c in enumerate(calls):
-            per_call[c].append(evs[i].elapsed_time(evs[i + 1]))
+        return a.elapsed_time(b)
+
+    if use_graph:
+        g_flush = reps_graph(lambda: None)
+        g_calls = {c: reps_graph(fns[c]) for c in calls}
+        torch.cuda.synchronize()
+        for _ in range(max(1, min(args.steps, 5))):
+            base = time_graph(g_flush)
+            for c in calls:
+                per_call[c].append(max(time_graph(g_calls[c]) - base, 0.0) / PER_CALL_REPS)
+        del g_flush, g_calls
+    else:
+        for _ in range(args.steps):
+            flush.zero_()
+            evs = [ev()]
+            for c in calls:
+                launch(c)
+                evs.append(ev())
+            torch.cuda.synchronize()
+            for i, c in enumerate(calls):
+                per_call[c].append(evs[i].elapsed_time(evs[i + 1]))
     # plain W4A4 linear (no RAC) and the RAC linear without weight prep, for the overhead
     plain_ms, rac_ms = [], []
     for _ in range(args.steps):
@@ -403,7 +433,7 @@ def run_ours(args, rank, world, local_rank):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4 (e2m1/ue4m3) x fp32 acc",
         "data": "synthetic (seeded channel-scaled heavy-tailed X, N(0,0.02) W; see DESIGN.md)",
         "config": {"workload": args.workload, "M": M, "K": K, "N": N, "k_percent": k, "n_sel": n_sel,
-                   "y_dtype": "bf16", "parallelism": f"replicas x{world}", "l2": "flushed between steps (256 MiB write)",
+                   "y_dtype": "bf16", "parallelism": f"replicas x{world}", "l2": "flushed between steps and before every per-call launch (256 MiB write)",
                    "cuda_graph": use_graph},
         "gemm_tflops": round(gemm_tflops, 1), "gemm_frac_fp4_peak": round(gemm_tflops / fp4_peak, 4),
         "quantizer_gbs": round(quant_gbs, 1), "quantizer_frac_hbm": round(quant_gbs / hbm_peak, 4),
