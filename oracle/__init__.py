@@ -32,4 +32,5 @@ from .formats import (bf16_to_f32, e2m1_decode, e2m1_encode, e4m3_decode,  # noq
 from .nvfp4 import amax, dequantize, quantize, quantize_tensor, tensor_scale  # noqa: F401
 from .rac import (channel_score, column_amax, gather_quantize, gemm_fp64,  # noqa: F401
                   moe_rac, n_selected, padded_width, quantize_activations,
-                  rac_linear, residual, select_channels, weight_qdq)
+                  rac_linear, residual, select_channels, weight_qdq,
+                  weight_sel_from_fp4)

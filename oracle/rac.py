@@ -116,6 +116,17 @@ def column_amax(w):
     return w.max(axis=0) if w.shape[0] else np.zeros(w.shape[1], F32)
 
 
+def weight_sel_from_fp4(w_codes, w_scales, w_st, sel, width: int):
+    """Variant of the weight-side second pass (not the pages' reading; an
+    option for rollouts that keep only Q(W)): W_sel is re-quantized from the
+    trainer's NVFP4 weights, DQ(Q(W))[:, sel] in fp32, zero-padded to
+    ``width``, with tensor scale RN(max over the selected columns of
+    max_n |DQ(Q(W))_nj| / 2688).  Returns (codes, scales, s_t)."""
+    dq = dequantize(w_codes, w_scales, w_st)
+    a = column_amax(dq)[np.asarray(sel, np.int64)].max() if len(sel) else F32(0.0)
+    return gather_quantize(dq, sel, width, a)
+
+
 def gemm_fp64(a_codes, a_scales, a_st, b_codes, b_scales, b_st, rows=None):
     """Y = s_ta * s_tb * sum_k a_ik b_jk in fp64, a and b the exact block
     values E2M1dec * E4M3dec.  ``rows`` restricts Y to those rows of A."""
@@ -154,13 +165,15 @@ def weight_qdq(w_bf16):
                 colamax=column_amax(w))
 
 
-def rac_linear(x_bf16, w_bf16, k_percent, rows=None, wq=None):
+def rac_linear(x_bf16, w_bf16, k_percent, rows=None, wq=None, wsel_source="bf16"):
     """One rollout linear Y = X W^T in NVFP4 W4A4 with RAC.
 
     ``rows`` restricts the fp64 products to a subset of output rows (all
     quantities that depend on every token, such as the scores and the mask,
     are still computed from all rows).  ``wq`` may pass a precomputed
-    ``weight_qdq(w_bf16)``.  Returns every intermediate."""
+    ``weight_qdq(w_bf16)``.  ``wsel_source="fp4"`` takes W_sel from Q(W)
+    (``weight_sel_from_fp4``) instead of bf16 W.  Returns every
+    intermediate."""
     qa = quantize_activations(x_bf16)
     M, K = qa["codes"].shape
     wq = weight_qdq(w_bf16) if wq is None else wq
@@ -179,9 +192,13 @@ def rac_linear(x_bf16, w_bf16, k_percent, rows=None, wq=None):
         return out
     r_amax = qa["res_colamax"][sel].max()
     r_codes, r_scales, r_st = gather_quantize(qa["dx"], sel, width, r_amax)
-    w = bf16_to_f32(w_bf16)
-    ws_amax = wq["colamax"][sel].max()
-    ws_codes, ws_scales, ws_st = gather_quantize(w, sel, width, ws_amax)
+    if wsel_source == "fp4":
+        ws_codes, ws_scales, ws_st = weight_sel_from_fp4(wq["codes"], wq["scales"], wq["s_t"], sel, width)
+        ws_amax = column_amax(dequantize(wq["codes"], wq["scales"], wq["s_t"]))[sel].max()
+    else:
+        w = bf16_to_f32(w_bf16)
+        ws_amax = wq["colamax"][sel].max()
+        ws_codes, ws_scales, ws_st = gather_quantize(w, sel, width, ws_amax)
     y_corr = gemm_fp64(r_codes, r_scales, r_st, ws_codes, ws_scales, ws_st, rows)
     out.update(r_codes=r_codes, r_scales=r_scales, r_st=r_st, r_amax=r_amax,
                ws_codes=ws_codes, ws_scales=ws_scales, ws_st=ws_st,

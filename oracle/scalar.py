@@ -84,9 +84,10 @@ def dequantize_rows(codes, scales, s_t):
              for j, c in enumerate(row)] for i, row in enumerate(codes)]
 
 
-def rac_linear(x_bits, w_bits, k_percent):
+def rac_linear(x_bits, w_bits, k_percent, wsel_source="bf16"):
     """x_bits [M][K], w_bits [N][K]: bf16 bit patterns.  Returns a dict with
-    the codes, scales, scores, sel and the fp64 outputs."""
+    the codes, scales, scores, sel and the fp64 outputs.  wsel_source="fp4"
+    takes the selected weight columns from the dequantized NVFP4 weights."""
     X = [[bf16_bits_to_float(b) for b in row] for row in x_bits]
     W = [[bf16_bits_to_float(b) for b in row] for row in w_bits]
     M, K, N = len(X), len(X[0]), len(W)
@@ -134,7 +135,8 @@ def rac_linear(x_bits, w_bits, k_percent):
         return out
     width = -(-n_sel // 64) * 64
     R = [[dx[i][j] for j in sel] + [0.0] * (width - n_sel) for i in range(M)]
-    Ws = [[W[n][j] for j in sel] + [0.0] * (width - n_sel) for n in range(N)]
+    Wsrc = dequantize_rows(cw, sw, stw) if wsel_source == "fp4" else W
+    Ws = [[Wsrc[n][j] for j in sel] + [0.0] * (width - n_sel) for n in range(N)]
     ar, str_ = t_scale(R)
     aws, stws = t_scale(Ws)
     cr, sr = quantize_rows(R, str_)

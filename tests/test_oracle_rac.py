@@ -163,3 +163,55 @@ def test_moe_groups_are_independent_linears():
         r = oracle.rac_linear(xb[off[e]:off[e + 1]], wb[e], 50.0)
         assert np.array_equal(y[off[e]:off[e + 1]], r["y"])
         assert np.array_equal(masks[e], r["mask"])
+
+
+@pytest.mark.parametrize("M,K,N,k", [(5, 64, 3, 50.0), (9, 32, 4, 25.0), (3, 80, 2, 100.0)])
+def test_wsel_from_fp4_scalar_restatement_agrees(M, K, N, k):
+    """The W_sel variant from Q(W) against the independent scalar
+    restatement (codes, scales, tensor scale and Y)."""
+    x = S.activations(M, K, seed=M + 2 * K)
+    w = S.weights(N, K, seed=N + 7)
+    xb, wb = S.bf16_bits(x), S.bf16_bits(w)
+    r = oracle.rac_linear(xb, wb, k, wsel_source="fp4")
+    s = scalar.rac_linear(xb.tolist(), wb.tolist(), k, wsel_source="fp4")
+    assert np.array_equal(r["ws_codes"], np.array(s["ws_codes"], np.uint8))
+    assert np.array_equal(r["ws_scales"], np.array(s["ws_scales"], np.uint8))
+    assert r["ws_st"] == s["ws_st"]
+    assert np.allclose(r["y"], np.array(s["y"]), rtol=1e-12, atol=1e-14)
+
+
+def test_wsel_from_fp4_equals_bf16_source_on_grid_weights():
+    """Weights already on the NVFP4 grid (W = DQ(Q(W0)), tensor scale a power
+    of two so every value is exact in bf16) quantize back to themselves
+    (Q(DQ(Q(w))) = Q(w)), so both sources of W_sel agree exactly."""
+    rng = np.random.default_rng(11)
+    N, K = 48, 256
+    w0 = rng.standard_normal((N, K)).astype(np.float32) * 0.05
+    amax = np.float32(2688.0 * 2.0 ** -10)                 # s_t = 2^-10 exactly
+    w0[3, 7] = amax
+    w0 = np.clip(w0, -amax, amax)
+    c0, s0, st0 = oracle.quantize_tensor(w0)
+    assert st0 == np.float32(2.0 ** -10)
+    dq = oracle.dequantize(c0, s0, st0)
+    wb = oracle.f32_to_bf16(dq)
+    assert np.array_equal(oracle.bf16_to_f32(wb), dq)       # exact in bf16
+    wq = oracle.weight_qdq(wb)
+    assert np.array_equal(wq["codes"], c0) and np.array_equal(wq["scales"], s0)
+    sel = np.sort(rng.choice(K, 100, replace=False)).astype(np.int32)
+    width = oracle.padded_width(len(sel))
+    a = oracle.weight_sel_from_fp4(wq["codes"], wq["scales"], wq["s_t"], sel, width)
+    b = oracle.gather_quantize(oracle.bf16_to_f32(wb), sel, width, wq["colamax"][sel].max())
+    for u, v in zip(a, b):
+        assert np.array_equal(u, v)
+
+
+def test_wsel_from_fp4_k0_is_plain_and_error_is_bounded():
+    x = S.activations(32, 128, seed=4)
+    w = S.weights(16, 128, seed=4)
+    xb, wb = S.bf16_bits(x), S.bf16_bits(w)
+    r0 = oracle.rac_linear(xb, wb, 0.0, wsel_source="fp4")
+    assert np.array_equal(r0["y"], r0["y_plain"])
+    # the FP4-sourced correction still reduces the error against bf16
+    ref = oracle.bf16_to_f32(xb).astype(np.float64) @ oracle.bf16_to_f32(wb).astype(np.float64).T
+    r50 = oracle.rac_linear(xb, wb, 50.0, wsel_source="fp4")
+    assert np.linalg.norm(r50["y"] - ref) <= np.linalg.norm(r0["y"] - ref)
