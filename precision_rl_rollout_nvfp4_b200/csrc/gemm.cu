@@ -31,7 +31,7 @@
 // CTA loads its own tiles (no load is shared between CTAs).  Every mbarrier
 // wait is bounded (see common.cuh).
 //
-// For dense activations with at least 512 rows a second kernel runs the same
+// For dense activations with at least 256 rows a second kernel runs the same
 // product on CTA pairs (tcgen05 cta_group::2): a pair computes a 256 x 256
 // tile, each CTA loading its own 128 rows of A and of B, so a pair fetches
 // half the operand bytes per FLOP of two 128 x 128 tiles; the leader's copier
@@ -946,9 +946,9 @@ cudaError_t launch_pair(const GemmArgs& a, cudaStream_t s) {
 }  // namespace
 
 cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s) {
-  // dense activations with enough rows for 256-row tiles, and row groups
+  // dense activations with at least one full 256-row tile, and row groups
   // (256-row tiles per group): the CTA-pair kernel
-  const bool pair_ok = a.g.off == nullptr ? a.M >= 512 : a.pair_start != nullptr;
+  const bool pair_ok = a.g.off == nullptr ? a.M >= 256 : a.pair_start != nullptr;
   if (pair_ok && !gemm_force_single_cta())
     return a.y_dtype == 0 ? launch_pair<4>(a, s) : launch_pair<2>(a, s);
   cudaError_t e = a.y_dtype == 0 ? prepare_kernel<4>() : prepare_kernel<2>();
