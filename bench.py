@@ -63,6 +63,8 @@ def parse_args():
     p.add_argument("--k", type=float, default=None, help="RAC k percent (default: workload's)")
     p.add_argument("--no-graph", action="store_true", help="issue calls directly, no CUDA graphs")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--wsel", choices=["bf16", "fp4"], default="bf16",
+                   help="W_sel source: the bf16 weight (default) or its NVFP4 codes (variant)")
     return p.parse_args()
 
 
@@ -76,13 +78,17 @@ def load_peaks():
 
 
 # ---------------------------------------------------------------- algorithmic work
-def work(M, K, N, n_sel, width):
-    """Algorithmic FLOPs / bytes per call (see the design notes)."""
+def work(M, K, N, n_sel, width, wsel="bf16"):
+    """Algorithmic FLOPs / bytes per call (see the design notes).  With
+    wsel="fp4" the weight preparation also reads Q(W) once for the DQ column
+    maxima, and W_sel is gathered from the 0.5625 B/element NVFP4 weight."""
+    fp4 = wsel == "fp4"
     return {
-        "prepare_weight": dict(bytes=6.5625 * N * K + 4 * K, bound="hbm"),
+        "prepare_weight": dict(bytes=6.5625 * N * K + 4 * K + (0.5625 * N * K + 4 * K if fp4 else 0.0),
+                               bound="hbm"),
         "quantize": dict(bytes=4.0 * M * K + 0.5625 * M * K + 12 * K, bound="hbm"),
         "select": dict(bytes=2.5625 * M * n_sel + 0.5625 * M * width + 12 * K + 4 * n_sel, bound="hbm"),
-        "weight_select": dict(bytes=2.0 * N * n_sel + 0.5625 * N * width, bound="hbm"),
+        "weight_select": dict(bytes=(0.5625 if fp4 else 2.0) * N * n_sel + 0.5625 * N * width, bound="hbm"),
         "gemm": dict(flops=2.0 * M * N * (K + n_sel), bytes=0.5625 * (M + N) * (K + width) + 2.0 * M * N,
                      bound="tensor"),
     }
@@ -257,7 +263,7 @@ def run_ours(args, rank, world, local_rank):
     w_host = S.weights(N, K, seed=seed).pin_memory()
     x = x_host.to(dev)
     w = w_host.to(dev)
-    plan = B.RacLinearPlan(M, K, N, k, out_dtype=torch.bfloat16, device=dev).bind(x, w)
+    plan = B.RacLinearPlan(M, K, N, k, out_dtype=torch.bfloat16, device=dev, wsel=args.wsel).bind(x, w)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
     calls = ["prepare_weight", "quantize", "select", "weight_select", "gemm"]
@@ -404,7 +410,7 @@ def run_ours(args, rank, world, local_rank):
     value = flops_step * world * args.steps / (total_ms * 1e-3) / 1e12
     e2e_value = flops_step * world * args.steps / (e2e_total * 1e-3) / 1e12
     med = {c: statistics.median(v) for c, v in per_call.items()}
-    wk = work(M, K, N, n_sel, width)
+    wk = work(M, K, N, n_sel, width, args.wsel)
     peaks, peak_kind = load_peaks()
     hbm_peak = peaks["hbm_gbs"]
     fp4_peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]) * FP4_OVER_BF16
@@ -425,7 +431,7 @@ def run_ours(args, rank, world, local_rank):
     gemm_tflops = wk["gemm"]["flops"] / (med["gemm"] * 1e-3) / 1e12
     quant_gbs = wk["quantize"]["bytes"] / (med["quantize"] * 1e-3) / 1e9
     rac_over = (statistics.median(rac_ms) - statistics.median(plain_ms)) / statistics.median(plain_ms)
-    launches_per_step = sum(B.RacLinearPlan.LAUNCHES[c] for c in calls) - (0 if n_sel else 2)
+    launches_per_step = sum(plan.launches[c] for c in calls) - (0 if n_sel else 2)
 
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s (effective 2MN(K+n_sel) per step)",
@@ -433,7 +439,7 @@ def run_ours(args, rank, world, local_rank):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4 (e2m1/ue4m3) x fp32 acc",
         "data": "synthetic (seeded channel-scaled heavy-tailed X, N(0,0.02) W; see DESIGN.md)",
         "config": {"workload": args.workload, "M": M, "K": K, "N": N, "k_percent": k, "n_sel": n_sel,
-                   "y_dtype": "bf16", "parallelism": f"replicas x{world}", "l2": "flushed between steps and before every per-call launch (256 MiB write)",
+                   "y_dtype": "bf16", "wsel": args.wsel, "parallelism": f"replicas x{world}", "l2": "flushed between steps and before every per-call launch (256 MiB write)",
                    "cuda_graph": use_graph},
         "gemm_tflops": round(gemm_tflops, 1), "gemm_frac_fp4_peak": round(gemm_tflops / fp4_peak, 4),
         "quantizer_gbs": round(quant_gbs, 1), "quantizer_frac_hbm": round(quant_gbs / hbm_peak, 4),
@@ -494,26 +500,34 @@ def run_moe(args, rank, world, local_rank):
         e.record(stream)
         return e
 
-    # weight preparation (per weight sync): Q(W) and colamax of every expert
+    # weight preparation (per weight sync): Q(W) and the column maxima of
+    # every expert (of W, or with --wsel fp4 of DQ(Q(W)))
+    fp4 = args.wsel == "fp4"
     wu_out, wd_out = torch.empty_like(wu), torch.empty_like(wd)
     prep = {}
     for _ in range(3):              # the last pass reuses cached buffers
         torch.cuda.synchronize()
         a = ev()
-        _, qu, cu = B.weight_qdq(wu, out=wu_out)
+        _, qu, cu = B.weight_qdq(wu, want_colamax=not fp4, out=wu_out)
+        if fp4:
+            cu = B.dq_colamax(qu, E)
         b = ev()
-        _, qd, cd = B.weight_qdq(wd, out=wd_out)
+        _, qd, cd = B.weight_qdq(wd, want_colamax=not fp4, out=wd_out)
+        if fp4:
+            cd = B.dq_colamax(qd, E)
         c = ev()
         torch.cuda.synchronize()
         prep = {"weight_qdq_up": a.elapsed_time(b) * 1e3, "weight_qdq_down": b.elapsed_time(c) * 1e3}
+    # W_sel source: the bf16 experts, or (None) their NVFP4 codes
+    wu_sel, wd_sel = (None, None) if fp4 else (wu, wd)
     yu = torch.empty(T, N_up, dtype=torch.bfloat16, device=dev)
     yd = torch.empty(T, N_dn, dtype=torch.bfloat16, device=dev)
 
     def up(kk=k):
-        B.moe_rac(xu, off, wu, qu, cu, kk, out_dtype=torch.bfloat16, masks=False, out=yu)
+        B.moe_rac(xu, off, wu_sel, qu, cu, kk, out_dtype=torch.bfloat16, masks=False, out=yu)
 
     def down(kk=k):
-        B.moe_rac(xd, off, wd, qd, cd, kk, out_dtype=torch.bfloat16, masks=False, out=yd)
+        B.moe_rac(xd, off, wd_sel, qd, cd, kk, out_dtype=torch.bfloat16, masks=False, out=yd)
 
     def step():
         up()
@@ -577,8 +591,8 @@ def run_moe(args, rank, world, local_rank):
     yu1, yd1 = torch.empty_like(yu), torch.empty_like(yd)
 
     def step1():
-        B.moe_rac(xu1, off, wu, qu, cu, k, out_dtype=torch.bfloat16, masks=False, out=yu1)
-        B.moe_rac(xd1, off, wd, qd, cd, k, out_dtype=torch.bfloat16, masks=False, out=yd1)
+        B.moe_rac(xu1, off, wu_sel, qu, cu, k, out_dtype=torch.bfloat16, masks=False, out=yu1)
+        B.moe_rac(xd1, off, wd_sel, qd, cd, k, out_dtype=torch.bfloat16, masks=False, out=yd1)
 
     sets = [{"h2d": [(xu, xu_host), (xd, xd_host)], "d2h": [(torch.empty(T, N_dn, dtype=torch.bfloat16).pin_memory(), yd)],
              "step": step},
@@ -604,7 +618,8 @@ def run_moe(args, rank, world, local_rank):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4 (e2m1/ue4m3) x fp32 acc",
         "data": "synthetic (seeded routing and activations; see DESIGN.md)",
         "config": {"workload": MOE_WORKLOAD, "tokens": cfg["T"], "topk": cfg["topk"], "routed_rows": T, "experts": E,
-                   "up": [K_up, N_up], "down": [K_dn, N_dn], "k_percent": k, "expert_rows_max": max(loads),
+                   "up": [K_up, N_up], "down": [K_dn, N_dn], "k_percent": k, "wsel": args.wsel,
+                   "expert_rows_max": max(loads),
                    "expert_rows_min": min(loads), "y_dtype": "bf16", "parallelism": f"replicas x{world}",
                    "l2": "inputs larger than L2 (402 MB per step)", "cuda_graph": use_graph},
         "per_call_us": {"up": round(1e3 * med["up"], 2), "down": round(1e3 * med["down"], 2),
@@ -627,7 +642,7 @@ def run_moe(args, rank, world, local_rank):
 
 
 # ---------------------------------------------------------------- oracle (CPU)
-def oracle_step_time(M, K, N, k, rows, seed=0):
+def oracle_step_time(M, K, N, k, rows, seed=0, wsel="bf16"):
     import numpy as np
 
     import oracle
@@ -636,7 +651,7 @@ def oracle_step_time(M, K, N, k, rows, seed=0):
     w = S.bf16_bits(S.weights(N, K, seed=seed))
     t0 = time.perf_counter()
     wq = oracle.weight_qdq(w)
-    r = oracle.rac_linear(x, w, k, wq=wq)
+    r = oracle.rac_linear(x, w, k, wq=wq, wsel_source=wsel)
     dt = time.perf_counter() - t0
     return dt, 2.0 * rows * N * (K + r["n_sel"]), np.asarray(r["y"]).shape
 
@@ -652,7 +667,7 @@ def blas_threads():
 _MOE_SAMPLE = {}
 
 
-def oracle_moe_time(k, n_experts=8, seed=0):
+def oracle_moe_time(k, n_experts=8, seed=0, wsel="bf16"):
     """Oracle up projection of the last n_experts experts (the smallest row
     groups) of the MoE workload: every step of the grouped RAC linear on those
     groups.  Returns (seconds, effective FLOPs, description)."""
@@ -669,7 +684,7 @@ def oracle_moe_time(k, n_experts=8, seed=0):
                                           off[e0:] - r0, r0, r1)
     x, w, sub_off, r0, r1 = _MOE_SAMPLE[(n_experts, seed)]
     t0 = time.perf_counter()
-    oracle.moe_rac(x, sub_off, w, k)
+    oracle.moe_rac(x, sub_off, w, k, wsel_source=wsel)
     dt = time.perf_counter() - t0
     K, N = cfg["hidden"], cfg["inter"]
     n_sel = oracle.n_selected(k, K)
@@ -681,7 +696,7 @@ def cpu_baseline(args, budget_s=12.0):
         k = args.k if args.k is not None else 50.0
         t, flops, n, desc = 0.0, 0.0, 0, ""
         while (t < budget_s and n < 4) or n == 0:
-            dt, f, desc = oracle_moe_time(k)
+            dt, f, desc = oracle_moe_time(k, wsel=args.wsel)
             t, flops, n = t + dt, flops + f, n + 1
         return {"value": round(flops / t / 1e12, 6), "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
                 "sample": f"{n} oracle run(s) of the grouped RAC linear: {desc} (numpy; fp64 product via BLAS)"}
@@ -690,7 +705,7 @@ def cpu_baseline(args, budget_s=12.0):
     rows = min(M, ORACLE_SAMPLE_ROWS)
     t, flops, n = 0.0, 0.0, 0
     while t < budget_s or n == 0:
-        dt, f, _ = oracle_step_time(M, K, N, k, rows)
+        dt, f, _ = oracle_step_time(M, K, N, k, rows, wsel=args.wsel)
         t += dt
         flops += f
         n += 1
@@ -705,10 +720,10 @@ def run_reference(args):
     if args.workload == MOE_WORKLOAD:
         k = args.k if args.k is not None else 50.0
         for _ in range(args.warmup):
-            oracle_moe_time(k)
+            oracle_moe_time(k, wsel=args.wsel)
         t, flops, desc = 0.0, 0.0, ""
         for _ in range(args.steps):
-            dt, f, desc = oracle_moe_time(k)
+            dt, f, desc = oracle_moe_time(k, wsel=args.wsel)
             t, flops = t + dt, flops + f
         value = flops / t / 1e12
         return {"impl": "reference", "metric": METRIC, "value": round(value, 6),
@@ -723,10 +738,10 @@ def run_reference(args):
     k = args.k if args.k is not None else k
     rows = min(M, ORACLE_SAMPLE_ROWS)
     for _ in range(args.warmup):
-        oracle_step_time(M, K, N, k, rows)
+        oracle_step_time(M, K, N, k, rows, wsel=args.wsel)
     t, flops = 0.0, 0.0
     for _ in range(args.steps):
-        dt, f, _ = oracle_step_time(M, K, N, k, rows)
+        dt, f, _ = oracle_step_time(M, K, N, k, rows, wsel=args.wsel)
         t += dt
         flops += f
     value = flops / t / 1e12

@@ -150,6 +150,31 @@ nvfp4_status rac_weight_quant(const uint16_t* w, int64_t N, int64_t K, int64_t l
                               nvfp4_tensor* q_wsel, void* stream);
 
 /*
+ * nvfp4_dq_colamax -- colamax [batch, cols] fp32, the column maxima
+ * max_n |DQ(Q(W))_nj| of `batch` stacked NVFP4 matrices of q->rows / batch
+ * rows each (tensor_scale[batch]).  The statistic rac_weight_quant_fp4 and
+ * the w == NULL forms below take as their column maxima; it changes only
+ * when the weights do.  Either scale layout.  colamax is overwritten.
+ */
+nvfp4_status nvfp4_dq_colamax(const nvfp4_tensor* q, int32_t batch, float* colamax, void* stream);
+
+/*
+ * rac_weight_quant_fp4 -- the second-pass quantization of the selected
+ * weight columns taken from the NVFP4 weights alone, for rollout engines that
+ * hold Q(W) but not the bf16 W: W_sel = DQ(Q(W))[:, sel] (exact fp32
+ * values), re-quantized with tensor scale RN(max_{j in sel} dq_colamax_j /
+ * 2688).  Pages: 2.2 B (second-pass quantization of the selected channels;
+ * the pages do not say where the weight values come from) and 2.1 (rollout
+ * and trainer share the weight QDQ path).  This is a variant beyond the
+ * plainest reading: Y differs from the bf16-sourced form by the weight's
+ * own quantization error in the correction term.
+ *   qw: the single weight's Q(W) (rows = N, cols = K, either scale layout);
+ *   dq_colamax: nvfp4_dq_colamax(qw, 1); q_wsel as for rac_weight_quant.
+ */
+nvfp4_status rac_weight_quant_fp4(const nvfp4_tensor* qw, const int32_t* sel, int64_t n_sel,
+                                  const float* dq_colamax, nvfp4_tensor* q_wsel, void* stream);
+
+/*
  * w4a4_rac_gemm -- Y = s_tX s_tW (A B^T) + s_tR s_tWs (R B_sel^T), one
  * block-scaled FP4 tensor-core GEMM over the K-concatenated operand
  * [Q(X) | Q(dX_sel)] x [Q(W) | Q(W_sel)] with two accumulators.
@@ -158,7 +183,9 @@ nvfp4_status rac_weight_quant(const uint16_t* w, int64_t N, int64_t K, int64_t l
  *   qx, qw: scale_layout 1; qx.cols == qw.cols == K; qw.rows == N.
  *   q_res_or_null / sel / n_sel: from rac_select; n_sel == 0 (or NULL q_res)
  *   gives plain W4A4.  w (bf16 [N, K], stride ldw) and w_colamax (fp32 [K])
- *   are used to quantize W_sel into the workspace when n_sel > 0.
+ *   are used to quantize W_sel into the workspace when n_sel > 0.  With
+ *   w == NULL, W_sel is taken from qw instead (rac_weight_quant_fp4) and
+ *   w_colamax must be nvfp4_dq_colamax(qw, 1).
  *   y: [M, N] fp32 (y_dtype 0) or bf16 (y_dtype 1, RN of the fp32 value),
  *   row stride ldy elements.  ws: NVFP4_OP_GEMM bytes for (N, K).
  */
@@ -188,7 +215,10 @@ nvfp4_status w4a4_gemm_quantized(const nvfp4_tensor* qa, const nvfp4_tensor* qb,
  *   device only; offsets_dev[0] == 0, offsets_dev[E] == T, non-decreasing).
  *   w [E, N, K] bf16 (row stride K), qw: the stacked Q(W) from weight_qdq
  *   with batch E (rows = E*N, cols = K, scale_layout 1, tensor_scale[E]),
- *   w_colamax [E, K].  y_perm [T, N] (dtype y_dtype), masks_or_null u8 [E, K].
+ *   w_colamax [E, K].  w == NULL takes every W_sel from qw instead (as
+ *   rac_weight_quant_fp4 does per expert) and then w_colamax must be
+ *   nvfp4_dq_colamax(qw, E).
+ *   y_perm [T, N] (dtype y_dtype), masks_or_null u8 [E, K].
  *   An empty expert writes no rows; its mask is the first n_sel channels.
  *   ws: nvfp4_workspace_size(NVFP4_OP_MOE, T, N, K, E) bytes.
  */

@@ -206,12 +206,12 @@ def rac_linear(x_bf16, w_bf16, k_percent, rows=None, wq=None, wsel_source="bf16"
     return out
 
 
-def moe_rac(x_perm_bf16, offsets, w_bf16, k_percent, wq=None):
+def moe_rac(x_perm_bf16, offsets, w_bf16, k_percent, wq=None, wsel_source="bf16"):
     """Grouped expert linears: rows offsets[e]:offsets[e+1] of the
     expert-contiguous activations go through expert e's own RAC linear (own
     amax, scores, mask and residual scale).  An empty group produces no rows;
     its mask is that of an all-zero score (the first n_sel channels).
-    Returns (y [T, N] fp64, masks [E, K], per-expert results)."""
+    ``wsel_source`` is passed to ``rac_linear``.  Returns (y [T, N] fp64, masks [E, K], per-expert results)."""
     E, N, K = w_bf16.shape
     T = x_perm_bf16.shape[0]
     y = np.zeros((T, N), np.float64)
@@ -226,7 +226,7 @@ def moe_rac(x_perm_bf16, offsets, w_bf16, k_percent, wq=None):
             masks[e] = mask
             per.append(None)
             continue
-        res = rac_linear(x_perm_bf16[r0:r1], w_bf16[e], k_percent, wq=wqe)
+        res = rac_linear(x_perm_bf16[r0:r1], w_bf16[e], k_percent, wq=wqe, wsel_source=wsel_source)
         y[r0:r1] = res["y"]
         masks[e] = res["mask"]
         per.append(res)

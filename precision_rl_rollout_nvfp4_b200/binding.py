@@ -29,7 +29,8 @@ EXPORTS = ["nvfp4_scale_bytes", "nvfp4_workspace_size", "nvfp4_quantize", "rac_s
            "nvfp4_rac_nsel", "nvfp4_rac_width", "rac_weight_quant", "w4a4_rac_gemm",
            "w4a4_gemm_quantized", "moe_grouped_w4a4_rac_gemm", "weight_qdq",
            "nvfp4_encode_e2m1", "nvfp4_encode_e4m3", "nvfp4_stream_status",
-           "nvfp4_check_bounded_wait", "nvfp4_status_string", "nvfp4_quantize_static_ws"]
+           "nvfp4_check_bounded_wait", "nvfp4_status_string", "nvfp4_quantize_static_ws",
+           "nvfp4_dq_colamax", "rac_weight_quant_fp4"]
 
 
 class _Tensor(ctypes.Structure):
@@ -49,6 +50,8 @@ _sig = {
     "nvfp4_rac_nsel": (I64, [F32, I64]),
     "nvfp4_rac_width": (I64, [I64]),
     "rac_weight_quant": (I32, [P, I64, I64, I64, P, I64, P, TP, P]),
+    "nvfp4_dq_colamax": (I32, [TP, I32, P, P]),
+    "rac_weight_quant_fp4": (I32, [TP, P, I64, P, TP, P]),
     "w4a4_rac_gemm": (I32, [TP, TP, P, I64, P, I64, I64, TP, P, P, I32, I64, P, SZ, P]),
     "w4a4_gemm_quantized": (I32, [TP, TP, TP, TP, P, I32, I64, P]),
     "moe_grouped_w4a4_rac_gemm": (I32, [P, I64, I64, P, I32, P, I64, TP, P, F32, P, I32, P, P, SZ, P]),
@@ -213,6 +216,25 @@ def rac_weight_quant(w, sel, n_sel, w_colamax, layout=1, out=None, stream=None):
     return q
 
 
+def dq_colamax(q, batch=1, out=None, stream=None):
+    """max_n |DQ(Q(W))_nk| per column of each of `batch` stacked matrices
+    held in the NVFP4 tensor q (rows = batch * N).  Returns fp32 [batch, K]."""
+    out = out if out is not None else torch.empty(batch, q.cols, dtype=torch.float32, device=q.codes.device)
+    qc = q.c()
+    _check(_lib.nvfp4_dq_colamax(ctypes.byref(qc), batch, _ptr(out), _stream(stream)), "nvfp4_dq_colamax")
+    return out
+
+
+def rac_weight_quant_fp4(qw, sel, n_sel, dq_cm, layout=1, out=None, stream=None):
+    """Q(W_sel) re-quantized from the NVFP4 weight qw alone (dq_cm from
+    dq_colamax(qw))."""
+    q = out if out is not None else NvFP4Tensor.empty(qw.rows, rac_width(n_sel), layout, device=qw.codes.device)
+    a, qs = qw.c(), q.c()
+    _check(_lib.rac_weight_quant_fp4(ctypes.byref(a), _ptr(sel), n_sel, _ptr(dq_cm), ctypes.byref(qs),
+                                     _stream(stream)), "rac_weight_quant_fp4")
+    return q
+
+
 def gemm_quantized(qa, qb, q_res=None, q_wsel=None, out_dtype=torch.float32, out=None, stream=None):
     y = out if out is not None else torch.empty(qa.rows, qb.rows, dtype=out_dtype, device=qa.codes.device)
     a, b = qa.c(), qb.c()
@@ -227,14 +249,17 @@ def gemm_quantized(qa, qb, q_res=None, q_wsel=None, out_dtype=torch.float32, out
 
 
 def rac_gemm(qx, q_res, sel, n_sel, w, qw, w_colamax, out_dtype=torch.float32, out=None, stream=None):
-    w = _bits(w)
-    N, K = w.shape
-    y = out if out is not None else torch.empty(qx.rows, N, dtype=out_dtype, device=w.device)
-    ws = _ws(workspace_size(OP_GEMM, 0, N, K), w.device)
+    """w = None takes W_sel from qw (then w_colamax = dq_colamax(qw))."""
+    N, K = qw.rows, qx.cols
+    dev = qx.codes.device
+    w = _bits(w) if w is not None else None
+    y = out if out is not None else torch.empty(qx.rows, N, dtype=out_dtype, device=dev)
+    ws = _ws(workspace_size(OP_GEMM, 0, N, K), dev)
     a, b = qx.c(), qw.c()
     r = q_res.c() if q_res is not None else None
     _check(_lib.w4a4_rac_gemm(ctypes.byref(a), ctypes.byref(r) if r is not None else None, _ptr(sel),
-                              n_sel, _ptr(w), N, w.stride(0), ctypes.byref(b), _ptr(w_colamax), _ptr(y),
+                              n_sel, _ptr(w), N, w.stride(0) if w is not None else K, ctypes.byref(b),
+                              _ptr(w_colamax), _ptr(y),
                               0 if y.dtype == torch.float32 else 1, y.stride(0), _ptr(ws), ws.numel(),
                               _stream(stream)), "w4a4_rac_gemm")
     return y
@@ -257,10 +282,16 @@ def weight_qdq(w, want_q=True, want_colamax=True, layout=1, out=None, stream=Non
 
 def moe_rac(x_perm, offsets, w, qw, w_colamax, k_percent, out_dtype=torch.float32, masks=True,
             out=None, stream=None):
-    """Grouped RAC linears of E experts.  offsets: int64 [E+1] on the device."""
-    x_perm, w = _bits(x_perm), _bits(w)
+    """Grouped RAC linears of E experts.  offsets: int64 [E+1] on the device.
+    w = None takes every W_sel from qw (then w_colamax = dq_colamax(qw, E))."""
+    x_perm = _bits(x_perm)
     T, K = x_perm.shape
-    E, N, _ = w.shape
+    if w is not None:
+        w = _bits(w)
+        E, N, _ = w.shape
+    else:
+        E = w_colamax.shape[0]
+        N = qw.rows // E
     y = out if out is not None else torch.empty(T, N, dtype=out_dtype, device=x_perm.device)
     mk = torch.empty(E, K, dtype=torch.uint8, device=x_perm.device) if masks else None
     ws = _ws(workspace_size(OP_MOE, T, N, K, E), x_perm.device)
@@ -272,17 +303,21 @@ def moe_rac(x_perm, offsets, w, qw, w_colamax, k_percent, out_dtype=torch.float3
     return y, mk
 
 
-def rac_linear(x, w, k_percent, out_dtype=torch.float32, prepared=None, stream=None):
+def rac_linear(x, w, k_percent, out_dtype=torch.float32, prepared=None, wsel="bf16", stream=None):
     """The whole rollout linear: weight prep (or `prepared` = (qw, colamax)),
-    Q(X) + scores, mask + Q(dX_sel), Q(W_sel), and the two-segment GEMM."""
+    Q(X) + scores, mask + Q(dX_sel), Q(W_sel), and the two-segment GEMM.
+    wsel="fp4" re-quantizes W_sel from Q(W) (colamax then holds the column
+    maxima of DQ(Q(W)))."""
+    assert wsel in ("bf16", "fp4")
     if prepared is None:
-        _, qw, colamax = weight_qdq(w, stream=stream)
-        colamax = colamax[0]
+        _, qw, colamax = weight_qdq(w, want_colamax=wsel == "bf16", stream=stream)
+        colamax = colamax[0] if wsel == "bf16" else dq_colamax(qw, stream=stream)[0]
     else:
         qw, colamax = prepared
     qx, score, rcm = quantize(x, stream=stream)
     mask, sel, n_sel, q_res = rac_select(x, qx, score, rcm, k_percent, stream=stream)
-    y = rac_gemm(qx, q_res, sel, n_sel, w, qw, colamax, out_dtype=out_dtype, stream=stream)
+    y = rac_gemm(qx, q_res, sel, n_sel, w if wsel == "bf16" else None, qw, colamax, out_dtype=out_dtype,
+                 stream=stream)
     return y, dict(qx=qx, score=score, res_colamax=rcm, mask=mask, sel=sel, n_sel=n_sel, q_res=q_res,
                    qw=qw, w_colamax=colamax)
 
@@ -323,16 +358,25 @@ class RacLinearPlan:
       select          rac_select -> mask, sel, Q(dX_sel)
       weight_select   rac_weight_quant -> Q(W_sel)
       gemm            w4a4_gemm_quantized -> Y
+    With wsel="fp4" the weight preparation also takes the column maxima of
+    DQ(Q(W)) (nvfp4_dq_colamax) and weight_select re-quantizes W_sel from
+    Q(W) (rac_weight_quant_fp4) instead of reading the bf16 W.
     """
 
-    def __init__(self, M, K, N, k_percent, out_dtype=torch.bfloat16, device="cuda"):
+    def __init__(self, M, K, N, k_percent, out_dtype=torch.bfloat16, device="cuda", wsel="bf16"):
+        assert wsel in ("bf16", "fp4")
         self.M, self.K, self.N, self.k = M, K, N, float(k_percent)
+        self.wsel = wsel
+        self.launches = dict(self.LAUNCHES)
+        if wsel == "fp4":
+            self.launches["prepare_weight"] += 1        # nvfp4_dq_colamax
         self.n_sel = rac_nsel(k_percent, K)
         self.width = rac_width(self.n_sel)
         dev = torch.device(device)
         self.qw = NvFP4Tensor.empty(N, K, 1, device=dev)
         self.w_out = torch.empty(N, K, dtype=torch.bfloat16, device=dev)
         self.w_colamax = torch.empty(K, dtype=torch.float32, device=dev)
+        self.dq_colamax = torch.empty(K, dtype=torch.float32, device=dev) if wsel == "fp4" else None
         self.qx = NvFP4Tensor.empty(M, K, 1, device=dev)
         self.score = torch.empty(K, dtype=torch.float64, device=dev)
         self.res_colamax = torch.empty(K, dtype=torch.float32, device=dev)
@@ -363,9 +407,13 @@ class RacLinearPlan:
         return self
 
     def prepare_weight(self, stream=None):
+        fp4 = self.wsel == "fp4"
         _check(_lib.weight_qdq(_ptr(self.w), self.N, self.K, self.w.stride(0), 1, _ptr(self.w_out),
-                               ctypes.byref(self._qw), _ptr(self.w_colamax), _ptr(self.ws_w),
-                               self.ws_w.numel(), _stream(stream)), "weight_qdq")
+                               ctypes.byref(self._qw), None if fp4 else _ptr(self.w_colamax),
+                               _ptr(self.ws_w), self.ws_w.numel(), _stream(stream)), "weight_qdq")
+        if fp4:
+            _check(_lib.nvfp4_dq_colamax(ctypes.byref(self._qw), 1, _ptr(self.dq_colamax), _stream(stream)),
+                   "nvfp4_dq_colamax")
 
     def quantize(self, stream=None, scores=True):
         _check(_lib.nvfp4_quantize(_ptr(self.x), self.M, self.K, self.x.stride(0), None, ctypes.byref(self._qx),
@@ -382,6 +430,11 @@ class RacLinearPlan:
 
     def weight_select(self, stream=None):
         if self.n_sel == 0:
+            return
+        if self.wsel == "fp4":
+            _check(_lib.rac_weight_quant_fp4(ctypes.byref(self._qw), _ptr(self.sel), self.n_sel,
+                                             _ptr(self.dq_colamax), ctypes.byref(self._qs), _stream(stream)),
+                   "rac_weight_quant_fp4")
             return
         _check(_lib.rac_weight_quant(_ptr(self.w), self.N, self.K, self.w.stride(0), _ptr(self.sel), self.n_sel,
                                      _ptr(self.w_colamax), ctypes.byref(self._qs), _stream(stream)),
@@ -422,4 +475,4 @@ class RacLinearPlan:
         self.gemm(stream, plain=True)
 
     # kernels each call launches (for launch accounting)
-    LAUNCHES = dict(prepare_weight=2, quantize=2, quantize_plain=2, select=2, weight_select=2, gemm=1)
+    LAUNCHES = dict(prepare_weight=2, quantize=2, quantize_plain=2, select=2, weight_select=1, gemm=1)

@@ -284,6 +284,36 @@ nvfp4_status rac_weight_quant(const uint16_t* w, int64_t N, int64_t K, int64_t l
   return NVFP4_OK;
 }
 
+nvfp4_status nvfp4_dq_colamax(const nvfp4_tensor* q, int32_t batch, float* colamax, void* stream) {
+  NV_CHECK(tensor_ok(q) && colamax, NVFP4_ERR_INVALID_ARG);
+  NV_CHECK(batch >= 1 && q->rows >= batch && q->rows % batch == 0 && q->cols >= 64 && q->cols % 64 == 0,
+           NVFP4_ERR_UNSUPPORTED_SHAPE);
+  NV_CHECK(aligned16(colamax), NVFP4_ERR_MISALIGNED);
+  const nvfp4_status d = device_ok();
+  if (d != NVFP4_OK) return d;
+  NV_TRY(launch_dq_colamax(q->codes, q->scales, q->scale_layout, q->tensor_scale, q->rows / batch, q->cols,
+                           batch, colamax, static_cast<cudaStream_t>(stream)));
+  return NVFP4_OK;
+}
+
+nvfp4_status rac_weight_quant_fp4(const nvfp4_tensor* qw, const int32_t* sel, int64_t n_sel,
+                                  const float* dq_colamax, nvfp4_tensor* q_wsel, void* stream) {
+  NV_CHECK(tensor_ok(qw) && sel && dq_colamax && tensor_ok(q_wsel), NVFP4_ERR_INVALID_ARG);
+  const int64_t N = qw->rows, K = qw->cols;
+  NV_CHECK(N >= 1 && K >= 64 && K % 64 == 0 && n_sel >= 1 && n_sel <= K, NVFP4_ERR_UNSUPPORTED_SHAPE);
+  const int64_t width = nvfp4_rac_width(n_sel);
+  NV_CHECK(q_wsel->rows == N && q_wsel->cols == width, NVFP4_ERR_UNSUPPORTED_SHAPE);
+  const nvfp4_status d = device_ok();
+  if (d != NVFP4_OK) return d;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (q_wsel->scale_layout == 1 && N % 128 != 0)
+    NV_TRY(cudaMemsetAsync(q_wsel->scales, 0, scale_bytes(N, width, 1), s));
+  NV_TRY(launch_weight_gather_fp4(qw->codes, qw->scales, qw->scale_layout, qw->tensor_scale, N, K, 1, sel,
+                                  n_sel, width, dq_colamax, q_wsel->tensor_scale, q_wsel->codes,
+                                  q_wsel->scales, q_wsel->scale_layout, s));
+  return NVFP4_OK;
+}
+
 static nvfp4_status gemm_checked(const nvfp4_tensor* qa, const nvfp4_tensor* qb, const nvfp4_tensor* qr,
                                  const nvfp4_tensor* qws, void* y, int32_t y_dtype, int64_t ldy,
                                  cudaStream_t s) {
@@ -340,13 +370,15 @@ nvfp4_status w4a4_rac_gemm(const nvfp4_tensor* qx, const nvfp4_tensor* q_res_or_
     return gemm_checked(qx, qw, nullptr, nullptr, y, y_dtype, ldy, s);
   const int64_t K = qx->cols;
   const int64_t width = nvfp4_rac_width(n_sel);
-  NV_CHECK(w && sel && w_colamax, NVFP4_ERR_INVALID_ARG);
-  NV_CHECK(n_sel <= K && q_res_or_null->cols == width, NVFP4_ERR_UNSUPPORTED_SHAPE);
+  NV_CHECK(sel && w_colamax, NVFP4_ERR_INVALID_ARG);
+  NV_CHECK(n_sel <= K && q_res_or_null->cols == width && qw->cols == K, NVFP4_ERR_UNSUPPORTED_SHAPE);
   Carver c(ws);
   const GemmWs gw = carve_gemm(c, N, width);
   NV_CHECK(ws != nullptr && ws_bytes >= c.off, NVFP4_ERR_WORKSPACE);
   nvfp4_tensor wsel{gw.codes, gw.scales, gw.st, N, width, 1};
-  const nvfp4_status r = rac_weight_quant(w, N, K, ldw, sel, n_sel, w_colamax, &wsel, stream);
+  // W_sel from the bf16 weight, or (w == NULL) from Q(W) itself
+  const nvfp4_status r = w ? rac_weight_quant(w, N, K, ldw, sel, n_sel, w_colamax, &wsel, stream)
+                           : rac_weight_quant_fp4(qw, sel, n_sel, w_colamax, &wsel, stream);
   if (r != NVFP4_OK) return r;
   return gemm_checked(qx, qw, q_res_or_null, &wsel, y, y_dtype, ldy, s);
 }
@@ -357,14 +389,14 @@ nvfp4_status moe_grouped_w4a4_rac_gemm(const uint16_t* x_perm, int64_t T, int64_
                                        float k_percent, void* y_perm, int32_t y_dtype,
                                        uint8_t* masks_or_null, void* ws, size_t ws_bytes,
                                        void* stream) {
-  NV_CHECK(x_perm && offsets_dev && w && tensor_ok(qw) && w_colamax && y_perm, NVFP4_ERR_INVALID_ARG);
+  NV_CHECK(x_perm && offsets_dev && tensor_ok(qw) && w_colamax && y_perm, NVFP4_ERR_INVALID_ARG);
   NV_CHECK(k_percent >= 0.0f && k_percent <= 100.0f && (y_dtype == 0 || y_dtype == 1),
            NVFP4_ERR_INVALID_ARG);
   NV_CHECK(E >= 1 && E <= 4096 && T >= 1 && K >= 64 && K % 64 == 0 && N >= 128 && N % 128 == 0,
            NVFP4_ERR_UNSUPPORTED_SHAPE);
   NV_CHECK(qw->scale_layout == 1 && qw->rows == static_cast<int64_t>(E) * N && qw->cols == K,
            NVFP4_ERR_UNSUPPORTED_SHAPE);
-  NV_CHECK(aligned16(x_perm) && aligned16(w) && aligned16(y_perm), NVFP4_ERR_MISALIGNED);
+  NV_CHECK(aligned16(x_perm) && aligned16(w) && aligned16(y_perm), NVFP4_ERR_MISALIGNED);   // w may be NULL
   const int64_t n_sel = nvfp4_rac_nsel(k_percent, K);
   const int64_t width = nvfp4_rac_width(n_sel);
   Carver c(ws);
@@ -395,8 +427,12 @@ nvfp4_status moe_grouped_w4a4_rac_gemm(const uint16_t* x_perm, int64_t T, int64_
   if (n_sel > 0) {
     NV_TRY(launch_residual_gather(x_perm, T, K, K, g, prows, m.qx_codes, m.qx_scales, 1, m.qx_st, m.sel,
                                   n_sel, width, m.r_st, m.r_codes, m.r_scales, 1, s));
-    NV_TRY(launch_weight_gather(w, N, K, K, E, m.sel, n_sel, width, w_colamax, m.ws_st, m.ws_codes,
-                                m.ws_scales, 1, s));
+    if (w)
+      NV_TRY(launch_weight_gather(w, N, K, K, E, m.sel, n_sel, width, w_colamax, m.ws_st, m.ws_codes,
+                                  m.ws_scales, 1, s));
+    else
+      NV_TRY(launch_weight_gather_fp4(qw->codes, qw->scales, 1, qw->tensor_scale, N, K, E, m.sel, n_sel,
+                                      width, w_colamax, m.ws_st, m.ws_codes, m.ws_scales, 1, s));
     a.a1 = {m.r_codes, m.r_scales, m.r_st, prows, width};
     a.b1 = {m.ws_codes, m.ws_scales, m.ws_st, static_cast<int64_t>(E) * N, width};
   }

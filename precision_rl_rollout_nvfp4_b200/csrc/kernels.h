@@ -124,6 +124,18 @@ cudaError_t launch_weight_gather(const uint16_t* w, int64_t N, int64_t K, int64_
                                  const float* colamax, float* s_t, uint8_t* codes, uint8_t* scales,
                                  int layout, cudaStream_t s);
 
+// W_sel re-quantized from the NVFP4 weight alone (codes, scales, tensor
+// scales w_st[E] of E stacked N x K matrices): the values are DQ(Q(W)) and
+// dq_colamax [E, K] holds max_n |DQ(Q(W))_nk| (launch_dq_colamax).
+cudaError_t launch_weight_gather_fp4(const uint8_t* w_codes, const uint8_t* w_scales, int w_layout,
+                                     const float* w_st, int64_t N, int64_t K, int32_t E,
+                                     const int32_t* sel, int64_t n_sel, int64_t width,
+                                     const float* dq_colamax, float* s_t, uint8_t* codes,
+                                     uint8_t* scales, int layout, cudaStream_t s);
+// colamax [batch, K] = max over the N rows of each stacked matrix of |DQ|.
+cudaError_t launch_dq_colamax(const uint8_t* codes, const uint8_t* scales, int layout, const float* st,
+                              int64_t N, int64_t K, int32_t batch, float* colamax, cudaStream_t s);
+
 // W' = bf16(DQ(Q(W))) for `batch` matrices; optional Q(W) and colamax
 // (colamax_bits zeroed beforehand, written as fp32 bits).  amax of matrix b:
 // max of amax_parts[b * n_parts .. + n_parts).

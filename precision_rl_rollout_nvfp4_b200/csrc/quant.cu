@@ -338,9 +338,15 @@ constexpr int kGThreads = 256;
 // Tiles are visited grid-stride.  With fuse_scale (one weight) the W_sel
 // tensor scale max_{j in sel} colamax_j / 2688 is reduced during the first
 // tile, its loads issued beside that tile's gather loads; CTA 0 publishes it.
+//
+// MODE 0: W_sel from the bf16 weight `src`;
+// MODE 1: the residual dX_sel from X (`src`) and Q(X) (`qx_*`);
+// MODE 2: W_sel from the NVFP4 weight alone: the gathered values are
+//         DQ(Q(W)) decoded from its codes and scales (`qx_*`, tensor scale
+//         qx_st[e]); `src` is unused and colamax holds max_n |DQ(Q(W))_nj|.
 constexpr int kGRows = 16, kGCols = 256;
 
-template <bool RESIDUAL>
+template <int MODE>
 __global__ void __launch_bounds__(kGThreads)
 gather_quant_kernel(const uint16_t* __restrict__ src, int64_t K, int64_t ld, RowGroups g,
                     int64_t N_per_group, const uint8_t* __restrict__ qx_codes,
@@ -349,6 +355,7 @@ gather_quant_kernel(const uint16_t* __restrict__ src, int64_t K, int64_t ld, Row
                     const float* __restrict__ colamax, int fuse_scale, float* __restrict__ out_st,
                     uint8_t* __restrict__ out_codes, uint8_t* __restrict__ out_scales, int out_layout,
                     int64_t out_rows, int64_t grid_rows) {
+  constexpr bool RESIDUAL = MODE == 1, FP4 = MODE == 2, CODES = MODE != 0;
   pdl_wait();
   pdl_launch_dependents();
   __shared__ __align__(16) float s_val[kGRows][kGCols + 4];
@@ -357,7 +364,7 @@ gather_quant_kernel(const uint16_t* __restrict__ src, int64_t K, int64_t ld, Row
   __shared__ float s_wm[kGThreads / 32];
   __shared__ ScaleTable T;
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-  if (RESIDUAL) {
+  if (CODES) {
     if (t < 16) s_e2m1[t] = e2m1_to_f32(static_cast<uint32_t>(t));
     if (t < 128) s_e4m3[t] = t < 127 ? e4m3_to_f32(static_cast<uint32_t>(t)) : 0.0f;
   }
@@ -402,7 +409,7 @@ gather_quant_kernel(const uint16_t* __restrict__ src, int64_t K, int64_t ld, Row
       fc[u] = (do_fuse && jf < n_sel) ? __ldg(sel + jf) : -1;
     }
     // level 2: the values (and the fused scale's colamax share)
-    const float st_x = (RESIDUAL && valid) ? qx_st[e] : 0.0f;
+    const float st_x = (CODES && valid) ? qx_st[e] : 0.0f;
     const int64_t k4 = (K + 63) / 64;
 #pragma unroll
     for (int rr = 0; rr < 2; ++rr) {
@@ -410,10 +417,10 @@ gather_quant_kernel(const uint16_t* __restrict__ src, int64_t K, int64_t ld, Row
       const int64_t srow = row_base + r;
       const int64_t prow = r0 + r;
       const bool live = valid && srow < row_end;
-      const uint16_t* xrow = src + srow * ld;
-      const uint8_t* crow = RESIDUAL ? qx_codes + prow * (K / 2) : nullptr;
+      const uint16_t* xrow = FP4 ? nullptr : src + srow * ld;
+      const uint8_t* crow = CODES ? qx_codes + prow * (K / 2) : nullptr;
       const uint8_t* srow_sc = nullptr;
-      if (RESIDUAL)
+      if (CODES)
         srow_sc = qx_layout == 1
                       ? qx_scales + ((prow >> 7) * k4) * 512 + (prow & 31) * 16 + ((prow & 127) >> 5) * 4
                       : qx_scales + prow * (K / kBlock);
@@ -422,8 +429,8 @@ gather_quant_kernel(const uint16_t* __restrict__ src, int64_t K, int64_t ld, Row
       for (int u = 0; u < 8; ++u) {
         const bool ok = live && static_cast<uint32_t>(c[u]) < K32;   // never false for a valid sel list
         const uint32_t cc = ok ? static_cast<uint32_t>(c[u]) : 0u;
-        xb[u] = ok ? __ldg(xrow + cc) : 0u;
-        if (RESIDUAL) {
+        xb[u] = (ok && !FP4) ? __ldg(xrow + cc) : 0u;
+        if (CODES) {
           cb[u] = ok ? __ldg(crow + (cc >> 1)) : 0u;
           const uint32_t so = qx_layout == 1 ? (cc >> 6) * 512u + ((cc >> 4) & 3u) : (cc >> 4);
           sb[u] = ok ? __ldg(srow_sc + so) : 0u;
@@ -433,10 +440,12 @@ gather_quant_kernel(const uint16_t* __restrict__ src, int64_t K, int64_t ld, Row
       for (int u = 0; u < 8; ++u) {
         float v = 0.0f;
         if (live && static_cast<uint32_t>(c[u]) < K32) {
-          v = bf16_bits_to_f32(xb[u]);
-          if (RESIDUAL) {
+          if (CODES) {
             const float q = s_e2m1[(cb[u] >> ((c[u] & 1) << 2)) & 15u];
-            v = __fsub_rn(v, __fmul_rn(__fmul_rn(q, s_e4m3[sb[u] & 127u]), st_x));
+            const float dq = __fmul_rn(__fmul_rn(q, s_e4m3[sb[u] & 127u]), st_x);
+            v = FP4 ? dq : __fsub_rn(bf16_bits_to_f32(xb[u]), dq);
+          } else {
+            v = bf16_bits_to_f32(xb[u]);
           }
         }
         s_val[r][lane + 32 * u] = v;
@@ -499,6 +508,62 @@ gather_quant_kernel(const uint16_t* __restrict__ src, int64_t K, int64_t ld, Row
 }
 
 // s_t[e] = RN(max_{j < n_sel} colamax[e*K + sel[e*n_sel + j]] / 2688), one CTA per group.
+// Column maxima of |DQ(Q(W))| for `batch` stacked NVFP4 matrices of N rows
+// each: colamax[e][j] = max_n |DQ_{e,n,j}|.  E2M1dec(code) * E4M3dec(scale)
+// is exact in fp32 (at most 6 significant bits) and RN(p * s_t) does not
+// decrease as p grows, so the maximum is taken over the exact products and
+// scaled once.  A CTA covers 128 rows x 64 columns: thread = (row t/4 and
+// t/4 + 64, 16-column block t%4); rows reduce by shuffles within the warp,
+// warps through shared memory, CTAs by an integer atomicMax on the bits of
+// the non-negative results (colamax zeroed beforehand).
+__global__ void __launch_bounds__(256)
+dq_colamax_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales, int layout,
+                  const float* __restrict__ st, int64_t N, int64_t K, unsigned* __restrict__ colamax) {
+  pdl_wait();
+  pdl_launch_dependents();
+  __shared__ float s_mag[8];
+  __shared__ float s_part[8][64];
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5, b = t & 3;
+  const int e = blockIdx.z;
+  const int64_t c0 = static_cast<int64_t>(blockIdx.x) * 64;
+  if (t < 8) s_mag[t] = e2m1_to_f32(static_cast<uint32_t>(t));
+  __syncthreads();
+  float m[16];
+#pragma unroll
+  for (int u = 0; u < 16; ++u) m[u] = 0.0f;
+#pragma unroll
+  for (int rr = 0; rr < 2; ++rr) {
+    const int64_t n = static_cast<int64_t>(blockIdx.y) * 128 + (t >> 2) + 64 * rr;
+    if (n < N) {
+      const int64_t row = static_cast<int64_t>(e) * N + n;
+      const uint2 w = __ldg(reinterpret_cast<const uint2*>(codes + row * (K / 2) + c0 / 2 + 8 * b));
+      const float sv = e4m3_to_f32(__ldg(scales + scale_offset(row, c0 / kBlock + b, K, layout)) & 127u);
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        const uint32_t word = u < 8 ? w.x : w.y;
+        m[u] = fmaxf(m[u], __fmul_rn(s_mag[(word >> (4 * (u & 7))) & 7u], sv));
+      }
+    }
+  }
+#pragma unroll
+  for (int u = 0; u < 16; ++u) {
+    m[u] = fmaxf(m[u], __shfl_xor_sync(0xFFFFFFFFu, m[u], 4));
+    m[u] = fmaxf(m[u], __shfl_xor_sync(0xFFFFFFFFu, m[u], 8));
+    m[u] = fmaxf(m[u], __shfl_xor_sync(0xFFFFFFFFu, m[u], 16));
+  }
+  if (lane < 4) {
+#pragma unroll
+    for (int u = 0; u < 16; ++u) s_part[warp][16 * lane + u] = m[u];
+  }
+  __syncthreads();
+  if (t < 64) {
+    float r = 0.0f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) r = fmaxf(r, s_part[w][t]);
+    atomicMax(colamax + static_cast<int64_t>(e) * K + c0 + t, __float_as_uint(__fmul_rn(r, st[e])));
+  }
+}
+
 __global__ void sel_tensor_scale_kernel(const float* __restrict__ colamax, int64_t K,
                                         const int32_t* __restrict__ sel, int64_t n_sel,
                                         float* __restrict__ s_t) {
@@ -742,7 +807,7 @@ cudaError_t launch_residual_gather(const uint16_t* x, int64_t rows, int64_t K, i
   // rows of the scale buffer are padded to 128 for the tiled layout
   const int64_t grid_rows = r_layout == 1 ? (prows + kTileRows - 1) / kTileRows * kTileRows : prows;
   {
-    const cudaError_t le = launch_k(gather_quant_kernel<true>, dim3(gather_grid(grid_rows, width)), dim3(kGThreads), 0, s, nullptr, 0,
+    const cudaError_t le = launch_k(gather_quant_kernel<1>, dim3(gather_grid(grid_rows, width)), dim3(kGThreads), 0, s, nullptr, 0,
                                    x, K, ldx, g, 0, qx_codes, qx_scales, qx_layout, qx_st, sel, n_sel,
                                    width, nullptr, 0, const_cast<float*>(r_st), r_codes, r_scales,
                                    r_layout, prows, grid_rows);
@@ -774,9 +839,47 @@ cudaError_t launch_weight_gather(const uint16_t* w, int64_t N, int64_t K, int64_
   const int64_t rows = static_cast<int64_t>(E) * N;
   RowGroups none{};
   {
-    const cudaError_t le = launch_k(gather_quant_kernel<false>, dim3(gather_grid(rows, width)), dim3(kGThreads), 0, s, nullptr, 0,
+    const cudaError_t le = launch_k(gather_quant_kernel<0>, dim3(gather_grid(rows, width)), dim3(kGThreads), 0, s, nullptr, 0,
                                    w, K, ldw, none, N, nullptr, nullptr, 0, nullptr, sel, n_sel, width,
                                    colamax, fuse, s_t, codes, scales, layout, rows, rows);
+    if (le != cudaSuccess) return le;
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_weight_gather_fp4(const uint8_t* w_codes, const uint8_t* w_scales, int w_layout,
+                                     const float* w_st, int64_t N, int64_t K, int32_t E,
+                                     const int32_t* sel, int64_t n_sel, int64_t width,
+                                     const float* dq_colamax, float* s_t, uint8_t* codes,
+                                     uint8_t* scales, int layout, cudaStream_t s) {
+  if (width == 0) return cudaSuccess;
+  const int fuse = E == 1 ? 1 : 0;
+  if (!fuse) {
+    cudaError_t e = launch_sel_tensor_scale(dq_colamax, K, sel, n_sel, E, s_t, s);
+    if (e != cudaSuccess) return e;
+  }
+  const int64_t rows = static_cast<int64_t>(E) * N;
+  RowGroups none{};
+  {
+    const cudaError_t le = launch_k(gather_quant_kernel<2>, dim3(gather_grid(rows, width)), dim3(kGThreads), 0, s, nullptr, 0,
+                                   nullptr, K, K, none, N, w_codes, w_scales, w_layout, w_st, sel, n_sel,
+                                   width, dq_colamax, fuse, s_t, codes, scales, layout, rows, rows);
+    if (le != cudaSuccess) return le;
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dq_colamax(const uint8_t* codes, const uint8_t* scales, int layout, const float* st,
+                              int64_t N, int64_t K, int32_t batch, float* colamax, cudaStream_t s) {
+  {
+    const cudaError_t me = cudaMemsetAsync(colamax, 0, sizeof(float) * K * batch, s);
+    if (me != cudaSuccess) return me;
+  }
+  dim3 grid(static_cast<unsigned>(K / 64), static_cast<unsigned>((N + 127) / 128),
+            static_cast<unsigned>(batch));
+  {
+    const cudaError_t le = launch_k(dq_colamax_kernel, dim3(grid), dim3(256), 0, s, nullptr, 0,
+                                   codes, scales, layout, st, N, K, reinterpret_cast<unsigned*>(colamax));
     if (le != cudaSuccess) return le;
   }
   return cudaGetLastError();
