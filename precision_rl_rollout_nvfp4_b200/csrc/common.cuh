@@ -188,18 +188,20 @@ __device__ __forceinline__ BlockQ block_q(float amax_b, const ScaleTable& T) {
   return q;
 }
 
-// Quotients of one block for four fp32 pairs: RN(|v| / sdec) with the sign
+// Quotients of one block for four fp32 pairs: RN(v / sdec) with the sign
 // bit of v (signed zeros when sdec == 0), through div_rn_pos's steps on both
-// lanes at once.
+// lanes at once.  Round-to-nearest-even and the FMA are symmetric under
+// negation, so the correction gives RN(v / sdec) for negative v as well; the
+// final OR only restores the sign of a zero quotient of v = -0 (whose
+// correction sum is +0).
 __device__ __forceinline__ void block_quotients(const uint64_t* x2, const BlockQ& q, uint64_t* out) {
   constexpr uint64_t kSign = 0x8000000080000000ull;
   if (q.sdec > 0.0f && q.rcp != 0.0f) {
     const uint64_t y2 = f2_pack(q.rcp, q.rcp), nb2 = f2_pack(-q.sdec, -q.sdec);
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const uint64_t a = f2_abs(x2[j]);
-      const uint64_t q0 = f2_mul(a, y2);
-      const uint64_t r = f2_fma(q0, nb2, a);          // a - q0 sdec, exact
+      const uint64_t q0 = f2_mul(x2[j], y2);
+      const uint64_t r = f2_fma(q0, nb2, x2[j]);      // v - q0 sdec, exact
       out[j] = f2_fma(r, y2, q0) | (x2[j] & kSign);
     }
   } else {

@@ -508,48 +508,300 @@ gather_quant_kernel(const uint16_t* __restrict__ src, int64_t K, int64_t ld, Row
 }
 
 // s_t[e] = RN(max_{j < n_sel} colamax[e*K + sel[e*n_sel + j]] / 2688), one CTA per group.
+constexpr int kWThreads = 256;
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async4(void* dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// W_sel, staged by rows: the gather + second quantization of the selected
+// weight columns, from the bf16 weight (FP4 = false) or from its NVFP4 codes
+// and scales (FP4 = true: the values are DQ(Q(W)) = RN(RN(e sbv) s_t)).
+//
+// A thread owns output 16-blocks and keeps their 16 channel indices in
+// registers for every row of the matrix (a padded channel reads element K of
+// the staged row, which is zero), so per element and row a gather is one
+// shared-memory load.  With nblk = width / 16 output blocks per row:
+//   nblk <= blockDim: P = blockDim / nblk threads share a block, each taking
+//                     the rows slot = phase + P k (k < RPT) of a pass;
+//   nblk >  blockDim: one thread per block and row (blocks t + blockDim i;
+//                     blockDim = nblk rounded up to 32, at most 512).
+// A pass is R = P RPT consecutive rows of one matrix (R | N when E > 1); a
+// CTA takes a contiguous range of passes and double-buffers them: the next
+// pass's rows are copied with cp.async (16-byte copies, 4-byte copies for
+// the NVFP4 scale words) while the current pass computes.  NVFP4 rows are
+// then expanded once per pass, cooperatively and coalesced, into the exact
+// products E2M1dec(code) E4M3dec(scale) as f16 (at most 6 significant bits
+// in [2^-10, 2688], so exact), through the hardware e2m1x2 / e4m3x2 -> f16x2
+// conversions; the gather reads those and applies RN(p s_t) in fp32.
+// With fuse_scale (one matrix) each CTA reduces the W_sel tensor scale
+// max_{j in sel} colamax_j / 2688 from its own blocks' channels.
+struct WselGeom {
+  int P, RPT, R, nob;          // threads per block, rows per thread, rows per pass, blocks per thread
+  uint32_t rowbytes, rawbytes; // staged row (2K + 16) and raw NVFP4 row (K/2 + K/16, to 16 bytes)
+};
+
+__device__ __forceinline__ uint32_t dup_e4m3_to_h2(uint32_t sb) {
+  uint32_t h;
+  const uint32_t two = (sb & 0x7Fu) * 0x0101u;
+  asm("{\n\t.reg .b16 t;\n\tcvt.u16.u32 t, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, t;\n\t}" : "=r"(h) : "r"(two));
+  return h;
+}
+__device__ __forceinline__ uint32_t e2m1x2_h2(uint32_t byte) {
+  uint32_t h;
+  asm("{\n\t.reg .b8 t;\n\tcvt.u8.u32 t, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, t;\n\t}" : "=r"(h) : "r"(byte));
+  return h;
+}
+__device__ __forceinline__ uint32_t h2mul(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+template <bool FP4>
+__global__ void __launch_bounds__(512, 2)
+wsel_rows_kernel(const uint16_t* __restrict__ w, int64_t ldw, const uint8_t* __restrict__ codes,
+                 const uint8_t* __restrict__ scales, int layout, const float* __restrict__ w_st, int64_t N,
+                 int64_t K, int32_t E, const int32_t* __restrict__ sel, int64_t n_sel, int64_t width,
+                 const float* __restrict__ colamax, int fuse_scale, float* __restrict__ out_st,
+                 uint8_t* __restrict__ out_codes, uint8_t* __restrict__ out_scales, int out_layout,
+                 WselGeom g) {
+  pdl_wait();
+  pdl_launch_dependents();
+  extern __shared__ __align__(16) uint8_t ws_smem[];
+  __shared__ ScaleTable T;
+  __shared__ float s_wm[32];
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5, nthr = blockDim.x;
+  const uint32_t Ku = static_cast<uint32_t>(K), half = Ku / 2u;
+  const int nblk = static_cast<int>(width / kBlock);
+  const uint32_t R = static_cast<uint32_t>(g.R);
+  // shared memory: [staged rows, 2 buffers (bf16) or 1 (NVFP4)][raw NVFP4 rows, 2 buffers]
+  const uint32_t nbuf_rows = FP4 ? 1u : 2u;
+  const uint32_t raw0 = nbuf_rows * R * g.rowbytes;
+  // zero the tails (element K onwards) of every staged row once: copies and
+  // the expansion write only elements 0 .. K-1
+  for (uint32_t r = t; r < nbuf_rows * R; r += nthr)
+    *reinterpret_cast<uint4*>(ws_smem + r * g.rowbytes + 2u * Ku) = make_uint4(0u, 0u, 0u, 0u);
+  // this thread's blocks and row phase
+  const bool shared_blocks = nblk <= nthr;
+  const int phase = shared_blocks ? t / nblk : 0;
+  const bool active = phase < g.P;
+  const int ob0 = shared_blocks ? t % nblk : t;
+  const int64_t rows = static_cast<int64_t>(E) * N;
+  const int64_t passes = (rows + R - 1) / R;
+  const int64_t p0 = static_cast<int64_t>(blockIdx.x) * passes / gridDim.x;
+  const int64_t p1 = static_cast<int64_t>(blockIdx.x + 1) * passes / gridDim.x;
+  auto stage = [&](int64_t p, uint32_t b) {
+    const int64_t r0 = p * R;
+    const uint32_t nrows = static_cast<uint32_t>(rows - r0 < R ? rows - r0 : R);
+    for (uint32_t r = 0; r < nrows; ++r) {
+      if (FP4) {
+        const uint32_t ro = raw0 + (b * R + r) * g.rawbytes;
+        const uint8_t* src = codes + (r0 + r) * static_cast<int64_t>(half);
+        for (uint32_t q = t; q < half / 16u; q += nthr) cp_async16(ws_smem + ro + 16u * q, src + 16u * q);
+        for (uint32_t q = t; q < Ku / 64u; q += nthr)
+          cp_async4(ws_smem + ro + half + 4u * q, scales + scale_offset(r0 + r, 4 * q, K, layout));
+      } else {
+        const uint32_t ro = (b * R + r) * g.rowbytes;
+        const uint16_t* src = w + (r0 + r) * ldw;
+        for (uint32_t q = t; q < Ku / 8u; q += nthr) cp_async16(ws_smem + ro + 16u * q, src + 8u * q);
+      }
+    }
+    cp_async_commit();
+  };
+  // channel indices of the thread's block ob (K for padding)
+  auto load_idx = [&](int e, int ob, uint32_t* c) {
+    const int32_t* sel_e = sel + static_cast<int64_t>(e) * n_sel;
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+      const int64_t j = static_cast<int64_t>(ob) * kBlock + u;
+      const int32_t v = j < n_sel ? __ldg(sel_e + j) : -1;
+      c[u] = (v >= 0 && v < K) ? static_cast<uint32_t>(v) : Ku;
+    }
+  };
+  uint32_t cidx[16];
+#pragma unroll
+  for (int u = 0; u < 16; ++u) cidx[u] = Ku;
+  if (p0 < p1) stage(p0, 0u);
+  int cur_e = -1;
+  float st_w = 0.0f;
+  for (int64_t p = p0; p < p1; ++p) {
+    const uint32_t b = static_cast<uint32_t>((p - p0) & 1);
+    if (p + 1 < p1) stage(p + 1, b ^ 1u);
+    const int64_t r0 = p * R;
+    const int e = static_cast<int>(r0 / N);
+    const uint32_t nrows = static_cast<uint32_t>(rows - r0 < R ? rows - r0 : R);
+    if (e != cur_e) {                              // uniform over the CTA; overlaps the copies in flight
+      if (g.nob == 1 && active && ob0 < nblk) load_idx(e, ob0, cidx);
+      float st;
+      if (fuse_scale) {
+        float m = 0.0f;
+        for (int i = 0; i < g.nob; ++i) {
+          const int ob = ob0 + i * nthr;
+          if (!active || phase != 0 || ob >= nblk) continue;
+          if (g.nob > 1) load_idx(e, ob, cidx);
+#pragma unroll
+          for (int u = 0; u < 16; ++u)
+            if (cidx[u] < Ku) m = fmaxf(m, __ldg(colamax + cidx[u]));
+        }
+        m = __uint_as_float(__reduce_max_sync(0xFFFFFFFFu, __float_as_uint(m)));
+        if (lane == 0) s_wm[warp] = m;
+        __syncthreads();
+        float r = 0.0f;
+        for (int k = 0; k < (nthr >> 5); ++k) r = fmaxf(r, s_wm[k]);
+        st = __fdiv_rn(r, kTensorScaleDiv);
+        if (blockIdx.x == 0 && t == 0) out_st[0] = st;
+      } else {
+        st = out_st[e];
+      }
+      __syncthreads();                             // the previous matrix's table is no longer read
+      build_scale_table(T, st, t);
+      if (FP4) st_w = w_st[e];
+      cur_e = e;
+    }
+    if (p + 1 < p1) {
+      cp_async_wait<1>();                          // this thread's copies of pass p are done
+    } else {
+      cp_async_wait<0>();
+    }
+    __syncthreads();                               // copies (and the scale table) are visible
+    const uint32_t rows0 = FP4 ? 0u : b * R * g.rowbytes;
+    if (FP4) {
+      // expand the raw rows into exact f16 products, 8 elements per step
+      const uint32_t steps = half / 4u;            // 32-bit code words per row
+      for (uint32_t r = 0; r < nrows; ++r) {
+        const uint32_t ro = raw0 + (b * R + r) * g.rawbytes;
+        uint8_t* dst = ws_smem + r * g.rowbytes;
+        for (uint32_t q = t; q < steps; q += nthr) {
+          const uint32_t wd = *reinterpret_cast<const uint32_t*>(ws_smem + ro + 4u * q);
+          const uint32_t sv = dup_e4m3_to_h2(ws_smem[ro + half + (q >> 1)]);
+          uint4 o;
+          o.x = h2mul(e2m1x2_h2(wd & 0xFFu), sv);
+          o.y = h2mul(e2m1x2_h2((wd >> 8) & 0xFFu), sv);
+          o.z = h2mul(e2m1x2_h2((wd >> 16) & 0xFFu), sv);
+          o.w = h2mul(e2m1x2_h2(wd >> 24), sv);
+          *reinterpret_cast<uint4*>(dst + 16u * q) = o;
+        }
+      }
+      __syncthreads();
+    }
+    if (active) {
+      for (int i = 0; i < g.nob; ++i) {
+        const int ob = ob0 + i * nthr;
+        if (ob >= nblk) break;
+        if (g.nob > 1) load_idx(e, ob, cidx);
+        for (int k = 0; k < g.RPT; ++k) {
+          const uint32_t slot = static_cast<uint32_t>(phase + g.P * k);
+          if (slot >= nrows) break;
+          const uint8_t* rb = ws_smem + rows0 + slot * g.rowbytes;
+          float v[16];
+          float am = 0.0f;
+#pragma unroll
+          for (int u = 0; u < 16; ++u) {
+            const uint32_t h = *reinterpret_cast<const uint16_t*>(rb + 2u * cidx[u]);
+            float x;
+            if (FP4)
+              x = __fmul_rn(__half2float(__ushort_as_half(static_cast<unsigned short>(h))), st_w);
+            else
+              x = __uint_as_float(h << 16);
+            v[u] = x;
+            am = fmaxf(am, fabsf(x));
+          }
+          const int64_t row = r0 + slot;
+          const BlockQ bq = block_q(am, T);
+          const uint32_t lo = encode8_q(v, bq), hi = encode8_q(v + 8, bq);
+          *reinterpret_cast<uint2*>(out_codes + row * (width / 2) + static_cast<int64_t>(ob) * 8) =
+              make_uint2(lo, hi);
+          out_scales[scale_offset(row, ob, width, out_layout)] = static_cast<uint8_t>(bq.sb);
+        }
+      }
+    }
+    __syncthreads();                               // staged rows and buffer b are free again
+  }
+}
+
+// Exact values of the two E2M1 codes of a byte (low nibble in the low half)
+// and of two E4M3 scale bytes (low byte in the low half) as f16x2, through
+// the hardware conversions; both are exact in f16.
+__device__ __forceinline__ uint32_t e2m1x2_to_h2(uint32_t byte) {
+  uint32_t h;
+  asm("{\n\t.reg .b8 t;\n\tcvt.u8.u32 t, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, t;\n\t}" : "=r"(h) : "r"(byte));
+  return h;
+}
+__device__ __forceinline__ uint32_t e4m3x2_to_h2(uint32_t two) {
+  uint32_t h;
+  asm("{\n\t.reg .b16 t;\n\tcvt.u16.u32 t, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, t;\n\t}" : "=r"(h) : "r"(two));
+  return h;
+}
+__device__ __forceinline__ uint32_t h2_mul(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+__device__ __forceinline__ uint32_t h2_max(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
 // Column maxima of |DQ(Q(W))| for `batch` stacked NVFP4 matrices of N rows
-// each: colamax[e][j] = max_n |DQ_{e,n,j}|.  E2M1dec(code) * E4M3dec(scale)
-// is exact in fp32 (at most 6 significant bits) and RN(p * s_t) does not
-// decrease as p grows, so the maximum is taken over the exact products and
-// scaled once.  A CTA covers 128 rows x 64 columns: thread = (row t/4 and
-// t/4 + 64, 16-column block t%4); rows reduce by shuffles within the warp,
-// warps through shared memory, CTAs by an integer atomicMax on the bits of
-// the non-negative results (colamax zeroed beforehand).
+// each: colamax[e][j] = max_n |DQ_{e,n,j}|.  |E2M1dec(code)| E4M3dec(scale)
+// has at most 6 significant bits and lies in [2^-10, 2688] (or is 0), so it
+// is exact in f16 and the products and their maxima run on f16 pairs; RN(p
+// s_t) does not decrease as p grows, so the maximum over the exact products
+// is scaled once, in fp32.  A CTA covers 128 columns x 256 rows: thread =
+// (32-column slice t%4, rows t/4 + 64 i), one 16-byte code load and one
+// 2-byte scale load per row; rows reduce by shuffles within the warp, warps
+// through shared memory, CTAs by an integer atomicMax on the bits of the
+// non-negative results (colamax zeroed beforehand).
+constexpr int kCmRows = 256;
+
 __global__ void __launch_bounds__(256)
 dq_colamax_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales, int layout,
                   const float* __restrict__ st, int64_t N, int64_t K, unsigned* __restrict__ colamax) {
   pdl_wait();
   pdl_launch_dependents();
-  __shared__ float s_mag[8];
-  __shared__ float s_part[8][64];
-  const int t = threadIdx.x, lane = t & 31, warp = t >> 5, b = t & 3;
+  __shared__ uint32_t s_part[8][64];
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5, cg = t & 3;
   const int e = blockIdx.z;
-  const int64_t c0 = static_cast<int64_t>(blockIdx.x) * 64;
-  if (t < 8) s_mag[t] = e2m1_to_f32(static_cast<uint32_t>(t));
-  __syncthreads();
-  float m[16];
+  const int64_t c0 = static_cast<int64_t>(blockIdx.x) * 128 + 32 * cg;   // first column of the slice
+  const bool cols_ok = c0 < K;
+  uint32_t m[16];
 #pragma unroll
-  for (int u = 0; u < 16; ++u) m[u] = 0.0f;
+  for (int u = 0; u < 16; ++u) m[u] = 0u;
+  if (cols_ok) {
 #pragma unroll
-  for (int rr = 0; rr < 2; ++rr) {
-    const int64_t n = static_cast<int64_t>(blockIdx.y) * 128 + (t >> 2) + 64 * rr;
-    if (n < N) {
-      const int64_t row = static_cast<int64_t>(e) * N + n;
-      const uint2 w = __ldg(reinterpret_cast<const uint2*>(codes + row * (K / 2) + c0 / 2 + 8 * b));
-      const float sv = e4m3_to_f32(__ldg(scales + scale_offset(row, c0 / kBlock + b, K, layout)) & 127u);
+    for (int i = 0; i < kCmRows / 64; ++i) {
+      const int64_t n = static_cast<int64_t>(blockIdx.y) * kCmRows + (t >> 2) + 64 * i;
+      if (n < N) {
+        const int64_t row = static_cast<int64_t>(e) * N + n;
+        const uint4 w = ld_nc_v4(codes + row * (K / 2) + c0 / 2);
+        const uint32_t sb2 = __ldg(reinterpret_cast<const uint16_t*>(scales + scale_offset(row, c0 / kBlock, K, layout)));
+        const uint32_t sv = e4m3x2_to_h2(sb2 & 0x7F7Fu);
+        const uint32_t sv0 = __byte_perm(sv, 0, 0x1010), sv1 = __byte_perm(sv, 0, 0x3232);
+        const uint32_t wd[4] = {w.x & 0x77777777u, w.y & 0x77777777u, w.z & 0x77777777u, w.w & 0x77777777u};
 #pragma unroll
-      for (int u = 0; u < 16; ++u) {
-        const uint32_t word = u < 8 ? w.x : w.y;
-        m[u] = fmaxf(m[u], __fmul_rn(s_mag[(word >> (4 * (u & 7))) & 7u], sv));
+        for (int q = 0; q < 4; ++q) {
+#pragma unroll
+          for (int b = 0; b < 4; ++b) {
+            const uint32_t pr = h2_mul(e2m1x2_to_h2((wd[q] >> (8 * b)) & 0xFFu), q < 2 ? sv0 : sv1);
+            m[4 * q + b] = h2_max(m[4 * q + b], pr);
+          }
+        }
       }
     }
   }
 #pragma unroll
   for (int u = 0; u < 16; ++u) {
-    m[u] = fmaxf(m[u], __shfl_xor_sync(0xFFFFFFFFu, m[u], 4));
-    m[u] = fmaxf(m[u], __shfl_xor_sync(0xFFFFFFFFu, m[u], 8));
-    m[u] = fmaxf(m[u], __shfl_xor_sync(0xFFFFFFFFu, m[u], 16));
+    m[u] = h2_max(m[u], __shfl_xor_sync(0xFFFFFFFFu, m[u], 4));
+    m[u] = h2_max(m[u], __shfl_xor_sync(0xFFFFFFFFu, m[u], 8));
+    m[u] = h2_max(m[u], __shfl_xor_sync(0xFFFFFFFFu, m[u], 16));
   }
   if (lane < 4) {
 #pragma unroll
@@ -557,10 +809,17 @@ dq_colamax_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__
   }
   __syncthreads();
   if (t < 64) {
-    float r = 0.0f;
+    uint32_t r = 0u;
 #pragma unroll
-    for (int w = 0; w < 8; ++w) r = fmaxf(r, s_part[w][t]);
-    atomicMax(colamax + static_cast<int64_t>(e) * K + c0 + t, __float_as_uint(__fmul_rn(r, st[e])));
+    for (int w = 0; w < 8; ++w) r = h2_max(r, s_part[w][t]);
+    const int64_t c = static_cast<int64_t>(blockIdx.x) * 128 + 2 * t;   // columns c, c + 1
+    if (c < K) {
+      const float s = st[e];
+      const float lo = __half2float(__ushort_as_half(static_cast<unsigned short>(r & 0xFFFFu)));
+      const float hi = __half2float(__ushort_as_half(static_cast<unsigned short>(r >> 16)));
+      atomicMax(colamax + static_cast<int64_t>(e) * K + c, __float_as_uint(__fmul_rn(lo, s)));
+      atomicMax(colamax + static_cast<int64_t>(e) * K + c + 1, __float_as_uint(__fmul_rn(hi, s)));
+    }
   }
 }
 
@@ -826,6 +1085,75 @@ cudaError_t launch_sel_tensor_scale(const float* colamax, int64_t K, const int32
   return cudaGetLastError();
 }
 
+namespace {
+// Launch shape of wsel_rows_kernel; ok == false when its shared memory would
+// not fit or K is past 16-bit channel offsets (the generic gather runs
+// instead).
+struct WselPlan {
+  WselGeom g;
+  int threads;
+  size_t smem;
+  bool ok;
+};
+WselPlan wsel_plan(int64_t N, int64_t K, int32_t E, int64_t width, bool fp4) {
+  // at most 54 KB of rows keeps four CTAs (the register limit) on an SM
+  constexpr size_t kBudget = 54 * 1024, kMax = 200 * 1024;
+  WselPlan w{};
+  const int64_t nblk = width / kBlock;
+  w.threads = nblk <= 256 ? 256 : static_cast<int>(nblk < 512 ? (nblk + 31) / 32 * 32 : 512);
+  int P = nblk <= w.threads ? static_cast<int>(w.threads / nblk) : 1;
+  if (E > 1)
+    while (P & (P - 1)) P &= P - 1;                // a power of two, so passes never straddle matrices
+  int RPT = 4;
+  w.g.rowbytes = static_cast<uint32_t>(2 * K + 16);
+  w.g.rawbytes = static_cast<uint32_t>((K / 2 + K / kBlock + 15) / 16 * 16);
+  auto bytes = [&](int r) {
+    return fp4 ? static_cast<size_t>(r) * (w.g.rowbytes + 2 * w.g.rawbytes)
+               : static_cast<size_t>(2 * r) * w.g.rowbytes;
+  };
+  while (bytes(P * RPT) > kBudget || (E > 1 && N % (P * RPT) != 0)) {
+    if (RPT > 1) RPT /= 2;
+    else if (P > 1) P /= 2;
+    else break;
+  }
+  w.g.P = P;
+  w.g.RPT = RPT;
+  w.g.R = P * RPT;
+  w.g.nob = static_cast<int>((nblk + w.threads - 1) / w.threads);
+  w.smem = bytes(w.g.R);
+  w.ok = K <= 65472 && w.smem <= kMax && (E == 1 || N % w.g.R == 0);
+  return w;
+}
+
+template <bool FP4>
+cudaError_t launch_wsel_rows(const WselPlan& wp, const uint16_t* w, int64_t ldw, const uint8_t* w_codes,
+                             const uint8_t* w_scales, int w_layout, const float* w_st, int64_t N, int64_t K,
+                             int32_t E, const int32_t* sel, int64_t n_sel, int64_t width,
+                             const float* colamax, int fuse, float* s_t, uint8_t* codes, uint8_t* scales,
+                             int layout, cudaStream_t s) {
+  static bool attr_set = false;
+  if (!attr_set) {
+    const cudaError_t ae = cudaFuncSetAttribute(wsel_rows_kernel<FP4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                200 * 1024);
+    if (ae != cudaSuccess) return ae;
+    attr_set = true;
+  }
+  int per_sm = 0;
+  const cudaError_t oe =
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, wsel_rows_kernel<FP4>, wp.threads, wp.smem);
+  if (oe != cudaSuccess) return oe;
+  const int64_t rows = static_cast<int64_t>(E) * N;
+  const int64_t passes = (rows + wp.g.R - 1) / wp.g.R;
+  const int64_t cap = static_cast<int64_t>(sm_count()) * (per_sm > 0 ? per_sm : 1);
+  const unsigned grid = static_cast<unsigned>(passes < cap ? passes : cap);
+  const cudaError_t le = launch_k(wsel_rows_kernel<FP4>, dim3(grid), dim3(wp.threads), wp.smem, s, nullptr, 0,
+                                  w, ldw, w_codes, w_scales, w_layout, w_st, N, K, E, sel, n_sel, width, colamax,
+                                  fuse, s_t, codes, scales, layout, wp.g);
+  if (le != cudaSuccess) return le;
+  return cudaGetLastError();
+}
+}  // namespace
+
 cudaError_t launch_weight_gather(const uint16_t* w, int64_t N, int64_t K, int64_t ldw, int32_t E,
                                  const int32_t* sel, int64_t n_sel, int64_t width,
                                  const float* colamax, float* s_t, uint8_t* codes, uint8_t* scales,
@@ -836,6 +1164,10 @@ cudaError_t launch_weight_gather(const uint16_t* w, int64_t N, int64_t K, int64_
     cudaError_t e = launch_sel_tensor_scale(colamax, K, sel, n_sel, E, s_t, s);
     if (e != cudaSuccess) return e;
   }
+  const WselPlan ws = wsel_plan(N, K, E, width, false);
+  if (ws.ok)
+    return launch_wsel_rows<false>(ws, w, ldw, nullptr, nullptr, 0, nullptr, N, K, E, sel, n_sel, width, colamax,
+                                   fuse, s_t, codes, scales, layout, s);
   const int64_t rows = static_cast<int64_t>(E) * N;
   RowGroups none{};
   {
@@ -859,6 +1191,10 @@ cudaError_t launch_weight_gather_fp4(const uint8_t* w_codes, const uint8_t* w_sc
     if (e != cudaSuccess) return e;
   }
   const int64_t rows = static_cast<int64_t>(E) * N;
+  const WselPlan ws = wsel_plan(N, K, E, width, true);
+  if (ws.ok)
+    return launch_wsel_rows<true>(ws, nullptr, 0, w_codes, w_scales, w_layout, w_st, N, K, E, sel, n_sel, width,
+                                  dq_colamax, fuse, s_t, codes, scales, layout, s);
   RowGroups none{};
   {
     const cudaError_t le = launch_k(gather_quant_kernel<2>, dim3(gather_grid(rows, width)), dim3(kGThreads), 0, s, nullptr, 0,
@@ -875,7 +1211,7 @@ cudaError_t launch_dq_colamax(const uint8_t* codes, const uint8_t* scales, int l
     const cudaError_t me = cudaMemsetAsync(colamax, 0, sizeof(float) * K * batch, s);
     if (me != cudaSuccess) return me;
   }
-  dim3 grid(static_cast<unsigned>(K / 64), static_cast<unsigned>((N + 127) / 128),
+  dim3 grid(static_cast<unsigned>((K + 127) / 128), static_cast<unsigned>((N + kCmRows - 1) / kCmRows),
             static_cast<unsigned>(batch));
   {
     const cudaError_t le = launch_k(dq_colamax_kernel, dim3(grid), dim3(256), 0, s, nullptr, 0,

@@ -53,7 +53,11 @@ def test_weight_qdq_in_place():
     assert np.array_equal(bits(wd), ref["w_out"])
 
 
-@pytest.mark.parametrize("N,K,k", [(512, 512, 50.0), (144, 1024, 25.0), (2048, 2048, 100.0), (300, 448, 12.5)])
+@pytest.mark.parametrize("N,K,k", [(512, 512, 50.0), (144, 1024, 25.0), (2048, 2048, 100.0), (300, 448, 12.5),
+                                   (11008, 4096, 50.0), (16, 64, 1.5625),
+                                   # one row per pass (shared-memory bound) and the generic
+                                   # gather (K beyond 16-bit channel indices)
+                                   (48, 16384, 0.5), (16, 65600, 0.1)])
 def test_weight_select_quant_matches_oracle(N, K, k):
     b = need_gpu()
     w = S.weights(N, K, seed=K)

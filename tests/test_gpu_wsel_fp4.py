@@ -59,7 +59,10 @@ def test_dq_colamax_matches_oracle(N, K, batch, layout):
 
 
 @pytest.mark.parametrize("N,K,k", [(512, 512, 50.0), (144, 1024, 25.0), (2048, 2048, 100.0),
-                                   (300, 448, 12.5), (16, 64, 1.5625), (11008, 4096, 50.0)])
+                                   (300, 448, 12.5), (16, 64, 1.5625), (11008, 4096, 50.0),
+                                   # 4 rows per pass (shared-memory bound) and the generic
+                                   # gather (K beyond 16-bit channel indices)
+                                   (48, 16384, 0.5), (16, 65600, 0.1)])
 def test_weight_select_fp4_matches_oracle(N, K, k):
     b = need_gpu()
     rng = np.random.default_rng(N * 3 + K)
