@@ -12,6 +12,8 @@ Modules
   rac      residual, channel score, top-k% mask, second-pass quantization,
            fp64 products, the trainer-side weight fake quantization, MoE.
   scalar   an independent pure-Python restatement for tiny shapes.
+  qat      the trainer-side QAT linear (W4A16, symmetric W4A4 ablation) with
+           the straight-through gradient.
 
 Floating point: the quantization steps are fp32 operations rounded to nearest
 even (numpy float32 arithmetic, no fused multiply-add, no flush to zero),
@@ -26,7 +28,7 @@ inputs, k = 0 / k = 100 reductions, the fp64 product against a plain loop,
 the scalar restatement, and "RAC error <= plain W4A4 error" against the bf16
 product.
 """
-from . import formats, nvfp4, rac, scalar  # noqa: F401
+from . import formats, nvfp4, qat, rac, scalar  # noqa: F401
 from .formats import (bf16_to_f32, e2m1_decode, e2m1_encode, e4m3_decode,  # noqa: F401
                       e4m3_encode, f32_to_bf16)
 from .nvfp4 import amax, dequantize, quantize, quantize_tensor, tensor_scale  # noqa: F401
