@@ -46,6 +46,8 @@ DEFAULT_WORKLOAD = "dense_rollout_projection"
 # grouped MoE expert FFN (up 2048 -> 1024, down 1024 -> 2048 over 64 experts,
 # 8192 tokens routed top-8): its own step, see run_moe
 MOE_WORKLOAD = "moe_expert_ffn"
+# trainer-side QAT step of one linear (forward + backward): (M, K, N, act_quant)
+QAT_WORKLOADS = {"qat_w4a16_step": (4096, 2048, 2048, False), "qat_w4a4_step": (4096, 2048, 2048, True)}
 FP4_OVER_BF16 = 4.0          # nominal dense FP4 / BF16 tensor ratio (9 / 2.25 PFLOP/s)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 ORACLE_SAMPLE_ROWS = 1024
@@ -59,7 +61,8 @@ def parse_args():
     p.add_argument("--steps", type=int, default=10)
     p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    p.add_argument("--workload", choices=sorted(WORKLOADS) + [MOE_WORKLOAD], default=DEFAULT_WORKLOAD)
+    p.add_argument("--workload", choices=sorted(WORKLOADS) + [MOE_WORKLOAD] + sorted(QAT_WORKLOADS),
+                   default=DEFAULT_WORKLOAD)
     p.add_argument("--k", type=float, default=None, help="RAC k percent (default: workload's)")
     p.add_argument("--no-graph", action="store_true", help="issue calls directly, no CUDA graphs")
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -641,6 +644,132 @@ def run_moe(args, rank, world, local_rank):
     }
 
 
+def run_qat(args, rank, world, local_rank):
+    """Trainer-side QAT step of one linear, forward and backward: Y = X' W'^T,
+    dX = dY W', dW = dY^T X' with W' = bf16(DQ(Q(W))) (the library's
+    weight_qdq, straight-through gradient) and, for the symmetric W4A4
+    ablation, X' = bf16(DQ(Q(X))); the three bf16 GEMMs are torch's.  Each
+    step (forward and backward) is replayed as one CUDA graph, so host-side
+    autograd does not enter the device time.  Timed with the same step
+    without fake quantization beside it; L2 flushed between steps."""
+    import torch
+    import torch.distributed as dist
+
+    from precision_rl_rollout_nvfp4_b200 import binding as B
+    from precision_rl_rollout_nvfp4_b200 import synthetic as S
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    M, K, N, act = QAT_WORKLOADS[args.workload]
+    seed = replica_seed(rank)
+    x_host = S.activations(M, K, seed=seed).pin_memory()
+    dy_host = (0.01 * torch.randn(M, N, generator=torch.Generator().manual_seed(seed))).to(torch.bfloat16).pin_memory()
+    w = S.weights(N, K, seed=seed).to(dev).requires_grad_(True)
+    x, dy = x_host.to(dev).requires_grad_(True), dy_host.to(dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(qat=True, xs=None, dys=None):
+        xs = x if xs is None else xs
+        dys = dy if dys is None else dys
+        xs.grad = None
+        w.grad = None
+        y = B.qat_linear(xs, w, act_quant=act) if qat else xs @ w.t()
+        y.backward(dys)
+        return y
+
+    def ev():
+        e = torch.cuda.Event(enable_timing=True)
+        e.record(stream)
+        return e
+
+    def timed(fn, reps):
+        ts = []
+        for _ in range(reps):
+            flush.zero_()
+            a = ev()
+            fn()
+            b = ev()
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        return ts
+
+    # warm-up on a side stream, then capture each step (autograd included)
+    side = torch.cuda.Stream(device=dev)
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        for _ in range(max(args.warmup, 3)):
+            step()
+            step(qat=False)
+            B.fake_quant(w.detach())
+    stream.wait_stream(side)
+    torch.cuda.synchronize()
+    if B.stream_status() != 0:
+        raise RuntimeError("device error word set during warm-up")
+    graphs = {}
+    for name, fn in [("qat", step), ("plain", lambda: step(qat=False)), ("fq", lambda: B.fake_quant(w.detach()))]:
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr):
+            fn()
+        graphs[name] = gr
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clocks:
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        qat_ms = timed(graphs["qat"].replay, args.steps)
+        if world > 1:
+            dist.barrier()
+    clock = clocks.summary()
+    total_ms = sum(qat_ms)
+    plain_ms = timed(graphs["plain"].replay, args.steps)
+    fq_ms = timed(graphs["fq"].replay, args.steps)
+    # end to end: X and dY from pinned host memory, a 4-byte loss-like scalar back
+    bufs = [(torch.empty_like(x), torch.empty_like(dy), torch.empty(1, dtype=torch.float32, device=dev))
+            for _ in range(2)]
+
+    def step_e2e(xb, dyb, out):
+        xs = xb.requires_grad_(True)
+        y = step(xs=xs, dys=dyb)
+        out.copy_(y.detach().float().sum().reshape(1))
+
+    sets = [{"h2d": [(xb.detach(), x_host), (dyb, dy_host)], "d2h": [(torch.empty(1).pin_memory(), out)],
+             "step": (lambda xb=xb, dyb=dyb, out=out: step_e2e(xb, dyb, out))} for xb, dyb, out in bufs]
+    e2e_ms = e2e_pipelined(sets, args.steps, max(args.warmup, 2))
+    if B.stream_status() != 0:
+        raise RuntimeError("device error word set during timing")
+    total_ms, e2e_total = max_over_ranks([total_ms, e2e_ms], world, dev)
+    flops = 6.0 * M * N * K
+    value = flops * world * args.steps / (total_ms * 1e-3) / 1e12
+    peaks, peak_kind = load_peaks()
+    med = {"qat_step": statistics.median(qat_ms), "plain_bf16_step": statistics.median(plain_ms),
+           "fake_quant_w": statistics.median(fq_ms)}
+    fq_bytes = 4.0 * N * K            # read W once, write W' once (algorithmic)
+    fq_gbs = fq_bytes / (med["fake_quant_w"] * 1e-3) / 1e9
+    return {
+        "metric": "QAT linear step TFLOP/s (6MNK per forward + backward)", "value": round(value, 2),
+        "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(total_ms / args.steps, 5), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16 GEMMs (torch) + nvfp4 fake quantization (library)",
+        "data": "synthetic (seeded channel-scaled heavy-tailed X, N(0,0.02) W, N(0,0.01) dY)",
+        "config": {"workload": args.workload, "M": M, "K": K, "N": N, "act_quant": act,
+                   "parallelism": f"replicas x{world}", "l2": "flushed before every timed step (256 MiB write)",
+                   "cuda_graph": True},
+        "per_call_us": {k: round(1e3 * v, 2) for k, v in med.items()},
+        "qdq_overhead_pct": round(100 * (med["qat_step"] - med["plain_bf16_step"]) / med["plain_bf16_step"], 1),
+        "roofline": {"kernel": "fake_quant(W): amax pass + weight_qdq", "bound": "hbm", "achieved": round(fq_gbs, 1),
+                     "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(fq_gbs / peaks["hbm_gbs"], 4),
+                     "traffic": None, "peak_source": f"{peak_kind}: hbm_gbs"},
+        "e2e": {"value": round(flops * world * args.steps / (e2e_total * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+                "h2d_bytes_per_step": int(2 * (x.numel() + dy.numel())), "d2h_bytes_per_step": 4,
+                "ms_per_step": round(e2e_total / args.steps, 4),
+                "pipelined": "2 buffer sets; H2D, compute and D2H on separate streams"},
+        # per step: fake quantization of W (2 launches) and, for W4A4, of X (2)
+        "gpu_launches": (4 if act else 2) * args.steps,
+        "clocks": clock,
+    }
+
+
 # ---------------------------------------------------------------- oracle (CPU)
 def oracle_step_time(M, K, N, k, rows, seed=0, wsel="bf16"):
     import numpy as np
@@ -654,6 +783,23 @@ def oracle_step_time(M, K, N, k, rows, seed=0, wsel="bf16"):
     r = oracle.rac_linear(x, w, k, wq=wq, wsel_source=wsel)
     dt = time.perf_counter() - t0
     return dt, 2.0 * rows * N * (K + r["n_sel"]), np.asarray(r["y"]).shape
+
+
+def oracle_qat_time(M, K, N, act, rows, seed=0):
+    """Oracle QAT step (fake quantization of the whole W, and of X for the
+    W4A4 ablation, then the fp64 forward and backward products) on the first
+    `rows` rows of X and dY."""
+    import torch
+
+    from oracle import qat
+    from precision_rl_rollout_nvfp4_b200 import synthetic as S
+    x = S.bf16_bits(S.activations(M, K, seed=seed))[:rows]
+    w = S.bf16_bits(S.weights(N, K, seed=seed))
+    dy = (0.01 * torch.randn(M, N, generator=torch.Generator().manual_seed(seed))).to(torch.bfloat16)
+    dy = dy.float().numpy()[:rows]
+    t0 = time.perf_counter()
+    qat.qat_linear(x, w, dy, act_quant=act)
+    return time.perf_counter() - t0, 6.0 * rows * N * K
 
 
 def blas_threads():
@@ -692,6 +838,16 @@ def oracle_moe_time(k, n_experts=8, seed=0, wsel="bf16"):
 
 
 def cpu_baseline(args, budget_s=12.0):
+    if args.workload in QAT_WORKLOADS:
+        M, K, N, act = QAT_WORKLOADS[args.workload]
+        rows = min(M, ORACLE_SAMPLE_ROWS)
+        t, flops, n = 0.0, 0.0, 0
+        while (t < budget_s and n < 8) or n == 0:
+            dt, f = oracle_qat_time(M, K, N, act, rows)
+            t, flops, n = t + dt, flops + f, n + 1
+        return {"value": round(flops / t / 1e12, 6), "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+                "sample": f"{n} oracle QAT step(s): fake quantization of W {N}x{K} and the fp64 forward and "
+                          f"backward on the first {rows} of {M} rows (numpy; products via BLAS)"}
     if args.workload == MOE_WORKLOAD:
         k = args.k if args.k is not None else 50.0
         t, flops, n, desc = 0.0, 0.0, 0, ""
@@ -717,6 +873,24 @@ def cpu_baseline(args, budget_s=12.0):
 
 
 def run_reference(args):
+    if args.workload in QAT_WORKLOADS:
+        M, K, N, act = QAT_WORKLOADS[args.workload]
+        rows = min(M, ORACLE_SAMPLE_ROWS)
+        for _ in range(args.warmup):
+            oracle_qat_time(M, K, N, act, rows)
+        t, flops = 0.0, 0.0
+        for _ in range(args.steps):
+            dt, f = oracle_qat_time(M, K, N, act, rows)
+            t, flops = t + dt, flops + f
+        value = flops / t / 1e12
+        return {"impl": "reference", "metric": "QAT linear step TFLOP/s (6MNK per forward + backward)",
+                "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": round(1e3 * t / args.steps, 3), "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f32 quantizer steps, f64 products",
+                "data": "synthetic", "config": {"workload": args.workload, "M": M, "K": K, "N": N, "act_quant": act},
+                "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+                                 "sample": f"the first {rows} of {M} rows per step (numpy oracle)"},
+                "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     if args.workload == MOE_WORKLOAD:
         k = args.k if args.k is not None else 50.0
         for _ in range(args.warmup):
@@ -773,7 +947,8 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=torch.device("cuda", local_rank))
     try:
-        line = (run_moe if args.workload == MOE_WORKLOAD else run_ours)(args, rank, world, local_rank)
+        runner = run_moe if args.workload == MOE_WORKLOAD else run_qat if args.workload in QAT_WORKLOADS else run_ours
+        line = runner(args, rank, world, local_rank)
         if rank == 0:
             if not args.no_cpu_baseline:
                 line["cpu_baseline"] = cpu_baseline(args)

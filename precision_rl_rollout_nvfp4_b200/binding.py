@@ -322,6 +322,36 @@ def rac_linear(x, w, k_percent, out_dtype=torch.float32, prepared=None, wsel="bf
                    qw=qw, w_colamax=colamax)
 
 
+class _FakeQuantSTE(torch.autograd.Function):
+    """bf16(DQ(Q(t))) of a 2-D bf16 tensor with its own tensor scale, by the
+    library's weight_qdq; backward: the straight-through estimator (the
+    gradient crosses the fake quantizer unchanged)."""
+
+    @staticmethod
+    def forward(ctx, t):
+        out, _, _ = weight_qdq(t.contiguous(), want_q=False, want_colamax=False)
+        return out
+
+    @staticmethod
+    def backward(ctx, g):
+        return g
+
+
+def fake_quant(t):
+    """Trainer-side NVFP4 fake quantization with a straight-through gradient."""
+    return _FakeQuantSTE.apply(t)
+
+
+def qat_linear(x, w, act_quant=False):
+    """Trainer-side QAT linear Y = X' W'^T as a bf16 GEMM (torch matmul):
+    W' = fake_quant(W) (asymmetric W4A16), and X' = fake_quant(X) for the
+    symmetric W4A4 ablation (act_quant=True), else X' = X.  Autograd gives
+    dX = dY W' and dW = dY^T X' through the straight-through quantizers."""
+    wq = fake_quant(w)
+    xq = fake_quant(x) if act_quant else x
+    return xq @ wq.t()
+
+
 def encode_e2m1(v: torch.Tensor, stream=None) -> torch.Tensor:
     out = torch.empty(v.numel(), dtype=torch.uint8, device=v.device)
     _check(_lib.nvfp4_encode_e2m1(_ptr(v), _ptr(out), v.numel(), _stream(stream)), "nvfp4_encode_e2m1")
