@@ -1164,8 +1164,12 @@ cudaError_t launch_weight_gather(const uint16_t* w, int64_t N, int64_t K, int64_
     cudaError_t e = launch_sel_tensor_scale(colamax, K, sel, n_sel, E, s_t, s);
     if (e != cudaSuccess) return e;
   }
+  // the row-staged kernel pays off once every CTA runs several passes; a
+  // weight with fewer rows than about two passes per resident CTA takes the
+  // tile gather (its fixed cost per CTA is lower)
   const WselPlan ws = wsel_plan(N, K, E, width, false);
-  if (ws.ok)
+  const int64_t passes_w = (static_cast<int64_t>(E) * N + ws.g.R - 1) / (ws.g.R > 0 ? ws.g.R : 1);
+  if (ws.ok && passes_w >= 2 * 4 * static_cast<int64_t>(sm_count()))
     return launch_wsel_rows<false>(ws, w, ldw, nullptr, nullptr, 0, nullptr, N, K, E, sel, n_sel, width, colamax,
                                    fuse, s_t, codes, scales, layout, s);
   const int64_t rows = static_cast<int64_t>(E) * N;
