@@ -68,3 +68,41 @@ def test_argument_errors_without_gpu(lib):
     s = lib.nvfp4_status_string
     s.restype, s.argtypes = ctypes.c_char_p, [ctypes.c_int32]
     assert s(6) == b"device-side wait timed out"
+
+
+class _T(ctypes.Structure):
+    _fields_ = [("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("tensor_scale", ctypes.c_void_p),
+                ("rows", ctypes.c_int64), ("cols", ctypes.c_int64), ("scale_layout", ctypes.c_int32)]
+
+
+def _fake_tensor(rows, cols, layout=1):
+    # aligned, never dereferenced: every call below returns before any CUDA work
+    return _T(0x10000, 0x20000, 0x30000, rows, cols, layout)
+
+
+def test_nvfp4_weight_variant_argument_errors_without_gpu(lib):
+    """nvfp4_dq_colamax and rac_weight_quant_fp4 reject bad arguments with
+    the documented codes before any CUDA call."""
+    TP = ctypes.POINTER(_T)
+    cm = lib.nvfp4_dq_colamax
+    cm.restype, cm.argtypes = ctypes.c_int32, [TP, ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p]
+    q = _fake_tensor(256, 512)
+    assert cm(None, 1, ctypes.c_void_p(0x40000), None) == 1            # null tensor
+    assert cm(ctypes.byref(q), 1, None, None) == 1                     # null output
+    assert cm(ctypes.byref(q), 0, ctypes.c_void_p(0x40000), None) == 3   # batch 0
+    assert cm(ctypes.byref(q), 3, ctypes.c_void_p(0x40000), None) == 3   # rows % batch
+    bad = _fake_tensor(256, 500)
+    assert cm(ctypes.byref(bad), 1, ctypes.c_void_p(0x40000), None) == 3  # cols % 64
+    assert cm(ctypes.byref(q), 1, ctypes.c_void_p(0x40004), None) == 2    # misaligned output
+    wq = lib.rac_weight_quant_fp4
+    wq.restype = ctypes.c_int32
+    wq.argtypes = [TP, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, TP, ctypes.c_void_p]
+    out = _fake_tensor(256, 256)
+    sel, dq = ctypes.c_void_p(0x50000), ctypes.c_void_p(0x60000)
+    assert wq(None, sel, 200, dq, ctypes.byref(out), None) == 1
+    assert wq(ctypes.byref(q), None, 200, dq, ctypes.byref(out), None) == 1
+    assert wq(ctypes.byref(q), sel, 0, dq, ctypes.byref(out), None) == 3       # n_sel 0
+    assert wq(ctypes.byref(q), sel, 513, dq, ctypes.byref(out), None) == 3     # n_sel > K
+    assert wq(ctypes.byref(q), sel, 100, dq, ctypes.byref(out), None) == 3     # width 128 != 256
+    wrong_rows = _fake_tensor(128, 256)
+    assert wq(ctypes.byref(q), sel, 200, dq, ctypes.byref(wrong_rows), None) == 3
