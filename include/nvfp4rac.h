@@ -133,6 +133,34 @@ nvfp4_status rac_select(const uint16_t* x, int64_t M, int64_t K, int64_t ldx,
                         float k_percent, uint8_t* mask, int32_t* sel, int64_t* n_sel_out,
                         nvfp4_tensor* q_res, void* ws, size_t ws_bytes, void* stream);
 
+/*
+ * rac_select_channels -- the first half of rac_select: the top-k% channel
+ * mask, sel and the residual tensor scale, without the residual gather, so
+ * that the gathers of the residual and of the weight (rac_residual_quant,
+ * rac_weight_quant) can run concurrently on two streams.  Pages: 2.2 B
+ * (binary channel mask, top k%).
+ *   score / res_colamax [K]: outputs of nvfp4_quantize.  mask u8 [K];
+ *   sel i32 [n_sel] ascending (may be NULL when n_sel == 0); *n_sel_out
+ *   (host) = floor(k K / 100).  res_tensor_scale (device fp32, required):
+ *   RN(max_{j in sel} res_colamax_j / 2688), the residual's tensor scale
+ *   (0 when n_sel == 0); pass q_res->tensor_scale to rac_residual_quant.
+ */
+nvfp4_status rac_select_channels(const double* score, const float* res_colamax, int64_t K, float k_percent,
+                                 uint8_t* mask, int32_t* sel, int64_t* n_sel_out, float* res_tensor_scale,
+                                 void* stream);
+
+/*
+ * rac_residual_quant -- the second half of rac_select: Q(dX_sel), the
+ * second-pass quantization of the residual's selected channels, with the
+ * tensor scale rac_select_channels wrote into q_res->tensor_scale (read on
+ * the device, so it must be ordered after that call).  Pages: 2.2 B
+ * (second-pass quantization of the high-residual channels).
+ *   x, qx as for rac_select; sel [n_sel], n_sel >= 1; q_res: rows = M,
+ *   cols = nvfp4_rac_width(n_sel), either scale layout.
+ */
+nvfp4_status rac_residual_quant(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, const nvfp4_tensor* qx,
+                                const int32_t* sel, int64_t n_sel, nvfp4_tensor* q_res, void* stream);
+
 /* n_sel for k_percent of K channels (exact floor), and the padded width of
  * the gathered residual / weight operands (n_sel rounded up to 64). */
 int64_t nvfp4_rac_nsel(float k_percent, int64_t K);

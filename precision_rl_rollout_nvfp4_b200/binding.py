@@ -30,7 +30,7 @@ EXPORTS = ["nvfp4_scale_bytes", "nvfp4_workspace_size", "nvfp4_quantize", "rac_s
            "w4a4_gemm_quantized", "moe_grouped_w4a4_rac_gemm", "weight_qdq",
            "nvfp4_encode_e2m1", "nvfp4_encode_e4m3", "nvfp4_stream_status",
            "nvfp4_check_bounded_wait", "nvfp4_status_string", "nvfp4_quantize_static_ws",
-           "nvfp4_dq_colamax", "rac_weight_quant_fp4"]
+           "nvfp4_dq_colamax", "rac_weight_quant_fp4", "rac_select_channels", "rac_residual_quant"]
 
 
 class _Tensor(ctypes.Structure):
@@ -51,6 +51,8 @@ _sig = {
     "nvfp4_rac_width": (I64, [I64]),
     "rac_weight_quant": (I32, [P, I64, I64, I64, P, I64, P, TP, P]),
     "nvfp4_dq_colamax": (I32, [TP, I32, P, P]),
+    "rac_select_channels": (I32, [P, P, I64, F32, P, P, ctypes.POINTER(I64), P, P]),
+    "rac_residual_quant": (I32, [P, I64, I64, I64, TP, P, I64, TP, P]),
     "rac_weight_quant_fp4": (I32, [TP, P, I64, P, TP, P]),
     "w4a4_rac_gemm": (I32, [TP, TP, P, I64, P, I64, I64, TP, P, P, I32, I64, P, SZ, P]),
     "w4a4_gemm_quantized": (I32, [TP, TP, TP, TP, P, I32, I64, P]),
@@ -204,6 +206,36 @@ def rac_select(x, qx, score, colamax, k_percent, layout=1, stream=None):
                            _stream(stream)), "rac_select")
     assert n_out.value == n_sel
     return mask, sel[:n_sel], n_sel, q_res
+
+
+def rac_select_channels(score, colamax, k_percent, res_tensor_scale=None, stream=None):
+    """Top-k% mask, sel and the residual tensor scale (the first half of
+    rac_select).  Returns (mask, sel [n_sel], n_sel, res_tensor_scale)."""
+    K = score.numel()
+    n_sel = rac_nsel(k_percent, K)
+    mask = torch.empty(K, dtype=torch.uint8, device=score.device)
+    sel = torch.empty(max(n_sel, 1), dtype=torch.int32, device=score.device)
+    st = res_tensor_scale if res_tensor_scale is not None else torch.empty(1, dtype=torch.float32,
+                                                                           device=score.device)
+    n_out = ctypes.c_int64(-1)
+    _check(_lib.rac_select_channels(_ptr(score), _ptr(colamax), K, float(k_percent), _ptr(mask), _ptr(sel),
+                                    ctypes.byref(n_out), _ptr(st), _stream(stream)), "rac_select_channels")
+    assert n_out.value == n_sel
+    return mask, sel[:n_sel], n_sel, st
+
+
+def rac_residual_quant(x, qx, sel, n_sel, res_tensor_scale, layout=1, out=None, stream=None):
+    """Q(dX_sel) (the second half of rac_select) with the residual tensor
+    scale written by rac_select_channels."""
+    x = _bits(x)
+    M, K = x.shape
+    q = out if out is not None else NvFP4Tensor.empty(M, rac_width(n_sel), layout, device=x.device)
+    if out is None:
+        q.tensor_scale.copy_(res_tensor_scale.reshape(1))
+    a, qs = qx.c(), q.c()
+    _check(_lib.rac_residual_quant(_ptr(x), M, K, x.stride(0), ctypes.byref(a), _ptr(sel), n_sel,
+                                   ctypes.byref(qs), _stream(stream)), "rac_residual_quant")
+    return q
 
 
 def rac_weight_quant(w, sel, n_sel, w_colamax, layout=1, out=None, stream=None):
@@ -386,6 +418,8 @@ class RacLinearPlan:
       prepare_weight  weight_qdq(W) -> Q(W), colamax_W     (per weight sync)
       quantize        nvfp4_quantize(X) -> Q(X), scores, residual col-max
       select          rac_select -> mask, sel, Q(dX_sel)
+                      (the steps call its halves, rac_select_channels and
+                      rac_residual_quant, so the two gathers overlap)
       weight_select   rac_weight_quant -> Q(W_sel)
       gemm            w4a4_gemm_quantized -> Y
     With wsel="fp4" the weight preparation also takes the column maxima of
@@ -423,6 +457,10 @@ class RacLinearPlan:
         self.side = torch.cuda.Stream(device=dev)
         self._fork = torch.cuda.Event()
         self._join = torch.cuda.Event()
+        self._sel_ready = torch.cuda.Event()
+        self._wsel_done = torch.cuda.Event()
+        self.res_st = (self.q_res.tensor_scale if self.q_res is not None
+                       else torch.empty(1, dtype=torch.float32, device=dev))
         self._qw, self._qx = self.qw.c(), self.qx.c()
         self._qr = self.q_res.c() if self.q_res is not None else None
         self._qs = self.q_wsel.c() if self.q_wsel is not None else None
@@ -458,6 +496,32 @@ class RacLinearPlan:
                                ctypes.byref(self._qr) if self._qr is not None else None,
                                _ptr(self.ws), self.ws.numel(), _stream(stream)), "rac_select")
 
+    def select_channels(self, stream=None):
+        _check(_lib.rac_select_channels(_ptr(self.score), _ptr(self.res_colamax), self.K, self.k, _ptr(self.mask),
+                                        _ptr(self.sel), ctypes.byref(self._nout), _ptr(self.res_st),
+                                        _stream(stream)), "rac_select_channels")
+
+    def residual_quant(self, stream=None):
+        if self.n_sel == 0:
+            return
+        _check(_lib.rac_residual_quant(_ptr(self.x), self.M, self.K, self.x.stride(0), ctypes.byref(self._qx),
+                                       _ptr(self.sel), self.n_sel, ctypes.byref(self._qr), _stream(stream)),
+               "rac_residual_quant")
+
+    def _gathers_overlapped(self):
+        """After select_channels: the W_sel gather on the side stream (after
+        any weight preparation queued there) concurrently with the residual
+        gather on the current stream; the current stream then waits for it."""
+        main = torch.cuda.current_stream()
+        if self.n_sel == 0:
+            return
+        self._sel_ready.record(main)
+        self.side.wait_event(self._sel_ready)
+        self.weight_select(stream=self.side)
+        self._wsel_done.record(self.side)
+        self.residual_quant()
+        main.wait_event(self._wsel_done)
+
     def weight_select(self, stream=None):
         if self.n_sel == 0:
             return
@@ -477,26 +541,32 @@ class RacLinearPlan:
                                         0 if self.y.dtype == torch.float32 else 1, self.y.stride(0),
                                         _stream(stream)), "w4a4_gemm_quantized")
 
-    def rollout_step(self, stream=None):
-        """The rollout linear on an already-prepared weight."""
-        self.quantize(stream)
-        self.select(stream)
-        self.weight_select(stream)
-        self.gemm(stream)
+    def rollout_step(self):
+        """The rollout linear on an already-prepared weight (on the current
+        stream; the two gathers overlap through the side stream)."""
+        main = torch.cuda.current_stream()
+        self._fork.record(main)
+        self.side.wait_event(self._fork)
+        self.quantize()
+        self.select_channels()
+        self._gathers_overlapped()
+        self.gemm()
 
     def full_step(self):
         """Weight preparation and the rollout linear, with the weight
         preparation (independent of X) on a side stream that forks from and
-        joins back into the current stream, so the two overlap on the GPU."""
+        joins back into the current stream, so the two overlap on the GPU;
+        the W_sel gather follows it on the side stream once sel exists, while
+        the residual gather runs on the current stream."""
         main = torch.cuda.current_stream()
         self._fork.record(main)
         self.side.wait_event(self._fork)
         self.prepare_weight(stream=self.side)
         self._join.record(self.side)
         self.quantize()
-        self.select()
+        self.select_channels()
+        self._gathers_overlapped()                 # W_sel queued behind the weight preparation
         main.wait_event(self._join)
-        self.weight_select()
         self.gemm()
 
     def plain_step(self, stream=None):

@@ -265,6 +265,37 @@ nvfp4_status rac_select(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, co
   return NVFP4_OK;
 }
 
+nvfp4_status rac_select_channels(const double* score, const float* res_colamax, int64_t K, float k_percent,
+                                 uint8_t* mask, int32_t* sel, int64_t* n_sel_out, float* res_tensor_scale,
+                                 void* stream) {
+  NV_CHECK(score && res_colamax && mask && n_sel_out && res_tensor_scale, NVFP4_ERR_INVALID_ARG);
+  NV_CHECK(k_percent >= 0.0f && k_percent <= 100.0f, NVFP4_ERR_INVALID_ARG);
+  NV_CHECK(K >= 64 && K % 64 == 0, NVFP4_ERR_UNSUPPORTED_SHAPE);
+  const int64_t n_sel = nvfp4_rac_nsel(k_percent, K);
+  NV_CHECK(n_sel == 0 || sel, NVFP4_ERR_INVALID_ARG);
+  const nvfp4_status d = device_ok();
+  if (d != NVFP4_OK) return d;
+  *n_sel_out = n_sel;
+  NV_TRY(launch_topk(score, res_colamax, K, 1, n_sel, mask, sel, res_tensor_scale,
+                     static_cast<cudaStream_t>(stream)));
+  return NVFP4_OK;
+}
+
+nvfp4_status rac_residual_quant(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, const nvfp4_tensor* qx,
+                                const int32_t* sel, int64_t n_sel, nvfp4_tensor* q_res, void* stream) {
+  NV_CHECK(x && tensor_ok(qx) && sel && tensor_ok(q_res), NVFP4_ERR_INVALID_ARG);
+  NV_CHECK(M >= 1 && K >= 64 && K % 64 == 0 && ldx >= K && qx->rows == M && qx->cols == K && n_sel >= 1 &&
+               n_sel <= K && q_res->rows == M && q_res->cols == nvfp4_rac_width(n_sel),
+           NVFP4_ERR_UNSUPPORTED_SHAPE);
+  NV_CHECK(aligned16(x) && ldx % 8 == 0, NVFP4_ERR_MISALIGNED);
+  const nvfp4_status d = device_ok();
+  if (d != NVFP4_OK) return d;
+  NV_TRY(launch_residual_gather(x, M, K, ldx, dense_groups(M), M, qx->codes, qx->scales, qx->scale_layout,
+                                qx->tensor_scale, sel, n_sel, q_res->cols, q_res->tensor_scale, q_res->codes,
+                                q_res->scales, q_res->scale_layout, static_cast<cudaStream_t>(stream)));
+  return NVFP4_OK;
+}
+
 nvfp4_status rac_weight_quant(const uint16_t* w, int64_t N, int64_t K, int64_t ldw, const int32_t* sel,
                               int64_t n_sel, const float* w_colamax, nvfp4_tensor* q_wsel,
                               void* stream) {

@@ -106,3 +106,27 @@ def test_nvfp4_weight_variant_argument_errors_without_gpu(lib):
     assert wq(ctypes.byref(q), sel, 100, dq, ctypes.byref(out), None) == 3     # width 128 != 256
     wrong_rows = _fake_tensor(128, 256)
     assert wq(ctypes.byref(q), sel, 200, dq, ctypes.byref(wrong_rows), None) == 3
+
+
+def test_split_select_argument_errors_without_gpu(lib):
+    f = lib.rac_select_channels
+    f.restype = ctypes.c_int32
+    f.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_float, ctypes.c_void_p,
+                  ctypes.c_void_p, ctypes.POINTER(ctypes.c_int64), ctypes.c_void_p, ctypes.c_void_p]
+    n = ctypes.c_int64(-1)
+    p = ctypes.c_void_p
+    assert f(None, p(0x100), 512, 50.0, p(0x200), p(0x300), ctypes.byref(n), p(0x400), None) == 1
+    assert f(p(0x100), p(0x100), 512, 50.0, p(0x200), p(0x300), ctypes.byref(n), None, None) == 1
+    assert f(p(0x100), p(0x100), 512, 150.0, p(0x200), p(0x300), ctypes.byref(n), p(0x400), None) == 1
+    assert f(p(0x100), p(0x100), 500, 50.0, p(0x200), p(0x300), ctypes.byref(n), p(0x400), None) == 3
+    assert f(p(0x100), p(0x100), 512, 50.0, p(0x200), None, ctypes.byref(n), p(0x400), None) == 1
+    g = lib.rac_residual_quant
+    TP = ctypes.POINTER(_T)
+    g.restype = ctypes.c_int32
+    g.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, TP, ctypes.c_void_p,
+                  ctypes.c_int64, TP, ctypes.c_void_p]
+    qx, qr = _fake_tensor(64, 512), _fake_tensor(64, 256)
+    assert g(None, 64, 512, 512, ctypes.byref(qx), p(0x300), 256, ctypes.byref(qr), None) == 1
+    assert g(p(0x1000), 64, 512, 512, ctypes.byref(qx), p(0x300), 300, ctypes.byref(qr), None) == 3   # width 320
+    assert g(p(0x1000), 64, 512, 512, ctypes.byref(qx), p(0x300), 0, ctypes.byref(qr), None) == 3
+    assert g(p(0x1008), 64, 512, 512, ctypes.byref(qx), p(0x300), 256, ctypes.byref(qr), None) == 2
