@@ -153,10 +153,15 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------- profile traffic
+KERNEL_SOURCES = ("common.cuh", "gemm.cu", "kernels.h", "quant.cu", "select.cu")
+
+
 def kernel_sources_hash():
+    """sha256 (first 16 hex digits) over the files that hold the kernels and
+    their launch code; the host-only ABI layer is not part of it."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "precision_rl_rollout_nvfp4_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in KERNEL_SOURCES:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
