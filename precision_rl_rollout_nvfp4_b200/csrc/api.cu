@@ -229,8 +229,7 @@ nvfp4_status nvfp4_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ldx
   }
   NV_TRY(launch_quant_score(x, M, K, ldx, g, amax_or_null, w.amax, n_parts, M, qx->codes, qx->scales,
                             qx->scale_layout, qx->tensor_scale, w.part_sum, w.part_max,
-                            scores ? w.counters : nullptr, score_or_null, res_colamax_or_null,
-                            device_error_word(), s));
+                            scores ? w.counters : nullptr, score_or_null, res_colamax_or_null, s));
   return NVFP4_OK;
 }
 
@@ -449,7 +448,7 @@ nvfp4_status moe_grouped_w4a4_rac_gemm(const uint16_t* x_perm, int64_t T, int64_
   NV_TRY(launch_amax(x_perm, T, K, K, g, m.amax, s));
   NV_TRY(launch_quant_score(x_perm, T, K, K, g, reinterpret_cast<const float*>(m.amax), nullptr, 0, prows,
                             m.qx_codes, m.qx_scales, 1, m.qx_st, m.part_sum, m.part_max, nullptr,
-                            nullptr, nullptr, device_error_word(), s));
+                            nullptr, nullptr, s));
   NV_TRY(launch_score_reduce(m.part_sum, m.part_max, K, g, tiles, m.score, m.colamax, m.qx_st, s));
   NV_TRY(launch_topk(m.score, m.colamax, K, E, n_sel, mask, m.sel, m.r_st, s));
   GemmArgs a{};

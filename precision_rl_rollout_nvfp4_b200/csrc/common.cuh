@@ -118,6 +118,32 @@ __device__ __forceinline__ uint64_t e2m1x2_to_f2(uint32_t byte) {
   return r;
 }
 
+// f16 pairs (one 32-bit register, element 2j in the low half).  The exact
+// values of the two E2M1 codes of a byte (low nibble in the low half) and of
+// two E4M3 scale bytes (low byte in the low half), through the hardware
+// conversions; both formats are exact in f16, and so is a product of an
+// E2M1 and an E4M3 value (at most 6 significant bits, in [2^-10, 2688]).
+__device__ __forceinline__ uint32_t e2m1x2_to_h2(uint32_t byte) {
+  uint32_t h;
+  asm("{\n\t.reg .b8 t;\n\tcvt.u8.u32 t, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, t;\n\t}" : "=r"(h) : "r"(byte));
+  return h;
+}
+__device__ __forceinline__ uint32_t e4m3x2_to_h2(uint32_t two) {
+  uint32_t h;
+  asm("{\n\t.reg .b16 t;\n\tcvt.u16.u32 t, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, t;\n\t}" : "=r"(h) : "r"(two));
+  return h;
+}
+__device__ __forceinline__ uint32_t h2_mul(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+__device__ __forceinline__ uint32_t h2_max(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
 // E2M1 codes of four fp32 pairs (8 elements) -> 4 bytes, element 2j in the
 // low nibble of byte j.
 __device__ __forceinline__ uint32_t e2m1x8_f2(const uint64_t* p) {

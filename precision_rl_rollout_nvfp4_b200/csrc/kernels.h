@@ -90,7 +90,7 @@ cudaError_t launch_quant_score(const uint16_t* x, int64_t rows, int64_t K, int64
                                int n_parts, int64_t codes_rows,
                                uint8_t* codes, uint8_t* scales, int layout, float* tensor_scale,
                                double* part_sum, float* part_max, unsigned* strip_count,
-                               double* score, float* colamax, unsigned* err, cudaStream_t s);
+                               double* score, float* colamax, cudaStream_t s);
 
 // score[e, j] = sum over the group's tiles of part_sum in tile order;
 // colamax[e, j] = max of part_max.  For empty groups (MoE) also writes

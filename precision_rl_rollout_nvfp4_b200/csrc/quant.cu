@@ -508,7 +508,6 @@ gather_quant_kernel(const uint16_t* __restrict__ src, int64_t K, int64_t ld, Row
 }
 
 // s_t[e] = RN(max_{j < n_sel} colamax[e*K + sel[e*n_sel + j]] / 2688), one CTA per group.
-constexpr int kWThreads = 256;
 
 __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
@@ -547,22 +546,8 @@ struct WselGeom {
   uint32_t rowbytes, rawbytes; // staged row (2K + 16) and raw NVFP4 row (K/2 + K/16, to 16 bytes)
 };
 
-__device__ __forceinline__ uint32_t dup_e4m3_to_h2(uint32_t sb) {
-  uint32_t h;
-  const uint32_t two = (sb & 0x7Fu) * 0x0101u;
-  asm("{\n\t.reg .b16 t;\n\tcvt.u16.u32 t, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, t;\n\t}" : "=r"(h) : "r"(two));
-  return h;
-}
-__device__ __forceinline__ uint32_t e2m1x2_h2(uint32_t byte) {
-  uint32_t h;
-  asm("{\n\t.reg .b8 t;\n\tcvt.u8.u32 t, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, t;\n\t}" : "=r"(h) : "r"(byte));
-  return h;
-}
-__device__ __forceinline__ uint32_t h2mul(uint32_t a, uint32_t b) {
-  uint32_t d;
-  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-  return d;
-}
+// Both halves of an f16 pair = E4M3dec(sb) of one scale byte (sign ignored).
+__device__ __forceinline__ uint32_t dup_e4m3_to_h2(uint32_t sb) { return e4m3x2_to_h2((sb & 0x7Fu) * 0x0101u); }
 
 template <bool FP4>
 __global__ void __launch_bounds__(512, 2)
@@ -682,10 +667,10 @@ wsel_rows_kernel(const uint16_t* __restrict__ w, int64_t ldw, const uint8_t* __r
           const uint32_t wd = *reinterpret_cast<const uint32_t*>(ws_smem + ro + 4u * q);
           const uint32_t sv = dup_e4m3_to_h2(ws_smem[ro + half + (q >> 1)]);
           uint4 o;
-          o.x = h2mul(e2m1x2_h2(wd & 0xFFu), sv);
-          o.y = h2mul(e2m1x2_h2((wd >> 8) & 0xFFu), sv);
-          o.z = h2mul(e2m1x2_h2((wd >> 16) & 0xFFu), sv);
-          o.w = h2mul(e2m1x2_h2(wd >> 24), sv);
+          o.x = h2_mul(e2m1x2_to_h2(wd & 0xFFu), sv);
+          o.y = h2_mul(e2m1x2_to_h2((wd >> 8) & 0xFFu), sv);
+          o.z = h2_mul(e2m1x2_to_h2((wd >> 16) & 0xFFu), sv);
+          o.w = h2_mul(e2m1x2_to_h2(wd >> 24), sv);
           *reinterpret_cast<uint4*>(dst + 16u * q) = o;
         }
       }
@@ -724,30 +709,6 @@ wsel_rows_kernel(const uint16_t* __restrict__ w, int64_t ldw, const uint8_t* __r
     }
     __syncthreads();                               // staged rows and buffer b are free again
   }
-}
-
-// Exact values of the two E2M1 codes of a byte (low nibble in the low half)
-// and of two E4M3 scale bytes (low byte in the low half) as f16x2, through
-// the hardware conversions; both are exact in f16.
-__device__ __forceinline__ uint32_t e2m1x2_to_h2(uint32_t byte) {
-  uint32_t h;
-  asm("{\n\t.reg .b8 t;\n\tcvt.u8.u32 t, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, t;\n\t}" : "=r"(h) : "r"(byte));
-  return h;
-}
-__device__ __forceinline__ uint32_t e4m3x2_to_h2(uint32_t two) {
-  uint32_t h;
-  asm("{\n\t.reg .b16 t;\n\tcvt.u16.u32 t, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, t;\n\t}" : "=r"(h) : "r"(two));
-  return h;
-}
-__device__ __forceinline__ uint32_t h2_mul(uint32_t a, uint32_t b) {
-  uint32_t d;
-  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-  return d;
-}
-__device__ __forceinline__ uint32_t h2_max(uint32_t a, uint32_t b) {
-  uint32_t d;
-  asm("max.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-  return d;
 }
 
 // Column maxima of |DQ(Q(W))| for `batch` stacked NVFP4 matrices of N rows
@@ -987,8 +948,7 @@ cudaError_t launch_quant_score(const uint16_t* x, int64_t rows, int64_t K, int64
                                int n_parts, int64_t codes_rows,
                                uint8_t* codes, uint8_t* scales, int layout, float* tensor_scale,
                                double* part_sum, float* part_max, unsigned* strip_count,
-                               double* score, float* colamax, unsigned* err, cudaStream_t s) {
-  (void)err;                                       // no waits in this kernel
+                               double* score, float* colamax, cudaStream_t s) {
   const int64_t tiles = max_tiles(g, rows);
   if (tiles == 0) return cudaSuccess;
   dim3 grid(static_cast<unsigned>(K / kQCols), static_cast<unsigned>(tiles));
