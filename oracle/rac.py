@@ -165,20 +165,29 @@ def weight_qdq(w_bf16):
                 colamax=column_amax(w))
 
 
-def rac_linear(x_bf16, w_bf16, k_percent, rows=None, wq=None, wsel_source="bf16"):
+def rac_linear(x_bf16, w_bf16, k_percent, rows=None, wq=None, wsel_source="bf16", sel=None):
     """One rollout linear Y = X W^T in NVFP4 W4A4 with RAC.
 
     ``rows`` restricts the fp64 products to a subset of output rows (all
     quantities that depend on every token, such as the scores and the mask,
     are still computed from all rows).  ``wq`` may pass a precomputed
     ``weight_qdq(w_bf16)``.  ``wsel_source="fp4"`` takes W_sel from Q(W)
-    (``weight_sel_from_fp4``) instead of bf16 W.  Returns every
-    intermediate."""
+    (``weight_sel_from_fp4``) instead of bf16 W.  ``sel`` (ascending channel
+    indices) replaces the top-k% selection of this X by a mask kept from an
+    earlier call (the mask-reuse variant); everything else (Q(X), dX, the
+    residual tensor scale over sel, both second passes) is this call's.
+    Returns every intermediate."""
     qa = quantize_activations(x_bf16)
     M, K = qa["codes"].shape
     wq = weight_qdq(w_bf16) if wq is None else wq
-    n_sel = n_selected(k_percent, K)
-    sel, mask = select_channels(qa["score"], n_sel)
+    if sel is None:
+        n_sel = n_selected(k_percent, K)
+        sel, mask = select_channels(qa["score"], n_sel)
+    else:
+        sel = np.asarray(sel, np.int32)
+        n_sel = len(sel)
+        mask = np.zeros(K, np.uint8)
+        mask[sel] = 1
     width = padded_width(n_sel)
     out = dict(qa)
     out.update(n_sel=n_sel, sel=sel, mask=mask, width=width, wq=wq)

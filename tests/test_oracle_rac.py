@@ -215,3 +215,38 @@ def test_wsel_from_fp4_k0_is_plain_and_error_is_bounded():
     ref = oracle.bf16_to_f32(xb).astype(np.float64) @ oracle.bf16_to_f32(wb).astype(np.float64).T
     r50 = oracle.rac_linear(xb, wb, 50.0, wsel_source="fp4")
     assert np.linalg.norm(r50["y"] - ref) <= np.linalg.norm(r0["y"] - ref)
+
+
+def test_reused_mask_equal_to_this_calls_mask_changes_nothing():
+    """The mask-reuse variant with the selection this X would make itself is
+    the per-call RAC linear, intermediate for intermediate."""
+    x = S.bf16_bits(S.activations(96, 256, seed=21))
+    w = S.bf16_bits(S.weights(64, 256, seed=21))
+    a = oracle.rac_linear(x, w, 50.0)
+    b = oracle.rac_linear(x, w, 50.0, sel=a["sel"])
+    for key in ("mask", "sel", "r_codes", "r_scales", "ws_codes", "ws_scales"):
+        assert np.array_equal(a[key], b[key]), key
+    assert a["r_st"] == b["r_st"] and a["ws_st"] == b["ws_st"]
+    assert np.array_equal(a["y"], b["y"])
+
+
+def test_reused_mask_from_another_batch():
+    """A mask kept from batch A applied to batch B: B's own residual (its
+    tensor scale is the maximum over the kept channels of B's residual
+    maxima), A's channels, and the plain W4A4 product when the mask is empty."""
+    xa = S.bf16_bits(S.activations(64, 256, seed=22))
+    xb = S.bf16_bits(S.activations(64, 256, seed=23))
+    w = S.bf16_bits(S.weights(32, 256, seed=22))
+    sel_a = oracle.rac_linear(xa, w, 25.0)["sel"]
+    r = oracle.rac_linear(xb, w, 25.0, sel=sel_a)
+    own = oracle.quantize_activations(xb)
+    assert np.array_equal(r["sel"], sel_a)
+    assert r["r_st"] == oracle.tensor_scale(own["res_colamax"][sel_a].max())
+    codes, scales, st = oracle.gather_quantize(own["dx"], sel_a, r["width"], own["res_colamax"][sel_a].max())
+    assert np.array_equal(r["r_codes"], codes) and np.array_equal(r["r_scales"], scales)
+    empty = oracle.rac_linear(xb, w, 25.0, sel=np.zeros(0, np.int32))
+    assert np.array_equal(empty["y"], empty["y_plain"])
+    # the kept mask is not this batch's own choice, and RAC with it still helps
+    assert not np.array_equal(sel_a, oracle.rac_linear(xb, w, 25.0)["sel"])
+    ref = oracle.bf16_to_f32(xb).astype(np.float64) @ oracle.bf16_to_f32(w).astype(np.float64).T
+    assert np.linalg.norm(r["y"] - ref) <= np.linalg.norm(r["y_plain"] - ref)
