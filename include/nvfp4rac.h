@@ -107,7 +107,10 @@ size_t nvfp4_workspace_size(int32_t op, int64_t M, int64_t N, int64_t K, int32_t
  *   supplied by the caller (skips the amax pass), or NULL.
  *   qx: rows = M, cols = K, codes/scales/tensor_scale written (either layout).
  *   score_or_null: fp64 [K] channel scores sum_i |dX_ij| in the fixed order;
- *   res_colamax_or_null: fp32 [K] max_i |dX_ij|.  Both or neither.
+ *   res_colamax_or_null: fp32 [K] max_i |dX_ij|.  Both, neither, or the
+ *   column maxima alone (a step that reuses an earlier channel mask needs
+ *   them for the residual tensor scale but no scores); scores without the
+ *   column maxima are refused.
  *   dX = RN(x - DQ(Q(x))) is formed in registers and never written.
  *   ws: nvfp4_workspace_size(NVFP4_OP_QUANTIZE, M, 0, K, 1) bytes.
  */
@@ -148,6 +151,18 @@ nvfp4_status rac_select(const uint16_t* x, int64_t M, int64_t K, int64_t ldx,
 nvfp4_status rac_select_channels(const double* score, const float* res_colamax, int64_t K, float k_percent,
                                  uint8_t* mask, int32_t* sel, int64_t* n_sel_out, float* res_tensor_scale,
                                  void* stream);
+
+/*
+ * rac_sel_tensor_scale -- tensor_scale (device fp32) = RN(max_{j in sel}
+ * colamax_j / 2688): the tensor scale of a second-pass operand over a given
+ * channel selection, e.g. the residual's for a step that reuses the channel
+ * mask of an earlier step (sel kept, colamax = this step's residual column
+ * maxima from nvfp4_quantize).  Pages: 2.2 B (second-pass quantization of
+ * the selected channels); keeping the mask across steps is a variant the
+ * pages do not describe.  sel: n_sel (>= 1) channel indices in [0, K).
+ */
+nvfp4_status rac_sel_tensor_scale(const float* colamax, int64_t K, const int32_t* sel, int64_t n_sel,
+                                  float* tensor_scale, void* stream);
 
 /*
  * rac_residual_quant -- the second half of rac_select: Q(dX_sel), the

@@ -30,7 +30,8 @@ EXPORTS = ["nvfp4_scale_bytes", "nvfp4_workspace_size", "nvfp4_quantize", "rac_s
            "w4a4_gemm_quantized", "moe_grouped_w4a4_rac_gemm", "weight_qdq",
            "nvfp4_encode_e2m1", "nvfp4_encode_e4m3", "nvfp4_stream_status",
            "nvfp4_check_bounded_wait", "nvfp4_status_string", "nvfp4_quantize_static_ws",
-           "nvfp4_dq_colamax", "rac_weight_quant_fp4", "rac_select_channels", "rac_residual_quant"]
+           "nvfp4_dq_colamax", "rac_weight_quant_fp4", "rac_select_channels", "rac_residual_quant",
+           "rac_sel_tensor_scale"]
 
 
 class _Tensor(ctypes.Structure):
@@ -53,6 +54,7 @@ _sig = {
     "nvfp4_dq_colamax": (I32, [TP, I32, P, P]),
     "rac_select_channels": (I32, [P, P, I64, F32, P, P, ctypes.POINTER(I64), P, P]),
     "rac_residual_quant": (I32, [P, I64, I64, I64, TP, P, I64, TP, P]),
+    "rac_sel_tensor_scale": (I32, [P, I64, P, I64, P, P]),
     "rac_weight_quant_fp4": (I32, [TP, P, I64, P, TP, P]),
     "w4a4_rac_gemm": (I32, [TP, TP, P, I64, P, I64, I64, TP, P, P, I32, I64, P, SZ, P]),
     "w4a4_gemm_quantized": (I32, [TP, TP, TP, TP, P, I32, I64, P]),
@@ -158,11 +160,12 @@ def _bits(x: torch.Tensor) -> torch.Tensor:
 
 def quantize(x, amax=None, layout=1, scores=True, out=None, stream=None):
     """Q(X) of bf16 x [M, K]; returns (qx, score fp64 [K], res_colamax fp32 [K])
-    (the last two None when scores=False)."""
+    (the last two None when scores=False; scores="colamax" gives the residual
+    column maxima without the scores)."""
     x = _bits(x)
     M, K = x.shape
     qx = out if out is not None else NvFP4Tensor.empty(M, K, layout, device=x.device)
-    score = torch.empty(K, dtype=torch.float64, device=x.device) if scores else None
+    score = torch.empty(K, dtype=torch.float64, device=x.device) if scores is True else None
     colamax = torch.empty(K, dtype=torch.float32, device=x.device) if scores else None
     nbytes = workspace_size(OP_QUANTIZE, M, 0, K)
     ws = _ws(nbytes, x.device)
@@ -222,6 +225,14 @@ def rac_select_channels(score, colamax, k_percent, res_tensor_scale=None, stream
                                     ctypes.byref(n_out), _ptr(st), _stream(stream)), "rac_select_channels")
     assert n_out.value == n_sel
     return mask, sel[:n_sel], n_sel, st
+
+
+def rac_sel_tensor_scale(colamax, sel, n_sel, out=None, stream=None):
+    """RN(max_{j in sel} colamax_j / 2688) as a device fp32 [1]."""
+    out = out if out is not None else torch.empty(1, dtype=torch.float32, device=colamax.device)
+    _check(_lib.rac_sel_tensor_scale(_ptr(colamax), colamax.numel(), _ptr(sel), n_sel, _ptr(out),
+                                     _stream(stream)), "rac_sel_tensor_scale")
+    return out
 
 
 def rac_residual_quant(x, qx, sel, n_sel, res_tensor_scale, layout=1, out=None, stream=None):
@@ -422,6 +433,11 @@ class RacLinearPlan:
                       rac_residual_quant, so the two gathers overlap)
       weight_select   rac_weight_quant -> Q(W_sel)
       gemm            w4a4_gemm_quantized -> Y
+    reuse_step() keeps the channel mask, sel and Q(W_sel) of the last step
+    that selected (the mask-reuse variant): it quantizes X with the residual
+    column maxima only (no scores, no top-k), takes the residual tensor scale
+    over the kept sel (rac_sel_tensor_scale), gathers Q(dX_sel) and runs the
+    GEMM.
     With wsel="fp4" the weight preparation also takes the column maxima of
     DQ(Q(W)) (nvfp4_dq_colamax) and weight_select re-quantizes W_sel from
     Q(W) (rac_weight_quant_fp4) instead of reading the bf16 W.
@@ -484,8 +500,10 @@ class RacLinearPlan:
                    "nvfp4_dq_colamax")
 
     def quantize(self, stream=None, scores=True):
+        """scores: True (scores and residual column maxima), False (codes
+        only) or "colamax" (residual column maxima only)."""
         _check(_lib.nvfp4_quantize(_ptr(self.x), self.M, self.K, self.x.stride(0), None, ctypes.byref(self._qx),
-                                   _ptr(self.score) if scores else None,
+                                   _ptr(self.score) if scores is True else None,
                                    _ptr(self.res_colamax) if scores else None, _ptr(self.ws),
                                    self.ws.numel(), _stream(stream)), "nvfp4_quantize")
 
@@ -569,10 +587,23 @@ class RacLinearPlan:
         main.wait_event(self._join)
         self.gemm()
 
+    def reuse_step(self):
+        """The rollout linear with the channel mask, sel and Q(W_sel) kept
+        from the last step that selected (see the class notes)."""
+        if self.n_sel == 0:
+            self.plain_step()
+            return
+        self.quantize(scores="colamax")
+        _check(_lib.rac_sel_tensor_scale(_ptr(self.res_colamax), self.K, _ptr(self.sel), self.n_sel,
+                                         _ptr(self.res_st), _stream(None)), "rac_sel_tensor_scale")
+        self.residual_quant()
+        self.gemm()
+
     def plain_step(self, stream=None):
         """Plain NVFP4 W4A4 (no RAC): Q(X) without scores, one-segment GEMM."""
         self.quantize(stream, scores=False)
         self.gemm(stream, plain=True)
 
     # kernels each call launches (for launch accounting)
-    LAUNCHES = dict(prepare_weight=2, quantize=2, quantize_plain=2, select=2, weight_select=1, gemm=1)
+    LAUNCHES = dict(prepare_weight=2, quantize=2, quantize_plain=2, select=2, weight_select=1, gemm=1,
+                    reuse_step=5)

@@ -205,13 +205,15 @@ nvfp4_status nvfp4_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ldx
                             const float* amax_or_null, nvfp4_tensor* qx, double* score_or_null,
                             float* res_colamax_or_null, void* ws, size_t ws_bytes, void* stream) {
   NV_CHECK(x && tensor_ok(qx), NVFP4_ERR_INVALID_ARG);
-  NV_CHECK((score_or_null == nullptr) == (res_colamax_or_null == nullptr), NVFP4_ERR_INVALID_ARG);
+  NV_CHECK(score_or_null == nullptr || res_colamax_or_null != nullptr, NVFP4_ERR_INVALID_ARG);
   NV_CHECK(M >= 1 && K >= 64 && K % 64 == 0 && ldx >= K && qx->rows == M && qx->cols == K,
            NVFP4_ERR_UNSUPPORTED_SHAPE);
   NV_CHECK(aligned16(x) && ldx % 8 == 0, NVFP4_ERR_MISALIGNED);
-  const bool scores = score_or_null != nullptr;
+  // stats: the residual column maxima (and with scores the channel sums)
+  // go through per-tile partials and the last CTA of each column strip
+  const bool scores = score_or_null != nullptr, stats = res_colamax_or_null != nullptr;
   Carver c(ws);
-  const QuantWs w = carve_quant(c, M, K, scores);
+  const QuantWs w = carve_quant(c, M, K, stats);
   NV_CHECK(ws != nullptr && ws_bytes >= c.off, NVFP4_ERR_WORKSPACE);
   const nvfp4_status d = device_ok();
   if (d != NVFP4_OK) return d;
@@ -223,13 +225,14 @@ nvfp4_status nvfp4_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ldx
   if (amax_or_null == nullptr) {
     n_parts = amax_parts_count(M, K);
     NV_TRY(launch_amax_partial(x, M, K, ldx, 1, 0, w.amax, n_parts, w.counters,
-                               scores ? static_cast<int>(K / 64) : 0, s));
-  } else if (scores) {
+                               stats ? static_cast<int>(K / 64) : 0, s));
+  } else if (stats) {
     NV_TRY(cudaMemsetAsync(w.counters, 0, sizeof(unsigned) * (K / 64), s));
   }
   NV_TRY(launch_quant_score(x, M, K, ldx, g, amax_or_null, w.amax, n_parts, M, qx->codes, qx->scales,
-                            qx->scale_layout, qx->tensor_scale, w.part_sum, w.part_max,
-                            scores ? w.counters : nullptr, score_or_null, res_colamax_or_null, s));
+                            qx->scale_layout, qx->tensor_scale, scores ? w.part_sum : nullptr,
+                            stats ? w.part_max : nullptr, stats ? w.counters : nullptr, score_or_null,
+                            res_colamax_or_null, s));
   return NVFP4_OK;
 }
 
@@ -292,6 +295,16 @@ nvfp4_status rac_residual_quant(const uint16_t* x, int64_t M, int64_t K, int64_t
   NV_TRY(launch_residual_gather(x, M, K, ldx, dense_groups(M), M, qx->codes, qx->scales, qx->scale_layout,
                                 qx->tensor_scale, sel, n_sel, q_res->cols, q_res->tensor_scale, q_res->codes,
                                 q_res->scales, q_res->scale_layout, static_cast<cudaStream_t>(stream)));
+  return NVFP4_OK;
+}
+
+nvfp4_status rac_sel_tensor_scale(const float* colamax, int64_t K, const int32_t* sel, int64_t n_sel,
+                                  float* tensor_scale, void* stream) {
+  NV_CHECK(colamax && sel && tensor_scale, NVFP4_ERR_INVALID_ARG);
+  NV_CHECK(K >= 1 && n_sel >= 1 && n_sel <= K, NVFP4_ERR_UNSUPPORTED_SHAPE);
+  const nvfp4_status d = device_ok();
+  if (d != NVFP4_OK) return d;
+  NV_TRY(launch_sel_tensor_scale(colamax, K, sel, n_sel, 1, tensor_scale, static_cast<cudaStream_t>(stream)));
   return NVFP4_OK;
 }
 

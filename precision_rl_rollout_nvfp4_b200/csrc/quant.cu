@@ -156,6 +156,9 @@ __device__ __forceinline__ float reduce_parts(const unsigned* parts, int n, uint
 // the tile's 32 group sums in order from shared memory.
 // ---------------------------------------------------------------------------
 // (4 CTAs per SM: measured faster than 3 with more registers)
+// SCORES: also the fp64 channel sums; without it the kernel writes the codes
+// alone (part_max == nullptr) or the codes and the residual column maxima.
+template <bool SCORES>
 __global__ void __launch_bounds__(kQThreads, 4)
 quant_score_kernel(const uint16_t* __restrict__ x, int64_t K, int64_t ldx, RowGroups g,
                    const float* __restrict__ amax, const unsigned* __restrict__ amax_parts,
@@ -225,8 +228,10 @@ quant_score_kernel(const uint16_t* __restrict__ x, int64_t K, int64_t ldx, RowGr
       f2_unpack(x2[j], x0, x1);
       const float d0 = fabsf(__fsub_rn(x0, __fmul_rn(p0, s_t)));
       const float d1 = fabsf(__fsub_rn(x1, __fmul_rn(p1, s_t)));
-      acc[2 * j] += static_cast<double>(d0);       // rows of the group in order
-      acc[2 * j + 1] += static_cast<double>(d1);
+      if (SCORES) {
+        acc[2 * j] += static_cast<double>(d0);     // rows of the group in order
+        acc[2 * j + 1] += static_cast<double>(d1);
+      }
       mx[2 * j] = fmaxf(mx[2 * j], d0);
       mx[2 * j + 1] = fmaxf(mx[2 * j + 1], d1);
     }
@@ -235,10 +240,12 @@ quant_score_kernel(const uint16_t* __restrict__ x, int64_t K, int64_t ldx, RowGr
     if ((cg & 1) == 0 && (layout == 1 || prow < codes_rows))
       scales[scale_offset(prow, col / kBlock, K, layout)] = static_cast<uint8_t>(bq.sb);
   }
-  if (part_sum == nullptr) return;
+  if (part_max == nullptr) return;
+  if (SCORES) {
 #pragma unroll
-  for (int j = 0; j < 8; j += 2)
-    *reinterpret_cast<double2*>(&gsum[grp][8 * cg + j]) = make_double2(acc[j], acc[j + 1]);
+    for (int j = 0; j < 8; j += 2)
+      *reinterpret_cast<double2*>(&gsum[grp][8 * cg + j]) = make_double2(acc[j], acc[j + 1]);
+  }
   *reinterpret_cast<float4*>(&gmax[grp][8 * cg]) = make_float4(mx[0], mx[1], mx[2], mx[3]);
   *reinterpret_cast<float4*>(&gmax[grp][8 * cg + 4]) = make_float4(mx[4], mx[5], mx[6], mx[7]);
   __syncthreads();
@@ -247,10 +254,10 @@ quant_score_kernel(const uint16_t* __restrict__ x, int64_t K, int64_t ldx, RowGr
     float m = 0.0f;
 #pragma unroll 8
     for (int q = 0; q < kGroups; ++q) {          // group order within the chunk
-      part += gsum[q][t];
+      if (SCORES) part += gsum[q][t];
       m = fmaxf(m, gmax[q][t]);
     }
-    part_sum[tile * K + col0 + t] = part;
+    if (SCORES) part_sum[tile * K + col0 + t] = part;
     part_max[tile * K + col0 + t] = m;
   }
   if (strip_count == nullptr) return;
@@ -281,19 +288,19 @@ quant_score_kernel(const uint16_t* __restrict__ x, int64_t K, int64_t ldx, RowGr
     __syncthreads();
     for (int k = t; k < nt * kQCols; k += kQThreads) {
       const int tt = k / kQCols, cc = k % kQCols;
-      ps[k] = __ldcg(part_sum + (c0 + tt) * K + col0 + cc);
+      if (SCORES) ps[k] = __ldcg(part_sum + (c0 + tt) * K + col0 + cc);
       pm[k] = __ldcg(part_max + (c0 + tt) * K + col0 + cc);
     }
     __syncthreads();
     if (t < kQCols) {
       for (int tt = 0; tt < nt; ++tt) {          // chunk order
-        total += ps[tt * kQCols + t];
+        if (SCORES) total += ps[tt * kQCols + t];
         tmax = fmaxf(tmax, pm[tt * kQCols + t]);
       }
     }
   }
   if (t < kQCols) {
-    score[static_cast<int64_t>(ti.e) * K + col0 + t] = total;
+    if (SCORES) score[static_cast<int64_t>(ti.e) * K + col0 + t] = total;
     colamax[static_cast<int64_t>(ti.e) * K + col0 + t] = tmax;
   }
   if (t == 0) *counter = 0;                      // ready for the next call
@@ -953,7 +960,8 @@ cudaError_t launch_quant_score(const uint16_t* x, int64_t rows, int64_t K, int64
   if (tiles == 0) return cudaSuccess;
   dim3 grid(static_cast<unsigned>(K / kQCols), static_cast<unsigned>(tiles));
   {
-    const cudaError_t le = launch_k(quant_score_kernel, dim3(grid), dim3(kQThreads), 0, s, nullptr, 0,
+    const cudaError_t le = launch_k(part_sum != nullptr ? quant_score_kernel<true> : quant_score_kernel<false>,
+                                    dim3(grid), dim3(kQThreads), 0, s, nullptr, 0,
                                    x, K, ldx, g, amax, amax_parts, n_parts, codes_rows, codes, scales,
                                    layout, tensor_scale, part_sum, part_max, strip_count, score, colamax);
     if (le != cudaSuccess) return le;

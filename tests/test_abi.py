@@ -130,3 +130,26 @@ def test_split_select_argument_errors_without_gpu(lib):
     assert g(p(0x1000), 64, 512, 512, ctypes.byref(qx), p(0x300), 300, ctypes.byref(qr), None) == 3   # width 320
     assert g(p(0x1000), 64, 512, 512, ctypes.byref(qx), p(0x300), 0, ctypes.byref(qr), None) == 3
     assert g(p(0x1008), 64, 512, 512, ctypes.byref(qx), p(0x300), 256, ctypes.byref(qr), None) == 2
+
+
+def test_sel_tensor_scale_argument_errors_without_gpu(lib):
+    f = lib.rac_sel_tensor_scale
+    f.restype = ctypes.c_int32
+    f.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p]
+    p = ctypes.c_void_p
+    assert f(None, 512, p(0x100), 8, p(0x200), None) == 1
+    assert f(p(0x100), 512, None, 8, p(0x200), None) == 1
+    assert f(p(0x100), 512, p(0x100), 8, None, None) == 1
+    assert f(p(0x100), 512, p(0x100), 0, p(0x200), None) == 3
+    assert f(p(0x100), 512, p(0x100), 513, p(0x200), None) == 3
+
+
+def test_quantize_refuses_scores_without_colamax(lib):
+    q = lib.nvfp4_quantize
+    q.restype = ctypes.c_int32
+    t = _fake_tensor(64, 64)
+    q.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p,
+                  ctypes.POINTER(_T), ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
+                  ctypes.c_void_p]
+    assert q(ctypes.c_void_p(0x1000), 64, 64, 64, None, ctypes.byref(t), ctypes.c_void_p(0x2000), None,
+             None, 0, None) == 1
