@@ -31,7 +31,8 @@
 // CTA loads its own tiles (no load is shared between CTAs).  Every mbarrier
 // wait is bounded (see common.cuh).
 //
-// For dense activations with at least 256 rows a second kernel runs the same
+// For dense activations with at least 256 rows (where its waves of tiles
+// take no longer; see dense_pair_pays) a second kernel runs the same
 // product on CTA pairs (tcgen05 cta_group::2): a pair computes a 256 x 256
 // tile, each CTA loading its own 128 rows of A and of B, so a pair fetches
 // half the operand bytes per FLOP of two 128 x 128 tiles; the leader's copier
@@ -945,10 +946,22 @@ cudaError_t launch_pair(const GemmArgs& a, cudaStream_t s) {
 
 }  // namespace
 
+// Dense: the CTA-pair kernel when its waves of 256 x 256 tiles over the SM
+// pairs take no longer than the single-CTA kernel's waves of 128 x 128
+// tiles over the SMs (a pair tile is twice a single tile's time on half as
+// many units), e.g. not for a 256-row product with few output columns.
+bool dense_pair_pays(int64_t M, int64_t N) {
+  if (M < 256) return false;
+  const int64_t sms = sm_count(), pairs = sms / 2;
+  const int64_t pt = ((M + 255) / 256) * ((N + 255) / 256);
+  const int64_t st = ((M + 127) / 128) * ((N + 127) / 128);
+  return 2 * ((pt + pairs - 1) / pairs) <= (st + sms - 1) / sms;
+}
+
 cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s) {
-  // dense activations with at least one full 256-row tile, and row groups
-  // (256-row tiles per group): the CTA-pair kernel
-  const bool pair_ok = a.g.off == nullptr ? a.M >= 256 : a.pair_start != nullptr;
+  // row groups (256-row tiles per group) and dense products where it pays:
+  // the CTA-pair kernel
+  const bool pair_ok = a.g.off == nullptr ? dense_pair_pays(a.M, a.N) : a.pair_start != nullptr;
   if (pair_ok && !gemm_force_single_cta())
     return a.y_dtype == 0 ? launch_pair<4>(a, s) : launch_pair<2>(a, s);
   cudaError_t e = a.y_dtype == 0 ? prepare_kernel<4>() : prepare_kernel<2>();

@@ -29,9 +29,11 @@ def _random_operand(b, rows, cols, rng, st):
 @pytest.mark.parametrize("M,N,K,W", [(128, 128, 256, 0), (128, 128, 64, 0), (256, 256, 512, 256),
                                      (300, 144, 320, 64), (1, 16, 64, 0), (130, 384, 1024, 192),
                                      (512, 512, 2048, 1024),
-                                     # M >= 256: CTA-pair kernel (256 x 256 tiles), ragged edges
                                      (600, 400, 320, 64), (1024, 2048, 4096, 0), (777, 272, 576, 448),
-                                     (512, 16, 64, 64)])
+                                     (512, 16, 64, 64),
+                                     # CTA-pair kernel (256 x 256 tiles: enough tiles for its waves
+                                     # to pay), ragged edges
+                                     (4000, 2000, 320, 64), (2560, 1040, 576, 448), (4096, 2048, 256, 0)])
 @pytest.mark.parametrize("out", ["f32", "bf16"])
 def test_gemm_on_random_operands(M, N, K, W, out):
     b = need_gpu()
