@@ -414,14 +414,8 @@ bool gemm_force_single_cta() {
 
 template <int YBYTES>
 cudaError_t prepare_kernel() {
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(w4a4_rac_gemm_kernel<YBYTES>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<YBYTES>::SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
-  return cudaSuccess;
+  static bool done[kMaxAttrDevices] = {};
+  return set_max_smem(w4a4_rac_gemm_kernel<YBYTES>, Cfg<YBYTES>::SMEM_BYTES, done);
 }
 
 // ===========================================================================
@@ -897,12 +891,10 @@ bool make_scale_map(CUtensorMap* tm, const uint8_t* scales, int64_t rows, int64_
 template <int YBYTES>
 cudaError_t launch_pair(const GemmArgs& a, cudaStream_t s) {
   using C = Cfg2<YBYTES>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(w4a4_rac_gemm_pair_kernel<YBYTES>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+  static bool done[kMaxAttrDevices] = {};
+  {
+    const cudaError_t e = set_max_smem(w4a4_rac_gemm_pair_kernel<YBYTES>, C::SMEM_BYTES, done);
     if (e != cudaSuccess) return e;
-    attr_set = true;
   }
   KParams2 p{};
   p.M = a.M;

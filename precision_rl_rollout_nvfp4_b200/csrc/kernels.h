@@ -19,6 +19,21 @@ namespace nvfp4 {
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn();
 int sm_count();
 
+// Kernel attributes (the dynamic shared-memory opt-in) belong to a device:
+// set_max_smem raises `kernel`'s limit to `bytes` once on each device the
+// library runs on (the flags of one kernel live in `done`, indexed by device).
+constexpr int kMaxAttrDevices = 64;
+template <typename... KArgs>
+cudaError_t set_max_smem(void (*kernel)(KArgs...), int bytes, bool (&done)[kMaxAttrDevices]) {
+  int dev = 0;
+  const cudaError_t ge = cudaGetDevice(&dev);
+  if (ge != cudaSuccess) return ge;
+  if (dev >= 0 && dev < kMaxAttrDevices && done[dev]) return cudaSuccess;
+  const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && dev >= 0 && dev < kMaxAttrDevices) done[dev] = true;
+  return e;
+}
+
 // Programmatic dependent launch is on unless NVFP4_NO_PDL=1.
 inline bool pdl_enabled() {
   static int v = -1;

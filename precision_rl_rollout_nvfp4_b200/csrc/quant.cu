@@ -1099,12 +1099,10 @@ cudaError_t launch_wsel_rows(const WselPlan& wp, const uint16_t* w, int64_t ldw,
                              int32_t E, const int32_t* sel, int64_t n_sel, int64_t width,
                              const float* colamax, int fuse, float* s_t, uint8_t* codes, uint8_t* scales,
                              int layout, cudaStream_t s) {
-  static bool attr_set = false;
-  if (!attr_set) {
-    const cudaError_t ae = cudaFuncSetAttribute(wsel_rows_kernel<FP4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                200 * 1024);
+  static bool done[kMaxAttrDevices] = {};
+  {
+    const cudaError_t ae = set_max_smem(wsel_rows_kernel<FP4>, 200 * 1024, done);
     if (ae != cudaSuccess) return ae;
-    attr_set = true;
   }
   int per_sm = 0;
   const cudaError_t oe =

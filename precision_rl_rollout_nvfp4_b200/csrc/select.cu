@@ -220,13 +220,12 @@ cudaError_t launch_topk(const double* score, const float* colamax, int64_t K, in
   const bool smem = K <= kMaxSmemKeys;
   const size_t bytes = smem ? static_cast<size_t>(K) * (sizeof(uint64_t) + sizeof(float)) : 0;
   // static plus dynamic shared memory can pass the 48 KB default: opt in
-  // once for the largest key buffer
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(kMaxSmemKeys * (sizeof(uint64_t) + sizeof(float))));
+  // once per device for the largest key buffer
+  static bool done[kMaxAttrDevices] = {};
+  {
+    const cudaError_t e =
+        set_max_smem(topk_kernel, static_cast<int>(kMaxSmemKeys * (sizeof(uint64_t) + sizeof(float))), done);
     if (e != cudaSuccess) return e;
-    attr_set = true;
   }
   {
     const cudaError_t le = launch_k(topk_kernel, dim3(E), dim3(kSelThreads), bytes, s, nullptr, 0,
