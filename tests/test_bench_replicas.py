@@ -53,3 +53,17 @@ def test_reference_arm_under_torchrun_prints_once():
     assert len(lines) == 1
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["value"] > 0 and d["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_reference_arm_of_the_variant_workloads():
+    """The oracle arm runs for the QAT workload and for the NVFP4-sourced
+    W_sel variant and prints one line each."""
+    for extra in (["--workload", "qat_w4a16_step"], ["--workload", "single_linear", "--wsel", "fp4"]):
+        cmd = [sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
+               "--warmup", "0", *extra]
+        r = subprocess.run(cmd, capture_output=True, text=True, timeout=300, cwd=ROOT)
+        assert r.returncode == 0, r.stderr[-2000:]
+        lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+        assert len(lines) == 1
+        d = json.loads(lines[0])
+        assert d["impl"] == "reference" and d["value"] > 0 and d["e2e"]["h2d_bytes_per_step"] == 0
