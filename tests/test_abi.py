@@ -153,3 +153,30 @@ def test_quantize_refuses_scores_without_colamax(lib):
                   ctypes.c_void_p]
     assert q(ctypes.c_void_p(0x1000), 64, 64, 64, None, ctypes.byref(t), ctypes.c_void_p(0x2000), None,
              None, 0, None) == 1
+
+
+def test_header_is_plain_c_and_links(tmp_path):
+    """include/nvfp4rac.h compiles as strict C99 and a C program links
+    against the library and calls its host-side size functions."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    src = tmp_path / "use_abi.c"
+    src.write_text(
+        '#include "nvfp4rac.h"\n'
+        "int main(void) {\n"
+        "  if (nvfp4_rac_width(1) != 64 || nvfp4_rac_width(65) != 128) return 1;\n"
+        "  if (nvfp4_rac_nsel(50.0f, 2048) != 1024) return 2;\n"
+        "  if (nvfp4_scale_bytes(300, 192, 1) != 384 * 4 * 3) return 3;\n"
+        "  if (nvfp4_workspace_size(99, 1, 1, 64, 1) != 0) return 4;\n"
+        "  return 0;\n}\n")
+    pkg = os.path.join(root, "precision_rl_rollout_nvfp4_b200")
+    exe = tmp_path / "use_abi"
+    cmd = [gcc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I", os.path.join(root, "include"),
+           str(src), os.path.join(pkg, "libnvfp4rac.so"), "-Wl,-rpath," + pkg, "-o", str(exe)]
+    r = subprocess.run(cmd, capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    assert subprocess.run([str(exe)]).returncode == 0
