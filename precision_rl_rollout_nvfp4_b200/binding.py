@@ -182,7 +182,7 @@ def quantize_static_ws(x, amax=None, layout=1, scores=True, out=None, stream=Non
     x = _bits(x)
     M, K = x.shape
     qx = out if out is not None else NvFP4Tensor.empty(M, K, layout, device=x.device)
-    score = torch.empty(K, dtype=torch.float64, device=x.device) if scores else None
+    score = torch.empty(K, dtype=torch.float64, device=x.device) if scores is True else None
     colamax = torch.empty(K, dtype=torch.float32, device=x.device) if scores else None
     st = qx.c()
     _check(_lib.nvfp4_quantize_static_ws(_ptr(x), M, K, x.stride(0), _ptr(amax), ctypes.byref(st),
