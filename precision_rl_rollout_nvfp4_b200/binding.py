@@ -483,11 +483,16 @@ class RacLinearPlan:
         self._nout = ctypes.c_int64(-1)
         self.x = None
         self.w = None
+        self.amax = None
 
-    def bind(self, x, w):
-        """Point the plan at device inputs x [M, K] and w [N, K] (bf16)."""
+    def bind(self, x, w, amax=None):
+        """Point the plan at device inputs x [M, K] and w [N, K] (bf16).
+        amax: optional device fp32 [1], a caller-supplied max|X| (e.g. from
+        calibration or an earlier step); the quantizer then skips its amax
+        pass (values above it saturate)."""
         assert tuple(x.shape) == (self.M, self.K) and tuple(w.shape) == (self.N, self.K)
         self.x, self.w = _bits(x), _bits(w)
+        self.amax = amax
         return self
 
     def prepare_weight(self, stream=None):
@@ -502,7 +507,8 @@ class RacLinearPlan:
     def quantize(self, stream=None, scores=True):
         """scores: True (scores and residual column maxima), False (codes
         only) or "colamax" (residual column maxima only)."""
-        _check(_lib.nvfp4_quantize(_ptr(self.x), self.M, self.K, self.x.stride(0), None, ctypes.byref(self._qx),
+        _check(_lib.nvfp4_quantize(_ptr(self.x), self.M, self.K, self.x.stride(0), _ptr(self.amax),
+                                   ctypes.byref(self._qx),
                                    _ptr(self.score) if scores is True else None,
                                    _ptr(self.res_colamax) if scores else None, _ptr(self.ws),
                                    self.ws.numel(), _stream(stream)), "nvfp4_quantize")
