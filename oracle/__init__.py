@@ -26,7 +26,11 @@ of 8 magnitudes per sign, round trips of every code under every scale,
 QDQ idempotence, the error bound of the grid, brute-force top-k on tiny
 inputs, k = 0 / k = 100 reductions, the fp64 product against a plain loop,
 the scalar restatement, and "RAC error <= plain W4A4 error" against the bf16
-product.
+product.  The opt-in variants are pinned the same way: W_sel from the NVFP4
+weights (scalar restatement, weights already on the grid), a channel mask
+kept from an earlier call (equal to the per-call linear under its own mask;
+an empty mask gives the plain product), and the QAT linear (grid-exact
+operands reduce it to the plain linear and the textbook gradients).
 """
 from . import formats, nvfp4, qat, rac, scalar  # noqa: F401
 from .formats import (bf16_to_f32, e2m1_decode, e2m1_encode, e4m3_decode,  # noqa: F401
