@@ -22,8 +22,8 @@
  *     sb = E4M3(RN(amax_b / RN(6 s_t))),  s_dec = RN(E4M3dec(sb) s_t),
  *     code = E2M1(RN(x / s_dec)),         DQ = RN(RN(E2M1dec E4M3dec) s_t),
  * channel scores score_j = sum_i |dX_ij| in fp64 (rows in chunks of 128
- * from row 0; a chunk is the in-order sum of its 32 groups of 4 rows, each
- * group summed in row order; chunk sums added in chunk order),
+ * from row 0, each chunk summed row by row in row order, the chunk sums
+ * added in chunk order; every addition rounded to nearest even),
  * n_sel = floor(k K / 100), ties to the lower channel, sel ascending, and
  * dX_sel / W_sel re-quantized with their own tensor scales.
  *

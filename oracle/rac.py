@@ -18,12 +18,12 @@ same product:
     Y = DQ(Q(X)) DQ(Q(W))^T + DQ(Q(dX_sel)) DQ(Q(W_sel))^T
 
 which is what this module computes.  Readings adopted where the pages are
-silent (each is listed with its reason in the design notes):
+silent (each is listed because the pages leave it open):
   * dX = RN(X - DQ(Q(X))) in fp32, never rounded to bf16;
   * score_j = sum over tokens of |dX_ij| in fp64, in a fixed order: rows in
-    consecutive chunks of 128 (from row 0); a chunk is 32 consecutive groups
-    of 4 rows, each group summed from 0.0 in row order, the group sums added
-    from 0.0 in group order; the chunk sums are added in chunk order;
+    consecutive chunks of 128 (from row 0), each chunk summed from 0.0 in row
+    order, then the chunk sums added from 0.0 in chunk order (one fixed
+    order, so that the ranking and the mask are reproducible bit for bit);
   * n_sel = floor(k * K / 100) with k taken exactly;
   * the n_sel largest scores win, ties to the lower channel index, and sel is
     listed in ascending channel order;
@@ -43,7 +43,6 @@ from .nvfp4 import (BLOCK, F32, amax, block_values, dequantize, quantize,
                     tensor_scale)
 
 SCORE_CHUNK = 128
-SCORE_GROUP = 4
 
 
 def n_selected(k_percent, K: int) -> int:
@@ -62,19 +61,16 @@ def residual(x, codes, scales, s_t):
 
 def channel_score(dx):
     """score_j (fp64, fixed order) and colamax_j = max_i |dX_ij| (fp32).
-    Order: chunks of 128 rows, each the sum in group order of its 32 groups
-    of 4 consecutive rows, each group summed in row order (rows past M add
-    nothing); chunk sums added in chunk order."""
+    Order: rows in chunks of 128 from row 0; a chunk is summed from 0.0 row
+    by row in row order; the chunk sums are added from 0.0 in chunk order.
+    Every addition is one fp64 operation rounded to nearest even."""
     a = np.abs(np.asarray(dx, F32))
     M, K = a.shape
     score = np.zeros(K, np.float64)
     for c0 in range(0, M, SCORE_CHUNK):
         part = np.zeros(K, np.float64)
-        for g0 in range(c0, min(c0 + SCORE_CHUNK, M), SCORE_GROUP):
-            grp = np.zeros(K, np.float64)
-            for r in range(g0, min(g0 + SCORE_GROUP, M)):
-                grp = grp + a[r].astype(np.float64)
-            part = part + grp
+        for r in range(c0, min(c0 + SCORE_CHUNK, M)):
+            part = part + a[r].astype(np.float64)
         score = score + part
     colamax = a.max(axis=0) if M else np.zeros(K, F32)
     return score, colamax.astype(F32)

@@ -105,11 +105,8 @@ def rac_linear(x_bits, w_bits, k_percent, wsel_source="bf16"):
         total = 0.0
         for c0 in range(0, M, 128):
             part = 0.0
-            for g0 in range(c0, min(c0 + 128, M), 4):
-                grp = 0.0
-                for i in range(g0, min(g0 + 4, M)):
-                    grp += abs(dx[i][j])
-                part += grp
+            for i in range(c0, min(c0 + 128, M)):
+                part += abs(dx[i][j])
             total += part
         score[j] = total
     n_sel = math.floor(k_percent * K / 100)

@@ -58,6 +58,50 @@ def test_score_order_and_bound():
     assert np.array_equal(qa["res_colamax"], np.abs(qa["dx"]).max(axis=0))
 
 
+def test_score_order_is_rows_then_chunks():
+    """channel_score adds the rows of each 128-row chunk one by one in row
+    order, then the chunk sums in chunk order, each addition rounded to the
+    nearest fp64 (ties to even).  The columns below are built so that this
+    order, a grouped order, a reversed order and the exactly rounded sum all
+    give different fp64 results; the expected values follow from IEEE
+    binary64 rounding alone (u = 2^-53 is half an ulp of 1.0):
+      col 0: 1, then 127 x u           -> 1 + u is a tie, rounds to 1 each
+                                          time: 1.0 (exact sum rounds to
+                                          1 + 2^-46; groups of 4 give
+                                          1 + 31 * 2^-51)
+      col 1: 127 x u, then 1           -> 127 u is exact; 1 + 127 u =
+                                          1 + 63.5 * 2^-52 ties to even:
+                                          1 + 2^-46 (reversed order gives 1)
+      col 2: 1 at row 0, u at rows 128 and 129
+                                       -> chunk sums 1 and 2u = 2^-52:
+                                          1 + 2^-52 (one sequential pass over
+                                          all rows would give 1)
+      col 3: 1, u, u in chunks 0, 1, 2  -> (1 + u) + u: 1.0 (adding the two
+                                          small chunks first gives 1 + 2^-52)
+    """
+    u = 2.0 ** -53
+    dx = np.zeros((3 * 128, 4), F32)
+    dx[0, 0] = 1.0
+    dx[1:128, 0] = u
+    dx[0:127, 1] = u
+    dx[127, 1] = 1.0
+    dx[0, 2] = 1.0
+    dx[128, 2] = u
+    dx[129, 2] = u
+    dx[0, 3] = 1.0
+    dx[128, 3] = u
+    dx[256, 3] = u
+    score, colamax = oracle.channel_score(-dx)          # |dX|: the sign does not matter
+    assert score[0] == 1.0
+    assert score[1] == 1.0 + 2.0 ** -46
+    assert score[2] == 1.0 + 2.0 ** -52
+    assert score[3] == 1.0
+    assert np.array_equal(colamax, np.array([1.0, 1.0, 1.0, 1.0], F32))
+    # the other orders named above really differ on these columns
+    assert math.fsum(dx[:, 0].astype(np.float64)) != score[0]
+    assert math.fsum(dx[:, 1].astype(np.float64)) == 1.0 + 2.0 ** -46
+
+
 def test_k0_is_plain_w4a4_and_k100_is_full_residual():
     x = S.activations(64, 128, seed=4)
     w = S.weights(96, 128, seed=4)
