@@ -1,17 +1,21 @@
 #!/usr/bin/env python
 """Benchmark of the NVFP4 W4A4 + RAC rollout linear on B200.
 
-One step = one pass of the whole path over one batch of the dense rollout
-projection (X bf16 4096 x 2048, W bf16 2048 x 2048, RAC k = 50%):
-    weight_qdq(W)                 W' , Q(W), colamax_W   (trainer-side QDQ)
+Default workload: large prefill + trainer QDQ.  One step is one pass of the
+whole path over one batch:
+    weight_qdq(W)                 W', Q(W), colamax_W   (weight preparation)
     nvfp4_quantize(X)             Q(X), channel scores, residual col-max
     rac_select                    top-k% mask, sel, Q(dX_sel)
     rac_weight_quant              Q(W_sel)
     w4a4_gemm_quantized           Y = s s' A B^T + s_R s_Ws R Ws^T  (bf16)
+for X bf16 32768 x 4096, W bf16 4096 x 4096, RAC k = 50%, plus the trainer's
+W4A16 fake quantization weight_qdq over 64 experts x (1024 x 2048 and
+2048 x 1024) bf16 weights (independent of the linear, on its own stream).
 The metric is the effective throughput of the RAC linear, 2 M N (K + n_sel)
 FLOPs per step over the whole step time, in TFLOP/s; the JSON line also
 carries the GEMM TFLOP/s, the quantizer GB/s, the RAC overhead over plain
-W4A4, per-call times and the roofline of the dominant kernel.
+W4A4, the expert QDQ time and GB/s, per-call times, a bf16 GEMM of the same
+shape for comparison and the roofline of the dominant kernel.
 
 Multi-GPU: every rank runs an independent replica on its own batch (the path
 has no exchange step), value = all ranks' FLOPs / max-over-ranks time.
@@ -42,7 +46,10 @@ WORKLOADS = {
     "single_linear": (64, 512, 512, 50.0),
     "large_prefill": (32768, 4096, 4096, 50.0),
 }
-DEFAULT_WORKLOAD = "dense_rollout_projection"
+DEFAULT_WORKLOAD = "large_prefill"
+# trainer-side W4A16 QDQ of a stacked expert weight set that runs with a
+# workload's step: workload -> (experts, [(N, K) of each stacked weight])
+QDQ_EXPERTS = {"large_prefill": (64, [(1024, 2048), (2048, 1024)])}
 # grouped MoE expert FFN (up 2048 -> 1024, down 1024 -> 2048 over 64 experts,
 # 8192 tokens routed top-8): its own step, see run_moe
 MOE_WORKLOAD = "moe_expert_ffn"
@@ -53,6 +60,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 ORACLE_SAMPLE_ROWS = 1024
 L2_FLUSH_BYTES = 256 << 20
 PER_CALL_REPS = 10
+PER_CALL_SAMPLES = 20       # per-call graphs of PER_CALL_REPS launches timed this many times
 
 
 def parse_args():
@@ -88,7 +96,11 @@ def load_peaks():
 
 # ---------------------------------------------------------------- algorithmic work
 def work(M, K, N, n_sel, width, wsel="bf16", static_amax=False):
-    """Algorithmic FLOPs / bytes per call (see the design notes).  With
+    """Algorithmic FLOPs / bytes per call.  Bytes count every tensor a call
+    must read or write once: X is read twice by the quantizer (its amax is a
+    global dependency of every code) unless the caller supplies amax; the
+    residual gather reads the selected channels of X plus their codes and
+    scales; the GEMM reads the FP4 operands and writes bf16 Y.  With
     wsel="fp4" the weight preparation also reads Q(W) once for the DQ column
     maxima, and W_sel is gathered from the 0.5625 B/element NVFP4 weight."""
     fp4 = wsel == "fp4"
@@ -104,20 +116,41 @@ def work(M, K, N, n_sel, width, wsel="bf16", static_amax=False):
 
 
 # ---------------------------------------------------------------- clocks
+def gpu_selector(local_rank):
+    """The `nvidia-smi -i` argument that names the GPU this process runs on:
+    its UUID ("GPU-..."), else its PCI bus id.  nvidia-smi ignores
+    CUDA_VISIBLE_DEVICES, so a bare index could name another GPU of the
+    machine.  None when neither is known."""
+    try:
+        import torch
+        props = torch.cuda.get_device_properties(local_rank)
+    except Exception:
+        return None
+    u = str(getattr(props, "uuid", "") or "")
+    if u:
+        return u if u.startswith("GPU-") else "GPU-" + u
+    try:
+        return f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+    except AttributeError:
+        return None
+
+
 class ClockSampler:
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, index):
-        self.index = index
+    def __init__(self, local_rank):
+        self.gpu = gpu_selector(local_rank)
         self.proc = None
         self.path = os.path.join("/tmp", f"nvfp4_clocks_{os.getpid()}.csv")
 
     def __enter__(self):
+        if self.gpu is None:              # unknown identity: sample nothing rather than another GPU
+            return self
         try:
             self.f = open(self.path, "w")
-            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", self.gpu, f"--query-gpu={self.FIELDS}",
                                           "--format=csv,noheader,nounits", "-lms", "100"],
                                          stdout=self.f, stderr=subprocess.DEVNULL)
             time.sleep(0.3)
@@ -152,7 +185,7 @@ class ClockSampler:
         loaded = [float(r[1]) for r in rows if re.match(r"^[0-9.]+$", r[3]) and float(r[3]) > 250.0]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.strip().lower() == "active"})
-        return {"sm_mhz": statistics.median(loaded or sm) if (loaded or sm) else None,
+        return {"gpu": self.gpu, "sm_mhz": statistics.median(loaded or sm) if (loaded or sm) else None,
                 "sm_max_mhz": float(rows[0][2]) if rows[0][2].replace(".", "").isdigit() else None,
                 "reasons": reasons, "samples": len(rows), "samples_under_load": len(loaded),
                 "power_w_max": max(power) if power else None}
@@ -261,6 +294,38 @@ def replica_seed(rank):
 
 
 # ---------------------------------------------------------------- ours
+class ExpertQDQ:
+    """The trainer-side W4A16 fake quantization of a stacked expert weight
+    set (one weight_qdq call per stacked weight shape), with preallocated
+    outputs and workspaces, so it can be captured in a CUDA graph."""
+
+    def __init__(self, B, experts, shapes, seed, dev, hosts=None):
+        import torch
+
+        from precision_rl_rollout_nvfp4_b200 import synthetic as S
+        self.B = B
+        self.hosts, self.w, self.out, self.ws = [], [], [], []
+        for i, (n, kk) in enumerate(shapes):
+            h = (S.weights(n, kk, seed, batch=experts, stream=S.STREAM_W + 10 * i).pin_memory()
+                 if hosts is None else hosts[i])
+            self.hosts.append(h)
+            self.w.append(h.to(dev))
+            self.out.append(torch.empty(experts, n, kk, dtype=torch.bfloat16, device=dev))
+            self.ws.append(torch.empty(B.workspace_size(B.OP_WEIGHT_QDQ, 0, n, kk, experts),
+                                       dtype=torch.uint8, device=dev))
+        self.shapes, self.experts = shapes, experts
+        self.elements = sum(experts * n * kk for n, kk in shapes)
+
+    def run(self, stream=None):
+        for w, out, ws in zip(self.w, self.out, self.ws):
+            self.B.weight_qdq(w, want_q=False, want_colamax=False, out=out, stream=stream, ws=ws)
+
+    def bytes(self):
+        """Algorithmic bytes: W read twice (amax, then the quantization) and
+        W' written once, 2 bytes each."""
+        return 6.0 * self.elements
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -285,14 +350,37 @@ def run_ours(args, rank, world, local_rank):
     calls = ["prepare_weight", "quantize", "select", "weight_select", "gemm"]
     fns = {"prepare_weight": plan.prepare_weight, "quantize": plan.quantize, "select": plan.select,
            "weight_select": plan.weight_select, "gemm": plan.gemm}
-
     reuse = args.mask == "reuse"
+    qdq = None
+    if args.workload in QDQ_EXPERTS and not reuse:
+        E_q, shapes = QDQ_EXPERTS[args.workload]
+        qdq = ExpertQDQ(B, E_q, shapes, seed, dev)
+        calls.append("qdq_experts")
+        fns["qdq_experts"] = qdq.run
+    qstream = torch.cuda.Stream(device=dev)
+    q_fork, q_join = torch.cuda.Event(), torch.cuda.Event()
+
+    def linear_step(p):
+        if reuse:
+            p.reuse_step()                    # mask, sel and Q(W_sel) kept from the warm-up
+        else:
+            p.full_step()                     # weight prep overlapped on a side stream
+
+    def step_with(p, q):
+        """The linear on the current stream; the expert QDQ (independent of
+        it) on its own stream, forked from and joined back into the current one."""
+        main = torch.cuda.current_stream()
+        if q is not None:
+            q_fork.record(main)
+            qstream.wait_event(q_fork)
+            q.run(stream=qstream)
+            q_join.record(qstream)
+        linear_step(p)
+        if q is not None:
+            main.wait_event(q_join)
 
     def full_step():
-        if reuse:
-            plan.reuse_step()                 # mask, sel and Q(W_sel) kept from the warm-up
-        else:
-            plan.full_step()                  # weight prep overlapped on a side stream
+        step_with(plan, qdq)
 
     # warm-up (also sets kernel attributes before any capture; with --mask
     # reuse the first full step selects the mask the timed steps keep)
@@ -362,7 +450,8 @@ def run_ours(args, rank, world, local_rank):
 
     # per-call breakdown: each call's average launch duration with L2
     # flushed before every launch, from one graph of PER_CALL_REPS (flush,
-    # call) pairs minus a graph of the flushes alone (no replay gaps inside)
+    # call) pairs minus a graph of the flushes alone (no replay gaps inside),
+    # sampled PER_CALL_SAMPLES times
     per_call = {c: [] for c in calls}
 
     def reps_graph(fn):
@@ -385,13 +474,13 @@ def run_ours(args, rank, world, local_rank):
         g_flush = reps_graph(lambda: None)
         g_calls = {c: reps_graph(fns[c]) for c in calls}
         torch.cuda.synchronize()
-        for _ in range(max(1, min(args.steps, 5))):
+        for _ in range(PER_CALL_SAMPLES):
             base = time_graph(g_flush)
             for c in calls:
                 per_call[c].append(max(time_graph(g_calls[c]) - base, 0.0) / PER_CALL_REPS)
         del g_flush, g_calls
     else:
-        for _ in range(args.steps):
+        for _ in range(max(args.steps, PER_CALL_SAMPLES)):
             flush.zero_()
             evs = [ev()]
             for c in calls:
@@ -410,28 +499,51 @@ def run_ours(args, rank, world, local_rank):
         if reuse:
             launch("step")
         else:
-            for name in calls[1:]:
+            for name in ("quantize", "select", "weight_select", "gemm"):
                 launch(name)
         d = ev()
         torch.cuda.synchronize()
         plain_ms.append(a.elapsed_time(b_))
         rac_ms.append(c.elapsed_time(d))
 
+    # bf16 comparator: the same product Y = X W^T as one torch (cuBLAS) bf16
+    # GEMM, timed the same way (a comparison only; not part of the step)
+    y_bf16 = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+
+    def bf16_gemm():
+        torch.matmul(x, w.t(), out=y_bf16)
+
+    bf16_gemm()
+    bf16_ms = []
+    for _ in range(max(args.steps, 5)):
+        flush.zero_()
+        a = ev(); bf16_gemm(); b_ = ev()
+        torch.cuda.synchronize()
+        bf16_ms.append(a.elapsed_time(b_))
+    del y_bf16
+
     # ---- end to end through the API from pinned host buffers (two buffer
     # sets, copies overlapped with the neighbouring steps' compute)
     x1, w1 = torch.empty_like(x), torch.empty_like(w)
     plan1 = B.RacLinearPlan(M, K, N, k, out_dtype=torch.bfloat16, device=dev, wsel=args.wsel).bind(x1, w1, amax)
+    qdq1 = ExpertQDQ(B, qdq.experts, qdq.shapes, seed, dev, hosts=qdq.hosts) if qdq is not None else None
     if reuse:                                 # weights resident; both plans select once, then reuse
         x1.copy_(x_host)
         w1.copy_(w_host)
         plan1.full_step()
         torch.cuda.synchronize()
-    sets = [{"h2d": [(x, x_host)] + ([] if reuse else [(w, w_host)]),
-             "d2h": [(torch.empty(M, N, dtype=torch.bfloat16).pin_memory(), plan.y)],
-             "step": plan.reuse_step if reuse else plan.full_step},
-            {"h2d": [(x1, x_host)] + ([] if reuse else [(w1, w_host)]),
-             "d2h": [(torch.empty(M, N, dtype=torch.bfloat16).pin_memory(), plan1.y)],
-             "step": plan1.reuse_step if reuse else plan1.full_step}]
+
+    def h2d(p_x, p_w, q):
+        pairs = [(p_x, x_host)] + ([] if reuse else [(p_w, w_host)])
+        if q is not None:
+            pairs += [(dst, src) for dst, src in zip(q.w, qdq.hosts)]
+        return pairs
+
+    sets = [{"h2d": h2d(x, w, qdq), "d2h": [(torch.empty(M, N, dtype=torch.bfloat16).pin_memory(), plan.y)],
+             "step": lambda: step_with(plan, qdq)},
+            {"h2d": h2d(x1, w1, qdq1), "d2h": [(torch.empty(M, N, dtype=torch.bfloat16).pin_memory(), plan1.y)],
+             "step": lambda: step_with(plan1, qdq1)}]
+    h2d_bytes = sum(dst.numel() * dst.element_size() for dst, _ in sets[0]["h2d"])
     e2e_ms = e2e_pipelined(sets, args.steps, max(args.warmup, 2))
     if B.stream_status() != 0:
         raise RuntimeError("device error word set during timing")
@@ -445,55 +557,82 @@ def run_ours(args, rank, world, local_rank):
     e2e_value = flops_step * world * args.steps / (e2e_total * 1e-3) / 1e12
     med = {c: statistics.median(v) for c, v in per_call.items()}
     wk = work(M, K, N, n_sel, width, args.wsel, args.static_amax)
+    if qdq is not None:
+        wk["qdq_experts"] = dict(bytes=qdq.bytes(), bound="hbm")
     peaks, peak_kind = load_peaks()
     hbm_peak = peaks["hbm_gbs"]
-    fp4_peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]) * FP4_OVER_BF16
+    # per-call kernels are timed alone, in bursts: the burst bf16 peak; the
+    # whole step is a long loop: the sustained one
+    fp4_burst = peaks["bf16_tflops"] * FP4_OVER_BF16
+    fp4_sustained = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]) * FP4_OVER_BF16
     dominant = max(med, key=med.get)
     d = wk[dominant]
     dur = med[dominant] * 1e-3
     traffic = profiled_traffic(dominant, args.workload)
+    traffic_source = (f"profiles/dram_traffic.md, ncu dram__bytes_read.sum + dram__bytes_write.sum per launch, "
+                      f"kernel sources sha256 {kernel_sources_hash()}") if traffic is not None else None
     if d["bound"] == "tensor":
         achieved = d["flops"] / dur / 1e12
         roof = {"kernel": dominant, "bound": "tensor", "achieved": round(achieved, 1),
-                "peak": round(fp4_peak, 1), "unit": "TFLOP/s", "frac": round(achieved / fp4_peak, 4),
-                "traffic": traffic, "peak_source": f"{peak_kind}: bf16 sustained x {FP4_OVER_BF16:g} (FP4/BF16 nominal)"}
+                "peak": round(fp4_burst, 1), "unit": "TFLOP/s", "frac": round(achieved / fp4_burst, 4),
+                "traffic": traffic, "traffic_source": traffic_source,
+                "peak_source": f"{peak_kind}: bf16 burst x {FP4_OVER_BF16:g} (FP4/BF16 nominal); kernel timed alone"}
     else:
         achieved = d["bytes"] / dur / 1e9
         roof = {"kernel": dominant, "bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak,
                 "unit": "GB/s", "frac": round(achieved / hbm_peak, 4), "traffic": traffic,
-                "peak_source": f"{peak_kind}: hbm_gbs"}
+                "traffic_source": traffic_source, "peak_source": f"{peak_kind}: hbm_gbs"}
     gemm_tflops = wk["gemm"]["flops"] / (med["gemm"] * 1e-3) / 1e12
     quant_gbs = wk["quantize"]["bytes"] / (med["quantize"] * 1e-3) / 1e9
     rac_over = (statistics.median(rac_ms) - statistics.median(plain_ms)) / statistics.median(plain_ms)
+    bf16_us = 1e3 * statistics.median(bf16_ms)
     launches_per_step = ((plan.launches["reuse_step"] if n_sel else 3) if reuse else
-                         sum(plan.launches[c] for c in calls) - (0 if n_sel else 2)) \
+                         sum(plan.launches[c] for c in calls if c in plan.launches) - (0 if n_sel else 2)) \
         - (1 if args.static_amax else 0)          # no amax pass
+    if qdq is not None:
+        launches_per_step += 2 * len(qdq.shapes)  # amax pass + quantization per stacked weight
 
+    cfg = {"workload": args.workload, "M": M, "K": K, "N": N, "k_percent": k, "n_sel": n_sel,
+           "y_dtype": "bf16", "wsel": args.wsel, "mask": args.mask,
+           "amax": "caller-supplied" if args.static_amax else "computed per call",
+           "parallelism": f"replicas x{world}",
+           "l2": "flushed between steps and before every per-call launch (256 MiB write)",
+           "cuda_graph": use_graph}
+    if qdq is not None:
+        cfg["qdq_experts"] = {"experts": qdq.experts, "shapes": [list(sh) for sh in qdq.shapes],
+                              "stream": "own stream, overlapped with the linear"}
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s (effective 2MN(K+n_sel) per step)",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4 (e2m1/ue4m3) x fp32 acc",
         "data": "synthetic, seeded: X = N(0,1) x per-channel exp(N(0,1)) scales with 1% outlier channels x20, W = N(0, 0.02^2), bf16",
-        "config": {"workload": args.workload, "M": M, "K": K, "N": N, "k_percent": k, "n_sel": n_sel,
-                   "y_dtype": "bf16", "wsel": args.wsel, "mask": args.mask,
-                   "amax": "caller-supplied" if args.static_amax else "computed per call",
-                   "parallelism": f"replicas x{world}", "l2": "flushed between steps and before every per-call launch (256 MiB write)",
-                   "cuda_graph": use_graph},
+        "config": cfg,
         "useful_tflops": round(2.0 * M * N * K * world * args.steps / (total_ms * 1e-3) / 1e12, 2),
-        "gemm_tflops": round(gemm_tflops, 1), "gemm_frac_fp4_peak": round(gemm_tflops / fp4_peak, 4),
+        "gemm_tflops": round(gemm_tflops, 1), "gemm_frac_fp4_peak": round(gemm_tflops / fp4_burst, 4),
         "quantizer_gbs": round(quant_gbs, 1), "quantizer_frac_hbm": round(quant_gbs / hbm_peak, 4),
         "rac_overhead_pct": round(100 * rac_over, 1),
         "plain_w4a4_linear_us": round(1e3 * statistics.median(plain_ms), 2),
         "rac_linear_us": round(1e3 * statistics.median(rac_ms), 2),
+        "bf16_gemm_us": round(bf16_us, 2),
+        "bf16_gemm_tflops": round(2.0 * M * N * K / (bf16_us * 1e-6) / 1e12, 1),
+        "fp4_gemm_speedup_over_bf16": round(bf16_us / (1e3 * med["gemm"]), 3),
         "per_call_us": {c: round(1e3 * v, 2) for c, v in med.items()},
+        "per_call_samples": len(next(iter(per_call.values()))),
+        "peaks": {"fp4_burst_tflops": round(fp4_burst, 1), "fp4_sustained_tflops": round(fp4_sustained, 1),
+                  "hbm_gbs": hbm_peak, "source": peak_kind},
         "roofline": roof,
         "e2e": {"value": round(e2e_value, 3), "unit": "TFLOP/s",
-                "h2d_bytes_per_step": int(2 * (M * K + (0 if reuse else N * K))),
-                "d2h_bytes_per_step": int(2 * M * N), "ms_per_step": round(e2e_total / args.steps, 4),
+                "h2d_bytes_per_step": int(h2d_bytes), "d2h_bytes_per_step": int(2 * M * N),
+                "ms_per_step": round(e2e_total / args.steps, 4),
                 "pipelined": "2 buffer sets; H2D, compute and D2H on separate streams"},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clock,
     }
+    if qdq is not None:
+        q_us = 1e3 * med["qdq_experts"]
+        line["qdq_experts_us"] = round(q_us, 2)
+        line["qdq_experts_gbs"] = round(qdq.bytes() / (q_us * 1e-6) / 1e9, 1)
+        line["qdq_experts_frac_hbm"] = round(qdq.bytes() / (q_us * 1e-6) / 1e9 / hbm_peak, 4)
     return line
 
 
@@ -808,18 +947,41 @@ def run_qat(args, rank, world, local_rank):
 
 
 # ---------------------------------------------------------------- oracle (CPU)
-def oracle_step_time(M, K, N, k, rows, seed=0, wsel="bf16"):
+_ORACLE_INPUTS = {}
+
+
+def oracle_step_time(M, K, N, k, rows, seed=0, wsel="bf16", qdq_shapes=()):
+    """One oracle step on a bounded sample of the workload: weight_qdq(W),
+    then the RAC linear of the first `rows` rows of X taken as a batch of
+    their own (their own amax, scores and mask), and weight_qdq of one expert
+    of every stacked shape in `qdq_shapes`."""
     import numpy as np
 
     import oracle
     from precision_rl_rollout_nvfp4_b200 import synthetic as S
-    x = S.bf16_bits(S.activations(M, K, seed=seed))[:rows]
-    w = S.bf16_bits(S.weights(N, K, seed=seed))
+    key = (M, K, N, rows, seed, tuple(qdq_shapes))
+    if key not in _ORACLE_INPUTS:
+        x = S.bf16_bits(S.activations(rows, K, seed=seed))     # the first `rows` rows of X
+        w = S.bf16_bits(S.weights(N, K, seed=seed))
+        experts = [S.bf16_bits(S.weights(n, kk, seed, batch=1, stream=S.STREAM_W + 10 * i))[0]
+                   for i, (n, kk) in enumerate(qdq_shapes)]
+        _ORACLE_INPUTS[key] = (x, w, experts)
+    x, w, experts = _ORACLE_INPUTS[key]
     t0 = time.perf_counter()
     wq = oracle.weight_qdq(w)
     r = oracle.rac_linear(x, w, k, wq=wq, wsel_source=wsel)
+    for we in experts:
+        oracle.weight_qdq(we)
     dt = time.perf_counter() - t0
     return dt, 2.0 * rows * N * (K + r["n_sel"]), np.asarray(r["y"]).shape
+
+
+def oracle_sample_text(M, K, N, rows, qdq_shapes):
+    t = (f"weight_qdq(W {N}x{K}) + the RAC linear of the first {rows} of {M} rows of X as a batch of "
+         f"their own (own amax, scores and mask)")
+    if qdq_shapes:
+        t += " + weight_qdq of one expert of each stacked shape " + ", ".join(f"{n}x{kk}" for n, kk in qdq_shapes)
+    return t + " (numpy oracle; fp64 product via BLAS)"
 
 
 def oracle_qat_time(M, K, N, act, rows, seed=0):
@@ -896,17 +1058,17 @@ def cpu_baseline(args, budget_s=12.0):
     M, K, N, k = WORKLOADS[args.workload]
     k = args.k if args.k is not None else k
     rows = min(M, ORACLE_SAMPLE_ROWS)
+    shapes = QDQ_EXPERTS[args.workload][1] if args.workload in QDQ_EXPERTS else ()
     t, flops, n = 0.0, 0.0, 0
     while t < budget_s or n == 0:
-        dt, f, _ = oracle_step_time(M, K, N, k, rows, wsel=args.wsel)
+        dt, f, _ = oracle_step_time(M, K, N, k, rows, wsel=args.wsel, qdq_shapes=shapes)
         t += dt
         flops += f
         n += 1
         if n >= 8:
             break
     return {"value": round(flops / t / 1e12, 6), "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
-            "sample": f"{n} oracle step(s) of weight_qdq(W {N}x{K}) + RAC linear on the first {rows} of {M} "
-                      f"rows of X (numpy; fp64 product via BLAS)"}
+            "sample": f"{n} oracle step(s) of " + oracle_sample_text(M, K, N, rows, shapes)}
 
 
 def run_reference(args):
@@ -948,17 +1110,17 @@ def run_reference(args):
     M, K, N, k = WORKLOADS[args.workload]
     k = args.k if args.k is not None else k
     rows = min(M, ORACLE_SAMPLE_ROWS)
+    shapes = QDQ_EXPERTS[args.workload][1] if args.workload in QDQ_EXPERTS else ()
     for _ in range(args.warmup):
-        oracle_step_time(M, K, N, k, rows, wsel=args.wsel)
+        oracle_step_time(M, K, N, k, rows, wsel=args.wsel, qdq_shapes=shapes)
     t, flops = 0.0, 0.0
     for _ in range(args.steps):
-        dt, f, _ = oracle_step_time(M, K, N, k, rows, wsel=args.wsel)
+        dt, f, _ = oracle_step_time(M, K, N, k, rows, wsel=args.wsel, qdq_shapes=shapes)
         t += dt
         flops += f
     value = flops / t / 1e12
     cores = blas_threads()
-    sample = (f"weight_qdq(W {N}x{K}) + RAC linear on the first {rows} of {M} rows of X per step "
-              f"(numpy oracle; fp64 product via BLAS)")
+    sample = oracle_sample_text(M, K, N, rows, shapes) + " per step"
     return {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s (effective 2MN(K+n_sel) per step)",
             "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * t / args.steps, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32 quantizer steps, f64 product",

@@ -308,15 +308,17 @@ def rac_gemm(qx, q_res, sel, n_sel, w, qw, w_colamax, out_dtype=torch.float32, o
     return y
 
 
-def weight_qdq(w, want_q=True, want_colamax=True, layout=1, out=None, stream=None):
+def weight_qdq(w, want_q=True, want_colamax=True, layout=1, out=None, stream=None, ws=None):
     """W4A16 fake quantization of bf16 w [N, K] or [batch, N, K].  Returns
-    (w_out bf16, qw or None, colamax fp32 [batch, K] or None)."""
+    (w_out bf16, qw or None, colamax fp32 [batch, K] or None).  ws: an
+    optional caller-owned uint8 workspace (else a shared per-device one)."""
     w = _bits(w)
     batch, N, K = (1, *w.shape) if w.dim() == 2 else w.shape
     w_out = out if out is not None else torch.empty_like(w)
     qw = NvFP4Tensor.empty(batch * N, K, layout, n_scales=batch, device=w.device) if want_q else None
     colamax = torch.empty(batch, K, dtype=torch.float32, device=w.device) if want_colamax else None
-    ws = _ws(workspace_size(OP_WEIGHT_QDQ, 0, N, K, batch), w.device)
+    if ws is None:
+        ws = _ws(workspace_size(OP_WEIGHT_QDQ, 0, N, K, batch), w.device)
     qs = qw.c() if qw is not None else None
     _check(_lib.weight_qdq(_ptr(w), N, K, K, batch, _ptr(w_out), ctypes.byref(qs) if qs is not None else None,
                            _ptr(colamax), _ptr(ws), ws.numel(), _stream(stream)), "weight_qdq")
