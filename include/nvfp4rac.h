@@ -242,6 +242,10 @@ nvfp4_status w4a4_rac_gemm(const nvfp4_tensor* qx, const nvfp4_tensor* q_res_or_
  * w4a4_gemm_quantized -- the GEMM alone, with every operand already
  * quantized (scale_layout 1): Y = s_tA s_tB A B^T [+ s_tR s_tWs R Ws^T].
  * q_res_or_null and q_wsel_or_null are both given (same cols) or both NULL.
+ * Each product of two tensor scales is applied as m 2^e (no fp32 underflow
+ * of s_tA s_tB while Y is representable).  A tensor scale of 0 must come
+ * with all-zero codes, as every quantizer of this library writes them (an
+ * all-zero X or W has an all-zero residual and W_sel too, and Y = 0).
  */
 nvfp4_status w4a4_gemm_quantized(const nvfp4_tensor* qa, const nvfp4_tensor* qb,
                                  const nvfp4_tensor* q_res_or_null,

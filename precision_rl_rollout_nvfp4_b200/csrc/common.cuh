@@ -252,6 +252,53 @@ __device__ __forceinline__ uint32_t encode8_q(const float* v, const BlockQ& q) {
   return e2m1x8_f2(o);
 }
 
+// ---- output scale of a block-scaled product --------------------------------
+// The product of two tensor scales s_a s_b is kept as m 2^e (m = RN(ma mb) in
+// [0.25, 1) from the frexp significands, e exact), so that it does not
+// underflow fp32 when both scales are tiny while Y itself is representable.
+struct ScaleProduct {
+  float m;
+  int e;
+};
+
+__device__ __forceinline__ ScaleProduct scale_product(float sa, float sb) {
+  int ea = 0, eb = 0;
+  const float ma = frexpf(sa, &ea), mb = frexpf(sb, &eb);
+  ScaleProduct r;
+  r.m = __fmul_rn(ma, mb);
+  r.e = r.m != 0.0f ? ea + eb : 0;
+  return r;
+}
+
+// 2^e as an fp32, e in [-149, 127] (a subnormal below -126).
+__device__ __forceinline__ float pow2f(int e) {
+  return e >= -126 ? __uint_as_float(static_cast<uint32_t>(e + 127) << 23)
+                   : __uint_as_float(1u << (e + 149));
+}
+
+// RN(t 2^e) as RN(RN(t p1) p2): p1 is 1 or an exact power-of-two pre-scale
+// (2^-64 / 2^64 when 2^e is outside fp32) that leaves every accumulator
+// value in range exact, and p2 carries the single rounding.
+struct Pow2Apply {
+  float p1, p2;
+  __device__ __forceinline__ float operator()(float t) const { return __fmul_rn(__fmul_rn(t, p1), p2); }
+};
+
+__device__ __forceinline__ Pow2Apply pow2_apply(int e) {
+  Pow2Apply a;
+  if (e > 127) {
+    a.p1 = pow2f(64);
+    a.p2 = pow2f(e - 64 < 127 ? e - 64 : 127);
+  } else if (e >= -149) {
+    a.p1 = 1.0f;
+    a.p2 = pow2f(e);
+  } else {
+    a.p1 = pow2f(-64);
+    a.p2 = pow2f(e + 64 > -149 ? e + 64 : -149);
+  }
+  return a;
+}
+
 // Byte offset of the scale of (row, block) in an NVFP4 scale buffer.
 __device__ __host__ __forceinline__ int64_t scale_offset(int64_t row, int64_t blk, int64_t cols,
                                                          int layout) {

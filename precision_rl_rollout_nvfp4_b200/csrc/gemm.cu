@@ -330,8 +330,14 @@ w4a4_rac_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_cons
       tc_fence_after();
       const int64_t mt = tile / p.n_tiles, nt = tile % p.n_tiles;
       const TileInfo ti = tile_info(p.g, mt);
-      const float al0 = __fmul_rn(p.sta[0][ti.e], p.stb[0][ti.e]);
-      const float al1 = nseg > 1 ? __fmul_rn(p.sta[1][ti.e], p.stb[1][ti.e]) : 0.0f;
+      // Y = a0 acc0 + a1 acc1 with a_s = s_tA,s s_tB,s = m_s 2^e_s: both
+      // segments in the units 2^E of the first nonzero one, then one
+      // power-of-two step (see Pow2Apply)
+      const ScaleProduct a0 = scale_product(p.sta[0][ti.e], p.stb[0][ti.e]);
+      const ScaleProduct a1 = nseg > 1 ? scale_product(p.sta[1][ti.e], p.stb[1][ti.e]) : ScaleProduct{0.0f, 0};
+      const int E = a0.m != 0.0f ? a0.e : a1.e;
+      const float c0 = a0.m, c1 = a1.m != 0.0f ? ldexpf(a1.m, a1.e - E) : 0.0f;
+      const Pow2Apply out = pow2_apply(E);
 #pragma unroll
       for (int c = 0; c < BN / 32; ++c) {
         float v[32], u[32];
@@ -340,10 +346,10 @@ w4a4_rac_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_cons
         tmem_ld_wait();
         if (nseg > 1) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = __fadd_rn(__fmul_rn(al0, v[i]), __fmul_rn(al1, u[i]));
+          for (int i = 0; i < 32; ++i) v[i] = out(__fadd_rn(__fmul_rn(c0, v[i]), __fmul_rn(c1, u[i])));
         } else {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(al0, v[i]);
+          for (int i = 0; i < 32; ++i) v[i] = out(__fmul_rn(c0, v[i]));
         }
         if (YBYTES == 4) {
 #pragma unroll
@@ -745,12 +751,16 @@ w4a4_rac_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid
     for (int tile = pair; tile < total; tile += npairs) {
       const int mt = tile / p.n_tiles, nt = tile % p.n_tiles;
       const PairRows pr = pair_rows(p, mt, rank);
-      const float al0 = __fmul_rn(p.sta[1][pr.e], p.stb[1][pr.e]);
-      const float al1 = has_res ? __fmul_rn(p.sta[0][pr.e], p.stb[0][pr.e]) : 0.0f;
-      // the residual is scaled to the plain segment's units, then Y = al0 acc;
-      // with al0 == 0 the plain operands are all zero codes and Y = al1 acc
-      const float ratio = al0 != 0.0f ? __fdiv_rn(al1, al0) : 1.0f;
-      const float fin = (has_res && al0 == 0.0f) ? al1 : al0;
+      // the residual is scaled to the plain segment's units (ratio =
+      // a_res / a_plain with a = s_tA s_tB = m 2^e), then Y = a_plain acc,
+      // applied as RN(acc m) and one power-of-two step (see Pow2Apply).  A
+      // zero plain scale means an all-zero X or W, whose residual and W_sel
+      // are zero as well: Y = 0.
+      const ScaleProduct ap = scale_product(p.sta[1][pr.e], p.stb[1][pr.e]);
+      const ScaleProduct ar = has_res ? scale_product(p.sta[0][pr.e], p.stb[0][pr.e]) : ScaleProduct{0.0f, 0};
+      const float ratio = (ap.m != 0.0f && ar.m != 0.0f) ? ldexpf(__fdiv_rn(ar.m, ap.m), ar.e - ap.e) : 0.0f;
+      const float fin = ap.m;
+      const Pow2Apply out = pow2_apply(ap.e);
       bool ok = true;
       if (has_res) {
         if (lane == 0) ok = mbar_wait(res_full, res_phase, p.err);
@@ -813,7 +823,7 @@ w4a4_rac_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid
             uint32_t w[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-              const float lo = __fmul_rn(fin, v[2 * i]), hi = __fmul_rn(fin, v[2 * i + 1]);
+              const float lo = out(__fmul_rn(fin, v[2 * i])), hi = out(__fmul_rn(fin, v[2 * i + 1]));
               asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(w[i]) : "f"(hi), "f"(lo));
             }
             if (h == 0) {
@@ -848,8 +858,8 @@ w4a4_rac_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid
 #pragma unroll
             for (int i = 0; i < 32; i += 4)
               *reinterpret_cast<float4*>(stg_row + (32 * c + i) * 4) =
-                  make_float4(__fmul_rn(fin, v[i]), __fmul_rn(fin, v[i + 1]), __fmul_rn(fin, v[i + 2]),
-                              __fmul_rn(fin, v[i + 3]));
+                  make_float4(out(__fmul_rn(fin, v[i])), out(__fmul_rn(fin, v[i + 1])),
+                              out(__fmul_rn(fin, v[i + 2])), out(__fmul_rn(fin, v[i + 3])));
           }
           if (h == 1) {
             tc_fence_before();

@@ -107,3 +107,24 @@ def test_bf16_output_is_rounded_fp32():
     y16, _ = b.rac_linear(x, w, 50.0, out_dtype=torch.bfloat16)
     torch.cuda.synchronize()
     assert torch.equal(y32.to(torch.bfloat16), y16)
+
+
+@pytest.mark.parametrize("M,K,N", [(4096, 1024, 2048),   # CTA-pair kernel
+                                   (128, 512, 256)])      # single-CTA kernel
+@pytest.mark.parametrize("k", [0.0, 50.0])
+def test_rac_linear_tiny_tensor_scales(M, K, N, k):
+    """X and W scaled by 2^-60 each (exact in bf16): the product of their
+    tensor scales, about 2^-140, is below fp32's normal range while Y (about
+    2^-120) is representable, so the output scale must not be formed as one
+    fp32 product."""
+    b = need_gpu()
+    x = (S.activations(M, K, seed=11).float() * 2.0 ** -60).to(torch.bfloat16)
+    w = (S.weights(N, K, seed=11).float() * 2.0 ** -60).to(torch.bfloat16)
+    y, st = b.rac_linear(x.cuda(), w.cuda(), k)
+    torch.cuda.synchronize()
+    assert b.stream_status() == 0
+    rows = np.unique(np.concatenate([[0, M - 1], np.random.default_rng(3).integers(0, M, 96)]))
+    ref = oracle.rac_linear(bits(x), bits(w), k, rows=rows)
+    assert np.array_equal(st["mask"].cpu().numpy(), ref["mask"])
+    assert float(st["qw"].tensor_scale.cpu()[0]) * float(st["qx"].tensor_scale.cpu()[0]) < 2.0 ** -126
+    assert rel_err(y.cpu().numpy()[rows], ref["y"]) < REL_TOL
