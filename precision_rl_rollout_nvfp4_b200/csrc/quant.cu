@@ -9,10 +9,10 @@
 // quantization (2.2 B).  The formulas are the reading in include/nvfp4rac.h.
 //
 // Layout of the quantize pass: a CTA of 256 threads owns a 128-row x 64-column
-// tile.  Thread t handles 8 consecutive columns (one 16-byte load) of rows
-// t/8 + 32 i, i = 0..3; the two halves of a 16-element block sit in threads
-// t and t^1 and meet through one shfl.xor.  |dX| goes to shared memory and 64
-// threads then sum their column over the 128 rows in row order in fp64.
+// tile.  Thread t handles 8 consecutive columns (one 16-byte load) of 4
+// consecutive rows; the two halves of a 16-element block sit in threads t and
+// t^1 and meet through one shfl.xor.  The channel score of the tile's 128 rows
+// is their fp64 sum in row order (see quant_score_kernel).
 #include "kernels.h"
 
 namespace nvfp4 {
@@ -150,11 +150,42 @@ __device__ __forceinline__ float reduce_parts(const unsigned* parts, int n, uint
 //
 // Thread t of the 256 owns 8 consecutive columns (one 16-byte load) of the 4
 // consecutive rows 4 (t/8) .. 4 (t/8) + 3 of the tile; the two halves of a
-// 16-element block sit in threads t and t^1.  The score order (4-row groups
-// summed in row order, group sums in group order, chunk sums in chunk order)
-// lets every thread sum its own group in fp64 registers; 64 threads then add
-// the tile's 32 group sums in order from shared memory.
+// 16-element block sit in threads t and t^1.
+//
+// The tile's rows are one 128-row chunk of the channel score, whose chunk sum
+// is defined as the fp64 sum of the chunk's |dX_ij| added one by one in row
+// order.  When the nonzero values of a column span at most 22 binades
+// (largest biased exponent minus smallest, a subnormal counted as exponent
+// 1), every partial sum of them is a multiple of the last bit of the
+// smallest and stays below 2^53 of those units, so every fp64 addition is
+// exact and any order of addition gives the row-order result: the tile then
+// adds the threads' 4-row sums through shared memory in two levels.  A
+// column whose values span more (a value far below the others; rare) is
+// summed again by one thread in row order, recomputing |dX| of each row from
+// X and the block's scale code with the same operations (so the same values).
 // ---------------------------------------------------------------------------
+constexpr int kSpanExact = 22;
+
+// |dX| of one element x (fp32 value of its bf16) in a block with scale code
+// sb: the scalar form of the quantize pass's arithmetic (block_quotients,
+// the E2M1 conversion, DQ and the difference), rounded the same way.
+__device__ __noinline__ float residual_abs_one(float xv, uint32_t sb, const ScaleTable& T) {
+  const float sbv = T.sbv[sb], sdec = T.sdec[sb], y = T.rcp[sb];
+  float q;
+  if (sdec > 0.0f && y != 0.0f) {
+    const float q0 = __fmul_rn(xv, y);
+    const float r = __fmaf_rn(q0, -sdec, xv);
+    q = __fmaf_rn(r, y, q0);
+  } else {
+    q = sdec > 0.0f ? div_slow(fabsf(xv), sdec) : 0.0f;
+  }
+  q = __uint_as_float(__float_as_uint(q) | (__float_as_uint(xv) & 0x80000000u));
+  float v[8] = {q, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  const uint32_t code = e2m1x8(v) & 15u;
+  const float p = __fmul_rn(e2m1_to_f32(code), sbv);
+  return fabsf(__fsub_rn(xv, __fmul_rn(p, T.s_t)));
+}
+
 // (4 CTAs per SM: measured faster than 3 with more registers)
 // SCORES: also the fp64 channel sums; without it the kernel writes the codes
 // alone (part_max == nullptr) or the codes and the residual column maxima.
@@ -175,6 +206,11 @@ quant_score_kernel(const uint16_t* __restrict__ x, int64_t K, int64_t ldx, RowGr
   constexpr int kGroups = kTileRows / 4;                          // 32 groups of 4 rows
   __shared__ __align__(16) double gsum[kGroups][kQCols];          // also tail staging
   __shared__ __align__(16) float gmax[kGroups][kQCols];
+  __shared__ __align__(16) uint32_t gmin[kGroups][kQCols];        // smallest nonzero |dX| bits - 1
+  __shared__ __align__(16) double qsum[4][kQCols];
+  __shared__ __align__(16) float qmax[4][kQCols];
+  __shared__ __align__(16) uint32_t qmin[4][kQCols];
+  __shared__ uint8_t s_sb[kTileRows][kQCols / kBlock];            // block scale codes of the tile
   __shared__ bool s_last;
   __shared__ ScaleTable T;
   const int t = threadIdx.x, cg = t & 7, grp = t >> 3;
@@ -196,8 +232,9 @@ quant_score_kernel(const uint16_t* __restrict__ x, int64_t K, int64_t ldx, RowGr
   uint8_t* code_base = codes + tile * kTileRows * (K / 2) + col / 2;
   double acc[8];
   float mx[8];
+  uint32_t mn[8];                                // min over nonzero |dX| of (bits - 1)
 #pragma unroll
-  for (int j = 0; j < 8; ++j) { acc[j] = 0.0; mx[j] = 0.0f; }
+  for (int j = 0; j < 8; ++j) { acc[j] = 0.0; mx[j] = 0.0f; mn[j] = 0xFFFFFFFFu; }
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int r = 4 * grp + i;
@@ -229,8 +266,10 @@ quant_score_kernel(const uint16_t* __restrict__ x, int64_t K, int64_t ldx, RowGr
       const float d0 = fabsf(__fsub_rn(x0, __fmul_rn(p0, s_t)));
       const float d1 = fabsf(__fsub_rn(x1, __fmul_rn(p1, s_t)));
       if (SCORES) {
-        acc[2 * j] += static_cast<double>(d0);     // rows of the group in order
+        acc[2 * j] += static_cast<double>(d0);     // exact whenever the span test passes
         acc[2 * j + 1] += static_cast<double>(d1);
+        mn[2 * j] = min(mn[2 * j], __float_as_uint(d0) - 1u);       // 0 wraps to ~0: ignored
+        mn[2 * j + 1] = min(mn[2 * j + 1], __float_as_uint(d1) - 1u);
       }
       mx[2 * j] = fmaxf(mx[2 * j], d0);
       mx[2 * j + 1] = fmaxf(mx[2 * j + 1], d1);
@@ -239,23 +278,68 @@ quant_score_kernel(const uint16_t* __restrict__ x, int64_t K, int64_t ldx, RowGr
       *reinterpret_cast<uint32_t*>(code_base + static_cast<uint32_t>(r) * static_cast<uint32_t>(K / 2)) = packed;
     if ((cg & 1) == 0 && (layout == 1 || prow < codes_rows))
       scales[scale_offset(prow, col / kBlock, K, layout)] = static_cast<uint8_t>(bq.sb);
+    if (SCORES && (cg & 1) == 0) s_sb[r][cg >> 1] = static_cast<uint8_t>(bq.sb);
   }
   if (part_max == nullptr) return;
+  // level 1: every thread's 4-row sums, maxima and minima to shared memory
   if (SCORES) {
 #pragma unroll
     for (int j = 0; j < 8; j += 2)
       *reinterpret_cast<double2*>(&gsum[grp][8 * cg + j]) = make_double2(acc[j], acc[j + 1]);
+    *reinterpret_cast<uint4*>(&gmin[grp][8 * cg]) = make_uint4(mn[0], mn[1], mn[2], mn[3]);
+    *reinterpret_cast<uint4*>(&gmin[grp][8 * cg + 4]) = make_uint4(mn[4], mn[5], mn[6], mn[7]);
   }
   *reinterpret_cast<float4*>(&gmax[grp][8 * cg]) = make_float4(mx[0], mx[1], mx[2], mx[3]);
   *reinterpret_cast<float4*>(&gmax[grp][8 * cg + 4]) = make_float4(mx[4], mx[5], mx[6], mx[7]);
   __syncthreads();
+  // level 2: thread (quarter t/64, column t%64) reduces 8 groups
+  {
+    const int c = t & (kQCols - 1), q4 = t >> 6;
+    double sum = 0.0;
+    float m = 0.0f;
+    uint32_t lo = 0xFFFFFFFFu;
+#pragma unroll
+    for (int gi = 8 * q4; gi < 8 * q4 + 8; ++gi) {
+      if (SCORES) {
+        sum += gsum[gi][c];
+        lo = min(lo, gmin[gi][c]);
+      }
+      m = fmaxf(m, gmax[gi][c]);
+    }
+    if (SCORES) {
+      qsum[q4][c] = sum;
+      qmin[q4][c] = lo;
+    }
+    qmax[q4][c] = m;
+  }
+  __syncthreads();
   if (t < kQCols) {
     double part = 0.0;
     float m = 0.0f;
-#pragma unroll 8
-    for (int q = 0; q < kGroups; ++q) {          // group order within the chunk
-      if (SCORES) part += gsum[q][t];
-      m = fmaxf(m, gmax[q][t]);
+    uint32_t lo = 0xFFFFFFFFu;
+#pragma unroll
+    for (int q4 = 0; q4 < 4; ++q4) {
+      if (SCORES) {
+        part += qsum[q4][t];
+        lo = min(lo, qmin[q4][t]);
+      }
+      m = fmaxf(m, qmax[q4][t]);
+    }
+    if (SCORES && lo != 0xFFFFFFFFu) {
+      const int e_hi = static_cast<int>(__float_as_uint(m) >> 23);
+      const int e_lo = max(static_cast<int>((lo + 1u) >> 23), 1);
+      if (e_hi - e_lo > kSpanExact) {
+        // the row-order sum itself, from X and the tile's block scales
+        const uint16_t* xc = x + col0 + t;
+        double chain = 0.0;
+        for (int r = 0; r < kTileRows; ++r) {
+          const int64_t row = ti.row0 + r;
+          if (row >= ti.row_end) break;
+          const float xv = bf16_bits_to_f32(__ldg(xc + row * ldx));
+          chain += static_cast<double>(residual_abs_one(xv, s_sb[r][t >> 4], T));
+        }
+        part = chain;
+      }
     }
     if (SCORES) part_sum[tile * K + col0 + t] = part;
     part_max[tile * K + col0 + t] = m;

@@ -97,3 +97,32 @@ def _boundary_tensor(s_t_target, seed):
 def test_quantize_rounding_boundaries(s_t, seed):
     b = need_gpu()
     _check_quant(b, _boundary_tensor(s_t, seed), 1)
+
+
+def test_score_row_order_on_wide_columns():
+    """Columns whose |dX| span far more than 22 binades take the kernel's
+    row-order path; their scores must still equal the oracle's (and the
+    values that IEEE rounding fixes for the plain order).  Column 0 holds 448
+    in every row, so every block's scale makes 1.0 and 2^-53 quantize to 0
+    and dX equals x there."""
+    b = need_gpu()
+    u = 2.0 ** -53
+    x = np.zeros((384, 64), np.float32)
+    x[:, 0] = 448.0
+    x[0, 1] = 1.0
+    x[1:128, 1] = u                      # 1 then 127 x u: every addition ties to 1.0
+    x[0:127, 2] = u
+    x[127, 2] = 1.0                      # 127 u then 1: 1 + 2^-46
+    x[0, 3] = 1.0
+    x[128, 3] = u
+    x[129, 3] = u                        # chunk sums 1 and 2u: 1 + 2^-52
+    x[0, 4] = 1.0
+    x[128, 4] = u
+    x[256, 4] = u                        # chunks 1, u, u in order: 1.0
+    xt = torch.from_numpy(x).to(torch.bfloat16)
+    _, score, _ = b.quantize(xt.cuda(), layout=1)
+    torch.cuda.synchronize()
+    got = score.cpu().numpy()
+    ref = oracle.quantize_activations(bits(xt))["score"]
+    assert np.array_equal(got, ref)
+    assert got[1] == 1.0 and got[2] == 1.0 + 2.0 ** -46 and got[3] == 1.0 + 2.0 ** -52 and got[4] == 1.0
