@@ -143,3 +143,32 @@ def rac_linear(x_bits, w_bits, k_percent, wsel_source="bf16"):
                ws_st=stws, y=[[y_plain[i][n] + y_corr[i][n] for n in range(N)]
                               for i in range(M)])
     return out
+
+
+def mxfp8_quantize_rows(rows):
+    """MXFP8 (E4M3 elements, one UE8M0 scale per 32 elements) of fp32 rows,
+    restated independently of oracle.mxfp8: the block exponent from a loop
+    over powers of two, the element code by exhaustive nearest search over
+    the 127 finite E4M3 magnitudes (ties to the even code, 448 saturates)."""
+    codes, scales = [], []
+    for row in rows:
+        rc, rs = [], []
+        for b0 in range(0, len(row), 32):
+            blk = row[b0:b0 + 32]
+            amax = max(abs(v) for v in blk)
+            if amax == 0.0:
+                e = -127
+            else:
+                p = 0
+                while 2.0 ** (p + 1) <= amax:
+                    p += 1
+                while 2.0 ** p > amax:
+                    p -= 1
+                e = max(-127, min(127, p - 8))
+            rs.append(e + 127)
+            for v in blk:
+                q = v / 2.0 ** e
+                rc.append(e4m3_code(abs(q)) | (0x80 if math.copysign(1.0, v) < 0 else 0))
+        codes.append(rc)
+        scales.append(rs)
+    return codes, scales
