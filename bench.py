@@ -470,15 +470,31 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.synchronize()
         return a.elapsed_time(b)
 
+    # comparators timed the same way (not part of the step): the plain W4A4
+    # GEMM alone, and the FP8 path on the same shape -- MXFP8 quantization of
+    # X and the kind::mxf8f6f4 W8A8 GEMM (W quantized once beforehand)
+    cmp_fns = {"gemm_plain": lambda: plan.gemm(plain=True)}
+    if K % 256 == 0:
+        qa8, qb8 = B.mxfp8_quantize(x), B.mxfp8_quantize(w)
+        y8 = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        cmp_fns["fp8_quantize"] = lambda: B.mxfp8_quantize(x, out=qa8)
+        cmp_fns["fp8_gemm"] = lambda: B.w8a8_gemm(qa8, qb8, out=y8)
+        for f in cmp_fns.values():
+            f()
+        torch.cuda.synchronize()
+    cmp_call = {c: [] for c in cmp_fns}
     if use_graph:
         g_flush = reps_graph(lambda: None)
         g_calls = {c: reps_graph(fns[c]) for c in calls}
+        g_cmp = {c: reps_graph(f) for c, f in cmp_fns.items()}
         torch.cuda.synchronize()
         for _ in range(PER_CALL_SAMPLES):
             base = time_graph(g_flush)
             for c in calls:
                 per_call[c].append(max(time_graph(g_calls[c]) - base, 0.0) / PER_CALL_REPS)
-        del g_flush, g_calls
+            for c in cmp_fns:
+                cmp_call[c].append(max(time_graph(g_cmp[c]) - base, 0.0) / PER_CALL_REPS)
+        del g_flush, g_calls, g_cmp
     else:
         for _ in range(max(args.steps, PER_CALL_SAMPLES)):
             flush.zero_()
@@ -489,6 +505,11 @@ def run_ours(args, rank, world, local_rank):
             torch.cuda.synchronize()
             for i, c in enumerate(calls):
                 per_call[c].append(evs[i].elapsed_time(evs[i + 1]))
+            for c, f in cmp_fns.items():
+                flush.zero_()
+                a = ev(); f(); b_ = ev()
+                torch.cuda.synchronize()
+                cmp_call[c].append(a.elapsed_time(b_))
     # plain W4A4 linear (no RAC) and the RAC linear without weight prep, for the overhead
     plain_ms, rac_ms = [], []
     for _ in range(args.steps):
@@ -628,6 +649,17 @@ def run_ours(args, rank, world, local_rank):
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clock,
     }
+    cmp_us = {c: 1e3 * statistics.median(v) for c, v in cmp_call.items() if v}
+    line["comparators_us"] = {c: round(v, 2) for c, v in cmp_us.items()}
+    if "fp8_gemm" in cmp_us:
+        fl = 2.0 * M * N * K
+        line["fp8_gemm_us"] = round(cmp_us["fp8_gemm"], 2)
+        line["fp8_gemm_tflops"] = round(fl / (cmp_us["fp8_gemm"] * 1e-6) / 1e12, 1)
+        line["fp4_gemm_plain_us"] = round(cmp_us["gemm_plain"], 2)
+        # throughput of the NVFP4 W4A4 GEMM over the MXFP8 W8A8 GEMM, same M, N, K
+        line["fp4_over_fp8"] = round(cmp_us["fp8_gemm"] / cmp_us["gemm_plain"], 3)
+        line["fp4_rac_over_fp8"] = round(cmp_us["fp8_gemm"] / (1e3 * med["gemm"]), 3)
+        line["fp8_linear_us"] = round(cmp_us["fp8_gemm"] + cmp_us["fp8_quantize"], 2)
     if qdq is not None:
         q_us = 1e3 * med["qdq_experts"]
         line["qdq_experts_us"] = round(q_us, 2)

@@ -316,6 +316,43 @@ nvfp4_status nvfp4_quantize_static_ws(const uint16_t* x, int64_t M, int64_t K, i
                                       void* stream);
 
 /*
+ * The FP8 comparator: MXFP8 operands and a W8A8 tensor-core GEMM, so that the
+ * NVFP4 path can be timed beside FP8 on the same shapes.  Pages: QUADS
+ * technical summary section 1 "Probleemstelling" (NVFP4 has about twice the
+ * GEMM throughput of FP8) and section 4 (about 16% faster rollout than FP8);
+ * the pages do not name the FP8 scheme.  The adopted one is the block-scaled
+ * FP8 that sm_100 tensor cores run natively, OCP MXFP8: E4M3 elements and
+ * one UE8M0 scale 2^E per 32 consecutive elements along K, with
+ * E = floor(log2 max|x_b|) - 8 clamped to [-127, 127] (-127 for an all-zero
+ * block) and code = E4M3(x / 2^E), nearest, ties to the even code,
+ * saturating at 448, the sign bit of x kept (so -0 stays -0).
+ */
+typedef struct {
+  uint8_t* codes;         /* device, rows x cols E4M3 bytes, row-major */
+  uint8_t* scales;        /* device, UE8M0 (E + 127) per 32-element block */
+  int64_t rows, cols;
+  int32_t scale_layout;   /* 0 canonical [rows][cols/32]; 1 MMA-tiled: rows
+                             padded to 128, the scale of (row r, block c) at
+                             ((r/128) * (cols/128) + c/4) * 512 + (r%32) * 16
+                             + ((r%128)/32) * 4 + c%4, padding written as 0 */
+} mxfp8_tensor;
+
+/* Bytes of the scale buffer of a rows x cols MXFP8 tensor in `layout`. */
+size_t mxfp8_scale_bytes(int64_t rows, int64_t cols, int32_t layout);
+
+/* mxfp8_quantize -- MXFP8 of bf16 x [M, K] (row stride ldx), K % 256 == 0;
+ * q: rows = M, cols = K, either scale layout.  Needs no workspace. */
+nvfp4_status mxfp8_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, mxfp8_tensor* q,
+                            void* stream);
+
+/* w8a8_gemm_quantized -- Y = A B^T with A [M, K] and B [N, K] MXFP8
+ * (scale_layout 1), K % 128 == 0, N % 16 == 0: a block-scaled E4M3 tensor-core
+ * GEMM (tcgen05 kind::mxf8f6f4) with fp32 accumulation; y fp32 (y_dtype 0)
+ * or bf16 (1, RN of the fp32 value), row stride ldy. */
+nvfp4_status w8a8_gemm_quantized(const mxfp8_tensor* qa, const mxfp8_tensor* qb, void* y, int32_t y_dtype,
+                                 int64_t ldy, void* stream);
+
+/*
  * Element converters used by the kernels, exposed for checking them:
  * nvfp4_encode_e2m1 writes one E2M1 code (0..15) per fp32 input,
  * nvfp4_encode_e4m3 one E4M3 code per fp32 input >= 0 (RN, saturating).

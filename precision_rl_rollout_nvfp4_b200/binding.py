@@ -31,7 +31,7 @@ EXPORTS = ["nvfp4_scale_bytes", "nvfp4_workspace_size", "nvfp4_quantize", "rac_s
            "nvfp4_encode_e2m1", "nvfp4_encode_e4m3", "nvfp4_stream_status",
            "nvfp4_check_bounded_wait", "nvfp4_status_string", "nvfp4_quantize_static_ws",
            "nvfp4_dq_colamax", "rac_weight_quant_fp4", "rac_select_channels", "rac_residual_quant",
-           "rac_sel_tensor_scale"]
+           "rac_sel_tensor_scale", "mxfp8_scale_bytes", "mxfp8_quantize", "w8a8_gemm_quantized"]
 
 
 class _Tensor(ctypes.Structure):
@@ -40,8 +40,14 @@ class _Tensor(ctypes.Structure):
                 ("cols", ctypes.c_int64), ("scale_layout", ctypes.c_int32)]
 
 
+class _MxTensor(ctypes.Structure):
+    _fields_ = [("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("rows", ctypes.c_int64),
+                ("cols", ctypes.c_int64), ("scale_layout", ctypes.c_int32)]
+
+
 P, I64, I32, F32, SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_float, ctypes.c_size_t
 TP = ctypes.POINTER(_Tensor)
+MP = ctypes.POINTER(_MxTensor)
 _sig = {
     "nvfp4_scale_bytes": (SZ, [I64, I64, I32]),
     "nvfp4_workspace_size": (SZ, [I32, I64, I64, I64, I32]),
@@ -65,6 +71,9 @@ _sig = {
     "nvfp4_stream_status": (I32, [P]),
     "nvfp4_check_bounded_wait": (I32, [I32, P]),
     "nvfp4_status_string": (ctypes.c_char_p, [I32]),
+    "mxfp8_scale_bytes": (SZ, [I64, I64, I32]),
+    "mxfp8_quantize": (I32, [P, I64, I64, I64, MP, P]),
+    "w8a8_gemm_quantized": (I32, [MP, MP, P, I32, I64, P]),
 }
 for _name, (_res, _args) in _sig.items():
     _f = getattr(_lib, _name)
@@ -395,6 +404,45 @@ def qat_linear(x, w, act_quant=False):
     wq = fake_quant(w)
     xq = fake_quant(x) if act_quant else x
     return xq @ wq.t()
+
+
+@dataclass
+class MxFP8Tensor:
+    """Device buffers of one MXFP8 tensor (mxfp8_tensor in the header): the
+    FP8 comparator's operand format."""
+    codes: torch.Tensor          # uint8 [rows, cols] E4M3
+    scales: torch.Tensor         # uint8 [mxfp8_scale_bytes] UE8M0
+    rows: int
+    cols: int
+    layout: int
+
+    @staticmethod
+    def empty(rows, cols, layout=1, device="cuda"):
+        return MxFP8Tensor(torch.empty(rows, cols, dtype=torch.uint8, device=device),
+                           torch.empty(max(int(_lib.mxfp8_scale_bytes(rows, cols, layout)), 1), dtype=torch.uint8,
+                                       device=device), rows, cols, layout)
+
+    def c(self) -> _MxTensor:
+        return _MxTensor(self.codes.data_ptr(), self.scales.data_ptr(), self.rows, self.cols, self.layout)
+
+
+def mxfp8_quantize(x, layout=1, out=None, stream=None):
+    """MXFP8 of bf16 x [M, K] (K % 256 == 0)."""
+    x = _bits(x)
+    M, K = x.shape
+    q = out if out is not None else MxFP8Tensor.empty(M, K, layout, device=x.device)
+    qs = q.c()
+    _check(_lib.mxfp8_quantize(_ptr(x), M, K, x.stride(0), ctypes.byref(qs), _stream(stream)), "mxfp8_quantize")
+    return q
+
+
+def w8a8_gemm(qa, qb, out_dtype=torch.float32, out=None, stream=None):
+    """Y = A B^T of two MXFP8 operands (the FP8 comparator GEMM)."""
+    y = out if out is not None else torch.empty(qa.rows, qb.rows, dtype=out_dtype, device=qa.codes.device)
+    a, b = qa.c(), qb.c()
+    _check(_lib.w8a8_gemm_quantized(ctypes.byref(a), ctypes.byref(b), _ptr(y), 0 if y.dtype == torch.float32 else 1,
+                                    y.stride(0), _stream(stream)), "w8a8_gemm_quantized")
+    return y
 
 
 def encode_e2m1(v: torch.Tensor, stream=None) -> torch.Tensor:

@@ -524,6 +524,57 @@ nvfp4_status weight_qdq(const uint16_t* w, int64_t N, int64_t K, int64_t ldw, in
   return NVFP4_OK;
 }
 
+size_t mxfp8_scale_bytes(int64_t rows, int64_t cols, int32_t layout) {
+  if (rows < 0 || cols < 0 || (layout != 0 && layout != 1)) return 0;
+  if (layout == 0) return static_cast<size_t>(rows * (cols / 32));
+  return static_cast<size_t>(ceil_div(rows, 128) * 128 * ceil_div(cols, 128) * 4);
+}
+
+static bool mx_tensor_ok(const mxfp8_tensor* t) {
+  return t && t->codes && t->scales && aligned16(t->codes) && aligned16(t->scales) &&
+         (t->scale_layout == 0 || t->scale_layout == 1);
+}
+
+nvfp4_status mxfp8_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, mxfp8_tensor* q, void* stream) {
+  NV_CHECK(x && mx_tensor_ok(q), NVFP4_ERR_INVALID_ARG);
+  NV_CHECK(M >= 1 && K >= 256 && K % 256 == 0 && ldx >= K && q->rows == M && q->cols == K,
+           NVFP4_ERR_UNSUPPORTED_SHAPE);
+  NV_CHECK(aligned16(x) && ldx % 8 == 0, NVFP4_ERR_MISALIGNED);
+  const nvfp4_status d = device_ok();
+  if (d != NVFP4_OK) return d;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (q->scale_layout == 1 && M % 128 != 0)
+    NV_TRY(cudaMemsetAsync(q->scales, 0, mxfp8_scale_bytes(M, K, 1), s));
+  NV_TRY(launch_mxfp8_quant(x, M, K, ldx, q->codes, q->scales, q->scale_layout, s));
+  return NVFP4_OK;
+}
+
+nvfp4_status w8a8_gemm_quantized(const mxfp8_tensor* qa, const mxfp8_tensor* qb, void* y, int32_t y_dtype,
+                                 int64_t ldy, void* stream) {
+  NV_CHECK(mx_tensor_ok(qa) && mx_tensor_ok(qb) && y, NVFP4_ERR_INVALID_ARG);
+  NV_CHECK(qa->scale_layout == 1 && qb->scale_layout == 1 && (y_dtype == 0 || y_dtype == 1),
+           NVFP4_ERR_INVALID_ARG);
+  const int64_t M = qa->rows, N = qb->rows, K = qa->cols;
+  NV_CHECK(M >= 1 && N >= 16 && N % 16 == 0 && K >= 128 && K % 128 == 0 && qb->cols == K && ldy >= N,
+           NVFP4_ERR_UNSUPPORTED_SHAPE);
+  NV_CHECK(aligned16(y) && ldy % 8 == 0, NVFP4_ERR_MISALIGNED);
+  const nvfp4_status d = device_ok();
+  if (d != NVFP4_OK) return d;
+  GemmArgs a{};
+  a.a0 = {qa->codes, qa->scales, nullptr, M, K};
+  a.b0 = {qb->codes, qb->scales, nullptr, N, K};
+  a.g = dense_groups(M);
+  a.M = M;
+  a.N = N;
+  a.m_tiles = ceil_div(M, 128);
+  a.y = y;
+  a.y_dtype = y_dtype;
+  a.ldy = ldy;
+  a.err = device_error_word();
+  NV_CHECK(a.err != nullptr, NVFP4_ERR_CUDA);
+  return cuda_status(launch_gemm_fp8(a, static_cast<cudaStream_t>(stream)));
+}
+
 nvfp4_status nvfp4_encode_e2m1(const float* in, uint8_t* out, int64_t n, void* stream) {
   NV_CHECK(in && out && n >= 0, NVFP4_ERR_INVALID_ARG);
   const nvfp4_status d = device_ok();

@@ -134,6 +134,20 @@ __device__ __forceinline__ void mma_fp4(uint32_t d, uint64_t a, uint64_t b, uint
       :: "r"(d), "l"(a), "l"(b), "r"(IDESC), "r"(accumulate), "r"(sfa), "r"(sfb) : "memory");
 }
 
+// kind::mxf8f6f4 instruction descriptor: E4M3 x E4M3 (format 0), UE8M0
+// scales (bit 23), both K-major, N = 128, M = 128.  Bits 29-30 / 4-5 select
+// which byte of a row's 32-bit scale word in TMEM the MMA reads (the j-th
+// 32-element block of a 128-element K step).
+constexpr uint32_t IDESC8 = (1u << 23) | (uint32_t(BN >> 3) << 17) | (uint32_t(BM >> 4) << 24);
+
+__device__ __forceinline__ void mma_fp8(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t sfa,
+                                        uint32_t sfb, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+      :: "r"(d), "l"(a), "l"(b), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb) : "memory");
+}
+
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
                :: "r"(smem_u32(bar)) : "memory");
@@ -160,12 +174,17 @@ __device__ __forceinline__ void tmem_ld_wait() {
 }
 
 // ---- the kernel -----------------------------------------------------------
-template <int YBYTES>
-__global__ void __launch_bounds__(THREADS1, 1)
-w4a4_rac_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
-                     const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
-                     const KParams p) {
+// The single-CTA kernel's body, for NVFP4 operands (FP8 = false: 256
+// elements per 128-byte K step, four kind::mxf4nvf4 MMAs of K = 64, one
+// 512-byte scale atom per MMA) or MXFP8 operands (FP8 = true: 128 elements
+// per K step, four kind::mxf8f6f4 MMAs of K = 32 reading the four bytes of
+// one scale atom, no residual segment).
+template <int YBYTES, bool FP8>
+__device__ __forceinline__ void gemm1_body(const CUtensorMap& tmA0, const CUtensorMap& tmB0,
+                                           const CUtensorMap& tmA1, const CUtensorMap& tmB1,
+                                           const KParams& p) {
   constexpr int STAGES = Cfg<YBYTES>::STAGES;
+  constexpr int SF_STEP = FP8 ? SF_ATOM : SF_STAGE;        // scale bytes per K step and operand
   constexpr int STG_STRIDE = Cfg<YBYTES>::STG_STRIDE;
   extern __shared__ uint8_t smem_raw[];
   // 128-byte swizzled tiles need 1024-byte aligned shared addresses
@@ -232,15 +251,15 @@ w4a4_rac_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_cons
           for (int kt = 0; kt < p.kt[seg]; ++kt) {
             if (!mbar_wait(&empty[stage], phase ^ 1, p.err)) { ok = false; break; }
             const int nkb = kt == p.kt[seg] - 1 ? p.kb_last[seg] : 4;
-            const uint32_t sf_bytes = nkb * SF_ATOM;
+            const uint32_t sf_bytes = FP8 ? SF_ATOM : nkb * SF_ATOM;
             const uint32_t fb = smem_u32(&full[stage]);
             mbar_arrive_expect_tx(&full[stage], A_STAGE + B_STAGE + 2 * sf_bytes);
             tma_load_2d(smem_u32(sA + stage * A_STAGE), tA, kt * BK_BYTES, static_cast<int>(mt * BM), fb);
             tma_load_2d(smem_u32(sB + stage * B_STAGE), tB, kt * BK_BYTES, static_cast<int>(b_row), fb);
-            bulk_load(smem_u32(sSFA + stage * SF_STAGE), p.sfa[seg] + mt * p.sfa_rb[seg] + kt * SF_STAGE,
+            bulk_load(smem_u32(sSFA + stage * SF_STAGE), p.sfa[seg] + mt * p.sfa_rb[seg] + kt * SF_STEP,
                       sf_bytes, fb);
             bulk_load(smem_u32(sSFB + stage * SF_STAGE),
-                      p.sfb[seg] + (b_row / BN) * p.sfb_rb[seg] + kt * SF_STAGE, sf_bytes, fb);
+                      p.sfb[seg] + (b_row / BN) * p.sfb_rb[seg] + kt * SF_STEP, sf_bytes, fb);
             armed |= 1u << stage;
             armed_phase = (armed_phase & ~(1u << stage)) | (phase << stage);
             if (++stage == STAGES) { stage = 0; phase ^= 1; }
@@ -271,9 +290,15 @@ w4a4_rac_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_cons
             const int nkb = kt == p.kt[seg] - 1 ? p.kb_last[seg] : 4;
             const uint32_t a0 = smem_u32(sA + stage * A_STAGE), b0 = smem_u32(sB + stage * B_STAGE);
             const uint32_t sfa = tmem + SF1_COL + SF1_STAGE_COLS * stage, sfb = sfa + 16;
-            for (int j = 0; j < nkb; ++j)
-              mma_fp4(d, desc_sw128(a0 + 32 * j), desc_sw128(b0 + 32 * j), sfa + 4 * j, sfb + 4 * j,
-                      (kt > 0 || j > 0) ? 1u : 0u);
+            for (int j = 0; j < nkb; ++j) {
+              if (FP8)
+                mma_fp8(d, desc_sw128(a0 + 32 * j), desc_sw128(b0 + 32 * j),
+                        IDESC8 | (static_cast<uint32_t>(j) << 29) | (static_cast<uint32_t>(j) << 4), sfa, sfb,
+                        (kt > 0 || j > 0) ? 1u : 0u);
+              else
+                mma_fp4(d, desc_sw128(a0 + 32 * j), desc_sw128(b0 + 32 * j), sfa + 4 * j, sfb + 4 * j,
+                        (kt > 0 || j > 0) ? 1u : 0u);
+            }
             umma_commit(&empty[stage]);
             if (++stage == STAGES) { stage = 0; phase ^= 1; }
           }
@@ -300,7 +325,7 @@ w4a4_rac_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_cons
             const int nkb = kt == p.kt[seg] - 1 ? p.kb_last[seg] : 4;
             const uint32_t fa = smem_u32(sSFA + stage * SF_STAGE), fb = smem_u32(sSFB + stage * SF_STAGE);
             const uint32_t sfa = tmem + SF1_COL + SF1_STAGE_COLS * stage, sfb = sfa + 16;
-            for (int j = 0; j < nkb; ++j) {
+            for (int j = 0; j < (FP8 ? 1 : nkb); ++j) {
               utccp_sf(sfa + 4 * j, desc_sf(fa + j * SF_ATOM));
               utccp_sf(sfb + 4 * j, desc_sf(fb + j * SF_ATOM));
             }
@@ -333,7 +358,8 @@ w4a4_rac_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_cons
       // Y = a0 acc0 + a1 acc1 with a_s = s_tA,s s_tB,s = m_s 2^e_s: both
       // segments in the units 2^E of the first nonzero one, then one
       // power-of-two step (see Pow2Apply)
-      const ScaleProduct a0 = scale_product(p.sta[0][ti.e], p.stb[0][ti.e]);
+      // (MXFP8 operands carry no tensor scale: the scale product is 1)
+      const ScaleProduct a0 = FP8 ? ScaleProduct{0.5f, 1} : scale_product(p.sta[0][ti.e], p.stb[0][ti.e]);
       const ScaleProduct a1 = nseg > 1 ? scale_product(p.sta[1][ti.e], p.stb[1][ti.e]) : ScaleProduct{0.0f, 0};
       const int E = a0.m != 0.0f ? a0.e : a1.e;
       const float c0 = a0.m, c1 = a1.m != 0.0f ? ldexpf(a1.m, a1.e - E) : 0.0f;
@@ -393,13 +419,32 @@ w4a4_rac_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_cons
   }
 }
 
+template <int YBYTES>
+__global__ void __launch_bounds__(THREADS1, 1)
+w4a4_rac_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
+                     const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
+                     const KParams p) {
+  gemm1_body<YBYTES, false>(tmA0, tmB0, tmA1, tmB1, p);
+}
+
+// MXFP8 x MXFP8 (the FP8 comparator): one K segment.
+template <int YBYTES>
+__global__ void __launch_bounds__(THREADS1, 1)
+w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
+                 const KParams p) {
+  gemm1_body<YBYTES, true>(tmA0, tmB0, tmA0, tmB0, p);
+}
+
 // ---- host side -------------------------------------------------------------
-// 2-D map over packed FP4 codes [rows, cols/2] bytes, box 128 B x box_rows.
-bool make_code_map(CUtensorMap* tm, const uint8_t* codes, int64_t rows, int64_t cols, int box_rows) {
+// 2-D map over packed FP4 codes [rows, cols/2] bytes (or, with row_bytes,
+// any byte matrix [rows, row_bytes]), box 128 B x box_rows.
+bool make_code_map(CUtensorMap* tm, const uint8_t* codes, int64_t rows, int64_t cols, int box_rows,
+                   int64_t row_bytes = -1) {
   auto fn = encode_fn();
   if (fn == nullptr) return false;
-  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols / 2), static_cast<cuuint64_t>(rows)};
-  cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols / 2)};
+  const int64_t rb = row_bytes >= 0 ? row_bytes : cols / 2;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(rb), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(rb)};
   cuuint32_t box[2] = {static_cast<cuuint32_t>(BK_BYTES), static_cast<cuuint32_t>(box_rows)};
   cuuint32_t estr[2] = {1, 1};
   return fn(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(codes), dims, strides, box, estr,
@@ -422,6 +467,12 @@ template <int YBYTES>
 cudaError_t prepare_kernel() {
   static bool done[kMaxAttrDevices] = {};
   return set_max_smem(w4a4_rac_gemm_kernel<YBYTES>, Cfg<YBYTES>::SMEM_BYTES, done);
+}
+
+template <int YBYTES>
+cudaError_t prepare_kernel8() {
+  static bool done[kMaxAttrDevices] = {};
+  return set_max_smem(w8a8_gemm_kernel<YBYTES>, Cfg<YBYTES>::SMEM_BYTES, done);
 }
 
 // ===========================================================================
@@ -1012,6 +1063,45 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s) {
                                      maps[0], maps[1], maps[2], maps[3], p);
       if (le != cudaSuccess) return le;
     }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gemm_fp8(const GemmArgs& a, cudaStream_t s) {
+  cudaError_t e = a.y_dtype == 0 ? prepare_kernel8<4>() : prepare_kernel8<2>();
+  if (e != cudaSuccess) return e;
+  KParams p{};
+  p.g = a.g;
+  p.N = a.N;
+  p.m_tiles_dense = (a.M + BM - 1) / BM;
+  p.n_tiles = static_cast<int>((a.N + BN - 1) / BN);
+  p.M = a.M;
+  const int64_t K = a.a0.cols;                   // multiple of 128: 4 MMAs of K = 32 per step
+  p.kt[0] = static_cast<int>(K / 128);
+  p.kt[1] = 0;
+  p.kb_last[0] = 4;
+  p.kb_last[1] = 4;
+  p.sfa[0] = p.sfa[1] = a.a0.scales;
+  p.sfb[0] = p.sfb[1] = a.b0.scales;
+  p.sfa_rb[0] = p.sfa_rb[1] = (K / 128) * SF_ATOM;   // one atom (128 rows x 4 blocks of 32) per step
+  p.sfb_rb[0] = p.sfb_rb[1] = (K / 128) * SF_ATOM;
+  CUtensorMap maps[2];
+  if (!make_code_map(&maps[0], a.a0.codes, a.a0.rows, K, BM, K) ||
+      !make_code_map(&maps[1], a.b0.codes, a.b0.rows, K, BN, K))
+    return cudaErrorInvalidValue;
+  p.y = a.y;
+  p.y_dtype = a.y_dtype;
+  p.ldy = a.ldy;
+  p.err = a.err;
+  const int64_t tiles = p.m_tiles_dense * p.n_tiles;
+  if (tiles == 0) return cudaSuccess;
+  const int grid = static_cast<int>(tiles < sm_count() ? tiles : sm_count());
+  const cudaError_t le =
+      a.y_dtype == 0
+          ? launch_k(w8a8_gemm_kernel<4>, dim3(grid), dim3(THREADS1), Cfg<4>::SMEM_BYTES, s, nullptr, 0, maps[0],
+                     maps[1], p)
+          : launch_k(w8a8_gemm_kernel<2>, dim3(grid), dim3(THREADS1), Cfg<2>::SMEM_BYTES, s, nullptr, 0, maps[0],
+                     maps[1], p);
+  if (le != cudaSuccess) return le;
   return cudaGetLastError();
 }
 

@@ -187,4 +187,16 @@ struct GemmArgs {
 
 cudaError_t launch_gemm(const GemmArgs& args, cudaStream_t s);
 
+// MXFP8 x MXFP8 comparator GEMM (single K segment, single-CTA kernel):
+// a0 / b0 codes are E4M3 bytes [rows, cols], scales UE8M0 in the MMA-tiled
+// layout with 32-element blocks; st unused; cols % 128 == 0; dense rows.
+cudaError_t launch_gemm_fp8(const GemmArgs& args, cudaStream_t s);
+
+// MXFP8 quantization of bf16 x [rows, K] (K % 128 == 0): codes [rows, K]
+// E4M3 bytes, scales UE8M0 per 32-element block in `layout` (0 canonical
+// [rows][K/32], 1 MMA-tiled: per 128-row block one 512-byte atom per 128
+// columns, row r at (r%32)*16 + ((r%128)/32)*4 + block%4).
+cudaError_t launch_mxfp8_quant(const uint16_t* x, int64_t rows, int64_t K, int64_t ldx, uint8_t* codes,
+                               uint8_t* scales, int layout, cudaStream_t s);
+
 }  // namespace nvfp4

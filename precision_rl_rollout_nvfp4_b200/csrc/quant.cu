@@ -983,6 +983,71 @@ weight_qdq_kernel(const uint16_t* w, int64_t N, int64_t K, int64_t ldw,
 }
 
 // ---------------------------------------------------------------------------
+// MXFP8 quantization (the FP8 comparator's operands): E4M3 elements, one
+// UE8M0 scale per 32 elements, E = floor(log2 amax_b) - 8 clamped to
+// [-127, 127] (-127 for an all-zero block), code = E4M3(x / 2^E) nearest-even
+// saturating, sign from x.  A warp covers 256 consecutive elements of a row
+// (8 blocks, 4 threads and one 16-byte load per thread and block quarter).
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256)
+mxfp8_quant_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t K, int64_t ldx,
+                   uint8_t* __restrict__ codes, uint8_t* __restrict__ scales, int layout) {
+  pdl_wait();
+  pdl_launch_dependents();
+  const int lane = threadIdx.x & 31;
+  const int64_t segs = K / 256;
+  const int64_t units = rows * segs;
+  const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  for (int64_t u = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); u < units;
+       u += warps) {
+    const int64_t row = u / segs;
+    const int64_t col = (u % segs) * 256 + 8 * lane;
+    const uint4 v = ld_nc_v4(x + row * ldx + col);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t m = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) m = max(m, max(w[j] & 0x7FFFu, (w[j] >> 16) & 0x7FFFu));
+    m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+    m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+    // floor(log2 amax) of the block (amax = bf16 bits m, as fp32 bits m << 16)
+    const uint32_t ab = m << 16;
+    const int eb = static_cast<int>(ab >> 23);
+    int E;
+    if (ab == 0) {
+      E = -127;
+    } else {
+      const int fl = eb != 0 ? eb - 127 : (31 - __clz(static_cast<int>(ab & 0x7FFFFFu))) - 149;
+      E = min(max(fl - 8, -127), 127);
+    }
+    const float inv = pow2f(-E);                   // exact power of two
+    uint32_t out[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      uint32_t packed = 0;
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const uint32_t wd = w[2 * h + j];
+        const float lo = __fmul_rn(__uint_as_float(wd << 16), inv);
+        const float hi = __fmul_rn(__uint_as_float(wd & 0xFFFF0000u), inv);
+        uint16_t r;
+        asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+        const uint32_t c2 = static_cast<uint32_t>(r) | ((wd >> 8) & 0x80u) | ((wd >> 16) & 0x8000u);
+        packed |= c2 << (16 * j);
+      }
+      out[h] = packed;
+    }
+    *reinterpret_cast<uint2*>(codes + row * K + col) = make_uint2(out[0], out[1]);
+    if ((lane & 3) == 0) {
+      const int64_t blk = col / 32;
+      const int64_t off = layout == 0 ? row * (K / 32) + blk
+                                      : ((row >> 7) * (K / 128) + (blk >> 2)) * 512 + (row & 31) * 16 +
+                                            ((row & 127) >> 5) * 4 + (blk & 3);
+      scales[off] = static_cast<uint8_t>(E + 127);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
 // element converters and the bounded-wait probe
 // ---------------------------------------------------------------------------
 __global__ void encode_kernel(const float* __restrict__ in, uint8_t* __restrict__ out, int64_t n,
@@ -1287,6 +1352,18 @@ cudaError_t launch_weight_qdq(const uint16_t* w, int64_t N, int64_t K, int64_t l
                                    tensor_scale, colamax_bits);
     if (le != cudaSuccess) return le;
   }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_mxfp8_quant(const uint16_t* x, int64_t rows, int64_t K, int64_t ldx, uint8_t* codes,
+                               uint8_t* scales, int layout, cudaStream_t s) {
+  const int64_t warps = rows * (K / 256);
+  if (warps == 0) return cudaSuccess;
+  const int64_t ctas = (warps + 7) / 8;
+  const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
+  const cudaError_t le = launch_k(mxfp8_quant_kernel, dim3(static_cast<unsigned>(ctas < cap ? ctas : cap)), dim3(256), 0,
+                                  s, nullptr, 0, x, rows, K, ldx, codes, scales, layout);
+  if (le != cudaSuccess) return le;
   return cudaGetLastError();
 }
 
