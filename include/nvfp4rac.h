@@ -297,11 +297,14 @@ nvfp4_status weight_qdq(const uint16_t* w, int64_t N, int64_t K, int64_t ldw, in
  * memory is entirely reserved by another runtime's allocator).  The pages
  * have no counterpart: this is a property of the library, not of the method.
  *   Scratch lives in one file-scope device array of 4 MiB that every GPU
- *   loading the library keeps until the process exits; shapes needing more
- *   (nvfp4_workspace_size(NVFP4_OP_QUANTIZE, M, 0, K, 1) > 4 MiB with scores,
- *   e.g. M * K above ~44.7 million elements) are refused with
- *   NVFP4_ERR_WORKSPACE before anything is queued.  The call allocates
- *   nothing and calls no allocating routine.
+ *   loading the library keeps until the process exits; shapes whose scratch
+ *   exceeds it are refused with NVFP4_ERR_WORKSPACE before anything is
+ *   queued.  The scratch is nvfp4_workspace_size(NVFP4_OP_QUANTIZE, M, 0, K,
+ *   1) minus that function's 256-byte alignment allowance (the array itself
+ *   is 256-byte aligned); with scores it is about 12 bytes per element of
+ *   ceil(M / 128) * 128 x K, so M * K up to about 44.7 million elements fit.
+ *   The call allocates nothing and calls no allocating routine; on a device
+ *   that is not sm_100 it returns NVFP4_ERR_DEVICE before touching it.
  *   The first call on a device looks up the array's device address
  *   (cudaGetSymbolAddress with that device current); make that first call
  *   before any stream capture.

@@ -44,6 +44,15 @@ nvfp4_status device_ok() {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+}  // namespace
+
+int nvfp4::device_check() {
+  const nvfp4_status d = device_ok();
+  return d == NVFP4_OK ? 0 : (d == NVFP4_ERR_DEVICE ? 1 : 2);
+}
+
+namespace {
+
 nvfp4_status cuda_status(cudaError_t e) { return e == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA; }
 
 #define NV_TRY(expr)                                  \

@@ -14,6 +14,10 @@
 
 namespace nvfp4 {
 
+// The current device is an sm_100 GPU: 0 yes, 1 another architecture, 2 the
+// query failed (cached per device; defined with the C ABI).
+int device_check();
+
 // cuTensorMapEncodeTiled through the runtime's driver entry point (null if
 // the driver does not provide it) and the current device's SM count.
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn();

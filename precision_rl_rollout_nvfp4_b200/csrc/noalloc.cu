@@ -29,7 +29,10 @@ void* scratch_address() {
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
   if (addr[dev] == nullptr) {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_quantize_scratch) != cudaSuccess) return nullptr;
+    if (cudaGetSymbolAddress(&p, g_quantize_scratch) != cudaSuccess) {
+      cudaGetLastError();              // leave no pending error behind for later calls to report
+      return nullptr;
+    }
     addr[dev] = p;
   }
   return addr[dev];
@@ -41,6 +44,9 @@ extern "C" nvfp4_status nvfp4_quantize_static_ws(const uint16_t* x, int64_t M, i
                                                  const float* amax_or_null, nvfp4_tensor* qx,
                                                  double* score_or_null, float* res_colamax_or_null,
                                                  void* stream) {
+  // the device first: on another architecture the symbol lookup itself would fail
+  const int dc = nvfp4::device_check();
+  if (dc != 0) return dc == 1 ? NVFP4_ERR_DEVICE : NVFP4_ERR_CUDA;
   void* ws = scratch_address();
   if (ws == nullptr) return NVFP4_ERR_CUDA;
   // nvfp4_quantize refuses (NVFP4_ERR_WORKSPACE, before anything is queued)

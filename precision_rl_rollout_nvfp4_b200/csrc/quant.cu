@@ -21,6 +21,16 @@ namespace {
 constexpr int kQThreads = 256;
 constexpr int kQCols = 64;
 
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async4(void* dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
 // ---------------------------------------------------------------------------
 // amax
 // ---------------------------------------------------------------------------
@@ -102,13 +112,15 @@ amax_partial_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t K, int
   const int64_t stride = static_cast<int64_t>(gridDim.x) * kQThreads;
   const bool flat = ldx == K;
   uint32_t m = 0;
+  // vectors are visited from the end of the matrix backwards, so that its
+  // first rows are the ones still in L2 when the next pass starts there
   for (int64_t v0 = static_cast<int64_t>(blockIdx.x) * kQThreads + threadIdx.x; v0 < nvec; v0 += 8 * stride) {
     uint4 r[8];
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
-      const int64_t v = v0 + u * stride;
+      const int64_t v = nvec - 1 - (v0 + u * stride);
       r[u] = make_uint4(0, 0, 0, 0);
-      if (v < nvec) {
+      if (v >= 0) {
         const int64_t off = flat ? v * 8 : (v / kv) * ldx + (v % kv) * 8;
         r[u] = ld_nc_v4(x + off);
       }
@@ -390,6 +402,252 @@ quant_score_kernel(const uint16_t* __restrict__ x, int64_t K, int64_t ldx, RowGr
   if (t == 0) *counter = 0;                      // ready for the next call
 }
 
+// ---------------------------------------------------------------------------
+// Persistent form of the quantize + residual + score pass.  The grid is a few
+// CTAs per SM; CTA b takes the (row tile, 64-column strip) pairs b, b + grid,
+// ... in row-tile-major order, so the whole grid sweeps X from its first rows
+// to its last (the amax pass walks X backwards, so the first rows are still
+// in L2 here).  Each thread copies the 4 rows x 16 bytes it will quantize in
+// the next tile into a shared double buffer with cp.async while it works on
+// the current one, so the loads of one tile overlap the arithmetic of the
+// other and need no barrier (every thread reads only its own copies).  The
+// tensor amax, s_t and the block-scale table are formed once per CTA (again
+// only when an MoE row group changes).  Per tile the arithmetic and the
+// score's exact two-level reduction / row-order fallback are those of
+// quant_score_kernel; the block-scale codes the fallback reads are
+// double-buffered by tile parity, because other threads start the next tile
+// while the fallback thread is still summing.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void cp_async16_zfill(uint32_t dst, const void* src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0)
+               : "memory");
+}
+
+template <bool SCORES>
+__global__ void __launch_bounds__(kQThreads, 3)
+quant_score2_kernel(const uint16_t* __restrict__ x, int64_t K, int64_t ldx, RowGroups g,
+                    const float* __restrict__ amax, const unsigned* __restrict__ amax_parts,
+                    int n_parts, int64_t codes_rows,
+                    uint8_t* __restrict__ codes, uint8_t* __restrict__ scales, int layout,
+                    float* __restrict__ tensor_scale, double* __restrict__ part_sum,
+                    float* __restrict__ part_max, unsigned* __restrict__ strip_count,
+                    double* __restrict__ score, float* __restrict__ colamax) {
+  pdl_wait();
+  pdl_launch_dependents();
+  constexpr int kGroups = kTileRows / 4;
+  extern __shared__ __align__(16) uint8_t q2_dyn[];                // 2 x 16 KB tile buffers
+  uint16_t (*xbuf)[kTileRows][kQCols] = reinterpret_cast<uint16_t (*)[kTileRows][kQCols]>(q2_dyn);
+  __shared__ __align__(16) double gsum[kGroups][kQCols];          // also tail staging
+  __shared__ __align__(16) float gmax[kGroups][kQCols];
+  __shared__ __align__(16) uint32_t gmin[kGroups][kQCols];
+  __shared__ __align__(16) double qsum[4][kQCols];
+  __shared__ __align__(16) float qmax[4][kQCols];
+  __shared__ __align__(16) uint32_t qmin[4][kQCols];
+  __shared__ uint8_t s_sb[2][kTileRows][kQCols / kBlock];
+  __shared__ uint32_t wscratch[kQThreads / 32];
+  __shared__ bool s_last;
+  __shared__ ScaleTable T;
+  const int t = threadIdx.x, cg = t & 7, grp = t >> 3;
+  const int64_t n_strips = K / kQCols;
+  const int64_t row_tiles = g.off == nullptr ? (g.M + kTileRows - 1) / kTileRows : g.tile_start[g.E];
+  const int64_t total = row_tiles * n_strips;
+  // the tensor amax once per CTA (dense: the max of the partial maxima)
+  const float a_dense = (g.off == nullptr && n_parts > 0) ? reduce_parts(amax_parts, n_parts, wscratch) : 0.0f;
+  int cur_e = -1;
+  float s_t = 0.0f;
+
+  auto prefetch = [&](int64_t idx, int b) {
+    const int64_t rt = idx / n_strips, strip = idx % n_strips;
+    const TileInfo ti = tile_info(g, rt);
+    const int64_t col = strip * kQCols + 8 * cg;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int r = 4 * grp + i;
+      const int64_t row = ti.row0 + r;
+      const bool ok = ti.valid && row < ti.row_end;
+      cp_async16_zfill(smem_u32(&xbuf[b][r][8 * cg]), ok ? static_cast<const void*>(x + row * ldx + col)
+                                                           : static_cast<const void*>(x), ok);
+    }
+    cp_async_commit();
+  };
+
+  int64_t idx = blockIdx.x;
+  if (idx < total) prefetch(idx, 0);
+  for (int it = 0; idx < total; ++it, idx += gridDim.x) {
+    const int b = it & 1;
+    const int64_t nidx = idx + gridDim.x;
+    if (nidx < total) {
+      prefetch(nidx, b ^ 1);
+      cp_async_wait<1>();                          // this thread's copies of the current tile landed
+    } else {
+      cp_async_wait<0>();
+    }
+    const int64_t tile = idx / n_strips, strip = idx % n_strips;
+    const TileInfo ti = tile_info(g, tile);
+    if (ti.e != cur_e) {                           // uniform over the CTA
+      const float a = g.off == nullptr ? (n_parts > 0 ? a_dense : amax[0]) : amax[ti.e];
+      s_t = __fdiv_rn(a, kTensorScaleDiv);
+      __syncthreads();                             // nobody reads the previous group's table any more
+      build_scale_table(T, s_t, t);
+      __syncthreads();
+      cur_e = ti.e;
+    }
+    const int64_t col0 = strip * kQCols;
+    const int64_t col = col0 + 8 * cg;
+    if (strip == 0 && t == 0 && (g.off == nullptr ? tile == 0 : tile == g.tile_start[ti.e]))
+      tensor_scale[ti.e] = s_t;
+    uint8_t* code_base = codes + tile * kTileRows * (K / 2) + col / 2;
+    double acc[8];
+    float mx[8];
+    uint32_t mn[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) { acc[j] = 0.0; mx[j] = 0.0f; mn[j] = 0xFFFFFFFFu; }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int r = 4 * grp + i;
+      const int64_t prow = tile * kTileRows + r;
+      const uint4 rv = *reinterpret_cast<const uint4*>(&xbuf[b][r][8 * cg]);
+      const uint32_t wv[4] = {rv.x, rv.y, rv.z, rv.w};
+      uint64_t x2[4];
+      uint32_t mbits = 0;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        x2[j] = bf16x2_to_f2(wv[j]);
+        mbits = __vmaxu2(mbits, wv[j] & 0x7FFF7FFFu);
+      }
+      float am = __uint_as_float(max(mbits & 0xFFFFu, mbits >> 16) << 16);
+      am = fmaxf(am, __shfl_xor_sync(0xFFFFFFFFu, am, 1));
+      const BlockQ bq = block_q(am, T);
+      uint64_t q2[4];
+      block_quotients(x2, bq, q2);
+      const uint32_t packed = e2m1x8_f2(q2);
+      const uint64_t sbv2 = f2_pack(bq.sbv, bq.sbv);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        float p0, p1, x0, x1;
+        f2_unpack(f2_mul(e2m1x2_to_f2((packed >> (8 * j)) & 0xFFu), sbv2), p0, p1);
+        f2_unpack(x2[j], x0, x1);
+        const float d0 = fabsf(__fsub_rn(x0, __fmul_rn(p0, s_t)));
+        const float d1 = fabsf(__fsub_rn(x1, __fmul_rn(p1, s_t)));
+        if (SCORES) {
+          acc[2 * j] += static_cast<double>(d0);
+          acc[2 * j + 1] += static_cast<double>(d1);
+          mn[2 * j] = min(mn[2 * j], __float_as_uint(d0) - 1u);
+          mn[2 * j + 1] = min(mn[2 * j + 1], __float_as_uint(d1) - 1u);
+        }
+        mx[2 * j] = fmaxf(mx[2 * j], d0);
+        mx[2 * j + 1] = fmaxf(mx[2 * j + 1], d1);
+      }
+      if (prow < codes_rows)
+        *reinterpret_cast<uint32_t*>(code_base + static_cast<uint32_t>(r) * static_cast<uint32_t>(K / 2)) = packed;
+      if ((cg & 1) == 0 && (layout == 1 || prow < codes_rows))
+        scales[scale_offset(prow, col / kBlock, K, layout)] = static_cast<uint8_t>(bq.sb);
+      if (SCORES && (cg & 1) == 0) s_sb[b][r][cg >> 1] = static_cast<uint8_t>(bq.sb);
+    }
+    if (part_max == nullptr) continue;
+    if (SCORES) {
+#pragma unroll
+      for (int j = 0; j < 8; j += 2)
+        *reinterpret_cast<double2*>(&gsum[grp][8 * cg + j]) = make_double2(acc[j], acc[j + 1]);
+      *reinterpret_cast<uint4*>(&gmin[grp][8 * cg]) = make_uint4(mn[0], mn[1], mn[2], mn[3]);
+      *reinterpret_cast<uint4*>(&gmin[grp][8 * cg + 4]) = make_uint4(mn[4], mn[5], mn[6], mn[7]);
+    }
+    *reinterpret_cast<float4*>(&gmax[grp][8 * cg]) = make_float4(mx[0], mx[1], mx[2], mx[3]);
+    *reinterpret_cast<float4*>(&gmax[grp][8 * cg + 4]) = make_float4(mx[4], mx[5], mx[6], mx[7]);
+    __syncthreads();
+    {
+      const int c = t & (kQCols - 1), q4 = t >> 6;
+      double sum = 0.0;
+      float m = 0.0f;
+      uint32_t lo = 0xFFFFFFFFu;
+#pragma unroll
+      for (int gi = 8 * q4; gi < 8 * q4 + 8; ++gi) {
+        if (SCORES) {
+          sum += gsum[gi][c];
+          lo = min(lo, gmin[gi][c]);
+        }
+        m = fmaxf(m, gmax[gi][c]);
+      }
+      if (SCORES) {
+        qsum[q4][c] = sum;
+        qmin[q4][c] = lo;
+      }
+      qmax[q4][c] = m;
+    }
+    __syncthreads();
+    if (t < kQCols) {
+      double part = 0.0;
+      float m = 0.0f;
+      uint32_t lo = 0xFFFFFFFFu;
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) {
+        if (SCORES) {
+          part += qsum[q4][t];
+          lo = min(lo, qmin[q4][t]);
+        }
+        m = fmaxf(m, qmax[q4][t]);
+      }
+      if (SCORES && lo != 0xFFFFFFFFu) {
+        const int e_hi = static_cast<int>(__float_as_uint(m) >> 23);
+        const int e_lo = max(static_cast<int>((lo + 1u) >> 23), 1);
+        if (e_hi - e_lo > kSpanExact) {
+          const uint16_t* xc = x + col0 + t;
+          double chain = 0.0;
+          for (int r = 0; r < kTileRows; ++r) {
+            const int64_t row = ti.row0 + r;
+            if (row >= ti.row_end) break;
+            const float xv = bf16_bits_to_f32(__ldg(xc + row * ldx));
+            chain += static_cast<double>(residual_abs_one(xv, s_sb[b][r][t >> 4], T));
+          }
+          part = chain;
+        }
+      }
+      if (SCORES) part_sum[tile * K + col0 + t] = part;
+      part_max[tile * K + col0 + t] = m;
+    }
+    if (strip_count == nullptr) continue;
+    __syncthreads();
+    const int64_t t0 = g.off == nullptr ? 0 : g.tile_start[ti.e];
+    const int64_t t1 = g.off == nullptr ? row_tiles : g.tile_start[ti.e + 1];
+    unsigned* counter = strip_count + static_cast<int64_t>(ti.e) * n_strips + strip;
+    if (t == 0) {
+      __threadfence();
+      const unsigned prev = atomicAdd(counter, 1u);
+      s_last = prev == static_cast<unsigned>(t1 - t0 - 1);
+    }
+    __syncthreads();
+    if (!s_last) continue;
+    __threadfence();
+    double* ps = &gsum[0][0];                      // [32 tiles][64 cols]
+    float* pm = &gmax[0][0];
+    double total_s = 0.0;
+    float tmax = 0.0f;
+    for (int64_t c0 = t0; c0 < t1; c0 += kGroups) {
+      const int nt = static_cast<int>(t1 - c0 < kGroups ? t1 - c0 : kGroups);
+      __syncthreads();
+      for (int k = t; k < nt * kQCols; k += kQThreads) {
+        const int tt = k / kQCols, cc = k % kQCols;
+        if (SCORES) ps[k] = __ldcg(part_sum + (c0 + tt) * K + col0 + cc);
+        pm[k] = __ldcg(part_max + (c0 + tt) * K + col0 + cc);
+      }
+      __syncthreads();
+      if (t < kQCols) {
+        for (int tt = 0; tt < nt; ++tt) {          // chunk order
+          if (SCORES) total_s += ps[tt * kQCols + t];
+          tmax = fmaxf(tmax, pm[tt * kQCols + t]);
+        }
+      }
+    }
+    if (t < kQCols) {
+      if (SCORES) score[static_cast<int64_t>(ti.e) * K + col0 + t] = total_s;
+      colamax[static_cast<int64_t>(ti.e) * K + col0 + t] = tmax;
+    }
+    if (t == 0) *counter = 0;                      // ready for the next call
+    __syncthreads();                               // staging buffers free before the next tile
+  }
+  cp_async_wait<0>();
+}
+
 __global__ void score_reduce_kernel(const double* __restrict__ part_sum,
                                     const float* __restrict__ part_max, int64_t K, RowGroups g,
                                     int64_t tiles, double* __restrict__ score,
@@ -600,15 +858,6 @@ gather_quant_kernel(const uint16_t* __restrict__ src, int64_t K, int64_t ld, Row
 
 // s_t[e] = RN(max_{j < n_sel} colamax[e*K + sel[e*n_sel + j]] / 2688), one CTA per group.
 
-__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async4(void* dst, const void* src) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 // W_sel, staged by rows: the gather + second quantization of the selected
 // weight columns, from the bf16 weight (FP4 = false) or from its NVFP4 codes
@@ -1099,6 +1348,17 @@ cudaError_t launch_group_tiles(const int64_t* off, int32_t E, int32_t* tile_star
   return cudaGetLastError();
 }
 
+// NVFP4_QUANT_V1=1 in the environment selects the one-tile-per-CTA form of
+// the quantize pass (kept to compare the two on the same build).
+bool quant_v1() {
+  static int v = -1;
+  if (v < 0) {
+    const char* e = getenv("NVFP4_QUANT_V1");
+    v = (e != nullptr && e[0] == '1') ? 1 : 0;
+  }
+  return v == 1;
+}
+
 cudaError_t launch_quant_score(const uint16_t* x, int64_t rows, int64_t K, int64_t ldx,
                                const RowGroups& g, const float* amax, const unsigned* amax_parts,
                                int n_parts, int64_t codes_rows,
@@ -1107,14 +1367,30 @@ cudaError_t launch_quant_score(const uint16_t* x, int64_t rows, int64_t K, int64
                                double* score, float* colamax, cudaStream_t s) {
   const int64_t tiles = max_tiles(g, rows);
   if (tiles == 0) return cudaSuccess;
-  dim3 grid(static_cast<unsigned>(K / kQCols), static_cast<unsigned>(tiles));
-  {
+  if (quant_v1()) {
+    dim3 grid(static_cast<unsigned>(K / kQCols), static_cast<unsigned>(tiles));
     const cudaError_t le = launch_k(part_sum != nullptr ? quant_score_kernel<true> : quant_score_kernel<false>,
                                     dim3(grid), dim3(kQThreads), 0, s, nullptr, 0,
                                    x, K, ldx, g, amax, amax_parts, n_parts, codes_rows, codes, scales,
                                    layout, tensor_scale, part_sum, part_max, strip_count, score, colamax);
     if (le != cudaSuccess) return le;
+    return cudaGetLastError();
   }
+  // persistent: a few CTAs per SM over every (row tile, strip) pair
+  constexpr int kDyn = 2 * kTileRows * kQCols * 2;
+  {
+    static bool done1[kMaxAttrDevices] = {}, done0[kMaxAttrDevices] = {};
+    const cudaError_t ae = part_sum != nullptr ? set_max_smem(quant_score2_kernel<true>, kDyn, done1)
+                                               : set_max_smem(quant_score2_kernel<false>, kDyn, done0);
+    if (ae != cudaSuccess) return ae;
+  }
+  const int64_t work = tiles * (K / kQCols);
+  const int64_t cap = static_cast<int64_t>(sm_count()) * 3;
+  const cudaError_t le = launch_k(part_sum != nullptr ? quant_score2_kernel<true> : quant_score2_kernel<false>,
+                                  dim3(static_cast<unsigned>(work < cap ? work : cap)), dim3(kQThreads), kDyn, s,
+                                  nullptr, 0, x, K, ldx, g, amax, amax_parts, n_parts, codes_rows, codes, scales,
+                                  layout, tensor_scale, part_sum, part_max, strip_count, score, colamax);
+  if (le != cudaSuccess) return le;
   return cudaGetLastError();
 }
 
