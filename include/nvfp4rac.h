@@ -74,7 +74,8 @@ typedef enum {
   NVFP4_ERR_WORKSPACE = 4,        /* workspace smaller than nvfp4_workspace_size() */
   NVFP4_ERR_CUDA = 5,             /* a CUDA runtime call or launch failed */
   NVFP4_ERR_TIMEOUT = 6,          /* a device-side bounded wait gave up */
-  NVFP4_ERR_DEVICE = 7            /* current device is not sm_100 */
+  NVFP4_ERR_DEVICE = 7,           /* current device is not sm_100 */
+  NVFP4_ERR_BOUNDS = 8            /* an index check of the checked build failed */
 } nvfp4_status;
 
 typedef struct {
@@ -364,13 +365,22 @@ nvfp4_status nvfp4_encode_e2m1(const float* in, uint8_t* out, int64_t n, void* s
 nvfp4_status nvfp4_encode_e4m3(const float* in, uint8_t* out, int64_t n, void* stream);
 
 /* Synchronize `stream`, then report (and clear) the device error word:
- * NVFP4_ERR_TIMEOUT if a bounded wait gave up since the last query. */
+ * NVFP4_ERR_TIMEOUT if a bounded wait gave up since the last query, and in
+ * the checked build NVFP4_ERR_BOUNDS if an index check failed (its source
+ * line is printed to stderr). */
 nvfp4_status nvfp4_stream_status(void* stream);
 
 /* Test hook for the bounded waits: launch one CTA that waits on an mbarrier
  * nothing arrives at, giving up after about timeout_ms milliseconds (capped
  * at 2000) and recording NVFP4_ERR_TIMEOUT in the device error word. */
 nvfp4_status nvfp4_check_bounded_wait(int32_t timeout_ms, void* stream);
+
+/* Build flags: bit 0 set in the checked build (libnvfp4rac_checked.so,
+ * compiled with NVFP4_CHECKS): every global-memory store and the gathered
+ * loads of the kernels test their index against the shapes of the call; a
+ * failing test skips the access, records the source line and makes
+ * nvfp4_stream_status return NVFP4_ERR_BOUNDS.  Nothing traps. */
+int32_t nvfp4_build_flags(void);
 
 const char* nvfp4_status_string(nvfp4_status s);
 

@@ -14,7 +14,9 @@ from dataclasses import dataclass
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libnvfp4rac.so")
+# NVFP4_LIB=checked loads the index-checked build (libnvfp4rac_checked.so)
+LIB_PATH = os.path.join(_PKG, "libnvfp4rac_checked.so" if os.environ.get("NVFP4_LIB") == "checked"
+                        else "libnvfp4rac.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"{LIB_PATH} is missing: build it with "
@@ -23,7 +25,8 @@ _lib = ctypes.CDLL(LIB_PATH)
 
 OK = 0
 STATUS_NAMES = {0: "ok", 1: "invalid argument", 2: "misaligned", 3: "unsupported shape",
-                4: "workspace too small", 5: "CUDA error", 6: "timeout", 7: "not sm_100"}
+                4: "workspace too small", 5: "CUDA error", 6: "timeout", 7: "not sm_100",
+                8: "index check failed"}
 OP_QUANTIZE, OP_RAC_SELECT, OP_GEMM, OP_MOE, OP_WEIGHT_QDQ = range(5)
 EXPORTS = ["nvfp4_scale_bytes", "nvfp4_workspace_size", "nvfp4_quantize", "rac_select",
            "nvfp4_rac_nsel", "nvfp4_rac_width", "rac_weight_quant", "w4a4_rac_gemm",
@@ -31,7 +34,8 @@ EXPORTS = ["nvfp4_scale_bytes", "nvfp4_workspace_size", "nvfp4_quantize", "rac_s
            "nvfp4_encode_e2m1", "nvfp4_encode_e4m3", "nvfp4_stream_status",
            "nvfp4_check_bounded_wait", "nvfp4_status_string", "nvfp4_quantize_static_ws",
            "nvfp4_dq_colamax", "rac_weight_quant_fp4", "rac_select_channels", "rac_residual_quant",
-           "rac_sel_tensor_scale", "mxfp8_scale_bytes", "mxfp8_quantize", "w8a8_gemm_quantized"]
+           "rac_sel_tensor_scale", "mxfp8_scale_bytes", "mxfp8_quantize", "w8a8_gemm_quantized",
+           "nvfp4_build_flags"]
 
 
 class _Tensor(ctypes.Structure):
@@ -72,6 +76,7 @@ _sig = {
     "nvfp4_check_bounded_wait": (I32, [I32, P]),
     "nvfp4_status_string": (ctypes.c_char_p, [I32]),
     "mxfp8_scale_bytes": (SZ, [I64, I64, I32]),
+    "nvfp4_build_flags": (I32, []),
     "mxfp8_quantize": (I32, [P, I64, I64, I64, MP, P]),
     "w8a8_gemm_quantized": (I32, [MP, MP, P, I32, I64, P]),
 }

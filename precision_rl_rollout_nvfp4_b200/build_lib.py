@@ -10,6 +10,9 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 SOURCES = ["api.cu", "quant.cu", "select.cu", "gemm.cu", "noalloc.cu"]
 LIB = os.path.join(PKG, "libnvfp4rac.so")
+# the index-checked build (NVFP4_CHECKS): same sources, every kernel store and
+# gathered load tests its index
+LIB_CHECKED = os.path.join(PKG, "libnvfp4rac_checked.so")
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-gencode", "arch=compute_100a,code=sm_100a",
          "-Xcompiler", "-fPIC", "-shared", "-Xptxas", "-warn-spills"]
 
@@ -21,28 +24,30 @@ def nvcc() -> str:
     raise RuntimeError("nvcc not found")
 
 
-def needs_build() -> bool:
-    if not os.path.exists(LIB):
+def needs_build(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     deps = [os.path.join(PKG, "csrc", f) for f in os.listdir(os.path.join(PKG, "csrc"))]
     deps.append(os.path.join(ROOT, "include", "nvfp4rac.h"))
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and not needs_build():
-        return LIB
-    cmd = [nvcc(), *FLAGS, "-I", os.path.join(ROOT, "include"),
-           *[os.path.join(PKG, "csrc", s) for s in SOURCES], "-o", LIB + ".tmp"]
+def build(force: bool = False, verbose: bool = False, checked: bool = False) -> str:
+    lib = LIB_CHECKED if checked else LIB
+    if not force and not needs_build(lib):
+        return lib
+    cmd = [nvcc(), *FLAGS, *(["-DNVFP4_CHECKS"] if checked else []), "-I", os.path.join(ROOT, "include"),
+           *[os.path.join(PKG, "csrc", s) for s in SOURCES], "-o", lib + ".tmp"]
     res = subprocess.run(cmd, capture_output=True, text=True)
     if res.returncode != 0:
         raise RuntimeError("nvcc failed:\n" + res.stdout + res.stderr)
     if verbose and (res.stdout or res.stderr):
         print(res.stdout + res.stderr)
-    os.replace(LIB + ".tmp", LIB)
-    return LIB
+    os.replace(lib + ".tmp", lib)
+    return lib
 
 
 if __name__ == "__main__":
     print(build(force=True, verbose=True))
+    print(build(force=True, verbose=True, checked=True))

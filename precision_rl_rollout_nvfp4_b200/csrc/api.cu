@@ -600,6 +600,16 @@ nvfp4_status nvfp4_encode_e4m3(const float* in, uint8_t* out, int64_t n, void* s
 
 nvfp4_status nvfp4_stream_status(void* stream) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return NVFP4_ERR_CUDA;
+  {
+    // index checks of the checked build (always 0 in the normal build)
+    unsigned l0 = 0, l1 = 0, l2 = 0;
+    const unsigned f = bounds_flags_quant(&l0) | bounds_flags_select(&l1) | bounds_flags_gemm(&l2);
+    if (f != 0) {
+      fprintf(stderr, "nvfp4: index check failed (quant.cu line %u, select.cu line %u, gemm.cu line %u)\n", l0,
+              l1, l2);
+      return NVFP4_ERR_BOUNDS;
+    }
+  }
   unsigned* word = device_error_word();
   if (word == nullptr) return NVFP4_ERR_CUDA;
   unsigned v = 0;
@@ -622,6 +632,14 @@ nvfp4_status nvfp4_check_bounded_wait(int32_t timeout_ms, void* stream) {
   return cuda_status(launch_wait_probe(ms * 1000000ull, word, static_cast<cudaStream_t>(stream)));
 }
 
+int32_t nvfp4_build_flags(void) {
+#ifdef NVFP4_CHECKS
+  return 1;
+#else
+  return 0;
+#endif
+}
+
 const char* nvfp4_status_string(nvfp4_status s) {
   switch (s) {
     case NVFP4_OK: return "ok";
@@ -632,6 +650,7 @@ const char* nvfp4_status_string(nvfp4_status s) {
     case NVFP4_ERR_CUDA: return "CUDA error";
     case NVFP4_ERR_TIMEOUT: return "device-side wait timed out";
     case NVFP4_ERR_DEVICE: return "device is not sm_100 (B200)";
+    case NVFP4_ERR_BOUNDS: return "index check failed (checked build)";
   }
   return "unknown status";
 }

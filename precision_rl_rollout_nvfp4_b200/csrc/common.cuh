@@ -23,6 +23,55 @@ constexpr float kTensorScaleDiv = 2688.0f;   // 6 (E2M1 max) x 448 (E4M3 max)
 constexpr unsigned kErrTimeout = 1u;
 
 // ---------------------------------------------------------------------------
+// Index checks of the checked build (compiled with -DNVFP4_CHECKS; the
+// library's memory-safety evidence where no sanitizer can run).  NV_IDX(c)
+// states the in-bounds condition of one global or shared memory access: in
+// the checked build a false condition sets this translation unit's flag word
+// and records the source line (the largest one seen), and the caller skips the
+// access; nothing traps.  nvfp4_stream_status reports it as
+// NVFP4_ERR_BOUNDS.  In the normal build NV_IDX(c) is the constant true.
+// ---------------------------------------------------------------------------
+#ifdef NVFP4_CHECKS
+static __device__ unsigned g_bounds_flag;
+static __device__ unsigned g_bounds_line;
+__device__ __forceinline__ bool idx_ok(bool ok, unsigned line) {
+  if (!ok) {
+    atomicOr(&g_bounds_flag, 1u);
+    atomicMax(&g_bounds_line, line);
+  }
+  return ok;
+}
+#define NV_IDX(cond) (::nvfp4::idx_ok(static_cast<bool>(cond), __LINE__))
+// host reader of this translation unit's flag word (and reset)
+#define NV_DEFINE_BOUNDS_READER(fname)                                                   \
+  unsigned fname(unsigned* line) {                                                       \
+    unsigned v = 0, l = 0, z = 0;                                                        \
+    if (cudaMemcpyFromSymbol(&v, g_bounds_flag, sizeof(v)) != cudaSuccess) return 0;     \
+    cudaMemcpyFromSymbol(&l, g_bounds_line, sizeof(l));                                  \
+    if (v) {                                                                             \
+      cudaMemcpyToSymbol(g_bounds_flag, &z, sizeof(z));                                  \
+      cudaMemcpyToSymbol(g_bounds_line, &z, sizeof(z));                                  \
+    }                                                                                    \
+    if (line) *line = l;                                                                 \
+    return v;                                                                            \
+  }
+#else
+#define NV_IDX(cond) (true)
+#define NV_DEFINE_BOUNDS_READER(fname) \
+  unsigned fname(unsigned* line) {     \
+    if (line) *line = 0;               \
+    return 0;                          \
+  }
+#endif
+
+// Bytes of a scale buffer of rows x cols with blocks of `blk` elements in
+// `layout` (0 canonical, 1 MMA-tiled with 128-row blocks of 4-block atoms).
+__device__ __host__ __forceinline__ int64_t scale_extent(int64_t rows, int64_t cols, int layout, int blk) {
+  if (layout == 0) return rows * (cols / blk);
+  return (rows + 127) / 128 * 128 * ((cols + 4 * blk - 1) / (4 * blk)) * 4;
+}
+
+// ---------------------------------------------------------------------------
 // Element formats.
 // ---------------------------------------------------------------------------
 

@@ -87,6 +87,7 @@ struct KParams {
   const uint8_t* sfa[2];
   const uint8_t* sfb[2];
   int64_t sfa_rb[2], sfb_rb[2];   // bytes per 128-row block of the scale buffers
+  int64_t sfa_bytes[2], sfb_bytes[2];   // sizes of the scale buffers (index checks)
   const float* sta[2];
   const float* stb[2];
   void* y;
@@ -253,13 +254,17 @@ __device__ __forceinline__ void gemm1_body(const CUtensorMap& tmA0, const CUtens
             const int nkb = kt == p.kt[seg] - 1 ? p.kb_last[seg] : 4;
             const uint32_t sf_bytes = FP8 ? SF_ATOM : nkb * SF_ATOM;
             const uint32_t fb = smem_u32(&full[stage]);
+            const int64_t sfa_off = mt * p.sfa_rb[seg] + kt * SF_STEP;
+            const int64_t sfb_off = (b_row / BN) * p.sfb_rb[seg] + kt * SF_STEP;
+            if (!NV_IDX(sfa_off + sf_bytes <= p.sfa_bytes[seg] && sfb_off + sf_bytes <= p.sfb_bytes[seg])) {
+              ok = false;                          // (checked build) never issue the out-of-range copy
+              break;
+            }
             mbar_arrive_expect_tx(&full[stage], A_STAGE + B_STAGE + 2 * sf_bytes);
             tma_load_2d(smem_u32(sA + stage * A_STAGE), tA, kt * BK_BYTES, static_cast<int>(mt * BM), fb);
             tma_load_2d(smem_u32(sB + stage * B_STAGE), tB, kt * BK_BYTES, static_cast<int>(b_row), fb);
-            bulk_load(smem_u32(sSFA + stage * SF_STAGE), p.sfa[seg] + mt * p.sfa_rb[seg] + kt * SF_STEP,
-                      sf_bytes, fb);
-            bulk_load(smem_u32(sSFB + stage * SF_STAGE),
-                      p.sfb[seg] + (b_row / BN) * p.sfb_rb[seg] + kt * SF_STEP, sf_bytes, fb);
+            bulk_load(smem_u32(sSFA + stage * SF_STAGE), p.sfa[seg] + sfa_off, sf_bytes, fb);
+            bulk_load(smem_u32(sSFB + stage * SF_STAGE), p.sfb[seg] + sfb_off, sf_bytes, fb);
             armed |= 1u << stage;
             armed_phase = (armed_phase & ~(1u << stage)) | (phase << stage);
             if (++stage == STAGES) { stage = 0; phase ^= 1; }
@@ -400,7 +405,7 @@ __device__ __forceinline__ void gemm1_body(const CUtensorMap& tmA0, const CUtens
 #pragma unroll 4
       for (int r = 0; r < 32; ++r) {
         const int64_t row = ti.row0 + 32 * q + r;
-        if (!ti.valid || row >= ti.row_end || !col_ok) continue;
+        if (!ti.valid || row >= ti.row_end || !col_ok || !NV_IDX(row < p.M)) continue;
         const uint8_t* src = stg_warp + r * STG_STRIDE + lane * 4 * YBYTES;
         if (YBYTES == 4)
           *reinterpret_cast<float4*>(static_cast<float*>(p.y) + row * p.ldy + col) = *reinterpret_cast<const float4*>(src);
@@ -852,6 +857,7 @@ w4a4_rac_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid
         for (int r = 0; r < 32; ++r) {
           if (lrow0 + r >= pr.m || !col_ok) continue;
           const int64_t row = pr.out0 + lrow0 + r;
+          if (!NV_IDX(row < p.M)) continue;
           const uint8_t* src = stg_warp + r * C::STG_STRIDE + lane * 4 * YBYTES;
           if (YBYTES == 4)
             *reinterpret_cast<float4*>(static_cast<float*>(p.y) + row * p.ldy + col) = *reinterpret_cast<const float4*>(src);
@@ -1038,6 +1044,8 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s) {
     p.sfb[seg] = B[sg]->scales;
     p.sfa_rb[seg] = (cols + 63) / 64 * SF_ATOM;
     p.sfb_rb[seg] = (B[sg]->cols + 63) / 64 * SF_ATOM;
+    p.sfa_bytes[seg] = scale_extent(A[sg]->rows, cols, 1, kBlock);
+    p.sfb_bytes[seg] = scale_extent(B[sg]->rows, B[sg]->cols, 1, kBlock);
     p.sta[seg] = A[sg]->st;
     p.stb[seg] = B[sg]->st;
     if (!make_code_map(&maps[2 * seg], A[sg]->codes, A[sg]->rows, cols, BM)) return cudaErrorInvalidValue;
@@ -1084,6 +1092,8 @@ cudaError_t launch_gemm_fp8(const GemmArgs& a, cudaStream_t s) {
   p.sfb[0] = p.sfb[1] = a.b0.scales;
   p.sfa_rb[0] = p.sfa_rb[1] = (K / 128) * SF_ATOM;   // one atom (128 rows x 4 blocks of 32) per step
   p.sfb_rb[0] = p.sfb_rb[1] = (K / 128) * SF_ATOM;
+  p.sfa_bytes[0] = p.sfa_bytes[1] = scale_extent(a.a0.rows, K, 1, 32);
+  p.sfb_bytes[0] = p.sfb_bytes[1] = scale_extent(a.b0.rows, K, 1, 32);
   CUtensorMap maps[2];
   if (!make_code_map(&maps[0], a.a0.codes, a.a0.rows, K, BM, K) ||
       !make_code_map(&maps[1], a.b0.codes, a.b0.rows, K, BN, K))
@@ -1104,5 +1114,7 @@ cudaError_t launch_gemm_fp8(const GemmArgs& a, cudaStream_t s) {
   if (le != cudaSuccess) return le;
   return cudaGetLastError();
 }
+
+NV_DEFINE_BOUNDS_READER(bounds_flags_gemm)
 
 }  // namespace nvfp4

@@ -14,6 +14,12 @@
 
 namespace nvfp4 {
 
+// Index-check flags of each translation unit's kernels (checked build; 0
+// otherwise), read and reset; *line gets the largest failing source line.
+unsigned bounds_flags_quant(unsigned* line);
+unsigned bounds_flags_select(unsigned* line);
+unsigned bounds_flags_gemm(unsigned* line);
+
 // The current device is an sm_100 GPU: 0 yes, 1 another architecture, 2 the
 // query failed (cached per device; defined with the C ABI).
 int device_check();

@@ -50,7 +50,7 @@ amax_kernel(const uint16_t* __restrict__ x, int64_t K, int64_t ldx, RowGroups g,
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int64_t row = ti.row0 + rr + 32 * i;
-    if (row < ti.row_end) {
+    if (row < ti.row_end && NV_IDX(col + 8 <= K)) {
       const uint4 v = ld_nc_v4(x + row * ldx + col);
       const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
@@ -67,7 +67,7 @@ amax_kernel(const uint16_t* __restrict__ x, int64_t K, int64_t ldx, RowGroups g,
   if (t == 0) {
     uint32_t r = 0;
     for (int i = 0; i < kQThreads / 32; ++i) r = max(r, wmax[i]);
-    if (r) atomicMax(amax_bits + ti.e, r << 16);   // |bf16| bits order like their values
+    if (r && NV_IDX(ti.e < g.E)) atomicMax(amax_bits + ti.e, r << 16);   // |bf16| bits order like their values
   }
 }
 
@@ -120,7 +120,7 @@ amax_partial_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t K, int
     for (int u = 0; u < 8; ++u) {
       const int64_t v = nvec - 1 - (v0 + u * stride);
       r[u] = make_uint4(0, 0, 0, 0);
-      if (v >= 0) {
+      if (v >= 0 && NV_IDX(v < nvec)) {
         const int64_t off = flat ? v * 8 : (v / kv) * ldx + (v % kv) * 8;
         r[u] = ld_nc_v4(x + off);
       }
@@ -464,7 +464,7 @@ quant_score2_kernel(const uint16_t* __restrict__ x, int64_t K, int64_t ldx, RowG
     for (int i = 0; i < 4; ++i) {
       const int r = 4 * grp + i;
       const int64_t row = ti.row0 + r;
-      const bool ok = ti.valid && row < ti.row_end;
+      const bool ok = ti.valid && row < ti.row_end && NV_IDX(col + 8 <= K);
       cp_async16_zfill(smem_u32(&xbuf[b][r][8 * cg]), ok ? static_cast<const void*>(x + row * ldx + col)
                                                            : static_cast<const void*>(x), ok);
     }
@@ -538,9 +538,10 @@ quant_score2_kernel(const uint16_t* __restrict__ x, int64_t K, int64_t ldx, RowG
         mx[2 * j] = fmaxf(mx[2 * j], d0);
         mx[2 * j + 1] = fmaxf(mx[2 * j + 1], d1);
       }
-      if (prow < codes_rows)
+      if (prow < codes_rows && NV_IDX(col + 8 <= K))
         *reinterpret_cast<uint32_t*>(code_base + static_cast<uint32_t>(r) * static_cast<uint32_t>(K / 2)) = packed;
-      if ((cg & 1) == 0 && (layout == 1 || prow < codes_rows))
+      if ((cg & 1) == 0 && (layout == 1 || prow < codes_rows) &&
+          NV_IDX(scale_offset(prow, col / kBlock, K, layout) < scale_extent(codes_rows, K, layout, kBlock)))
         scales[scale_offset(prow, col / kBlock, K, layout)] = static_cast<uint8_t>(bq.sb);
       if (SCORES && (cg & 1) == 0) s_sb[b][r][cg >> 1] = static_cast<uint8_t>(bq.sb);
     }
@@ -595,15 +596,17 @@ quant_score2_kernel(const uint16_t* __restrict__ x, int64_t K, int64_t ldx, RowG
           double chain = 0.0;
           for (int r = 0; r < kTileRows; ++r) {
             const int64_t row = ti.row0 + r;
-            if (row >= ti.row_end) break;
+            if (row >= ti.row_end || !NV_IDX(col0 + t < K)) break;
             const float xv = bf16_bits_to_f32(__ldg(xc + row * ldx));
             chain += static_cast<double>(residual_abs_one(xv, s_sb[b][r][t >> 4], T));
           }
           part = chain;
         }
       }
-      if (SCORES) part_sum[tile * K + col0 + t] = part;
-      part_max[tile * K + col0 + t] = m;
+      if (NV_IDX(tile < row_tiles && col0 + t < K)) {
+        if (SCORES) part_sum[tile * K + col0 + t] = part;
+        part_max[tile * K + col0 + t] = m;
+      }
     }
     if (strip_count == nullptr) continue;
     __syncthreads();
@@ -638,7 +641,7 @@ quant_score2_kernel(const uint16_t* __restrict__ x, int64_t K, int64_t ldx, RowG
         }
       }
     }
-    if (t < kQCols) {
+    if (t < kQCols && NV_IDX(ti.e < g.E && col0 + t < K)) {
       if (SCORES) score[static_cast<int64_t>(ti.e) * K + col0 + t] = total_s;
       colamax[static_cast<int64_t>(ti.e) * K + col0 + t] = tmax;
     }
@@ -749,6 +752,7 @@ gather_quant_kernel(const uint16_t* __restrict__ src, int64_t K, int64_t ld, Row
     for (int u = 0; u < 8; ++u) {
       const int64_t j = j0 + lane + 32 * u;
       c[u] = (valid && j < n_sel) ? __ldg(sel_e + j) : -1;
+      if (valid && j < n_sel && !NV_IDX(c[u] >= 0 && c[u] < K)) c[u] = -1;
     }
     const bool do_fuse = fuse && first;
     int32_t fc[8];
@@ -849,8 +853,10 @@ gather_quant_kernel(const uint16_t* __restrict__ src, int64_t K, int64_t ld, Row
         for (int u = 0; u < 16; ++u) am = fmaxf(am, fabsf(v[u]));
         const BlockQ bq = block_q(am, T);
         const uint32_t lo = encode8_q(v, bq), hi = encode8_q(v + 8, bq);
-        if (in_rows) *reinterpret_cast<uint2*>(out_codes + prow * (width / 2) + blk * 8) = make_uint2(lo, hi);
-        out_scales[scale_offset(prow, blk, width, out_layout)] = static_cast<uint8_t>(bq.sb);
+        if (in_rows && NV_IDX(blk * kBlock + 16 <= width))
+          *reinterpret_cast<uint2*>(out_codes + prow * (width / 2) + blk * 8) = make_uint2(lo, hi);
+        if (NV_IDX(scale_offset(prow, blk, width, out_layout) < scale_extent(grid_rows, width, out_layout, kBlock)))
+          out_scales[scale_offset(prow, blk, width, out_layout)] = static_cast<uint8_t>(bq.sb);
       }
     }
   }
@@ -948,6 +954,7 @@ wsel_rows_kernel(const uint16_t* __restrict__ w, int64_t ldw, const uint8_t* __r
       const int64_t j = static_cast<int64_t>(ob) * kBlock + u;
       const int32_t v = j < n_sel ? __ldg(sel_e + j) : -1;
       c[u] = (v >= 0 && v < K) ? static_cast<uint32_t>(v) : Ku;
+      if (j < n_sel && !NV_IDX(v >= 0 && v < K)) c[u] = Ku;
     }
   };
   uint32_t cidx[16];
@@ -1041,9 +1048,11 @@ wsel_rows_kernel(const uint16_t* __restrict__ w, int64_t ldw, const uint8_t* __r
           const int64_t row = r0 + slot;
           const BlockQ bq = block_q(am, T);
           const uint32_t lo = encode8_q(v, bq), hi = encode8_q(v + 8, bq);
-          *reinterpret_cast<uint2*>(out_codes + row * (width / 2) + static_cast<int64_t>(ob) * 8) =
-              make_uint2(lo, hi);
-          out_scales[scale_offset(row, ob, width, out_layout)] = static_cast<uint8_t>(bq.sb);
+          if (NV_IDX(row < rows && (ob + 1) * kBlock <= width)) {
+            *reinterpret_cast<uint2*>(out_codes + row * (width / 2) + static_cast<int64_t>(ob) * 8) =
+                make_uint2(lo, hi);
+            out_scales[scale_offset(row, ob, width, out_layout)] = static_cast<uint8_t>(bq.sb);
+          }
         }
       }
     }
@@ -1133,7 +1142,7 @@ __global__ void sel_tensor_scale_kernel(const float* __restrict__ colamax, int64
   float m = 0.0f;
   for (int64_t j = threadIdx.x; j < n_sel; j += blockDim.x) {
     const int64_t c = sel[e * n_sel + j];
-    if (c >= 0 && c < K) m = fmaxf(m, colamax[e * K + c]);
+    if (NV_IDX(c >= 0 && c < K)) m = fmaxf(m, colamax[e * K + c]);
   }
   m = __uint_as_float(__reduce_max_sync(0xFFFFFFFFu, __float_as_uint(m)));
   __shared__ float wm[32];
@@ -1208,8 +1217,10 @@ weight_qdq_kernel(const uint16_t* w, int64_t N, int64_t K, int64_t ldw,
         f2_unpack(f2_mul(f2_mul(e2m1x2_to_f2((q >> (8 * j)) & 0xFFu), sbv2), st2), d0, d1);
         asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(o[j]) : "f"(d1), "f"(d0));   // d0 in the low half
       }
-      *reinterpret_cast<uint4*>(w_out + off) = make_uint4(o[0], o[1], o[2], o[3]);
-      if (codes) *reinterpret_cast<uint32_t*>(codes + qrow * (K / 2) + col / 2) = q;
+      if (NV_IDX(col + 8 <= K)) {
+        *reinterpret_cast<uint4*>(w_out + off) = make_uint4(o[0], o[1], o[2], o[3]);
+        if (codes) *reinterpret_cast<uint32_t*>(codes + qrow * (K / 2) + col / 2) = q;
+      }
     }
     // rows past N belong to the next matrix: only live rows write (the caller
     // zero-fills the padding of a tiled scale buffer beforehand)
@@ -1285,13 +1296,14 @@ mxfp8_quant_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t K, int6
       }
       out[h] = packed;
     }
-    *reinterpret_cast<uint2*>(codes + row * K + col) = make_uint2(out[0], out[1]);
+    if (NV_IDX(row < rows && col + 8 <= K))
+      *reinterpret_cast<uint2*>(codes + row * K + col) = make_uint2(out[0], out[1]);
     if ((lane & 3) == 0) {
       const int64_t blk = col / 32;
       const int64_t off = layout == 0 ? row * (K / 32) + blk
                                       : ((row >> 7) * (K / 128) + (blk >> 2)) * 512 + (row & 31) * 16 +
                                             ((row & 127) >> 5) * 4 + (blk & 3);
-      scales[off] = static_cast<uint8_t>(E + 127);
+      if (NV_IDX(off < scale_extent(rows, K, layout, 32))) scales[off] = static_cast<uint8_t>(E + 127);
     }
   }
 }
@@ -1653,5 +1665,7 @@ cudaError_t launch_wait_probe(uint64_t limit_ns, unsigned* err, cudaStream_t s) 
   wait_probe_kernel<<<1, 32, 0, s>>>(limit_ns, err);
   return cudaGetLastError();
 }
+
+NV_DEFINE_BOUNDS_READER(bounds_flags_quant)
 
 }  // namespace nvfp4

@@ -197,7 +197,7 @@ topk_kernel(const double* __restrict__ score, const float* __restrict__ colamax,
     }
     mk[j] = m ? 1 : 0;
     if (m) {
-      if (p < n_sel) sl[p] = static_cast<int32_t>(j);
+      if (NV_IDX(p < n_sel)) sl[p] = static_cast<int32_t>(j);
       ++p;
       mx = fmaxf(mx, cm[j]);
     }
@@ -234,5 +234,7 @@ cudaError_t launch_topk(const double* score, const float* colamax, int64_t K, in
   }
   return cudaGetLastError();
 }
+
+NV_DEFINE_BOUNDS_READER(bounds_flags_select)
 
 }  // namespace nvfp4
