@@ -104,7 +104,7 @@ def work(M, K, N, n_sel, width, wsel="bf16", static_amax=False):
     wsel="fp4" the weight preparation also reads Q(W) once for the DQ column
     maxima, and W_sel is gathered from the 0.5625 B/element NVFP4 weight."""
     fp4 = wsel == "fp4"
-    return {
+    d = {
         "prepare_weight": dict(bytes=6.5625 * N * K + 4 * K + (0.5625 * N * K + 4 * K if fp4 else 0.0),
                                bound="hbm"),
         "quantize": dict(bytes=(2.0 if static_amax else 4.0) * M * K + 0.5625 * M * K + 12 * K, bound="hbm"),
@@ -113,6 +113,11 @@ def work(M, K, N, n_sel, width, wsel="bf16", static_amax=False):
         "gemm": dict(flops=2.0 * M * N * (K + n_sel), bytes=0.5625 * (M + N) * (K + width) + 2.0 * M * N,
                      bound="tensor"),
     }
+    # the fused calls of the step: quantize + selection, and both second passes
+    d["quantize_select"] = dict(bytes=d["quantize"]["bytes"] + 4 * n_sel + K, bound="hbm")
+    d["second_pass"] = dict(bytes=d["select"]["bytes"] - 12 * K - 4 * n_sel + 4 * n_sel + d["weight_select"]["bytes"],
+                            bound="hbm")
+    return d
 
 
 # ---------------------------------------------------------------- clocks
@@ -276,6 +281,27 @@ def e2e_pipelined(sets, steps, warmup):
     return t0.elapsed_time(t1)
 
 
+# ---------------------------------------------------------------- launches
+def graph_kernel_count(g):
+    """Kernel nodes in a captured torch CUDA graph (None when the graph or
+    cuda-python cannot tell)."""
+    if g is None:
+        return None
+    try:
+        from cuda.bindings import runtime as rt
+        raw = g.raw_cuda_graph()
+        err, nodes, n = rt.cudaGraphGetNodes(raw, 0)
+        err, nodes, n = rt.cudaGraphGetNodes(raw, n)
+        count = 0
+        for nd in nodes[:n]:
+            err, ty = rt.cudaGraphNodeGetType(nd)
+            if ty == rt.cudaGraphNodeType.cudaGraphNodeTypeKernel:
+                count += 1
+        return count
+    except Exception:
+        return None
+
+
 # ---------------------------------------------------------------- ranks
 def max_over_ranks(values, world, device="cpu"):
     """Element-wise max of per-rank timings (every rank gets the result)."""
@@ -347,9 +373,11 @@ def run_ours(args, rank, world, local_rank):
     plan = B.RacLinearPlan(M, K, N, k, out_dtype=torch.bfloat16, device=dev, wsel=args.wsel).bind(x, w, amax)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
-    calls = ["prepare_weight", "quantize", "select", "weight_select", "gemm"]
-    fns = {"prepare_weight": plan.prepare_weight, "quantize": plan.quantize, "select": plan.select,
-           "weight_select": plan.weight_select, "gemm": plan.gemm}
+    # the calls of one step, each timed alone below: weight preparation, the
+    # quantize pass with the fused top-k selection, both second passes, GEMM
+    calls = ["prepare_weight", "quantize_select", "second_pass", "gemm"]
+    fns = {"prepare_weight": plan.prepare_weight, "quantize_select": plan.quantize_select,
+           "second_pass": plan.second_pass, "gemm": plan.gemm}
     reuse = args.mask == "reuse"
     qdq = None
     if args.workload in QDQ_EXPERTS and not reuse:
@@ -473,7 +501,7 @@ def run_ours(args, rank, world, local_rank):
     # comparators timed the same way (not part of the step): the plain W4A4
     # GEMM alone, and the FP8 path on the same shape -- MXFP8 quantization of
     # X and the kind::mxf8f6f4 W8A8 GEMM (W quantized once beforehand)
-    cmp_fns = {"gemm_plain": lambda: plan.gemm(plain=True)}
+    cmp_fns = {"gemm_plain": lambda: plan.gemm(plain=True), "quantize": plan.quantize}
     if K % 256 == 0:
         qa8, qb8 = B.mxfp8_quantize(x), B.mxfp8_quantize(w)
         y8 = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
@@ -510,6 +538,15 @@ def run_ours(args, rank, world, local_rank):
                 a = ev(); f(); b_ = ev()
                 torch.cuda.synchronize()
                 cmp_call[c].append(a.elapsed_time(b_))
+    # the RAC linear without weight preparation as one graph (launch count)
+    g_rac = None
+    if use_graph and not reuse:
+        g_rac = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_rac):
+            plan.quantize_select()
+            plan.second_pass()
+            plan.gemm()
+        torch.cuda.synchronize()
     # plain W4A4 linear (no RAC) and the RAC linear without weight prep, for the overhead
     plain_ms, rac_ms = [], []
     for _ in range(args.steps):
@@ -520,7 +557,7 @@ def run_ours(args, rank, world, local_rank):
         if reuse:
             launch("step")
         else:
-            for name in ("quantize", "select", "weight_select", "gemm"):
+            for name in ("quantize_select", "second_pass", "gemm"):
                 launch(name)
         d = ev()
         torch.cuda.synchronize()
@@ -604,14 +641,17 @@ def run_ours(args, rank, world, local_rank):
                 "unit": "GB/s", "frac": round(achieved / hbm_peak, 4), "traffic": traffic,
                 "traffic_source": traffic_source, "peak_source": f"{peak_kind}: hbm_gbs"}
     gemm_tflops = wk["gemm"]["flops"] / (med["gemm"] * 1e-3) / 1e12
-    quant_gbs = wk["quantize"]["bytes"] / (med["quantize"] * 1e-3) / 1e9
+    quant_gbs = wk["quantize"]["bytes"] / (statistics.median(cmp_call["quantize"])) / 1e6
     rac_over = (statistics.median(rac_ms) - statistics.median(plain_ms)) / statistics.median(plain_ms)
     bf16_us = 1e3 * statistics.median(bf16_ms)
-    launches_per_step = ((plan.launches["reuse_step"] if n_sel else 3) if reuse else
-                         sum(plan.launches[c] for c in calls if c in plan.launches) - (0 if n_sel else 2)) \
-        - (1 if args.static_amax else 0)          # no amax pass
-    if qdq is not None:
-        launches_per_step += 2 * len(qdq.shapes)  # amax pass + quantization per stacked weight
+    launches_per_step = graph_kernel_count(graphs.get("step")) if use_graph else None
+    if launches_per_step is None:                 # static count of the step's calls
+        launches_per_step = ((plan.launches["reuse_step"] if n_sel else 3) if reuse else
+                             sum(plan.launches[c] for c in calls if c in plan.launches) - (0 if n_sel else 1)) \
+            - (1 if args.static_amax else 0)      # no amax pass
+        if qdq is not None:
+            launches_per_step += 2 * len(qdq.shapes)  # amax pass + quantization per stacked weight
+    rac_launches = graph_kernel_count(g_rac) if use_graph else None
 
     cfg = {"workload": args.workload, "M": M, "K": K, "N": N, "k_percent": k, "n_sel": n_sel,
            "y_dtype": "bf16", "wsel": args.wsel, "mask": args.mask,
@@ -647,8 +687,12 @@ def run_ours(args, rank, world, local_rank):
                 "ms_per_step": round(e2e_total / args.steps, 4),
                 "pipelined": "2 buffer sets; H2D, compute and D2H on separate streams"},
         "gpu_launches": launches_per_step * args.steps,
+        "launches_per_step": launches_per_step,
+        "rac_linear_launches": rac_launches,
         "clocks": clock,
     }
+    if "quantize_select" in med:
+        line["quantize_select_gbs"] = round(wk["quantize"]["bytes"] / (med["quantize_select"] * 1e-3) / 1e9, 1)
     cmp_us = {c: 1e3 * statistics.median(v) for c, v in cmp_call.items() if v}
     line["comparators_us"] = {c: round(v, 2) for c, v in cmp_us.items()}
     if "fp8_gemm" in cmp_us:

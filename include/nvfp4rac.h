@@ -177,6 +177,40 @@ nvfp4_status rac_sel_tensor_scale(const float* colamax, int64_t K, const int32_t
 nvfp4_status rac_residual_quant(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, const nvfp4_tensor* qx,
                                 const int32_t* sel, int64_t n_sel, nvfp4_tensor* q_res, void* stream);
 
+/*
+ * rac_quantize_select -- nvfp4_quantize (with scores and residual column
+ * maxima) and rac_select_channels in one pass over X: the CTA that finishes
+ * the last column strip of the quantize pass runs the top-k% selection on the
+ * finished scores, so mask, sel and the residual tensor scale come out of the
+ * same launch (plus the amax pass unless amax_or_null is given).  Pages:
+ * 2.2 B (residual magnitude, binary channel mask of the top k%; the pages'
+ * implementation fuses its kernels to keep the overhead low).  Arguments as
+ * for the two calls; the outputs are identical to theirs.
+ *   ws: nvfp4_workspace_size(NVFP4_OP_QUANTIZE, M, 0, K, 1) bytes.
+ */
+nvfp4_status rac_quantize_select(const uint16_t* x, int64_t M, int64_t K, int64_t ldx,
+                                 const float* amax_or_null, nvfp4_tensor* qx, double* score,
+                                 float* res_colamax, float k_percent, uint8_t* mask, int32_t* sel,
+                                 int64_t* n_sel_out, float* res_tensor_scale, void* ws, size_t ws_bytes,
+                                 void* stream);
+
+/*
+ * rac_second_pass -- both second-pass quantizations of a RAC linear in one
+ * call: Q(dX_sel) exactly as rac_residual_quant (q_res->tensor_scale must
+ * hold the residual tensor scale already) and Q(W_sel) exactly as
+ * rac_weight_quant from bf16 w [N, K] (stride ldw), or, with w == NULL, as
+ * rac_weight_quant_fp4 from qw (w_colamax then nvfp4_dq_colamax(qw, 1)).
+ * One kernel launch runs both when the weight side uses the tile gather
+ * (weights of up to about 9000 rows at K = 4096), two otherwise.  Pages: 2.2 B
+ * (second-pass quantization of the selected channels).
+ *   q_res: rows = M, cols = nvfp4_rac_width(n_sel); q_wsel: rows = N, same
+ *   cols, scale_layout 1 for the GEMM.
+ */
+nvfp4_status rac_second_pass(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, const nvfp4_tensor* qx,
+                             const int32_t* sel, int64_t n_sel, nvfp4_tensor* q_res, const uint16_t* w,
+                             int64_t N, int64_t ldw, const nvfp4_tensor* qw, const float* w_colamax,
+                             nvfp4_tensor* q_wsel, void* stream);
+
 /* n_sel for k_percent of K channels (exact floor), and the padded width of
  * the gathered residual / weight operands (n_sel rounded up to 64). */
 int64_t nvfp4_rac_nsel(float k_percent, int64_t K);

@@ -35,7 +35,7 @@ EXPORTS = ["nvfp4_scale_bytes", "nvfp4_workspace_size", "nvfp4_quantize", "rac_s
            "nvfp4_check_bounded_wait", "nvfp4_status_string", "nvfp4_quantize_static_ws",
            "nvfp4_dq_colamax", "rac_weight_quant_fp4", "rac_select_channels", "rac_residual_quant",
            "rac_sel_tensor_scale", "mxfp8_scale_bytes", "mxfp8_quantize", "w8a8_gemm_quantized",
-           "nvfp4_build_flags"]
+           "nvfp4_build_flags", "rac_quantize_select", "rac_second_pass"]
 
 
 class _Tensor(ctypes.Structure):
@@ -77,6 +77,8 @@ _sig = {
     "nvfp4_status_string": (ctypes.c_char_p, [I32]),
     "mxfp8_scale_bytes": (SZ, [I64, I64, I32]),
     "nvfp4_build_flags": (I32, []),
+    "rac_quantize_select": (I32, [P, I64, I64, I64, P, TP, P, P, F32, P, P, ctypes.POINTER(I64), P, P, SZ, P]),
+    "rac_second_pass": (I32, [P, I64, I64, I64, TP, P, I64, TP, P, I64, I64, TP, P, TP, P]),
     "mxfp8_quantize": (I32, [P, I64, I64, I64, MP, P]),
     "w8a8_gemm_quantized": (I32, [MP, MP, P, I32, I64, P]),
 }
@@ -223,6 +225,45 @@ def rac_select(x, qx, score, colamax, k_percent, layout=1, stream=None):
                            _stream(stream)), "rac_select")
     assert n_out.value == n_sel
     return mask, sel[:n_sel], n_sel, q_res
+
+
+def quantize_select(x, k_percent, amax=None, layout=1, stream=None):
+    """Q(X), scores and the top-k% selection in one pass (rac_quantize_select).
+    Returns (qx, score, res_colamax, mask, sel [n_sel], n_sel, res_tensor_scale)."""
+    x = _bits(x)
+    M, K = x.shape
+    n_sel = rac_nsel(k_percent, K)
+    qx = NvFP4Tensor.empty(M, K, layout, device=x.device)
+    score = torch.empty(K, dtype=torch.float64, device=x.device)
+    colamax = torch.empty(K, dtype=torch.float32, device=x.device)
+    mask = torch.empty(K, dtype=torch.uint8, device=x.device)
+    sel = torch.empty(max(n_sel, 1), dtype=torch.int32, device=x.device)
+    st = torch.empty(1, dtype=torch.float32, device=x.device)
+    ws = _ws(workspace_size(OP_QUANTIZE, M, 0, K), x.device)
+    n_out = ctypes.c_int64(-1)
+    q = qx.c()
+    _check(_lib.rac_quantize_select(_ptr(x), M, K, x.stride(0), _ptr(amax), ctypes.byref(q), _ptr(score),
+                                    _ptr(colamax), float(k_percent), _ptr(mask), _ptr(sel), ctypes.byref(n_out),
+                                    _ptr(st), _ptr(ws), ws.numel(), _stream(stream)), "rac_quantize_select")
+    assert n_out.value == n_sel
+    return qx, score, colamax, mask, sel[:n_sel], n_sel, st
+
+
+def second_pass(x, qx, sel, n_sel, res_tensor_scale, w, qw, w_colamax, layout=1, stream=None):
+    """Q(dX_sel) and Q(W_sel) in one call (rac_second_pass); w = None takes
+    W_sel from qw (w_colamax = dq_colamax(qw)).  Returns (q_res, q_wsel)."""
+    x = _bits(x)
+    M, K = x.shape
+    N = qw.rows
+    q_res = NvFP4Tensor.empty(M, rac_width(n_sel), layout, device=x.device)
+    q_res.tensor_scale.copy_(res_tensor_scale.reshape(1))
+    q_ws = NvFP4Tensor.empty(N, rac_width(n_sel), layout, device=x.device)
+    a, r, wq, ws_ = qx.c(), q_res.c(), qw.c(), q_ws.c()
+    w = _bits(w) if w is not None else None
+    _check(_lib.rac_second_pass(_ptr(x), M, K, x.stride(0), ctypes.byref(a), _ptr(sel), n_sel, ctypes.byref(r),
+                                _ptr(w), N, w.stride(0) if w is not None else K, ctypes.byref(wq), _ptr(w_colamax),
+                                ctypes.byref(ws_), _stream(stream)), "rac_second_pass")
+    return q_res, q_ws
 
 
 def rac_select_channels(score, colamax, k_percent, res_tensor_scale=None, stream=None):
@@ -575,6 +616,25 @@ class RacLinearPlan:
                                ctypes.byref(self._qr) if self._qr is not None else None,
                                _ptr(self.ws), self.ws.numel(), _stream(stream)), "rac_select")
 
+    def quantize_select(self, stream=None):
+        """Q(X), scores, mask, sel and the residual tensor scale in one pass."""
+        _check(_lib.rac_quantize_select(_ptr(self.x), self.M, self.K, self.x.stride(0), _ptr(self.amax),
+                                        ctypes.byref(self._qx), _ptr(self.score), _ptr(self.res_colamax), self.k,
+                                        _ptr(self.mask), _ptr(self.sel), ctypes.byref(self._nout),
+                                        _ptr(self.res_st), _ptr(self.ws), self.ws.numel(), _stream(stream)),
+               "rac_quantize_select")
+
+    def second_pass(self, stream=None):
+        """Q(dX_sel) and Q(W_sel) in one call."""
+        if self.n_sel == 0:
+            return
+        fp4 = self.wsel == "fp4"
+        _check(_lib.rac_second_pass(_ptr(self.x), self.M, self.K, self.x.stride(0), ctypes.byref(self._qx),
+                                    _ptr(self.sel), self.n_sel, ctypes.byref(self._qr),
+                                    None if fp4 else _ptr(self.w), self.N, self.K if fp4 else self.w.stride(0),
+                                    ctypes.byref(self._qw), _ptr(self.dq_colamax if fp4 else self.w_colamax),
+                                    ctypes.byref(self._qs), _stream(stream)), "rac_second_pass")
+
     def select_channels(self, stream=None):
         _check(_lib.rac_select_channels(_ptr(self.score), _ptr(self.res_colamax), self.K, self.k, _ptr(self.mask),
                                         _ptr(self.sel), ctypes.byref(self._nout), _ptr(self.res_st),
@@ -621,22 +681,30 @@ class RacLinearPlan:
                                         _stream(stream)), "w4a4_gemm_quantized")
 
     def rollout_step(self):
-        """The rollout linear on an already-prepared weight (on the current
-        stream; the two gathers overlap through the side stream)."""
-        main = torch.cuda.current_stream()
-        self._fork.record(main)
-        self.side.wait_event(self._fork)
-        self.quantize()
-        self.select_channels()
-        self._gathers_overlapped()
+        """The rollout linear on an already-prepared weight: quantize with the
+        fused selection, both second passes, the GEMM (current stream)."""
+        self.quantize_select()
+        self.second_pass()
         self.gemm()
 
     def full_step(self):
-        """Weight preparation and the rollout linear, with the weight
-        preparation (independent of X) on a side stream that forks from and
-        joins back into the current stream, so the two overlap on the GPU;
-        the W_sel gather follows it on the side stream once sel exists, while
-        the residual gather runs on the current stream."""
+        """Weight preparation and the rollout linear.  The weight preparation
+        (independent of X) runs on a side stream that forks from the current
+        stream and joins it before the second passes, which read Q(W)'s
+        source and the weight's column maxima; it overlaps the quantize pass."""
+        main = torch.cuda.current_stream()
+        self._fork.record(main)
+        self.side.wait_event(self._fork)
+        self.prepare_weight(stream=self.side)
+        self._join.record(self.side)
+        self.quantize_select()
+        main.wait_event(self._join)
+        self.second_pass()
+        self.gemm()
+
+    def split_step(self):
+        """The same linear as full_step through the separate calls (quantize,
+        select_channels, the two gathers on two streams, GEMM)."""
         main = torch.cuda.current_stream()
         self._fork.record(main)
         self.side.wait_event(self._fork)
@@ -667,4 +735,4 @@ class RacLinearPlan:
 
     # kernels each call launches (for launch accounting)
     LAUNCHES = dict(prepare_weight=2, quantize=2, quantize_plain=2, select=2, weight_select=1, gemm=1,
-                    reuse_step=5)
+                    reuse_step=5, quantize_select=2, second_pass=1)

@@ -103,7 +103,7 @@ struct QuantWs {
 QuantWs carve_quant(Carver& c, int64_t M, int64_t K, bool scores) {
   QuantWs w{};
   const int64_t tiles = ceil_div(M, kTileRows);
-  w.counters = c.take<unsigned>(K / 64);      // one counter per 64-column strip
+  w.counters = c.take<unsigned>(K / 64 + 1);  // one counter per 64-column strip, then the strips-done count
   w.amax = c.take<unsigned>(amax_parts_count(M, K));   // partial maxima
   if (scores) {
     w.part_sum = c.take<double>(tiles * K);
@@ -234,14 +234,73 @@ nvfp4_status nvfp4_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ldx
   if (amax_or_null == nullptr) {
     n_parts = amax_parts_count(M, K);
     NV_TRY(launch_amax_partial(x, M, K, ldx, 1, 0, w.amax, n_parts, w.counters,
-                               stats ? static_cast<int>(K / 64) : 0, s));
+                               stats ? static_cast<int>(K / 64 + 1) : 0, s));
   } else if (stats) {
-    NV_TRY(cudaMemsetAsync(w.counters, 0, sizeof(unsigned) * (K / 64), s));
+    NV_TRY(cudaMemsetAsync(w.counters, 0, sizeof(unsigned) * (K / 64 + 1), s));
   }
   NV_TRY(launch_quant_score(x, M, K, ldx, g, amax_or_null, w.amax, n_parts, M, qx->codes, qx->scales,
                             qx->scale_layout, qx->tensor_scale, scores ? w.part_sum : nullptr,
                             stats ? w.part_max : nullptr, stats ? w.counters : nullptr, score_or_null,
                             res_colamax_or_null, s));
+  return NVFP4_OK;
+}
+
+nvfp4_status rac_quantize_select(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, const float* amax_or_null,
+                                 nvfp4_tensor* qx, double* score, float* res_colamax, float k_percent, uint8_t* mask,
+                                 int32_t* sel, int64_t* n_sel_out, float* res_tensor_scale, void* ws,
+                                 size_t ws_bytes, void* stream) {
+  NV_CHECK(x && tensor_ok(qx) && score && res_colamax && mask && n_sel_out && res_tensor_scale,
+           NVFP4_ERR_INVALID_ARG);
+  NV_CHECK(k_percent >= 0.0f && k_percent <= 100.0f, NVFP4_ERR_INVALID_ARG);
+  NV_CHECK(M >= 1 && K >= 64 && K % 64 == 0 && ldx >= K && qx->rows == M && qx->cols == K,
+           NVFP4_ERR_UNSUPPORTED_SHAPE);
+  NV_CHECK(aligned16(x) && ldx % 8 == 0, NVFP4_ERR_MISALIGNED);
+  const int64_t n_sel = nvfp4_rac_nsel(k_percent, K);
+  NV_CHECK(n_sel == 0 || sel, NVFP4_ERR_INVALID_ARG);
+  Carver c(ws);
+  const QuantWs w = carve_quant(c, M, K, true);
+  NV_CHECK(ws != nullptr && ws_bytes >= c.off, NVFP4_ERR_WORKSPACE);
+  const nvfp4_status d = device_ok();
+  if (d != NVFP4_OK) return d;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int n_parts = 0;
+  if (amax_or_null == nullptr) {
+    n_parts = amax_parts_count(M, K);
+    NV_TRY(launch_amax_partial(x, M, K, ldx, 1, 0, w.amax, n_parts, w.counters, static_cast<int>(K / 64 + 1), s));
+  } else {
+    NV_TRY(cudaMemsetAsync(w.counters, 0, sizeof(unsigned) * (K / 64 + 1), s));
+  }
+  const FusedSelect fs{n_sel, mask, sel, res_tensor_scale, w.counters + K / 64};
+  *n_sel_out = n_sel;
+  NV_TRY(launch_quant_score(x, M, K, ldx, dense_groups(M), amax_or_null, w.amax, n_parts, M, qx->codes, qx->scales,
+                            qx->scale_layout, qx->tensor_scale, w.part_sum, w.part_max, w.counters, score,
+                            res_colamax, s, &fs));
+  return NVFP4_OK;
+}
+
+nvfp4_status rac_second_pass(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, const nvfp4_tensor* qx,
+                             const int32_t* sel, int64_t n_sel, nvfp4_tensor* q_res, const uint16_t* w, int64_t N,
+                             int64_t ldw, const nvfp4_tensor* qw, const float* w_colamax, nvfp4_tensor* q_wsel,
+                             void* stream) {
+  NV_CHECK(x && tensor_ok(qx) && sel && tensor_ok(q_res) && tensor_ok(q_wsel) && w_colamax, NVFP4_ERR_INVALID_ARG);
+  NV_CHECK(w != nullptr || tensor_ok(qw), NVFP4_ERR_INVALID_ARG);
+  const int64_t width = nvfp4_rac_width(n_sel);
+  NV_CHECK(M >= 1 && K >= 64 && K % 64 == 0 && ldx >= K && qx->rows == M && qx->cols == K && n_sel >= 1 &&
+               n_sel <= K && q_res->rows == M && q_res->cols == width && N >= 1 && q_wsel->rows == N &&
+               q_wsel->cols == width && (w == nullptr ? (qw->rows == N && qw->cols == K) : ldw >= K),
+           NVFP4_ERR_UNSUPPORTED_SHAPE);
+  NV_CHECK(aligned16(x) && ldx % 8 == 0 && (w == nullptr || (aligned16(w) && ldw % 8 == 0)), NVFP4_ERR_MISALIGNED);
+  const nvfp4_status d = device_ok();
+  if (d != NVFP4_OK) return d;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (q_wsel->scale_layout == 1 && N % 128 != 0)
+    NV_TRY(cudaMemsetAsync(q_wsel->scales, 0, scale_bytes(N, width, 1), s));
+  NV_TRY(launch_second_pass(x, M, K, ldx, qx->codes, qx->scales, qx->scale_layout, qx->tensor_scale, sel, n_sel,
+                            width, q_res->tensor_scale, q_res->codes, q_res->scales, q_res->scale_layout, w, N,
+                            w != nullptr ? ldw : K, w == nullptr ? qw->codes : nullptr,
+                            w == nullptr ? qw->scales : nullptr, w == nullptr ? qw->scale_layout : 0,
+                            w == nullptr ? qw->tensor_scale : nullptr, w_colamax, q_wsel->tensor_scale,
+                            q_wsel->codes, q_wsel->scales, q_wsel->scale_layout, s));
   return NVFP4_OK;
 }
 

@@ -109,13 +109,25 @@ cudaError_t launch_amax_partial(const uint16_t* x, int64_t rows, int64_t K, int6
                                 int64_t mat_stride, unsigned* parts, int n_parts, unsigned* zero_ptr,
                                 int n_zero, cudaStream_t s);
 
+// The top-k% selection fused into the quantize pass (dense, with scores and
+// strip counters): mask [K], sel [n_sel], residual tensor scale s_t; the
+// counter strips_done must be zero on entry and is left zero.
+struct FusedSelect {
+  int64_t n_sel;
+  uint8_t* mask;
+  int32_t* sel;
+  float* s_t;
+  unsigned* strips_done;
+};
+
 // amax: fp32 per group, or (n_parts > 0) the max of amax_parts[0 .. n_parts).
 cudaError_t launch_quant_score(const uint16_t* x, int64_t rows, int64_t K, int64_t ldx,
                                const RowGroups& g, const float* amax, const unsigned* amax_parts,
                                int n_parts, int64_t codes_rows,
                                uint8_t* codes, uint8_t* scales, int layout, float* tensor_scale,
                                double* part_sum, float* part_max, unsigned* strip_count,
-                               double* score, float* colamax, cudaStream_t s);
+                               double* score, float* colamax, cudaStream_t s,
+                               const FusedSelect* fused = nullptr);
 
 // score[e, j] = sum over the group's tiles of part_sum in tile order;
 // colamax[e, j] = max of part_max.  For empty groups (MoE) also writes
@@ -136,6 +148,18 @@ cudaError_t launch_residual_gather(const uint16_t* x, int64_t rows, int64_t K, i
                                    const float* qx_st, const int32_t* sel, int64_t n_sel,
                                    int64_t width, const float* r_st, uint8_t* r_codes,
                                    uint8_t* r_scales, int r_layout, cudaStream_t s);
+
+// Both second passes of a dense RAC linear: Q(dX_sel) into r_* (as
+// launch_residual_gather) and Q(W_sel) into ws_* from bf16 w, or from the
+// NVFP4 weight w_codes / w_scales / w_st when w is null (w_colamax then holds
+// the DQ column maxima).  One launch when the weight side takes the tile
+// gather, two when it takes the row-staged kernel.
+cudaError_t launch_second_pass(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, const uint8_t* qx_codes,
+                               const uint8_t* qx_scales, int qx_layout, const float* qx_st, const int32_t* sel,
+                               int64_t n_sel, int64_t width, const float* r_st, uint8_t* r_codes, uint8_t* r_scales,
+                               int r_layout, const uint16_t* w, int64_t N, int64_t ldw, const uint8_t* w_codes,
+                               const uint8_t* w_scales, int w_layout, const float* w_st, const float* w_colamax,
+                               float* ws_st, uint8_t* ws_codes, uint8_t* ws_scales, int ws_layout, cudaStream_t s);
 
 // s_t[e] = RN(max_{j < n_sel} colamax[e*K + sel[e*n_sel + j]] / 2688).
 cudaError_t launch_sel_tensor_scale(const float* colamax, int64_t K, const int32_t* sel,

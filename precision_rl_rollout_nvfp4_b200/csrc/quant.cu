@@ -14,6 +14,7 @@
 // t^1 and meet through one shfl.xor.  The channel score of the tile's 128 rows
 // is their fp64 sum in row order (see quant_score_kernel).
 #include "kernels.h"
+#include "topk.cuh"
 
 namespace nvfp4 {
 namespace {
@@ -177,6 +178,15 @@ __device__ __forceinline__ float reduce_parts(const unsigned* parts, int n, uint
 // X and the block's scale code with the same operations (so the same values).
 // ---------------------------------------------------------------------------
 constexpr int kSpanExact = 22;
+
+// Optional top-k% selection fused into the quantize pass's tail.
+struct SelectOut {
+  int64_t n_sel;            // < 0: no selection
+  uint8_t* mask;
+  int32_t* sel;
+  float* s_t;               // residual tensor scale
+  unsigned* strips_done;    // zero on entry, left zero
+};
 
 // |dX| of one element x (fp32 value of its bf16) in a block with scale code
 // sb: the scalar form of the quantize pass's arithmetic (block_quotients,
@@ -423,6 +433,8 @@ __device__ __forceinline__ void cp_async16_zfill(uint32_t dst, const void* src, 
                : "memory");
 }
 
+// With sel_out.n_sel >= 0 (dense only) the CTA that completes the last
+// column strip also runs the top-k% selection over the finished scores.
 template <bool SCORES>
 __global__ void __launch_bounds__(kQThreads, 3)
 quant_score2_kernel(const uint16_t* __restrict__ x, int64_t K, int64_t ldx, RowGroups g,
@@ -431,7 +443,7 @@ quant_score2_kernel(const uint16_t* __restrict__ x, int64_t K, int64_t ldx, RowG
                     uint8_t* __restrict__ codes, uint8_t* __restrict__ scales, int layout,
                     float* __restrict__ tensor_scale, double* __restrict__ part_sum,
                     float* __restrict__ part_max, unsigned* __restrict__ strip_count,
-                    double* __restrict__ score, float* __restrict__ colamax) {
+                    double* __restrict__ score, float* __restrict__ colamax, SelectOut sel_out) {
   pdl_wait();
   pdl_launch_dependents();
   constexpr int kGroups = kTileRows / 4;
@@ -647,6 +659,21 @@ quant_score2_kernel(const uint16_t* __restrict__ x, int64_t K, int64_t ldx, RowG
     }
     if (t == 0) *counter = 0;                      // ready for the next call
     __syncthreads();                               // staging buffers free before the next tile
+    if (SCORES && sel_out.n_sel >= 0) {
+      // the last strip to finish selects the channels; its scores were
+      // published like the partials (barrier, then one thread's fence before
+      // the counter moves)
+      if (t == 0) {
+        __threadfence();
+        s_last = atomicAdd(sel_out.strips_done, 1u) == static_cast<unsigned>(n_strips - 1);
+      }
+      __syncthreads();
+      if (s_last) {
+        __threadfence();
+        topk_select(score, colamax, K, sel_out.n_sel, sel_out.mask, sel_out.sel, sel_out.s_t, 0, nullptr, true);
+        if (t == 0) *sel_out.strips_done = 0;
+      }
+    }
   }
   cp_async_wait<0>();
 }
@@ -698,23 +725,59 @@ constexpr int kGThreads = 256;
 //         qx_st[e]); `src` is unused and colamax holds max_n |DQ(Q(W))_nj|.
 constexpr int kGRows = 16, kGCols = 256;
 
+// Arguments of one second-pass gather (see gather_quant_body).
+struct GatherArgs {
+  const uint16_t* src;
+  int64_t K, ld;
+  RowGroups g;
+  int64_t N_per_group;
+  const uint8_t* qx_codes;
+  const uint8_t* qx_scales;
+  int qx_layout;
+  const float* qx_st;
+  const int32_t* sel;
+  int64_t n_sel, width;
+  const float* colamax;
+  int fuse_scale;
+  float* out_st;
+  uint8_t* out_codes;
+  uint8_t* out_scales;
+  int out_layout;
+  int64_t out_rows, grid_rows;
+};
+
+struct GatherSmem {
+  __align__(16) float s_val[kGRows][kGCols + 4];
+  float s_e2m1[16];                                // E2M1 value of every code
+  float s_e4m3[128];                               // E4M3 value of every scale byte
+  float s_wm[kGThreads / 32];
+  ScaleTable T;
+};
+
+// The residual's tiles run from the last rows of X to the first (the
+// quantize pass that precedes them ends on the last rows, which are then
+// still in L2); the weight's in order.
 template <int MODE>
-__global__ void __launch_bounds__(kGThreads)
-gather_quant_kernel(const uint16_t* __restrict__ src, int64_t K, int64_t ld, RowGroups g,
-                    int64_t N_per_group, const uint8_t* __restrict__ qx_codes,
-                    const uint8_t* __restrict__ qx_scales, int qx_layout, const float* __restrict__ qx_st,
-                    const int32_t* __restrict__ sel, int64_t n_sel, int64_t width,
-                    const float* __restrict__ colamax, int fuse_scale, float* __restrict__ out_st,
-                    uint8_t* __restrict__ out_codes, uint8_t* __restrict__ out_scales, int out_layout,
-                    int64_t out_rows, int64_t grid_rows) {
+__device__ __forceinline__ void gather_quant_body(const GatherArgs& A, GatherSmem& sm, int cta, int ncta) {
   constexpr bool RESIDUAL = MODE == 1, FP4 = MODE == 2, CODES = MODE != 0;
-  pdl_wait();
-  pdl_launch_dependents();
-  __shared__ __align__(16) float s_val[kGRows][kGCols + 4];
-  __shared__ float s_e2m1[16];                     // E2M1 value of every code
-  __shared__ float s_e4m3[128];                    // E4M3 value of every scale byte
-  __shared__ float s_wm[kGThreads / 32];
-  __shared__ ScaleTable T;
+  const uint16_t* __restrict__ src = A.src;
+  const int64_t K = A.K, ld = A.ld, N_per_group = A.N_per_group, n_sel = A.n_sel, width = A.width;
+  const RowGroups& g = A.g;
+  const uint8_t* __restrict__ qx_codes = A.qx_codes;
+  const uint8_t* __restrict__ qx_scales = A.qx_scales;
+  const int qx_layout = A.qx_layout, fuse_scale = A.fuse_scale, out_layout = A.out_layout;
+  const float* __restrict__ qx_st = A.qx_st;
+  const int32_t* __restrict__ sel = A.sel;
+  const float* __restrict__ colamax = A.colamax;
+  float* __restrict__ out_st = A.out_st;
+  uint8_t* __restrict__ out_codes = A.out_codes;
+  uint8_t* __restrict__ out_scales = A.out_scales;
+  const int64_t out_rows = A.out_rows, grid_rows = A.grid_rows;
+  float (&s_val)[kGRows][kGCols + 4] = sm.s_val;
+  float* s_e2m1 = sm.s_e2m1;
+  float* s_e4m3 = sm.s_e4m3;
+  float* s_wm = sm.s_wm;
+  ScaleTable& T = sm.T;
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
   if (CODES) {
     if (t < 16) s_e2m1[t] = e2m1_to_f32(static_cast<uint32_t>(t));
@@ -726,8 +789,9 @@ gather_quant_kernel(const uint16_t* __restrict__ src, int64_t K, int64_t ld, Row
   const uint32_t K32 = static_cast<uint32_t>(K);
   const int64_t row_tiles = (grid_rows + kGRows - 1) / kGRows;
   const int64_t col_tiles = (width + kGCols - 1) / kGCols;
-  for (int64_t tile = blockIdx.x; tile < row_tiles * col_tiles; tile += gridDim.x) {
-    const int64_t r0 = (tile / col_tiles) * kGRows, j0 = (tile % col_tiles) * kGCols;
+  for (int64_t tile = cta; tile < row_tiles * col_tiles; tile += ncta) {
+    const int64_t rt = RESIDUAL ? row_tiles - 1 - tile / col_tiles : tile / col_tiles;
+    const int64_t r0 = rt * kGRows, j0 = (tile % col_tiles) * kGCols;
     // rows of this tile belong to one group: 16 divides 128 and N % 16 == 0
     int e;
     int64_t row_base, row_end;     // source row of r0, end of the group's rows
@@ -827,7 +891,7 @@ gather_quant_kernel(const uint16_t* __restrict__ src, int64_t K, int64_t ld, Row
 #pragma unroll
       for (int k = 0; k < kGThreads / 32; ++k) r = fmaxf(r, s_wm[k]);
       fused_st = __fdiv_rn(r, kTensorScaleDiv);
-      if (blockIdx.x == 0 && t == 0) out_st[0] = fused_st;
+      if (cta == 0 && t == 0) out_st[0] = fused_st;
     }
     first = false;
     float st = 0.0f;
@@ -860,6 +924,28 @@ gather_quant_kernel(const uint16_t* __restrict__ src, int64_t K, int64_t ld, Row
       }
     }
   }
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(kGThreads) gather_quant_kernel(GatherArgs A) {
+  pdl_wait();
+  pdl_launch_dependents();
+  __shared__ GatherSmem sm;
+  gather_quant_body<MODE>(A, sm, blockIdx.x, gridDim.x);
+}
+
+// Both second passes of a RAC linear in one launch: CTAs [0, n_res) run the
+// residual's tiles (MODE 1), the others the weight's (MODE 0, or 2 from the
+// NVFP4 weight).
+template <int WMODE>
+__global__ void __launch_bounds__(kGThreads) gather_pair_kernel(GatherArgs R, GatherArgs W, int n_res) {
+  pdl_wait();
+  pdl_launch_dependents();
+  __shared__ GatherSmem sm;
+  if (static_cast<int>(blockIdx.x) < n_res)
+    gather_quant_body<1>(R, sm, blockIdx.x, n_res);
+  else
+    gather_quant_body<WMODE>(W, sm, blockIdx.x - n_res, gridDim.x - n_res);
 }
 
 // s_t[e] = RN(max_{j < n_sel} colamax[e*K + sel[e*n_sel + j]] / 2688), one CTA per group.
@@ -1376,10 +1462,10 @@ cudaError_t launch_quant_score(const uint16_t* x, int64_t rows, int64_t K, int64
                                int n_parts, int64_t codes_rows,
                                uint8_t* codes, uint8_t* scales, int layout, float* tensor_scale,
                                double* part_sum, float* part_max, unsigned* strip_count,
-                               double* score, float* colamax, cudaStream_t s) {
+                               double* score, float* colamax, cudaStream_t s, const FusedSelect* fused) {
   const int64_t tiles = max_tiles(g, rows);
   if (tiles == 0) return cudaSuccess;
-  if (quant_v1()) {
+  if (quant_v1() && fused == nullptr) {
     dim3 grid(static_cast<unsigned>(K / kQCols), static_cast<unsigned>(tiles));
     const cudaError_t le = launch_k(part_sum != nullptr ? quant_score_kernel<true> : quant_score_kernel<false>,
                                     dim3(grid), dim3(kQThreads), 0, s, nullptr, 0,
@@ -1398,10 +1484,12 @@ cudaError_t launch_quant_score(const uint16_t* x, int64_t rows, int64_t K, int64
   }
   const int64_t work = tiles * (K / kQCols);
   const int64_t cap = static_cast<int64_t>(sm_count()) * 3;
+  SelectOut so{-1, nullptr, nullptr, nullptr, nullptr};
+  if (fused != nullptr) so = SelectOut{fused->n_sel, fused->mask, fused->sel, fused->s_t, fused->strips_done};
   const cudaError_t le = launch_k(part_sum != nullptr ? quant_score2_kernel<true> : quant_score2_kernel<false>,
                                   dim3(static_cast<unsigned>(work < cap ? work : cap)), dim3(kQThreads), kDyn, s,
                                   nullptr, 0, x, K, ldx, g, amax, amax_parts, n_parts, codes_rows, codes, scales,
-                                  layout, tensor_scale, part_sum, part_max, strip_count, score, colamax);
+                                  layout, tensor_scale, part_sum, part_max, strip_count, score, colamax, so);
   if (le != cudaSuccess) return le;
   return cudaGetLastError();
 }
@@ -1471,10 +1559,10 @@ cudaError_t launch_residual_gather(const uint16_t* x, int64_t rows, int64_t K, i
   // rows of the scale buffer are padded to 128 for the tiled layout
   const int64_t grid_rows = r_layout == 1 ? (prows + kTileRows - 1) / kTileRows * kTileRows : prows;
   {
-    const cudaError_t le = launch_k(gather_quant_kernel<1>, dim3(gather_grid(grid_rows, width)), dim3(kGThreads), 0, s, nullptr, 0,
-                                   x, K, ldx, g, 0, qx_codes, qx_scales, qx_layout, qx_st, sel, n_sel,
-                                   width, nullptr, 0, const_cast<float*>(r_st), r_codes, r_scales,
-                                   r_layout, prows, grid_rows);
+    const GatherArgs A{x, K, ldx, g, 0, qx_codes, qx_scales, qx_layout, qx_st, sel, n_sel,
+                       width, nullptr, 0, const_cast<float*>(r_st), r_codes, r_scales, r_layout, prows, grid_rows};
+    const cudaError_t le = launch_k(gather_quant_kernel<1>, dim3(gather_grid(grid_rows, width)), dim3(kGThreads), 0, s,
+                                    nullptr, 0, A);
     if (le != cudaSuccess) return le;
   }
   return cudaGetLastError();
@@ -1578,9 +1666,10 @@ cudaError_t launch_weight_gather(const uint16_t* w, int64_t N, int64_t K, int64_
   const int64_t rows = static_cast<int64_t>(E) * N;
   RowGroups none{};
   {
-    const cudaError_t le = launch_k(gather_quant_kernel<0>, dim3(gather_grid(rows, width)), dim3(kGThreads), 0, s, nullptr, 0,
-                                   w, K, ldw, none, N, nullptr, nullptr, 0, nullptr, sel, n_sel, width,
-                                   colamax, fuse, s_t, codes, scales, layout, rows, rows);
+    const GatherArgs A{w, K, ldw, none, N, nullptr, nullptr, 0, nullptr, sel, n_sel, width,
+                       colamax, fuse, s_t, codes, scales, layout, rows, rows};
+    const cudaError_t le = launch_k(gather_quant_kernel<0>, dim3(gather_grid(rows, width)), dim3(kGThreads), 0, s,
+                                    nullptr, 0, A);
     if (le != cudaSuccess) return le;
   }
   return cudaGetLastError();
@@ -1604,9 +1693,10 @@ cudaError_t launch_weight_gather_fp4(const uint8_t* w_codes, const uint8_t* w_sc
                                   dq_colamax, fuse, s_t, codes, scales, layout, s);
   RowGroups none{};
   {
-    const cudaError_t le = launch_k(gather_quant_kernel<2>, dim3(gather_grid(rows, width)), dim3(kGThreads), 0, s, nullptr, 0,
-                                   nullptr, K, K, none, N, w_codes, w_scales, w_layout, w_st, sel, n_sel,
-                                   width, dq_colamax, fuse, s_t, codes, scales, layout, rows, rows);
+    const GatherArgs A{nullptr, K, K, none, N, w_codes, w_scales, w_layout, w_st, sel, n_sel,
+                       width, dq_colamax, fuse, s_t, codes, scales, layout, rows, rows};
+    const cudaError_t le = launch_k(gather_quant_kernel<2>, dim3(gather_grid(rows, width)), dim3(kGThreads), 0, s,
+                                    nullptr, 0, A);
     if (le != cudaSuccess) return le;
   }
   return cudaGetLastError();
@@ -1663,6 +1753,49 @@ cudaError_t launch_encode(const float* in, uint8_t* out, int64_t n, int which, c
 
 cudaError_t launch_wait_probe(uint64_t limit_ns, unsigned* err, cudaStream_t s) {
   wait_probe_kernel<<<1, 32, 0, s>>>(limit_ns, err);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_second_pass(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, const uint8_t* qx_codes,
+                               const uint8_t* qx_scales, int qx_layout, const float* qx_st, const int32_t* sel,
+                               int64_t n_sel, int64_t width, const float* r_st, uint8_t* r_codes, uint8_t* r_scales,
+                               int r_layout, const uint16_t* w, int64_t N, int64_t ldw, const uint8_t* w_codes,
+                               const uint8_t* w_scales, int w_layout, const float* w_st, const float* w_colamax,
+                               float* ws_st, uint8_t* ws_codes, uint8_t* ws_scales, int ws_layout, cudaStream_t s) {
+  if (width == 0) return cudaSuccess;
+  const RowGroups dense{nullptr, nullptr, 1, M};
+  const int64_t grid_rows = r_layout == 1 ? (M + kTileRows - 1) / kTileRows * kTileRows : M;
+  // the weight side takes the row-staged kernel when it pays (see
+  // launch_weight_gather): then the two passes are two launches
+  const WselPlan wp = wsel_plan(N, K, 1, width, w == nullptr);
+  const int64_t passes_w = (N + wp.g.R - 1) / (wp.g.R > 0 ? wp.g.R : 1);
+  const bool rows_kernel = w != nullptr ? (wp.ok && passes_w >= 2 * 4 * static_cast<int64_t>(sm_count())) : wp.ok;
+  if (rows_kernel) {
+    cudaError_t e = launch_residual_gather(x, M, K, ldx, dense, M, qx_codes, qx_scales, qx_layout, qx_st, sel, n_sel,
+                                           width, r_st, r_codes, r_scales, r_layout, s);
+    if (e != cudaSuccess) return e;
+    return w != nullptr ? launch_weight_gather(w, N, K, ldw, 1, sel, n_sel, width, w_colamax, ws_st, ws_codes,
+                                               ws_scales, ws_layout, s)
+                        : launch_weight_gather_fp4(w_codes, w_scales, w_layout, w_st, N, K, 1, sel, n_sel, width,
+                                                   w_colamax, ws_st, ws_codes, ws_scales, ws_layout, s);
+  }
+  const RowGroups none{};
+  const GatherArgs R{x, K, ldx, dense, 0, qx_codes, qx_scales, qx_layout, qx_st, sel, n_sel,
+                     width, nullptr, 0, const_cast<float*>(r_st), r_codes, r_scales, r_layout, M, grid_rows};
+  const GatherArgs W{w, K, ldw, none, N, w_codes, w_scales, w_layout, w_st, sel, n_sel,
+                     width, w_colamax, 1, ws_st, ws_codes, ws_scales, ws_layout, N, N};
+  const int64_t ct = (width + kGCols - 1) / kGCols;
+  const int64_t rt = (grid_rows + kGRows - 1) / kGRows * ct, wt = (N + kGRows - 1) / kGRows * ct;
+  const int64_t cap = 8 * static_cast<int64_t>(sm_count());
+  const int64_t grid = rt + wt < cap ? rt + wt : cap;
+  int64_t n_res = (grid * rt + (rt + wt) / 2) / (rt + wt);
+  n_res = n_res < 1 ? 1 : (n_res > grid - 1 ? grid - 1 : n_res);
+  const cudaError_t le =
+      w != nullptr ? launch_k(gather_pair_kernel<0>, dim3(static_cast<unsigned>(grid)), dim3(kGThreads), 0, s, nullptr,
+                              0, R, W, static_cast<int>(n_res))
+                   : launch_k(gather_pair_kernel<2>, dim3(static_cast<unsigned>(grid)), dim3(kGThreads), 0, s, nullptr,
+                              0, R, W, static_cast<int>(n_res));
+  if (le != cudaSuccess) return le;
   return cudaGetLastError();
 }
 

@@ -16,6 +16,7 @@
 // s_tR = RN(max_{j in sel} colamax_j / 2688).  Keys and colamax sit in shared
 // memory when they fit.
 #include "kernels.h"
+#include "topk.cuh"
 
 namespace nvfp4 {
 namespace {
@@ -23,193 +24,14 @@ namespace {
 constexpr int kSelThreads = 512;
 constexpr int64_t kMaxSmemKeys = 16384;          // 16384 x (8 + 4) bytes = 192 KB
 
-// Exclusive prefix sum of v over the CTA in thread order; `total` receives
-// the CTA-wide sum.  Every thread of the CTA must call it.
-__device__ long long block_excl_scan(long long v, long long& total, long long* wsum) {
-  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
-  const int nw = blockDim.x >> 5;
-  long long incl = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const long long n = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-    if (lane >= o) incl += n;
-  }
-  if (lane == 31) wsum[w] = incl;
-  __syncthreads();
-  if (w == 0) {
-    long long x = lane < nw ? wsum[lane] : 0;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const long long n = __shfl_up_sync(0xFFFFFFFFu, x, o);
-      if (lane >= o) x += n;
-    }
-    if (lane < nw) wsum[lane] = x;                 // inclusive over warps
-  }
-  __syncthreads();
-  const long long before = (w == 0 ? 0 : wsum[w - 1]) + incl - v;
-  total = wsum[nw - 1];
-  __syncthreads();
-  return before;
-}
-
 __global__ void __launch_bounds__(kSelThreads)
 topk_kernel(const double* __restrict__ score, const float* __restrict__ colamax, int64_t K,
             int64_t n_sel, uint8_t* __restrict__ mask, int32_t* __restrict__ sel,
             float* __restrict__ s_t_out, int in_smem) {
   pdl_wait();
   pdl_launch_dependents();
-  const int64_t e = blockIdx.x;
-  const uint64_t* gkeys = reinterpret_cast<const uint64_t*>(score + e * K);
-  const float* gcm = colamax + e * K;
   extern __shared__ uint64_t skeys[];            // [K] keys, then [K] colamax
-  float* scm = reinterpret_cast<float*>(skeys + (in_smem ? K : 0));
-  if (in_smem) {
-    for (int64_t j = threadIdx.x; j < K; j += blockDim.x) {
-      skeys[j] = __ldg(gkeys + j);
-      scm[j] = __ldg(gcm + j);
-    }
-    __syncthreads();
-  }
-  const uint64_t* keys = in_smem ? skeys : gkeys;
-  const float* cm = in_smem ? scm : gcm;
-  uint8_t* mk = mask + e * K;
-  int32_t* sl = sel + e * n_sel;
-  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
-
-  __shared__ unsigned hist[256];
-  __shared__ long long wsum[32];
-  __shared__ unsigned long long s_and, s_or, s_prefix;
-  __shared__ long long s_remaining;
-  __shared__ bool s_ge;
-  __shared__ float s_max[32];
-
-  // After each pass `prefix` holds the leading bits of the n_sel-th largest
-  // key and `remaining` how many keys with that prefix are still to be
-  // taken.  If every key of the chosen bin is taken, the selection is simply
-  // key >= (prefix, zeros) (ge_mode); otherwise, once every bit is fixed, T
-  // is the exact n_sel-th largest key and ties at T go to the lower channels.
-  uint64_t prefix = 0;
-  long long remaining = n_sel;
-  bool ge_mode = n_sel >= K;                     // all selected: key >= 0
-  if (n_sel > 0 && n_sel < K) {
-    if (tid == 0) {
-      s_and = ~0ull;
-      s_or = 0ull;
-    }
-    __syncthreads();
-    uint64_t a = ~0ull, o = 0ull;
-    for (int64_t j = tid; j < K; j += blockDim.x) {
-      const uint64_t k = keys[j];
-      a &= k;
-      o |= k;
-    }
-    const uint32_t ahi = __reduce_and_sync(0xFFFFFFFFu, static_cast<uint32_t>(a >> 32));
-    const uint32_t alo = __reduce_and_sync(0xFFFFFFFFu, static_cast<uint32_t>(a));
-    const uint32_t ohi = __reduce_or_sync(0xFFFFFFFFu, static_cast<uint32_t>(o >> 32));
-    const uint32_t olo = __reduce_or_sync(0xFFFFFFFFu, static_cast<uint32_t>(o));
-    if (lane == 0) {
-      atomicAnd(&s_and, (static_cast<unsigned long long>(ahi) << 32) | alo);
-      atomicOr(&s_or, (static_cast<unsigned long long>(ohi) << 32) | olo);
-    }
-    __syncthreads();
-    const uint64_t diff = s_and ^ s_or;
-    int pos = diff == 0 ? 0 : 64 - __clzll(static_cast<long long>(diff));   // free low bits
-    uint64_t pmask = pos == 64 ? 0ull : ~((1ull << pos) - 1ull);
-    prefix = s_and & pmask;
-    while (pos > 0 && !ge_mode) {
-      const int D = pos < 8 ? pos : 8;
-      const int shift = pos - D;
-      const int nb = 1 << D;
-      if (tid < 256) hist[tid] = 0;
-      __syncthreads();
-      for (int64_t j = tid; j < K; j += blockDim.x) {
-        const uint64_t k = keys[j];
-        if ((k & pmask) == prefix) atomicAdd(&hist[(k >> shift) & static_cast<uint64_t>(nb - 1)], 1u);
-      }
-      __syncthreads();
-      // threads 0..nb-1 own bins nb-1-tid (largest first); an inclusive scan
-      // over them finds the bin that holds the remaining-th largest key
-      unsigned h = 0, incl = 0;
-      if (tid < 256) {
-        h = tid < nb ? hist[nb - 1 - tid] : 0u;
-        incl = h;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-          const unsigned n = __shfl_up_sync(0xFFFFFFFFu, incl, off);
-          if (lane >= off) incl += n;
-        }
-        if (lane == 31) wsum[w] = incl;
-      }
-      __syncthreads();
-      if (tid < nb) {
-        long long before_warp = 0;
-        for (int i = 0; i < w; ++i) before_warp += wsum[i];
-        const long long upto = before_warp + incl;     // inclusive
-        const long long before = upto - h;
-        if (before < remaining && remaining <= upto) {
-          s_prefix = prefix | (static_cast<uint64_t>(nb - 1 - tid) << shift);
-          s_remaining = remaining - before;
-          s_ge = (remaining - before) == static_cast<long long>(h);
-        }
-      }
-      __syncthreads();
-      prefix = s_prefix;
-      remaining = s_remaining;
-      ge_mode = s_ge;
-      pmask |= static_cast<uint64_t>(nb - 1) << shift;
-      pos = shift;
-      __syncthreads();
-    }
-  }
-  const uint64_t T = prefix;
-  const long long need_eq = ge_mode ? 0 : remaining;   // keys == T still to take
-
-  // classification: thread tid owns channels [jb, je)
-  const int64_t per = (K + blockDim.x - 1) / blockDim.x;
-  const int64_t jb = tid * per < K ? tid * per : K;
-  const int64_t je = jb + per < K ? jb + per : K;
-  const bool none = n_sel == 0;
-  long long n_gt = 0, n_eq = 0;
-  if (!none) {
-    for (int64_t j = jb; j < je; ++j) {
-      const uint64_t k = keys[j];
-      if (ge_mode ? k >= T : k > T) ++n_gt;
-      else if (!ge_mode && k == T) ++n_eq;
-    }
-  }
-  long long tot;
-  const long long eq_before = ge_mode || none ? 0 : block_excl_scan(n_eq, tot, wsum);
-  long long take_eq = need_eq - eq_before;
-  take_eq = take_eq < 0 ? 0 : (take_eq > n_eq ? n_eq : take_eq);
-  long long p = block_excl_scan(n_gt + take_eq, tot, wsum);
-  float mx = 0.0f;
-  long long eq_seen = 0;
-  for (int64_t j = jb; j < je; ++j) {
-    bool m = false;
-    if (!none) {
-      const uint64_t k = keys[j];
-      if (ge_mode ? k >= T : k > T) {
-        m = true;
-      } else if (!ge_mode && k == T) {
-        m = eq_seen < take_eq;
-        ++eq_seen;
-      }
-    }
-    mk[j] = m ? 1 : 0;
-    if (m) {
-      if (NV_IDX(p < n_sel)) sl[p] = static_cast<int32_t>(j);
-      ++p;
-      mx = fmaxf(mx, cm[j]);
-    }
-  }
-  mx = __uint_as_float(__reduce_max_sync(0xFFFFFFFFu, __float_as_uint(mx)));
-  if (lane == 0) s_max[w] = mx;
-  __syncthreads();
-  if (tid == 0) {
-    float r = 0.0f;
-    for (int i = 0; i < static_cast<int>(blockDim.x >> 5); ++i) r = fmaxf(r, s_max[i]);
-    s_t_out[e] = __fdiv_rn(r, kTensorScaleDiv);
-  }
+  topk_select(score, colamax, K, n_sel, mask, sel, s_t_out, blockIdx.x, in_smem ? skeys : nullptr, false);
 }
 
 }  // namespace
