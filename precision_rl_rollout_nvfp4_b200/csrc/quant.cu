@@ -670,7 +670,10 @@ quant_score2_kernel(const uint16_t* __restrict__ x, int64_t K, int64_t ldx, RowG
       __syncthreads();
       if (s_last) {
         __threadfence();
-        topk_select(score, colamax, K, sel_out.n_sel, sel_out.mask, sel_out.sel, sel_out.s_t, 0, nullptr, true);
+        // keys in the (now idle) tile buffers when they fit, column maxima from L2
+        const bool fit = K * static_cast<int64_t>(sizeof(uint64_t)) <= 2 * kTileRows * kQCols * 2;
+        topk_select(score, colamax, K, sel_out.n_sel, sel_out.mask, sel_out.sel, sel_out.s_t, 0,
+                    fit ? reinterpret_cast<uint64_t*>(q2_dyn) : nullptr, true, false);
         if (t == 0) *sel_out.strips_done = 0;
       }
     }

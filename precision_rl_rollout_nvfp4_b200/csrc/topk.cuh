@@ -49,27 +49,28 @@ static __device__ __forceinline__ long long block_excl_scan(long long v, long lo
   return before;
 }
 
-// Selection of group e over K keys.  skeys: shared memory for K keys and K
-// column maxima, or null to read them from global memory.  coherent: the
-// scores were written by the same kernel (read through L2, not the read-only
-// path).  Every thread of the CTA calls it.
+// Selection of group e over K keys.  skeys: shared memory for K keys (and,
+// with cm_too, K column maxima after them), or null to read them from global
+// memory.  coherent: the scores were written by the same kernel (read through
+// L2, not the read-only path).  Every thread of the CTA calls it.
 static __device__ __noinline__ void topk_select(const double* __restrict__ score, const float* __restrict__ colamax,
                                          int64_t K, int64_t n_sel, uint8_t* __restrict__ mask,
                                          int32_t* __restrict__ sel, float* __restrict__ s_t_out, int64_t e,
-                                         uint64_t* skeys, bool coherent) {
+                                         uint64_t* skeys, bool coherent, bool cm_too = true) {
   const uint64_t* gkeys = reinterpret_cast<const uint64_t*>(score + e * K);
   const float* gcm = colamax + e * K;
   const bool in_smem = skeys != nullptr;
+  const bool cm_smem = in_smem && cm_too;
   float* scm = reinterpret_cast<float*>(skeys + (in_smem ? K : 0));
   if (in_smem) {
     for (int64_t j = threadIdx.x; j < K; j += blockDim.x) {
       skeys[j] = coherent ? __ldcg(gkeys + j) : __ldg(gkeys + j);
-      scm[j] = coherent ? __ldcg(gcm + j) : __ldg(gcm + j);
+      if (cm_smem) scm[j] = coherent ? __ldcg(gcm + j) : __ldg(gcm + j);
     }
     __syncthreads();
   }
   const uint64_t* keys = in_smem ? skeys : gkeys;
-  const float* cm = in_smem ? scm : gcm;
+  const float* cm = cm_smem ? scm : gcm;
   uint8_t* mk = mask + e * K;
   int32_t* sl = sel + e * n_sel;
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
@@ -120,6 +121,7 @@ static __device__ __noinline__ void topk_select(const double* __restrict__ score
       const int nb = 1 << D;
       if (tid < 256) hist[tid] = 0;
       __syncthreads();
+#pragma unroll 8
       for (int64_t j = tid; j < K; j += blockDim.x) {
         const uint64_t k = in_smem ? keys[j] : __ldcg(keys + j);
         if ((k & pmask) == prefix) atomicAdd(&hist[(k >> shift) & static_cast<uint64_t>(nb - 1)], 1u);
@@ -197,7 +199,7 @@ static __device__ __noinline__ void topk_select(const double* __restrict__ score
     if (m) {
       if (NV_IDX(p < n_sel)) sl[p] = static_cast<int32_t>(j);
       ++p;
-      mx = fmaxf(mx, in_smem ? cm[j] : __ldcg(cm + j));
+      mx = fmaxf(mx, cm_smem ? cm[j] : __ldcg(cm + j));
     }
   }
   mx = __uint_as_float(__reduce_max_sync(0xFFFFFFFFu, __float_as_uint(mx)));
