@@ -12,7 +12,7 @@
 // tile.  Thread t handles 8 consecutive columns (one 16-byte load) of 4
 // consecutive rows; the two halves of a 16-element block sit in threads t and
 // t^1 and meet through one shfl.xor.  The channel score of the tile's 128 rows
-// is their fp64 sum in row order (see quant_score_kernel).
+// is their fp64 sum in row order (see quant_score2_kernel).
 #include "kernels.h"
 #include "topk.cuh"
 
@@ -208,212 +208,8 @@ __device__ __noinline__ float residual_abs_one(float xv, uint32_t sb, const Scal
   return fabsf(__fsub_rn(xv, __fmul_rn(p, T.s_t)));
 }
 
-// (4 CTAs per SM: measured faster than 3 with more registers)
-// SCORES: also the fp64 channel sums; without it the kernel writes the codes
-// alone (part_max == nullptr) or the codes and the residual column maxima.
-template <bool SCORES>
-__global__ void __launch_bounds__(kQThreads, 4)
-quant_score_kernel(const uint16_t* __restrict__ x, int64_t K, int64_t ldx, RowGroups g,
-                   const float* __restrict__ amax, const unsigned* __restrict__ amax_parts,
-                   int n_parts, int64_t codes_rows,
-                   uint8_t* __restrict__ codes, uint8_t* __restrict__ scales, int layout,
-                   float* __restrict__ tensor_scale, double* __restrict__ part_sum,
-                   float* __restrict__ part_max, unsigned* __restrict__ strip_count,
-                   double* __restrict__ score, float* __restrict__ colamax) {
-  pdl_wait();
-  pdl_launch_dependents();
-  const int64_t tile = blockIdx.y;
-  const TileInfo ti = tile_info(g, tile);
-  if (!ti.valid) return;
-  constexpr int kGroups = kTileRows / 4;                          // 32 groups of 4 rows
-  __shared__ __align__(16) double gsum[kGroups][kQCols];          // also tail staging
-  __shared__ __align__(16) float gmax[kGroups][kQCols];
-  __shared__ __align__(16) uint32_t gmin[kGroups][kQCols];        // smallest nonzero |dX| bits - 1
-  __shared__ __align__(16) double qsum[4][kQCols];
-  __shared__ __align__(16) float qmax[4][kQCols];
-  __shared__ __align__(16) uint32_t qmin[4][kQCols];
-  __shared__ uint8_t s_sb[kTileRows][kQCols / kBlock];            // block scale codes of the tile
-  __shared__ bool s_last;
-  __shared__ ScaleTable T;
-  const int t = threadIdx.x, cg = t & 7, grp = t >> 3;
-  const int64_t col0 = static_cast<int64_t>(blockIdx.x) * kQCols;
-  const int64_t col = col0 + 8 * cg;
-  uint4 raw[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int64_t row = ti.row0 + 4 * grp + i;
-    raw[i] = row < ti.row_end ? ld_nc_v4(x + row * ldx + col) : make_uint4(0, 0, 0, 0);
-  }
-  __shared__ uint32_t wscratch[kQThreads / 32];
-  const float a = n_parts > 0 ? reduce_parts(amax_parts, n_parts, wscratch) : amax[ti.e];
-  const float s_t = __fdiv_rn(a, kTensorScaleDiv);
-  if (blockIdx.x == 0 && t == 0 && (g.off == nullptr ? tile == 0 : tile == g.tile_start[ti.e]))
-    tensor_scale[ti.e] = s_t;
-  build_scale_table(T, s_t, t);
-  __syncthreads();                               // table ready
-  uint8_t* code_base = codes + tile * kTileRows * (K / 2) + col / 2;
-  double acc[8];
-  float mx[8];
-  uint32_t mn[8];                                // min over nonzero |dX| of (bits - 1)
-#pragma unroll
-  for (int j = 0; j < 8; ++j) { acc[j] = 0.0; mx[j] = 0.0f; mn[j] = 0xFFFFFFFFu; }
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int r = 4 * grp + i;
-    const int64_t prow = tile * kTileRows + r;
-    const uint32_t wv[4] = {raw[i].x, raw[i].y, raw[i].z, raw[i].w};
-    uint64_t x2[4];
-    uint32_t mbits = 0;                            // max |bf16| bits, two lanes
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      x2[j] = bf16x2_to_f2(wv[j]);
-      mbits = __vmaxu2(mbits, wv[j] & 0x7FFF7FFFu);
-    }
-    float am = __uint_as_float(max(mbits & 0xFFFFu, mbits >> 16) << 16);
-    am = fmaxf(am, __shfl_xor_sync(0xFFFFFFFFu, am, 1));
-    const BlockQ bq = block_q(am, T);
-    uint64_t q2[4];
-    block_quotients(x2, bq, q2);
-    const uint32_t packed = e2m1x8_f2(q2);
-    const uint64_t sbv2 = f2_pack(bq.sbv, bq.sbv);
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      // |dX| = |RN(x - RN(p * s_t))| with p = E2M1dec * E4M3dec (exact, both
-      // lanes at once).  The last product and the difference stay scalar:
-      // the packed forms of a product followed by a difference are fused
-      // into one rounding by the code generator, which changes dX.
-      float p0, p1, x0, x1;
-      f2_unpack(f2_mul(e2m1x2_to_f2((packed >> (8 * j)) & 0xFFu), sbv2), p0, p1);
-      f2_unpack(x2[j], x0, x1);
-      const float d0 = fabsf(__fsub_rn(x0, __fmul_rn(p0, s_t)));
-      const float d1 = fabsf(__fsub_rn(x1, __fmul_rn(p1, s_t)));
-      if (SCORES) {
-        acc[2 * j] += static_cast<double>(d0);     // exact whenever the span test passes
-        acc[2 * j + 1] += static_cast<double>(d1);
-        mn[2 * j] = min(mn[2 * j], __float_as_uint(d0) - 1u);       // 0 wraps to ~0: ignored
-        mn[2 * j + 1] = min(mn[2 * j + 1], __float_as_uint(d1) - 1u);
-      }
-      mx[2 * j] = fmaxf(mx[2 * j], d0);
-      mx[2 * j + 1] = fmaxf(mx[2 * j + 1], d1);
-    }
-    if (prow < codes_rows)
-      *reinterpret_cast<uint32_t*>(code_base + static_cast<uint32_t>(r) * static_cast<uint32_t>(K / 2)) = packed;
-    if ((cg & 1) == 0 && (layout == 1 || prow < codes_rows))
-      scales[scale_offset(prow, col / kBlock, K, layout)] = static_cast<uint8_t>(bq.sb);
-    if (SCORES && (cg & 1) == 0) s_sb[r][cg >> 1] = static_cast<uint8_t>(bq.sb);
-  }
-  if (part_max == nullptr) return;
-  // level 1: every thread's 4-row sums, maxima and minima to shared memory
-  if (SCORES) {
-#pragma unroll
-    for (int j = 0; j < 8; j += 2)
-      *reinterpret_cast<double2*>(&gsum[grp][8 * cg + j]) = make_double2(acc[j], acc[j + 1]);
-    *reinterpret_cast<uint4*>(&gmin[grp][8 * cg]) = make_uint4(mn[0], mn[1], mn[2], mn[3]);
-    *reinterpret_cast<uint4*>(&gmin[grp][8 * cg + 4]) = make_uint4(mn[4], mn[5], mn[6], mn[7]);
-  }
-  *reinterpret_cast<float4*>(&gmax[grp][8 * cg]) = make_float4(mx[0], mx[1], mx[2], mx[3]);
-  *reinterpret_cast<float4*>(&gmax[grp][8 * cg + 4]) = make_float4(mx[4], mx[5], mx[6], mx[7]);
-  __syncthreads();
-  // level 2: thread (quarter t/64, column t%64) reduces 8 groups
-  {
-    const int c = t & (kQCols - 1), q4 = t >> 6;
-    double sum = 0.0;
-    float m = 0.0f;
-    uint32_t lo = 0xFFFFFFFFu;
-#pragma unroll
-    for (int gi = 8 * q4; gi < 8 * q4 + 8; ++gi) {
-      if (SCORES) {
-        sum += gsum[gi][c];
-        lo = min(lo, gmin[gi][c]);
-      }
-      m = fmaxf(m, gmax[gi][c]);
-    }
-    if (SCORES) {
-      qsum[q4][c] = sum;
-      qmin[q4][c] = lo;
-    }
-    qmax[q4][c] = m;
-  }
-  __syncthreads();
-  if (t < kQCols) {
-    double part = 0.0;
-    float m = 0.0f;
-    uint32_t lo = 0xFFFFFFFFu;
-#pragma unroll
-    for (int q4 = 0; q4 < 4; ++q4) {
-      if (SCORES) {
-        part += qsum[q4][t];
-        lo = min(lo, qmin[q4][t]);
-      }
-      m = fmaxf(m, qmax[q4][t]);
-    }
-    if (SCORES && lo != 0xFFFFFFFFu) {
-      const int e_hi = static_cast<int>(__float_as_uint(m) >> 23);
-      const int e_lo = max(static_cast<int>((lo + 1u) >> 23), 1);
-      if (e_hi - e_lo > kSpanExact) {
-        // the row-order sum itself, from X and the tile's block scales
-        const uint16_t* xc = x + col0 + t;
-        double chain = 0.0;
-        for (int r = 0; r < kTileRows; ++r) {
-          const int64_t row = ti.row0 + r;
-          if (row >= ti.row_end) break;
-          const float xv = bf16_bits_to_f32(__ldg(xc + row * ldx));
-          chain += static_cast<double>(residual_abs_one(xv, s_sb[r][t >> 4], T));
-        }
-        part = chain;
-      }
-    }
-    if (SCORES) part_sum[tile * K + col0 + t] = part;
-    part_max[tile * K + col0 + t] = m;
-  }
-  if (strip_count == nullptr) return;
-  // The last CTA of this group's column strip sums the group's partials in
-  // tile order (so the result does not depend on which CTA finishes last).
-  // The barrier orders the 64 writers' partials before thread 0's fence, so
-  // the fence publishes them all (cumulativity) before the counter moves.
-  __syncthreads();
-  const int64_t t0 = g.off == nullptr ? 0 : g.tile_start[ti.e];
-  const int64_t t1 = g.off == nullptr ? (g.M + kTileRows - 1) / kTileRows : g.tile_start[ti.e + 1];
-  unsigned* counter = strip_count + static_cast<int64_t>(ti.e) * gridDim.x + blockIdx.x;
-  if (t == 0) {
-    __threadfence();
-    const unsigned prev = atomicAdd(counter, 1u);
-    s_last = prev == static_cast<unsigned>(t1 - t0 - 1);
-  }
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  // stage up to 32 tiles' partials of this strip in shared memory (all 256
-  // threads load), then 64 threads add them in tile order
-  double* ps = &gsum[0][0];                      // [32 tiles][64 cols]
-  float* pm = &gmax[0][0];
-  double total = 0.0;
-  float tmax = 0.0f;
-  for (int64_t c0 = t0; c0 < t1; c0 += kGroups) {
-    const int nt = static_cast<int>(t1 - c0 < kGroups ? t1 - c0 : kGroups);
-    __syncthreads();
-    for (int k = t; k < nt * kQCols; k += kQThreads) {
-      const int tt = k / kQCols, cc = k % kQCols;
-      if (SCORES) ps[k] = __ldcg(part_sum + (c0 + tt) * K + col0 + cc);
-      pm[k] = __ldcg(part_max + (c0 + tt) * K + col0 + cc);
-    }
-    __syncthreads();
-    if (t < kQCols) {
-      for (int tt = 0; tt < nt; ++tt) {          // chunk order
-        if (SCORES) total += ps[tt * kQCols + t];
-        tmax = fmaxf(tmax, pm[tt * kQCols + t]);
-      }
-    }
-  }
-  if (t < kQCols) {
-    if (SCORES) score[static_cast<int64_t>(ti.e) * K + col0 + t] = total;
-    colamax[static_cast<int64_t>(ti.e) * K + col0 + t] = tmax;
-  }
-  if (t == 0) *counter = 0;                      // ready for the next call
-}
-
 // ---------------------------------------------------------------------------
-// Persistent form of the quantize + residual + score pass.  The grid is a few
+// The quantize + residual + score pass (persistent).  The grid is a few
 // CTAs per SM; CTA b takes the (row tile, 64-column strip) pairs b, b + grid,
 // ... in row-tile-major order, so the whole grid sweeps X from its first rows
 // to its last (the amax pass walks X backwards, so the first rows are still
@@ -422,11 +218,8 @@ quant_score_kernel(const uint16_t* __restrict__ x, int64_t K, int64_t ldx, RowGr
 // the current one, so the loads of one tile overlap the arithmetic of the
 // other and need no barrier (every thread reads only its own copies).  The
 // tensor amax, s_t and the block-scale table are formed once per CTA (again
-// only when an MoE row group changes).  Per tile the arithmetic and the
-// score's exact two-level reduction / row-order fallback are those of
-// quant_score_kernel; the block-scale codes the fallback reads are
-// double-buffered by tile parity, because other threads start the next tile
-// while the fallback thread is still summing.
+// only when an MoE row group changes).  The tile's channel score is the exact
+// two-level reduction or the row-order sum described above.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void cp_async16_zfill(uint32_t dst, const void* src, bool valid) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0)
@@ -456,6 +249,8 @@ quant_score2_kernel(const uint16_t* __restrict__ x, int64_t K, int64_t ldx, RowG
   __shared__ __align__(16) float qmax[4][kQCols];
   __shared__ __align__(16) uint32_t qmin[4][kQCols];
   __shared__ uint8_t s_sb[2][kTileRows][kQCols / kBlock];
+  __shared__ float s_dxcol[kTileRows];             // |dX| of one column for the row-order sum
+  __shared__ uint8_t s_wide[kQCols];
   __shared__ uint32_t wscratch[kQThreads / 32];
   __shared__ bool s_last;
   __shared__ ScaleTable T;
@@ -588,6 +383,7 @@ quant_score2_kernel(const uint16_t* __restrict__ x, int64_t K, int64_t ldx, RowG
       qmax[q4][c] = m;
     }
     __syncthreads();
+    int wide = 0;
     if (t < kQCols) {
       double part = 0.0;
       float m = 0.0f;
@@ -603,21 +399,33 @@ quant_score2_kernel(const uint16_t* __restrict__ x, int64_t K, int64_t ldx, RowG
       if (SCORES && lo != 0xFFFFFFFFu) {
         const int e_hi = static_cast<int>(__float_as_uint(m) >> 23);
         const int e_lo = max(static_cast<int>((lo + 1u) >> 23), 1);
-        if (e_hi - e_lo > kSpanExact) {
-          const uint16_t* xc = x + col0 + t;
-          double chain = 0.0;
-          for (int r = 0; r < kTileRows; ++r) {
-            const int64_t row = ti.row0 + r;
-            if (row >= ti.row_end || !NV_IDX(col0 + t < K)) break;
-            const float xv = bf16_bits_to_f32(__ldg(xc + row * ldx));
-            chain += static_cast<double>(residual_abs_one(xv, s_sb[b][r][t >> 4], T));
-          }
-          part = chain;
-        }
+        wide = e_hi - e_lo > kSpanExact;
       }
+      if (SCORES) s_wide[t] = static_cast<uint8_t>(wide);
       if (NV_IDX(tile < row_tiles && col0 + t < K)) {
-        if (SCORES) part_sum[tile * K + col0 + t] = part;
+        if (SCORES && !wide) part_sum[tile * K + col0 + t] = part;
         part_max[tile * K + col0 + t] = m;
+      }
+    }
+    // columns whose values span more than kSpanExact binades: the row-order
+    // sum itself.  The tile is still in this parity's buffer (its next use
+    // is the prefetch two tiles ahead, issued after this point by every
+    // thread), so 128 threads recompute the column's |dX| from it and the
+    // tile's block-scale codes, and one thread adds them in row order.
+    if (SCORES && __syncthreads_or(wide)) {
+      for (int c = 0; c < kQCols; ++c) {
+        if (!s_wide[c]) continue;                  // uniform: every thread reads the same flag
+        if (t < kTileRows) {
+          const float xv = bf16_bits_to_f32(xbuf[b][t][c]);   // rows past the end were zero-filled
+          s_dxcol[t] = residual_abs_one(xv, s_sb[b][t][c >> 4], T);
+        }
+        __syncthreads();
+        if (t == 0) {
+          double chain = 0.0;
+          for (int r = 0; r < kTileRows; ++r) chain += static_cast<double>(s_dxcol[r]);
+          if (NV_IDX(tile < row_tiles && col0 + c < K)) part_sum[tile * K + col0 + c] = chain;
+        }
+        __syncthreads();
       }
     }
     if (strip_count == nullptr) continue;
@@ -1449,17 +1257,6 @@ cudaError_t launch_group_tiles(const int64_t* off, int32_t E, int32_t* tile_star
   return cudaGetLastError();
 }
 
-// NVFP4_QUANT_V1=1 in the environment selects the one-tile-per-CTA form of
-// the quantize pass (kept to compare the two on the same build).
-bool quant_v1() {
-  static int v = -1;
-  if (v < 0) {
-    const char* e = getenv("NVFP4_QUANT_V1");
-    v = (e != nullptr && e[0] == '1') ? 1 : 0;
-  }
-  return v == 1;
-}
-
 cudaError_t launch_quant_score(const uint16_t* x, int64_t rows, int64_t K, int64_t ldx,
                                const RowGroups& g, const float* amax, const unsigned* amax_parts,
                                int n_parts, int64_t codes_rows,
@@ -1468,15 +1265,6 @@ cudaError_t launch_quant_score(const uint16_t* x, int64_t rows, int64_t K, int64
                                double* score, float* colamax, cudaStream_t s, const FusedSelect* fused) {
   const int64_t tiles = max_tiles(g, rows);
   if (tiles == 0) return cudaSuccess;
-  if (quant_v1() && fused == nullptr) {
-    dim3 grid(static_cast<unsigned>(K / kQCols), static_cast<unsigned>(tiles));
-    const cudaError_t le = launch_k(part_sum != nullptr ? quant_score_kernel<true> : quant_score_kernel<false>,
-                                    dim3(grid), dim3(kQThreads), 0, s, nullptr, 0,
-                                   x, K, ldx, g, amax, amax_parts, n_parts, codes_rows, codes, scales,
-                                   layout, tensor_scale, part_sum, part_max, strip_count, score, colamax);
-    if (le != cudaSuccess) return le;
-    return cudaGetLastError();
-  }
   // persistent: a few CTAs per SM over every (row tile, strip) pair
   constexpr int kDyn = 2 * kTileRows * kQCols * 2;
   {
