@@ -35,7 +35,8 @@ def main(argv=None):
                            device=dev).bind(x, w)
     fns = {"prepare_weight": plan.prepare_weight, "quantize": plan.quantize, "select": plan.select,
            "weight_select": plan.weight_select, "gemm": plan.gemm, "gemm_plain": lambda: plan.gemm(plain=True),
-           "quantize_plain": lambda: plan.quantize(scores=False)}
+           "quantize_plain": lambda: plan.quantize(scores=False), "quantize_select": plan.quantize_select,
+           "second_pass": plan.second_pass}
     calls = [c for c in a.calls.split(",") if c]
     # the steps depend on each other: one full pass first
     plan.prepare_weight()
