@@ -483,13 +483,15 @@ cudaError_t prepare_kernel8() {
 // ===========================================================================
 // CTA-pair kernel (tcgen05 cta_group::2), dense activations.
 // ===========================================================================
-template <int YBYTES>
+// FP8 = true: MXFP8 operands (the FP8 comparator): one scale atom per 128
+// rows and K step (4 blocks of 32), four kind::mxf8f6f4 MMAs reading its bytes.
+template <int YBYTES, bool FP8 = false>
 struct Cfg2 {
   static constexpr int STAGES = YBYTES == 2 ? 5 : 4;
   static constexpr int A_ST = 128 * BK_BYTES;          // own 128 rows of A
   static constexpr int B_ST = 128 * BK_BYTES;          // own 128 rows (N half) of B
-  static constexpr int SFA_ST = 4 * SF_ATOM;           // own 128 rows x 4 K blocks
-  static constexpr int SFB_ST = 8 * SF_ATOM;           // all 256 N rows x 4 K blocks
+  static constexpr int SFA_ST = (FP8 ? 1 : 4) * SF_ATOM;   // own 128 rows x 4 K blocks
+  static constexpr int SFB_ST = (FP8 ? 2 : 8) * SF_ATOM;   // all 256 N rows x 4 K blocks
   static constexpr int STAGE = A_ST + B_ST + SFA_ST + SFB_ST;
   static constexpr int STG_STRIDE = 128 * YBYTES + 16; // staging: 128 columns per half tile
   static constexpr int STG_BYTES = 128 * STG_STRIDE;
@@ -506,6 +508,9 @@ constexpr int THREADS2 = 224;
 constexpr uint32_t ACC2_COL = 0, SF2_COL = 256, SF2_STAGE_COLS = 48;
 // kind::mxf4nvf4, M = 256 (pair), N = 256, both K-major, ue4m3 scales.
 constexpr uint32_t IDESC2 = (1u << 7) | (1u << 10) | (uint32_t(256 >> 3) << 17) | (uint32_t(256 >> 4) << 24);
+// kind::mxf8f6f4, M = 256, N = 256: E4M3 x E4M3, UE8M0 scales (bit 23); bits
+// 29-30 / 4-5 pick the byte of the scale word (see IDESC8).
+constexpr uint32_t IDESC2_8 = (1u << 23) | (uint32_t(256 >> 3) << 17) | (uint32_t(256 >> 4) << 24);
 
 struct KParams2 {
   int64_t M, N;
@@ -587,6 +592,14 @@ __device__ __forceinline__ void utccp_sf_pair(uint32_t taddr, uint64_t sdesc) {
   asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" :: "r"(taddr), "l"(sdesc) : "memory");
 }
 
+__device__ __forceinline__ void mma_fp8_pair(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t sfa,
+                                             uint32_t sfb, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+      :: "r"(d), "l"(a), "l"(b), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb) : "memory");
+}
+
 __device__ __forceinline__ void mma_fp4_pair(uint32_t d, uint64_t a, uint64_t b, uint32_t sfa, uint32_t sfb,
                                              uint32_t accumulate) {
   asm volatile(
@@ -619,14 +632,12 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
       : "memory");
 }
 
-template <int YBYTES>
-__global__ void __launch_bounds__(THREADS2, 1)
-w4a4_rac_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
-                          const __grid_constant__ CUtensorMap tmSA0, const __grid_constant__ CUtensorMap tmSB0,
-                          const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
-                          const __grid_constant__ CUtensorMap tmSA1, const __grid_constant__ CUtensorMap tmSB1,
-                          const KParams2 p) {
-  using C = Cfg2<YBYTES>;
+template <int YBYTES, bool FP8>
+__device__ __forceinline__ void gemm2_body(const CUtensorMap& tmA0, const CUtensorMap& tmB0, const CUtensorMap& tmSA0,
+                                           const CUtensorMap& tmSB0, const CUtensorMap& tmA1, const CUtensorMap& tmB1,
+                                           const CUtensorMap& tmSA1, const CUtensorMap& tmSB1, const KParams2& p) {
+  using C = Cfg2<YBYTES, FP8>;
+  constexpr int SF_X = FP8 ? 64 : 256;          // scale-map x extent of one K step (int64 units)
   constexpr int STAGES = C::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -702,8 +713,8 @@ w4a4_rac_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid
             uint8_t* st = sStage + stage * C::STAGE;
             tma_load_2d_pair(smem_u32(st), tA, kt * BK_BYTES, a_row, lead_full);
             tma_load_2d_pair(smem_u32(st + C::A_ST), tB, kt * BK_BYTES, b_row, lead_full);
-            tma_load_2d_pair(smem_u32(st + C::A_ST + C::B_ST), tSA, kt * 256, a_row / 128, lead_full);
-            tma_load_2d_pair(smem_u32(st + C::A_ST + C::B_ST + C::SFA_ST), tSB, kt * 256, b_row0 / 128, lead_full);
+            tma_load_2d_pair(smem_u32(st + C::A_ST + C::B_ST), tSA, kt * SF_X, a_row / 128, lead_full);
+            tma_load_2d_pair(smem_u32(st + C::A_ST + C::B_ST + C::SFA_ST), tSB, kt * SF_X, b_row0 / 128, lead_full);
             armed |= 1u << stage;
             armed_phase = (armed_phase & ~(1u << stage)) | (phase << stage);
             if (++stage == STAGES) { stage = 0; phase ^= 1; }
@@ -742,8 +753,13 @@ w4a4_rac_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
               const uint32_t accum = (seg == 1 && has_res) ? 1u : ((kt > 0 || j > 0) ? 1u : 0u);
-              mma_fp4_pair(tmem + ACC2_COL, desc_sw128(a0 + 32 * j), desc_sw128(b0 + 32 * j),
-                           sfa + 4 * j, sfb + 8 * j, accum);
+              if (FP8)
+                mma_fp8_pair(tmem + ACC2_COL, desc_sw128(a0 + 32 * j), desc_sw128(b0 + 32 * j),
+                             IDESC2_8 | (static_cast<uint32_t>(j) << 29) | (static_cast<uint32_t>(j) << 4), sfa, sfb,
+                             accum);
+              else
+                mma_fp4_pair(tmem + ACC2_COL, desc_sw128(a0 + 32 * j), desc_sw128(b0 + 32 * j),
+                             sfa + 4 * j, sfb + 8 * j, accum);
             }
             umma_commit_pair(&empty[stage]);
             if (++stage == STAGES) { stage = 0; phase ^= 1; }
@@ -779,11 +795,19 @@ w4a4_rac_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid
             tc_fence_after();
             const uint32_t fa = smem_u32(sStage + stage * C::STAGE) + C::A_ST + C::B_ST, fb = fa + C::SFA_ST;
             const uint32_t sfa = tmem + SF2_COL + SF2_STAGE_COLS * stage, sfb = sfa + 16;
+            if (FP8) {
+              // one atom of A, the two 128-row atoms of B; every MMA of the
+              // step reads these columns (its own byte of each word)
+              utccp_sf_pair(sfa, desc_sf(fa));
+              utccp_sf_pair(sfb, desc_sf(fb));
+              utccp_sf_pair(sfb + 4, desc_sf(fb + SF_ATOM));
+            } else {
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              utccp_sf_pair(sfa + 4 * j, desc_sf(fa + j * SF_ATOM));
-              utccp_sf_pair(sfb + 8 * j, desc_sf(fb + j * SF_ATOM));
-              utccp_sf_pair(sfb + 8 * j + 4, desc_sf(fb + 4 * SF_ATOM + j * SF_ATOM));
+              for (int j = 0; j < 4; ++j) {
+                utccp_sf_pair(sfa + 4 * j, desc_sf(fa + j * SF_ATOM));
+                utccp_sf_pair(sfb + 8 * j, desc_sf(fb + j * SF_ATOM));
+                utccp_sf_pair(sfb + 8 * j + 4, desc_sf(fb + 4 * SF_ATOM + j * SF_ATOM));
+              }
             }
             asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];"
                          :: "r"(smem_u32(&sf_ready[stage])) : "memory");
@@ -812,7 +836,7 @@ w4a4_rac_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid
       // applied as RN(acc m) and one power-of-two step (see Pow2Apply).  A
       // zero plain scale means an all-zero X or W, whose residual and W_sel
       // are zero as well: Y = 0.
-      const ScaleProduct ap = scale_product(p.sta[1][pr.e], p.stb[1][pr.e]);
+      const ScaleProduct ap = FP8 ? ScaleProduct{0.5f, 1} : scale_product(p.sta[1][pr.e], p.stb[1][pr.e]);
       const ScaleProduct ar = has_res ? scale_product(p.sta[0][pr.e], p.stb[0][pr.e]) : ScaleProduct{0.0f, 0};
       const float ratio = (ap.m != 0.0f && ar.m != 0.0f) ? ldexpf(__fdiv_rn(ar.m, ap.m), ar.e - ap.e) : 0.0f;
       const float fin = ap.m;
@@ -940,15 +964,37 @@ w4a4_rac_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid
   }
 }
 
+template <int YBYTES>
+__global__ void __launch_bounds__(THREADS2, 1)
+w4a4_rac_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
+                          const __grid_constant__ CUtensorMap tmSA0, const __grid_constant__ CUtensorMap tmSB0,
+                          const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
+                          const __grid_constant__ CUtensorMap tmSA1, const __grid_constant__ CUtensorMap tmSB1,
+                          const KParams2 p) {
+  gemm2_body<YBYTES, false>(tmA0, tmB0, tmSA0, tmSB0, tmA1, tmB1, tmSA1, tmSB1, p);
+}
+
+// MXFP8 x MXFP8 on CTA pairs (the FP8 comparator): one K segment.
+template <int YBYTES>
+__global__ void __launch_bounds__(THREADS2, 1)
+w8a8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
+                      const __grid_constant__ CUtensorMap tmSA0, const __grid_constant__ CUtensorMap tmSB0,
+                      const KParams2 p) {
+  gemm2_body<YBYTES, true>(tmA0, tmB0, tmSA0, tmSB0, tmA0, tmB0, tmSA0, tmSB0, p);
+}
+
 // 2-D map over a tiled scale buffer seen as int64 elements: one row per
 // 128-row block (all its 512-byte atoms), box = 4 atoms x box_rows blocks.
-bool make_scale_map(CUtensorMap* tm, const uint8_t* scales, int64_t rows, int64_t cols, int box_rows) {
+// atom_cols: K elements one atom covers (64 for NVFP4, 128 for MXFP8);
+// box_x: int64 elements of one K step's scales (4 atoms, or 1).
+bool make_scale_map(CUtensorMap* tm, const uint8_t* scales, int64_t rows, int64_t cols, int box_rows,
+                    int64_t atom_cols = 64, uint32_t box_x = 256u) {
   auto fn = encode_fn();
   if (fn == nullptr) return false;
-  const int64_t atoms = (cols + 63) / 64;
+  const int64_t atoms = (cols + atom_cols - 1) / atom_cols;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(atoms * 64), static_cast<cuuint64_t>((rows + 127) / 128)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(atoms * 512)};
-  cuuint32_t box[2] = {256u, static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t box[2] = {box_x, static_cast<cuuint32_t>(box_rows)};
   cuuint32_t estr[2] = {1, 1};
   return fn(tm, CU_TENSOR_MAP_DATA_TYPE_INT64, 2, const_cast<uint8_t*>(scales), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -1074,7 +1120,48 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s) {
   return cudaGetLastError();
 }
 
+template <int YBYTES>
+cudaError_t launch_pair_fp8(const GemmArgs& a, cudaStream_t s) {
+  using C = Cfg2<YBYTES, true>;
+  static bool done[kMaxAttrDevices] = {};
+  {
+    const cudaError_t e = set_max_smem(w8a8_gemm_pair_kernel<YBYTES>, C::SMEM_BYTES, done);
+    if (e != cudaSuccess) return e;
+  }
+  const int64_t K = a.a0.cols;
+  KParams2 p{};
+  p.M = a.M;
+  p.N = a.N;
+  p.g = a.g;
+  p.m_tiles = static_cast<int>((a.M + 255) / 256);
+  p.n_tiles = static_cast<int>((a.N + 255) / 256);
+  p.kt[0] = 0;
+  p.kt[1] = static_cast<int>(K / 128);
+  CUtensorMap maps[4];
+  if (!make_code_map(&maps[0], a.a0.codes, a.a0.rows, K, 128, K) ||
+      !make_code_map(&maps[1], a.b0.codes, a.b0.rows, K, 128, K) ||
+      !make_scale_map(&maps[2], a.a0.scales, a.a0.rows, K, 1, 128, 64u) ||
+      !make_scale_map(&maps[3], a.b0.scales, a.b0.rows, K, 2, 128, 64u))
+    return cudaErrorInvalidValue;
+  p.y = a.y;
+  p.ldy = a.ldy;
+  p.err = a.err;
+  const int tiles = p.m_tiles * p.n_tiles;
+  const int pairs = tiles < sm_count() / 2 ? tiles : sm_count() / 2;
+  if (pairs == 0) return cudaSuccess;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  return launch_k(w8a8_gemm_pair_kernel<YBYTES>, dim3(static_cast<unsigned>(2 * pairs)), dim3(THREADS2),
+                  C::SMEM_BYTES, s, attr, 1, maps[0], maps[1], maps[2], maps[3], p);
+}
+
 cudaError_t launch_gemm_fp8(const GemmArgs& a, cudaStream_t s) {
+  // CTA pairs where their waves pay, as for NVFP4 (NVFP4_GEMM_SINGLE_CTA=1 keeps the single-CTA form)
+  if (dense_pair_pays(a.M, a.N) && !gemm_force_single_cta())
+    return a.y_dtype == 0 ? launch_pair_fp8<4>(a, s) : launch_pair_fp8<2>(a, s);
   cudaError_t e = a.y_dtype == 0 ? prepare_kernel8<4>() : prepare_kernel8<2>();
   if (e != cudaSuccess) return e;
   KParams p{};

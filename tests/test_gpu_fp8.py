@@ -53,6 +53,7 @@ def test_mxfp8_quantize_edges():
 
 
 @pytest.mark.parametrize("M,N,K", [(128, 128, 256), (300, 144, 512), (1, 16, 256), (1024, 2048, 4096),
+                                   (4000, 2000, 512), (2560, 1040, 256),   # CTA-pair kernel, ragged
                                    (256, 11008, 4096)])
 @pytest.mark.parametrize("out", ["f32", "bf16"])
 def test_w8a8_gemm_matches_oracle(M, N, K, out):
