@@ -792,24 +792,56 @@ struct WselGeom {
 // Both halves of an f16 pair = E4M3dec(sb) of one scale byte (sign ignored).
 __device__ __forceinline__ uint32_t dup_e4m3_to_h2(uint32_t sb) { return e4m3x2_to_h2((sb & 0x7Fu) * 0x0101u); }
 
-template <bool FP4>
-__global__ void __launch_bounds__(512, 2)
-wsel_rows_kernel(const uint16_t* __restrict__ w, int64_t ldw, const uint8_t* __restrict__ codes,
-                 const uint8_t* __restrict__ scales, int layout, const float* __restrict__ w_st, int64_t N,
-                 int64_t K, int32_t E, const int32_t* __restrict__ sel, int64_t n_sel, int64_t width,
-                 const float* __restrict__ colamax, int fuse_scale, float* __restrict__ out_st,
-                 uint8_t* __restrict__ out_codes, uint8_t* __restrict__ out_scales, int out_layout,
-                 WselGeom g) {
-  pdl_wait();
-  pdl_launch_dependents();
-  extern __shared__ __align__(16) uint8_t ws_smem[];
-  __shared__ ScaleTable T;
-  __shared__ float s_wm[32];
+// MODE 0: W_sel from bf16 rows w; MODE 1: W_sel from the NVFP4 weight
+// (codes / scales / w_st); MODE 2: the residual dX_sel of dense activations:
+// rows of X (w, stride ldw) and of Q(X) (codes / scales / w_st = its tensor
+// scale) are staged side by side, each gathered element is x - DQ decoded
+// from the staged code nibble and scale byte (the product E2M1 E4M3 exact in
+// f16, then RN(p s_t) and RN(x - dq) in fp32, as the quantize pass forms dX),
+// and the passes of each CTA run from its last rows to its first.
+struct RowsArgs {
+  const uint16_t* w;
+  int64_t ldw;
+  const uint8_t* codes;
+  const uint8_t* scales;
+  int layout;
+  const float* w_st;
+  int64_t N, K;
+  int32_t E;
+  const int32_t* sel;
+  int64_t n_sel, width;
+  const float* colamax;
+  int fuse_scale;
+  float* out_st;
+  uint8_t* out_codes;
+  uint8_t* out_scales;
+  int out_layout;
+  WselGeom g;
+};
+
+template <int MODE>
+__device__ __forceinline__ void wsel_rows_body(const RowsArgs& A, uint8_t* ws_smem, ScaleTable& T, float* s_wm,
+                                               int cta, int ncta) {
+  constexpr bool FP4 = MODE == 1, RES = MODE == 2;
+  const uint16_t* __restrict__ w = A.w;
+  const int64_t ldw = A.ldw, N = A.N, K = A.K, n_sel = A.n_sel, width = A.width;
+  const uint8_t* __restrict__ codes = A.codes;
+  const uint8_t* __restrict__ scales = A.scales;
+  const int layout = A.layout, fuse_scale = A.fuse_scale, out_layout = A.out_layout;
+  const float* __restrict__ w_st = A.w_st;
+  const int32_t E = A.E;
+  const int32_t* __restrict__ sel = A.sel;
+  const float* __restrict__ colamax = A.colamax;
+  float* __restrict__ out_st = A.out_st;
+  uint8_t* __restrict__ out_codes = A.out_codes;
+  uint8_t* __restrict__ out_scales = A.out_scales;
+  const WselGeom& g = A.g;
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5, nthr = blockDim.x;
   const uint32_t Ku = static_cast<uint32_t>(K), half = Ku / 2u;
   const int nblk = static_cast<int>(width / kBlock);
   const uint32_t R = static_cast<uint32_t>(g.R);
   // shared memory: [staged rows, 2 buffers (bf16) or 1 (NVFP4)][raw NVFP4 rows, 2 buffers]
+  // (residual: bf16 rows of X, 2 buffers, then the raw Q(X) rows, 2 buffers)
   const uint32_t nbuf_rows = FP4 ? 1u : 2u;
   const uint32_t raw0 = nbuf_rows * R * g.rowbytes;
   // zero the tails (element K onwards) of every staged row once: copies and
@@ -823,19 +855,22 @@ wsel_rows_kernel(const uint16_t* __restrict__ w, int64_t ldw, const uint8_t* __r
   const int ob0 = shared_blocks ? t % nblk : t;
   const int64_t rows = static_cast<int64_t>(E) * N;
   const int64_t passes = (rows + R - 1) / R;
-  const int64_t p0 = static_cast<int64_t>(blockIdx.x) * passes / gridDim.x;
-  const int64_t p1 = static_cast<int64_t>(blockIdx.x + 1) * passes / gridDim.x;
+  const int64_t p0 = static_cast<int64_t>(cta) * passes / ncta;
+  const int64_t p1 = static_cast<int64_t>(cta + 1) * passes / ncta;
+  // the i-th pass of this CTA (the residual walks its range backwards)
+  auto pass_of = [&](int64_t i) { return RES ? p1 - 1 - (i - p0) : i; };
   auto stage = [&](int64_t p, uint32_t b) {
     const int64_t r0 = p * R;
     const uint32_t nrows = static_cast<uint32_t>(rows - r0 < R ? rows - r0 : R);
     for (uint32_t r = 0; r < nrows; ++r) {
-      if (FP4) {
+      if (FP4 || RES) {
         const uint32_t ro = raw0 + (b * R + r) * g.rawbytes;
         const uint8_t* src = codes + (r0 + r) * static_cast<int64_t>(half);
         for (uint32_t q = t; q < half / 16u; q += nthr) cp_async16(ws_smem + ro + 16u * q, src + 16u * q);
         for (uint32_t q = t; q < Ku / 64u; q += nthr)
           cp_async4(ws_smem + ro + half + 4u * q, scales + scale_offset(r0 + r, 4 * q, K, layout));
-      } else {
+      }
+      if (!FP4) {
         const uint32_t ro = (b * R + r) * g.rowbytes;
         const uint16_t* src = w + (r0 + r) * ldw;
         for (uint32_t q = t; q < Ku / 8u; q += nthr) cp_async16(ws_smem + ro + 16u * q, src + 8u * q);
@@ -857,12 +892,13 @@ wsel_rows_kernel(const uint16_t* __restrict__ w, int64_t ldw, const uint8_t* __r
   uint32_t cidx[16];
 #pragma unroll
   for (int u = 0; u < 16; ++u) cidx[u] = Ku;
-  if (p0 < p1) stage(p0, 0u);
+  if (p0 < p1) stage(pass_of(p0), 0u);
   int cur_e = -1;
   float st_w = 0.0f;
-  for (int64_t p = p0; p < p1; ++p) {
-    const uint32_t b = static_cast<uint32_t>((p - p0) & 1);
-    if (p + 1 < p1) stage(p + 1, b ^ 1u);
+  for (int64_t pi = p0; pi < p1; ++pi) {
+    const int64_t p = pass_of(pi);
+    const uint32_t b = static_cast<uint32_t>((pi - p0) & 1);
+    if (pi + 1 < p1) stage(pass_of(pi + 1), b ^ 1u);
     const int64_t r0 = p * R;
     const int e = static_cast<int>(r0 / N);
     const uint32_t nrows = static_cast<uint32_t>(rows - r0 < R ? rows - r0 : R);
@@ -885,16 +921,16 @@ wsel_rows_kernel(const uint16_t* __restrict__ w, int64_t ldw, const uint8_t* __r
         float r = 0.0f;
         for (int k = 0; k < (nthr >> 5); ++k) r = fmaxf(r, s_wm[k]);
         st = __fdiv_rn(r, kTensorScaleDiv);
-        if (blockIdx.x == 0 && t == 0) out_st[0] = st;
+        if (cta == 0 && t == 0) out_st[0] = st;
       } else {
         st = out_st[e];
       }
       __syncthreads();                             // the previous matrix's table is no longer read
       build_scale_table(T, st, t);
-      if (FP4) st_w = w_st[e];
+      if (FP4 || RES) st_w = w_st[e];
       cur_e = e;
     }
-    if (p + 1 < p1) {
+    if (pi + 1 < p1) {
       cp_async_wait<1>();                          // this thread's copies of pass p are done
     } else {
       cp_async_wait<0>();
@@ -929,16 +965,29 @@ wsel_rows_kernel(const uint16_t* __restrict__ w, int64_t ldw, const uint8_t* __r
           const uint32_t slot = static_cast<uint32_t>(phase + g.P * k);
           if (slot >= nrows) break;
           const uint8_t* rb = ws_smem + rows0 + slot * g.rowbytes;
+          const uint8_t* raw = ws_smem + raw0 + (b * R + slot) * g.rawbytes;
           float v[16];
           float am = 0.0f;
 #pragma unroll
           for (int u = 0; u < 16; ++u) {
             const uint32_t h = *reinterpret_cast<const uint16_t*>(rb + 2u * cidx[u]);
             float x;
-            if (FP4)
+            if (FP4) {
               x = __fmul_rn(__half2float(__ushort_as_half(static_cast<unsigned short>(h))), st_w);
-            else
+            } else if (RES) {
+              // padded channels read element K of the x row (zero) and a code
+              // and scale past the row's data; their product is discarded
+              const uint32_t c = cidx[u];
+              const bool real = c < Ku;
+              const uint32_t cb = real ? raw[c >> 1] : 0u;
+              const uint32_t sb = real ? raw[half + (c >> 4)] : 0u;
+              const uint32_t pr = h2_mul(e2m1x2_to_h2(cb), dup_e4m3_to_h2(sb));
+              const uint32_t ph = (c & 1u) ? (pr >> 16) : (pr & 0xFFFFu);
+              const float dq = __fmul_rn(__half2float(__ushort_as_half(static_cast<unsigned short>(ph))), st_w);
+              x = __fsub_rn(__uint_as_float(h << 16), dq);
+            } else {
               x = __uint_as_float(h << 16);
+            }
             v[u] = x;
             am = fmaxf(am, fabsf(x));
           }
@@ -955,6 +1004,32 @@ wsel_rows_kernel(const uint16_t* __restrict__ w, int64_t ldw, const uint8_t* __r
     }
     __syncthreads();                               // staged rows and buffer b are free again
   }
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(512, 2) wsel_rows_kernel(RowsArgs A) {
+  pdl_wait();
+  pdl_launch_dependents();
+  extern __shared__ __align__(16) uint8_t ws_smem[];
+  __shared__ ScaleTable T;
+  __shared__ float s_wm[32];
+  wsel_rows_body<MODE>(A, ws_smem, T, s_wm, blockIdx.x, gridDim.x);
+}
+
+// Both second passes of a dense RAC linear, row-staged, in one launch: CTAs
+// [0, n_res) run the residual (MODE 2), the others W_sel (WMODE 0 from the
+// bf16 weight, 1 from the NVFP4 weight).
+template <int WMODE>
+__global__ void __launch_bounds__(512, 2) rows_pair_kernel(RowsArgs Rr, RowsArgs Wr, int n_res) {
+  pdl_wait();
+  pdl_launch_dependents();
+  extern __shared__ __align__(16) uint8_t ws_smem[];
+  __shared__ ScaleTable T;
+  __shared__ float s_wm[32];
+  if (static_cast<int>(blockIdx.x) < n_res)
+    wsel_rows_body<2>(Rr, ws_smem, T, s_wm, blockIdx.x, n_res);
+  else
+    wsel_rows_body<WMODE>(Wr, ws_smem, T, s_wm, blockIdx.x - n_res, gridDim.x - n_res);
 }
 
 // Column maxima of |DQ(Q(W))| for `batch` stacked NVFP4 matrices of N rows
@@ -1379,9 +1454,13 @@ struct WselPlan {
   size_t smem;
   bool ok;
 };
-WselPlan wsel_plan(int64_t N, int64_t K, int32_t E, int64_t width, bool fp4) {
-  // at most 54 KB of rows keeps four CTAs (the register limit) on an SM
-  constexpr size_t kBudget = 54 * 1024, kMax = 200 * 1024;
+// mode 0: bf16 weight rows; 1: NVFP4 weight rows; 2: the residual (bf16 X
+// rows and raw Q(X) rows, both double-buffered).
+WselPlan wsel_plan(int64_t N, int64_t K, int32_t E, int64_t width, int mode) {
+  const bool fp4 = mode == 1;
+  // at most 54 KB of rows keeps four CTAs (the register limit) on an SM; the
+  // residual's rows are larger: up to 110 KB (two CTAs of 256 threads)
+  const size_t kBudget = mode == 2 ? 110 * 1024 : 54 * 1024, kMax = 200 * 1024;
   WselPlan w{};
   const int64_t nblk = width / kBlock;
   w.threads = nblk <= 256 ? 256 : static_cast<int>(nblk < 512 ? (nblk + 31) / 32 * 32 : 512);
@@ -1392,6 +1471,7 @@ WselPlan wsel_plan(int64_t N, int64_t K, int32_t E, int64_t width, bool fp4) {
   w.g.rowbytes = static_cast<uint32_t>(2 * K + 16);
   w.g.rawbytes = static_cast<uint32_t>((K / 2 + K / kBlock + 15) / 16 * 16);
   auto bytes = [&](int r) {
+    if (mode == 2) return static_cast<size_t>(2 * r) * (w.g.rowbytes + w.g.rawbytes);
     return fp4 ? static_cast<size_t>(r) * (w.g.rowbytes + 2 * w.g.rawbytes)
                : static_cast<size_t>(2 * r) * w.g.rowbytes;
   };
@@ -1409,7 +1489,7 @@ WselPlan wsel_plan(int64_t N, int64_t K, int32_t E, int64_t width, bool fp4) {
   return w;
 }
 
-template <bool FP4>
+template <int MODE>
 cudaError_t launch_wsel_rows(const WselPlan& wp, const uint16_t* w, int64_t ldw, const uint8_t* w_codes,
                              const uint8_t* w_scales, int w_layout, const float* w_st, int64_t N, int64_t K,
                              int32_t E, const int32_t* sel, int64_t n_sel, int64_t width,
@@ -1417,20 +1497,20 @@ cudaError_t launch_wsel_rows(const WselPlan& wp, const uint16_t* w, int64_t ldw,
                              int layout, cudaStream_t s) {
   static bool done[kMaxAttrDevices] = {};
   {
-    const cudaError_t ae = set_max_smem(wsel_rows_kernel<FP4>, 200 * 1024, done);
+    const cudaError_t ae = set_max_smem(wsel_rows_kernel<MODE>, 200 * 1024, done);
     if (ae != cudaSuccess) return ae;
   }
   int per_sm = 0;
   const cudaError_t oe =
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, wsel_rows_kernel<FP4>, wp.threads, wp.smem);
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, wsel_rows_kernel<MODE>, wp.threads, wp.smem);
   if (oe != cudaSuccess) return oe;
   const int64_t rows = static_cast<int64_t>(E) * N;
   const int64_t passes = (rows + wp.g.R - 1) / wp.g.R;
   const int64_t cap = static_cast<int64_t>(sm_count()) * (per_sm > 0 ? per_sm : 1);
   const unsigned grid = static_cast<unsigned>(passes < cap ? passes : cap);
-  const cudaError_t le = launch_k(wsel_rows_kernel<FP4>, dim3(grid), dim3(wp.threads), wp.smem, s, nullptr, 0,
-                                  w, ldw, w_codes, w_scales, w_layout, w_st, N, K, E, sel, n_sel, width, colamax,
-                                  fuse, s_t, codes, scales, layout, wp.g);
+  const RowsArgs A{w, ldw, w_codes, w_scales, w_layout, w_st, N, K, E, sel, n_sel, width, colamax,
+                   fuse, s_t, codes, scales, layout, wp.g};
+  const cudaError_t le = launch_k(wsel_rows_kernel<MODE>, dim3(grid), dim3(wp.threads), wp.smem, s, nullptr, 0, A);
   if (le != cudaSuccess) return le;
   return cudaGetLastError();
 }
@@ -1449,10 +1529,10 @@ cudaError_t launch_weight_gather(const uint16_t* w, int64_t N, int64_t K, int64_
   // the row-staged kernel pays off once every CTA runs several passes; a
   // weight with fewer rows than about two passes per resident CTA takes the
   // tile gather (its fixed cost per CTA is lower)
-  const WselPlan ws = wsel_plan(N, K, E, width, false);
+  const WselPlan ws = wsel_plan(N, K, E, width, 0);
   const int64_t passes_w = (static_cast<int64_t>(E) * N + ws.g.R - 1) / (ws.g.R > 0 ? ws.g.R : 1);
   if (ws.ok && passes_w >= 2 * 4 * static_cast<int64_t>(sm_count()))
-    return launch_wsel_rows<false>(ws, w, ldw, nullptr, nullptr, 0, nullptr, N, K, E, sel, n_sel, width, colamax,
+    return launch_wsel_rows<0>(ws, w, ldw, nullptr, nullptr, 0, nullptr, N, K, E, sel, n_sel, width, colamax,
                                    fuse, s_t, codes, scales, layout, s);
   const int64_t rows = static_cast<int64_t>(E) * N;
   RowGroups none{};
@@ -1478,9 +1558,9 @@ cudaError_t launch_weight_gather_fp4(const uint8_t* w_codes, const uint8_t* w_sc
     if (e != cudaSuccess) return e;
   }
   const int64_t rows = static_cast<int64_t>(E) * N;
-  const WselPlan ws = wsel_plan(N, K, E, width, true);
+  const WselPlan ws = wsel_plan(N, K, E, width, 1);
   if (ws.ok)
-    return launch_wsel_rows<true>(ws, nullptr, 0, w_codes, w_scales, w_layout, w_st, N, K, E, sel, n_sel, width,
+    return launch_wsel_rows<1>(ws, nullptr, 0, w_codes, w_scales, w_layout, w_st, N, K, E, sel, n_sel, width,
                                   dq_colamax, fuse, s_t, codes, scales, layout, s);
   RowGroups none{};
   {
@@ -1556,11 +1636,56 @@ cudaError_t launch_second_pass(const uint16_t* x, int64_t M, int64_t K, int64_t 
   if (width == 0) return cudaSuccess;
   const RowGroups dense{nullptr, nullptr, 1, M};
   const int64_t grid_rows = r_layout == 1 ? (M + kTileRows - 1) / kTileRows * kTileRows : M;
+  const int wmode = w != nullptr ? 0 : 1;
+  const int64_t sms = sm_count();
+  // large activations: the residual row-staged (whole rows of X and Q(X)
+  // read once, coalesced); with it the weight row-staged in the same launch
+  const WselPlan rp = wsel_plan(M, K, 1, width, 2);
+  const WselPlan wq = wsel_plan(N, K, 1, width, wmode);
+  const int64_t passes_r = (M + rp.g.R - 1) / (rp.g.R > 0 ? rp.g.R : 1);
+  const int64_t passes_w = (N + wq.g.R - 1) / (wq.g.R > 0 ? wq.g.R : 1);
+  // (the row-staged residual writes real rows only: with a tiled layout the
+  // padding rows of the scale buffer would stay unwritten unless M % 128 == 0)
+  if (rp.ok && wq.ok && rp.threads == wq.threads && passes_r >= 2 * sms &&
+      (r_layout == 0 || M % kTileRows == 0)) {
+    const size_t smem = rp.smem > wq.smem ? rp.smem : wq.smem;
+    static bool done0[kMaxAttrDevices] = {}, done1[kMaxAttrDevices] = {};
+    {
+      const cudaError_t ae = wmode == 0 ? set_max_smem(rows_pair_kernel<0>, 200 * 1024, done0)
+                                        : set_max_smem(rows_pair_kernel<1>, 200 * 1024, done1);
+      if (ae != cudaSuccess) return ae;
+    }
+    int per_sm = 0;
+    const cudaError_t oe = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+        &per_sm, wmode == 0 ? rows_pair_kernel<0> : rows_pair_kernel<1>, rp.threads, smem);
+    if (oe != cudaSuccess) return oe;
+    const int64_t total = sms * (per_sm > 0 ? per_sm : 1);
+    // CTAs in proportion to the bytes each side reads
+    const double rb = static_cast<double>(M) * 2.5625 * K;
+    const double wb = static_cast<double>(N) * (wmode == 0 ? 2.0 : 0.5625) * K;
+    int64_t n_res = static_cast<int64_t>(static_cast<double>(total) * rb / (rb + wb) + 0.5);
+    n_res = n_res < 1 ? 1 : (n_res > total - 1 ? total - 1 : n_res);
+    if (n_res > passes_r) n_res = passes_r;
+    int64_t n_w = total - n_res;
+    if (n_w > passes_w) n_w = passes_w;
+    if (n_w < 1) n_w = 1;
+    const RowsArgs Rr{x, ldx, qx_codes, qx_scales, qx_layout, qx_st, M, K, 1, sel, n_sel, width, nullptr, 0,
+                      const_cast<float*>(r_st), r_codes, r_scales, r_layout, rp.g};
+    const RowsArgs Wr{w, ldw, w_codes, w_scales, w_layout, w_st, N, K, 1, sel, n_sel, width, w_colamax, 1,
+                      ws_st, ws_codes, ws_scales, ws_layout, wq.g};
+    const cudaError_t le =
+        wmode == 0 ? launch_k(rows_pair_kernel<0>, dim3(static_cast<unsigned>(n_res + n_w)), dim3(rp.threads), smem, s,
+                              nullptr, 0, Rr, Wr, static_cast<int>(n_res))
+                   : launch_k(rows_pair_kernel<1>, dim3(static_cast<unsigned>(n_res + n_w)), dim3(rp.threads), smem, s,
+                              nullptr, 0, Rr, Wr, static_cast<int>(n_res));
+    if (le != cudaSuccess) return le;
+    return cudaGetLastError();
+  }
   // the weight side takes the row-staged kernel when it pays (see
   // launch_weight_gather): then the two passes are two launches
-  const WselPlan wp = wsel_plan(N, K, 1, width, w == nullptr);
-  const int64_t passes_w = (N + wp.g.R - 1) / (wp.g.R > 0 ? wp.g.R : 1);
-  const bool rows_kernel = w != nullptr ? (wp.ok && passes_w >= 2 * 4 * static_cast<int64_t>(sm_count())) : wp.ok;
+  const WselPlan wp = wsel_plan(N, K, 1, width, wmode);
+  const int64_t passes_wt = (N + wp.g.R - 1) / (wp.g.R > 0 ? wp.g.R : 1);
+  const bool rows_kernel = w != nullptr ? (wp.ok && passes_wt >= 2 * 4 * sms) : wp.ok;
   if (rows_kernel) {
     cudaError_t e = launch_residual_gather(x, M, K, ldx, dense, M, qx_codes, qx_scales, qx_layout, qx_st, sel, n_sel,
                                            width, r_st, r_codes, r_scales, r_layout, s);

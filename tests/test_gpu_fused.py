@@ -39,7 +39,9 @@ def test_quantize_select_matches_separate_calls(M, K, k, caller_amax):
 
 
 @pytest.mark.parametrize("M,K,N,k", [(300, 192, 144, 50.0), (4096, 2048, 2048, 50.0), (256, 4096, 11008, 50.0),
-                                     (64, 512, 512, 25.0)])
+                                     (64, 512, 512, 25.0),
+                                     # row-staged residual with the weight in the same launch
+                                     (8192, 1024, 640, 25.0), (16384, 4096, 4096, 50.0)])
 @pytest.mark.parametrize("wsel", ["bf16", "fp4"])
 def test_second_pass_matches_separate_calls(M, K, N, k, wsel):
     b = need_gpu()
