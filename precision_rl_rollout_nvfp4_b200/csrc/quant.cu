@@ -263,8 +263,11 @@ quant_score2_kernel(const uint16_t* __restrict__ x, int64_t K, int64_t ldx, RowG
   int cur_e = -1;
   float s_t = 0.0f;
 
+  // tile and strip counts fit in 32 bits: 32-bit division per tile
+  const uint32_t ns32 = static_cast<uint32_t>(n_strips);
   auto prefetch = [&](int64_t idx, int b) {
-    const int64_t rt = idx / n_strips, strip = idx % n_strips;
+    const uint32_t i32 = static_cast<uint32_t>(idx);
+    const int64_t rt = i32 / ns32, strip = i32 % ns32;
     const TileInfo ti = tile_info(g, rt);
     const int64_t col = strip * kQCols + 8 * cg;
 #pragma unroll
@@ -289,7 +292,7 @@ quant_score2_kernel(const uint16_t* __restrict__ x, int64_t K, int64_t ldx, RowG
     } else {
       cp_async_wait<0>();
     }
-    const int64_t tile = idx / n_strips, strip = idx % n_strips;
+    const int64_t tile = static_cast<uint32_t>(idx) / ns32, strip = static_cast<uint32_t>(idx) % ns32;
     const TileInfo ti = tile_info(g, tile);
     if (ti.e != cur_e) {                           // uniform over the CTA
       const float a = g.off == nullptr ? (n_parts > 0 ? a_dense : amax[0]) : amax[ti.e];
@@ -1349,6 +1352,7 @@ cudaError_t launch_quant_score(const uint16_t* x, int64_t rows, int64_t K, int64
     if (ae != cudaSuccess) return ae;
   }
   const int64_t work = tiles * (K / kQCols);
+  if (work >= (int64_t(1) << 31)) return cudaErrorInvalidValue;   // tile indices are 32-bit in the kernel
   const int64_t cap = static_cast<int64_t>(sm_count()) * 3;
   SelectOut so{-1, nullptr, nullptr, nullptr, nullptr};
   if (fused != nullptr) so = SelectOut{fused->n_sel, fused->mask, fused->sel, fused->s_t, fused->strips_done};
