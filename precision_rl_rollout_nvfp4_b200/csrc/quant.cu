@@ -481,10 +481,13 @@ quant_score2_kernel(const uint16_t* __restrict__ x, int64_t K, int64_t ldx, RowG
       __syncthreads();
       if (s_last) {
         __threadfence();
-        // keys in the (now idle) tile buffers when they fit, column maxima from L2
-        const bool fit = K * static_cast<int64_t>(sizeof(uint64_t)) <= 2 * kTileRows * kQCols * 2;
+        // keys in the (now idle) tile buffers and column maxima in the idle
+        // partial-sum buffer when they fit (K <= 4096), else read from L2
+        const bool fit = K * static_cast<int64_t>(sizeof(uint64_t)) <= 2 * kTileRows * kQCols * 2 &&
+                         K * static_cast<int64_t>(sizeof(float)) <= static_cast<int64_t>(sizeof(gsum));
         topk_select(score, colamax, K, sel_out.n_sel, sel_out.mask, sel_out.sel, sel_out.s_t, 0,
-                    fit ? reinterpret_cast<uint64_t*>(q2_dyn) : nullptr, true, false);
+                    fit ? reinterpret_cast<uint64_t*>(q2_dyn) : nullptr,
+                    fit ? reinterpret_cast<float*>(&gsum[0][0]) : nullptr, true);
         if (t == 0) *sel_out.strips_done = 0;
       }
     }

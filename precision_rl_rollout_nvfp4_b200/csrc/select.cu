@@ -31,7 +31,8 @@ topk_kernel(const double* __restrict__ score, const float* __restrict__ colamax,
   pdl_wait();
   pdl_launch_dependents();
   extern __shared__ uint64_t skeys[];            // [K] keys, then [K] colamax
-  topk_select(score, colamax, K, n_sel, mask, sel, s_t_out, blockIdx.x, in_smem ? skeys : nullptr, false);
+  topk_select(score, colamax, K, n_sel, mask, sel, s_t_out, blockIdx.x, in_smem ? skeys : nullptr,
+              in_smem ? reinterpret_cast<float*>(skeys + K) : nullptr, false);
 }
 
 }  // namespace

@@ -49,23 +49,39 @@ static __device__ __forceinline__ long long block_excl_scan(long long v, long lo
   return before;
 }
 
-// Selection of group e over K keys.  skeys: shared memory for K keys (and,
-// with cm_too, K column maxima after them), or null to read them from global
-// memory.  coherent: the scores were written by the same kernel (read through
-// L2, not the read-only path).  Every thread of the CTA calls it.
+// Selection of group e over K keys.  skeys / scm: shared memory for the K
+// keys and the K column maxima, or null to read them from global memory.
+// coherent: the scores were written by the same kernel (read through L2, not
+// the read-only path).  Every thread of the CTA calls it.
 static __device__ __noinline__ void topk_select(const double* __restrict__ score, const float* __restrict__ colamax,
                                          int64_t K, int64_t n_sel, uint8_t* __restrict__ mask,
                                          int32_t* __restrict__ sel, float* __restrict__ s_t_out, int64_t e,
-                                         uint64_t* skeys, bool coherent, bool cm_too = true) {
+                                         uint64_t* skeys, float* scm, bool coherent) {
   const uint64_t* gkeys = reinterpret_cast<const uint64_t*>(score + e * K);
   const float* gcm = colamax + e * K;
   const bool in_smem = skeys != nullptr;
-  const bool cm_smem = in_smem && cm_too;
-  float* scm = reinterpret_cast<float*>(skeys + (in_smem ? K : 0));
-  if (in_smem) {
-    for (int64_t j = threadIdx.x; j < K; j += blockDim.x) {
-      skeys[j] = coherent ? __ldcg(gkeys + j) : __ldg(gkeys + j);
-      if (cm_smem) scm[j] = coherent ? __ldcg(gcm + j) : __ldg(gcm + j);
+  const bool cm_smem = scm != nullptr;
+  if (in_smem || cm_smem) {
+    // eight loads in flight per thread, then the stores
+    for (int64_t j0 = threadIdx.x; j0 < K; j0 += 8 * static_cast<int64_t>(blockDim.x)) {
+      uint64_t kv[8];
+      float cv[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int64_t j = j0 + u * static_cast<int64_t>(blockDim.x);
+        if (j < K) {
+          if (in_smem) kv[u] = coherent ? __ldcg(gkeys + j) : __ldg(gkeys + j);
+          if (cm_smem) cv[u] = coherent ? __ldcg(gcm + j) : __ldg(gcm + j);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int64_t j = j0 + u * static_cast<int64_t>(blockDim.x);
+        if (j < K) {
+          if (in_smem) skeys[j] = kv[u];
+          if (cm_smem) scm[j] = cv[u];
+        }
+      }
     }
     __syncthreads();
   }
@@ -97,6 +113,7 @@ static __device__ __noinline__ void topk_select(const double* __restrict__ score
     }
     __syncthreads();
     uint64_t a = ~0ull, o = 0ull;
+#pragma unroll 8
     for (int64_t j = tid; j < K; j += blockDim.x) {
       const uint64_t k = in_smem ? keys[j] : __ldcg(keys + j);
       a &= k;
@@ -171,6 +188,7 @@ static __device__ __noinline__ void topk_select(const double* __restrict__ score
   const bool none = n_sel == 0;
   long long n_gt = 0, n_eq = 0;
   if (!none) {
+#pragma unroll 8
     for (int64_t j = jb; j < je; ++j) {
       const uint64_t k = in_smem ? keys[j] : __ldcg(keys + j);
       if (ge_mode ? k >= T : k > T) ++n_gt;
