@@ -289,7 +289,7 @@ def graph_kernel_count(g):
         return None
     try:
         from cuda.bindings import runtime as rt
-        raw = g.raw_cuda_graph()
+        raw = rt.cudaGraph_t(init_value=int(g.raw_cuda_graph()))
         err, nodes, n = rt.cudaGraphGetNodes(raw, 0)
         err, nodes, n = rt.cudaGraphGetNodes(raw, n)
         count = 0
@@ -426,9 +426,11 @@ def run_ours(args, rank, world, local_rank):
     if use_graph:
         try:
             for name, fn in [("step", full_step), ("plain", plan.plain_step)] + [(c, fns[c]) for c in calls]:
-                g = torch.cuda.CUDAGraph()
+                g = torch.cuda.CUDAGraph(keep_graph=(name == "step"))   # kept: its kernel nodes are counted
                 with torch.cuda.graph(g):
                     fn()
+                if name == "step":
+                    g.instantiate()
                 graphs[name] = g
             torch.cuda.synchronize()
         except Exception as exc:  # capture not possible: time direct calls
@@ -541,11 +543,12 @@ def run_ours(args, rank, world, local_rank):
     # the RAC linear without weight preparation as one graph (launch count)
     g_rac = None
     if use_graph and not reuse:
-        g_rac = torch.cuda.CUDAGraph()
+        g_rac = torch.cuda.CUDAGraph(keep_graph=True)
         with torch.cuda.graph(g_rac):
             plan.quantize_select()
             plan.second_pass()
             plan.gemm()
+        g_rac.instantiate()
         torch.cuda.synchronize()
     # plain W4A4 linear (no RAC) and the RAC linear without weight prep, for the overhead
     plain_ms, rac_ms = [], []
