@@ -1026,7 +1026,7 @@ __global__ void __launch_bounds__(512, 2) wsel_rows_kernel(RowsArgs A) {
 // [0, n_res) run the residual (MODE 2), the others W_sel (WMODE 0 from the
 // bf16 weight, 1 from the NVFP4 weight).
 template <int WMODE>
-__global__ void __launch_bounds__(512, 2) rows_pair_kernel(RowsArgs Rr, RowsArgs Wr, int n_res) {
+__global__ void __launch_bounds__(512, 1) rows_pair_kernel(RowsArgs Rr, RowsArgs Wr, int n_res) {
   pdl_wait();
   pdl_launch_dependents();
   extern __shared__ __align__(16) uint8_t ws_smem[];
