@@ -70,9 +70,9 @@ constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC0_COL = 0, ACC1_COL = 128;   // two 128-column fp32 accumulators
 // block scales: per pipeline stage 32 columns (16 for A, 16 for B)
 constexpr uint32_t SF1_COL = 256, SF1_STAGE_COLS = 32;
-// warps of the single-CTA kernel: 0 TMA producer, 1 MMA issuer (which also
-// copies each stage's block scales into TMEM), 2..5 epilogue
-constexpr int THREADS1 = 192;
+// warps of the single-CTA kernel: 0 TMA producer, 1 MMA issuer, 2..5
+// epilogue, 6 scale-factor copier
+constexpr int THREADS1 = 224;
 
 // kind::mxf4nvf4 instruction descriptor: E2M1 x E2M1, ue4m3 scales, both
 // K-major, N = 128, M = 128.
@@ -197,20 +197,24 @@ __device__ __forceinline__ void gemm1_body(const CUtensorMap& tmA0, const CUtens
   uint8_t* sOut = sSFB + STAGES * SF_STAGE;                     // epilogue staging
   uint64_t* full = reinterpret_cast<uint64_t*>(sOut + Cfg<YBYTES>::STG_BYTES);
   uint64_t* empty = full + STAGES;
-  uint64_t* tmem_full = empty + STAGES;
+  uint64_t* sf_ready = empty + STAGES;       // the stage's scales are in TMEM
+  uint64_t* tmem_full = sf_ready + STAGES;
   uint64_t* tmem_empty = tmem_full + 1;
   uint64_t* drain = tmem_empty + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* drain_cp = drain + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_cp + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
+      mbar_init(&sf_ready[s], 1);
     }
     mbar_init(tmem_full, 1);
     mbar_init(tmem_empty, 128);
     mbar_init(drain, 1);
+    mbar_init(drain_cp, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
@@ -274,13 +278,6 @@ __device__ __forceinline__ void gemm1_body(const CUtensorMap& tmA0, const CUtens
   } else if (warp == 1) {
     if (lane == 0) {
       // ------------------------------ MMA issuer
-      // Per stage: the block scales go smem -> TMEM (tcgen05.cp), then the
-      // MMAs that read them.  Both are issued by this one thread, and a
-      // tcgen05.cp followed by a tcgen05.mma from the same thread executes in
-      // issue order, so no barrier stands between them and the tensor pipe
-      // never drains between K steps.  A stage's TMEM scale columns are
-      // rewritten only after its smem was refilled, i.e. after the MMAs that
-      // read them completed (empty[stage]).
       int stage = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
@@ -290,16 +287,14 @@ __device__ __forceinline__ void gemm1_body(const CUtensorMap& tmA0, const CUtens
         for (int seg = 0; seg < nseg && ok; ++seg) {
           const uint32_t d = tmem + (seg ? ACC1_COL : ACC0_COL);
           for (int kt = 0; kt < p.kt[seg]; ++kt) {
-            if (!mbar_wait(&full[stage], phase, p.err)) { ok = false; break; }
+            if (!mbar_wait(&full[stage], phase, p.err) || !mbar_wait(&sf_ready[stage], phase, p.err)) {
+              ok = false;
+              break;
+            }
             tc_fence_after();
             const int nkb = kt == p.kt[seg] - 1 ? p.kb_last[seg] : 4;
             const uint32_t a0 = smem_u32(sA + stage * A_STAGE), b0 = smem_u32(sB + stage * B_STAGE);
             const uint32_t sfa = tmem + SF1_COL + SF1_STAGE_COLS * stage, sfb = sfa + 16;
-            const uint32_t fa = smem_u32(sSFA + stage * SF_STAGE), fb = smem_u32(sSFB + stage * SF_STAGE);
-            for (int j = 0; j < (FP8 ? 1 : nkb); ++j) {
-              utccp_sf(sfa + 4 * j, desc_sf(fa + j * SF_ATOM));
-              utccp_sf(sfb + 4 * j, desc_sf(fb + j * SF_ATOM));
-            }
             for (int j = 0; j < nkb; ++j) {
               if (FP8)
                 mma_fp8(d, desc_sw128(a0 + 32 * j), desc_sw128(b0 + 32 * j),
@@ -318,6 +313,34 @@ __device__ __forceinline__ void gemm1_body(const CUtensorMap& tmA0, const CUtens
       }
       umma_commit(drain);                 // all issued tensor-core work done
       mbar_wait(drain, 0, p.err);
+    }
+  } else if (warp == 6) {
+    if (lane == 0) {
+      // ------------------------------ scale-factor copier: smem -> TMEM
+      // copies of the stage's block scales; completion arrives on
+      // sf_ready[stage], which the MMA issuer waits for
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int64_t tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        for (int seg = 0; seg < nseg && ok; ++seg) {
+          for (int kt = 0; kt < p.kt[seg]; ++kt) {
+            if (!mbar_wait(&full[stage], phase, p.err)) { ok = false; break; }
+            tc_fence_after();
+            const int nkb = kt == p.kt[seg] - 1 ? p.kb_last[seg] : 4;
+            const uint32_t fa = smem_u32(sSFA + stage * SF_STAGE), fb = smem_u32(sSFB + stage * SF_STAGE);
+            const uint32_t sfa = tmem + SF1_COL + SF1_STAGE_COLS * stage, sfb = sfa + 16;
+            for (int j = 0; j < (FP8 ? 1 : nkb); ++j) {
+              utccp_sf(sfa + 4 * j, desc_sf(fa + j * SF_ATOM));
+              utccp_sf(sfb + 4 * j, desc_sf(fb + j * SF_ATOM));
+            }
+            umma_commit(&sf_ready[stage]);
+            if (++stage == STAGES) { stage = 0; phase ^= 1; }
+          }
+        }
+      }
+      umma_commit(drain_cp);
+      mbar_wait(drain_cp, 0, p.err);
     }
   } else {
     // ------------------------------ epilogue (warps 2..5)
@@ -476,11 +499,12 @@ struct Cfg2 {
   static constexpr uint32_t TX = 2 * STAGE;            // bytes landing per stage (both CTAs)
 };
 
-// Warps of the pair kernel: 0 TMA producer, 1 MMA issuer (leader CTA; it
-// also copies each stage's block scales into TMEM), 2..5 epilogue.
-constexpr int THREADS2 = 192;
+// Warps of the pair kernel: 0 TMA producer, 1 MMA issuer, 2..5 epilogue,
+// 6 scale-factor copier (leader CTA).
+constexpr int THREADS2 = 224;
 // TMEM columns: the 256-column accumulator, then per pipeline stage 48
-// columns of block scales (16 for A, 32 for B).
+// columns of block scales (16 for A, 32 for B), so the copies for later
+// stages run while the MMAs of earlier ones read theirs.
 constexpr uint32_t ACC2_COL = 0, SF2_COL = 256, SF2_STAGE_COLS = 48;
 // kind::mxf4nvf4, M = 256 (pair), N = 256, both K-major, ue4m3 scales.
 constexpr uint32_t IDESC2 = (1u << 7) | (1u << 10) | (uint32_t(256 >> 3) << 17) | (uint32_t(256 >> 4) << 24);
@@ -621,12 +645,14 @@ __device__ __forceinline__ void gemm2_body(const CUtensorMap& tmA0, const CUtens
   uint8_t* sOut = smem + STAGES * C::STAGE;
   uint64_t* full = reinterpret_cast<uint64_t*>(sOut + C::STG_BYTES);
   uint64_t* empty = full + STAGES;
-  uint64_t* tmem_full = empty + STAGES;
+  uint64_t* sf_ready = empty + STAGES;   // the stage's scales are in TMEM
+  uint64_t* tmem_full = sf_ready + STAGES;
   uint64_t* tmem_empty = tmem_full + 1;
   uint64_t* res_full = tmem_empty + 1;
   uint64_t* res_done = res_full + 1;
   uint64_t* drain = res_done + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* drain_cp = drain + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_cp + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_rank();
@@ -635,12 +661,14 @@ __device__ __forceinline__ void gemm2_body(const CUtensorMap& tmA0, const CUtens
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
+      mbar_init(&sf_ready[s], 1);
     }
     mbar_init(tmem_full, 1);
     mbar_init(tmem_empty, 8);          // one arrival per epilogue warp of both CTAs
     mbar_init(res_full, 1);
     mbar_init(res_done, 8);
     mbar_init(drain, 1);
+    mbar_init(drain_cp, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   cluster_sync_all();                  // barriers of both CTAs initialised
@@ -706,12 +734,6 @@ __device__ __forceinline__ void gemm2_body(const CUtensorMap& tmA0, const CUtens
   } else if (warp == 1) {
     if (lane == 0 && rank == 0) {
       // ------------------------------ MMA issuer (leader CTA only)
-      // Per stage: both CTAs' block scales smem -> TMEM (tcgen05.cp), then
-      // the MMAs that read them, all from this thread: a tcgen05.cp and a
-      // later tcgen05.mma of the same thread execute in issue order, so the
-      // tensor pipe is fed without a barrier between K steps.  A stage's
-      // TMEM scale columns are rewritten only after its smem was refilled,
-      // i.e. after the MMAs that read them completed (empty[stage]).
       int stage = 0;
       uint32_t phase = 0, acc_phase = 0, res_phase = 0;
       bool ok = true;
@@ -720,26 +742,14 @@ __device__ __forceinline__ void gemm2_body(const CUtensorMap& tmA0, const CUtens
         tc_fence_after();
         for (int seg = has_res ? 0 : 1; seg < 2 && ok; ++seg) {
           for (int kt = 0; kt < p.kt[seg]; ++kt) {
-            if (!mbar_wait(&full[stage], phase, p.err)) { ok = false; break; }
+            if (!mbar_wait(&full[stage], phase, p.err) || !mbar_wait(&sf_ready[stage], phase, p.err)) {
+              ok = false;
+              break;
+            }
             tc_fence_after();
             const uint32_t st = smem_u32(sStage + stage * C::STAGE);
             const uint32_t a0 = st, b0 = st + C::A_ST;
             const uint32_t sfa = tmem + SF2_COL + SF2_STAGE_COLS * stage, sfb = sfa + 16;
-            const uint32_t fa = st + C::A_ST + C::B_ST, fb = fa + C::SFA_ST;
-            if (FP8) {
-              // one atom of A, the two 128-row atoms of B; every MMA of the
-              // step reads these columns (its own byte of each word)
-              utccp_sf_pair(sfa, desc_sf(fa));
-              utccp_sf_pair(sfb, desc_sf(fb));
-              utccp_sf_pair(sfb + 4, desc_sf(fb + SF_ATOM));
-            } else {
-#pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                utccp_sf_pair(sfa + 4 * j, desc_sf(fa + j * SF_ATOM));
-                utccp_sf_pair(sfb + 8 * j, desc_sf(fb + j * SF_ATOM));
-                utccp_sf_pair(sfb + 8 * j + 4, desc_sf(fb + 4 * SF_ATOM + j * SF_ATOM));
-              }
-            }
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
               const uint32_t accum = (seg == 1 && has_res) ? 1u : ((kt > 0 || j > 0) ? 1u : 0u);
@@ -769,6 +779,45 @@ __device__ __forceinline__ void gemm2_body(const CUtensorMap& tmA0, const CUtens
       asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];"
                    :: "r"(smem_u32(drain)) : "memory");
       mbar_wait(drain, 0, p.err);
+    }
+  } else if (warp == 6) {
+    if (lane == 0 && rank == 0) {
+      // ------------------------------ scale-factor copier (leader CTA only)
+      // smem -> TMEM copies of both CTAs' block scales for each stage; their
+      // completion arrives on sf_ready[stage], which the MMA issuer waits for
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int tile = pair; tile < total && ok; tile += npairs) {
+        for (int seg = has_res ? 0 : 1; seg < 2 && ok; ++seg) {
+          for (int kt = 0; kt < p.kt[seg]; ++kt) {
+            if (!mbar_wait(&full[stage], phase, p.err)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t fa = smem_u32(sStage + stage * C::STAGE) + C::A_ST + C::B_ST, fb = fa + C::SFA_ST;
+            const uint32_t sfa = tmem + SF2_COL + SF2_STAGE_COLS * stage, sfb = sfa + 16;
+            if (FP8) {
+              // one atom of A, the two 128-row atoms of B; every MMA of the
+              // step reads these columns (its own byte of each word)
+              utccp_sf_pair(sfa, desc_sf(fa));
+              utccp_sf_pair(sfb, desc_sf(fb));
+              utccp_sf_pair(sfb + 4, desc_sf(fb + SF_ATOM));
+            } else {
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                utccp_sf_pair(sfa + 4 * j, desc_sf(fa + j * SF_ATOM));
+                utccp_sf_pair(sfb + 8 * j, desc_sf(fb + j * SF_ATOM));
+                utccp_sf_pair(sfb + 8 * j + 4, desc_sf(fb + 4 * SF_ATOM + j * SF_ATOM));
+              }
+            }
+            asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                         :: "r"(smem_u32(&sf_ready[stage])) : "memory");
+            if (++stage == STAGES) { stage = 0; phase ^= 1; }
+          }
+        }
+      }
+      asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                   :: "r"(smem_u32(drain_cp)) : "memory");
+      mbar_wait(drain_cp, 0, p.err);
     }
   } else {
     // ------------------------------ epilogue (warps 2..5 of both CTAs)
