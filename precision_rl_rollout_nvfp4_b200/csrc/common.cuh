@@ -124,9 +124,11 @@ __device__ __forceinline__ uint32_t e2m1x8(const float* v) {
 // sm_100a executes mul / fma (and add / sub) on two fp32 lanes in one
 // instruction (.f32x2, each lane rounded to nearest even like the scalar
 // form).  A pair lives in one 64-bit register: element 2j in the low half.
-// A packed product that feeds a packed sum or difference can be fused into
-// one rounding by the code generator, so only products whose result is
-// consumed by something other than an addition use the packed form.
+// A packed product that feeds a packed sum or difference is fused into one
+// rounding by the code generator (measured: a mul.rn.f32x2 feeding an
+// add.rn.f32x2 changed the residual's last bits), so only products whose
+// result is consumed by something other than an addition use the packed
+// form, and there is no packed add here.
 __device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
   uint64_t r;
   asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));

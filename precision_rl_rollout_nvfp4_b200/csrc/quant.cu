@@ -178,6 +178,10 @@ __device__ __forceinline__ float reduce_parts(const unsigned* parts, int n, uint
 // X and the block's scale code with the same operations (so the same values).
 // ---------------------------------------------------------------------------
 constexpr int kSpanExact = 22;
+// tensor scales from 2^-55 up: every nonzero block decode scale
+// RN(E4M3dec(sb) s_t) >= 2^-9 2^-55 = 2^-64, so its reciprocal table entry
+// serves the quotient (Markstein) and no division fallback is needed
+constexpr float kFastScale = 2.7755575615628914e-17f;   // 2^-55
 
 // Optional top-k% selection fused into the quantize pass's tail.
 struct SelectOut {
@@ -226,6 +230,93 @@ __device__ __forceinline__ void cp_async16_zfill(uint32_t dst, const void* src, 
                : "memory");
 }
 
+// The row-order sums of the tile's wide columns (a column whose nonzero
+// |dX| span more than kSpanExact binades): the tile is still in its shared
+// buffer xt, so 128 threads recompute the column's |dX| from it and the
+// tile's block-scale codes sbt, and one thread adds them in row order.
+// Kept out of line like finish_strip (it never runs on most inputs).
+static __device__ __noinline__ void wide_columns(const uint16_t (*xt)[kQCols], const uint8_t (*sbt)[kQCols / kBlock],
+                                                 const uint8_t* s_wide, float* s_dxcol, const ScaleTable& T,
+                                                 int64_t tile, int64_t row_tiles, int64_t col0, int64_t K,
+                                                 double* part_sum) {
+  const int t = threadIdx.x;
+  for (int c = 0; c < kQCols; ++c) {
+    if (!s_wide[c]) continue;                      // uniform: every thread reads the same flag
+    if (t < kTileRows) {
+      const float xv = bf16_bits_to_f32(xt[t][c]);   // rows past the end were zero-filled
+      s_dxcol[t] = residual_abs_one(xv, sbt[t][c >> 4], T);
+    }
+    __syncthreads();
+    if (t == 0) {
+      double chain = 0.0;
+      for (int r = 0; r < kTileRows; ++r) chain += static_cast<double>(s_dxcol[r]);
+      if (NV_IDX(tile < row_tiles && col0 + c < K)) part_sum[tile * K + col0 + c] = chain;
+    }
+    __syncthreads();
+  }
+}
+
+// The last CTA to finish a column strip of a row group: the chunk-order
+// totals of the strip's partial sums and maxima (staged through the idle
+// partial buffers ps / pm, 32 chunks at a time), and, when a selection is
+// fused, the top-k% selection by the last strip overall.  Kept out of line:
+// it runs once per strip and should not weigh on the registers of the
+// tile loop.
+template <bool SCORES>
+static __device__ __noinline__ void finish_strip(int64_t t0, int64_t t1, unsigned* counter, double* ps, float* pm,
+                                                 const double* part_sum, const float* part_max, int64_t K,
+                                                 int64_t col0, double* score, float* colamax, int e, int E,
+                                                 SelectOut sel_out, int64_t n_strips, uint8_t* keys, bool* s_last) {
+  constexpr int kGroups = kTileRows / 4;
+  const int t = threadIdx.x;
+  __threadfence();
+  double total_s = 0.0;
+  float tmax = 0.0f;
+  for (int64_t c0 = t0; c0 < t1; c0 += kGroups) {
+    const int nt = static_cast<int>(t1 - c0 < kGroups ? t1 - c0 : kGroups);
+    __syncthreads();
+    for (int k = t; k < nt * kQCols; k += kQThreads) {
+      const int tt = k / kQCols, cc = k % kQCols;
+      if (SCORES) ps[k] = __ldcg(part_sum + (c0 + tt) * K + col0 + cc);
+      pm[k] = __ldcg(part_max + (c0 + tt) * K + col0 + cc);
+    }
+    __syncthreads();
+    if (t < kQCols) {
+      for (int tt = 0; tt < nt; ++tt) {          // chunk order
+        if (SCORES) total_s += ps[tt * kQCols + t];
+        tmax = fmaxf(tmax, pm[tt * kQCols + t]);
+      }
+    }
+  }
+  if (t < kQCols && NV_IDX(e < E && col0 + t < K)) {
+    if (SCORES) score[static_cast<int64_t>(e) * K + col0 + t] = total_s;
+    colamax[static_cast<int64_t>(e) * K + col0 + t] = tmax;
+  }
+  if (t == 0) *counter = 0;                      // ready for the next call
+  __syncthreads();                               // staging buffers free before the next tile
+  if (SCORES && sel_out.n_sel >= 0) {
+    // the last strip to finish selects the channels; its scores were
+    // published like the partials (barrier, then one thread's fence before
+    // the counter moves)
+    if (t == 0) {
+      __threadfence();
+      *s_last = atomicAdd(sel_out.strips_done, 1u) == static_cast<unsigned>(n_strips - 1);
+    }
+    __syncthreads();
+    if (*s_last) {
+      __threadfence();
+      // keys in the (now idle) tile buffers and column maxima in the idle
+      // partial-sum buffer when they fit (K <= 4096), else read from L2
+      const bool fit = K * static_cast<int64_t>(sizeof(uint64_t)) <= 2 * kTileRows * kQCols * 2 &&
+                       K * static_cast<int64_t>(sizeof(float)) <= static_cast<int64_t>(kGroups * kQCols * sizeof(double));
+      topk_select(score, colamax, K, sel_out.n_sel, sel_out.mask, sel_out.sel, sel_out.s_t, 0,
+                  fit ? reinterpret_cast<uint64_t*>(keys) : nullptr,
+                  fit ? reinterpret_cast<float*>(ps) : nullptr, true);
+      if (t == 0) *sel_out.strips_done = 0;
+    }
+  }
+}
+
 // With sel_out.n_sel >= 0 (dense only) the CTA that completes the last
 // column strip also runs the top-k% selection over the finished scores.
 template <bool SCORES>
@@ -248,12 +339,13 @@ quant_score2_kernel(const uint16_t* __restrict__ x, int64_t K, int64_t ldx, RowG
   __shared__ __align__(16) double qsum[4][kQCols];
   __shared__ __align__(16) float qmax[4][kQCols];
   __shared__ __align__(16) uint32_t qmin[4][kQCols];
-  __shared__ uint8_t s_sb[2][kTileRows][kQCols / kBlock];
+  __shared__ __align__(16) uint8_t s_sb[2][kTileRows][kQCols / kBlock];
   __shared__ float s_dxcol[kTileRows];             // |dX| of one column for the row-order sum
   __shared__ uint8_t s_wide[kQCols];
   __shared__ uint32_t wscratch[kQThreads / 32];
   __shared__ bool s_last;
   __shared__ ScaleTable T;
+  __shared__ float4 T4[128];                       // {sbv, sdec, -rcp} per scale code
   const int t = threadIdx.x, cg = t & 7, grp = t >> 3;
   const int64_t n_strips = K / kQCols;
   const int64_t row_tiles = g.off == nullptr ? (g.M + kTileRows - 1) / kTileRows : g.tile_start[g.E];
@@ -261,7 +353,8 @@ quant_score2_kernel(const uint16_t* __restrict__ x, int64_t K, int64_t ldx, RowG
   // the tensor amax once per CTA (dense: the max of the partial maxima)
   const float a_dense = (g.off == nullptr && n_parts > 0) ? reduce_parts(amax_parts, n_parts, wscratch) : 0.0f;
   int cur_e = -1;
-  float s_t = 0.0f;
+  float s_t = 0.0f, dd = 0.0f, rcpd = 0.0f;
+  bool fast = false;
 
   // tile and strip counts fit in 32 bits: 32-bit division per tile
   const uint32_t ns32 = static_cast<uint32_t>(n_strips);
@@ -299,8 +392,12 @@ quant_score2_kernel(const uint16_t* __restrict__ x, int64_t K, int64_t ldx, RowG
       s_t = __fdiv_rn(a, kTensorScaleDiv);
       __syncthreads();                             // nobody reads the previous group's table any more
       build_scale_table(T, s_t, t);
+      if (t < 128) T4[t] = make_float4(T.sbv[t], T.sdec[t], -T.rcp[t], 0.0f);   // this thread's own entries
       __syncthreads();
       cur_e = ti.e;
+      fast = s_t >= kFastScale;
+      dd = T.d;
+      rcpd = T.rcp_d;
     }
     const int64_t col0 = strip * kQCols;
     const int64_t col = col0 + 8 * cg;
@@ -327,13 +424,41 @@ quant_score2_kernel(const uint16_t* __restrict__ x, int64_t K, int64_t ldx, RowG
       }
       float am = __uint_as_float(max(mbits & 0xFFFFu, mbits >> 16) << 16);
       am = fmaxf(am, __shfl_xor_sync(0xFFFFFFFFu, am, 1));
-      const BlockQ bq = block_q(am, T);
-      uint64_t q2[4];
-      block_quotients(x2, bq, q2);
-      const uint32_t packed = e2m1x8_f2(q2);
-      const uint64_t sbv2 = f2_pack(bq.sbv, bq.sbv);
+      uint32_t packed, sb;
+      float sbv;
+      if (fast) {
+        // every block decode scale is 0 or >= 2^-64: the quotients need no
+        // division fallback.  sb = E4M3(RN(am / d)) by Markstein's
+        // correction; the element quotients are formed negated, c = -q with
+        // q = RN(x / sdec) (a = RN(-x y) = -q0, the remainder x - q0 sdec
+        // is exact, c = RN(-(r y + q0))), which also gives signed zeros the
+        // right sign: E2M1(c) with every sign bit flipped is E2M1(q).
+        const float q0 = __fmul_rn(am, rcpd);
+        const float rr = __fmaf_rn(-q0, dd, am);
+        sb = f32_to_e4m3(__fmaf_rn(rr, rcpd, q0));
+        const float4 tv = T4[sb];
+        const uint64_t ny2 = f2_pack(tv.z, tv.z), sd2 = f2_pack(tv.y, tv.y);
+        uint64_t c2[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint64_t a = f2_mul(x2[j], ny2);
+          c2[j] = f2_fma(f2_fma(a, sd2, x2[j]), ny2, a);
+        }
+        packed = e2m1x8_f2(c2) ^ 0x88888888u;
+        sbv = tv.x;
+      } else {
+        const BlockQ bq = block_q(am, T);
+        uint64_t q2[4];
+        block_quotients(x2, bq, q2);
+        packed = e2m1x8_f2(q2);
+        sb = bq.sb;
+        sbv = bq.sbv;
+      }
+      const uint64_t sbv2 = f2_pack(sbv, sbv);
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
+        // dX = RN(x - RN(p s_t)) with p = E2M1dec E4M3dec exact (scalar
+        // product and difference: two roundings)
         float p0, p1, x0, x1;
         f2_unpack(f2_mul(e2m1x2_to_f2((packed >> (8 * j)) & 0xFFu), sbv2), p0, p1);
         f2_unpack(x2[j], x0, x1);
@@ -350,22 +475,36 @@ quant_score2_kernel(const uint16_t* __restrict__ x, int64_t K, int64_t ldx, RowG
       }
       if (prow < codes_rows && NV_IDX(col + 8 <= K))
         *reinterpret_cast<uint32_t*>(code_base + static_cast<uint32_t>(r) * static_cast<uint32_t>(K / 2)) = packed;
-      if ((cg & 1) == 0 && (layout == 1 || prow < codes_rows) &&
-          NV_IDX(scale_offset(prow, col / kBlock, K, layout) < scale_extent(codes_rows, K, layout, kBlock)))
-        scales[scale_offset(prow, col / kBlock, K, layout)] = static_cast<uint8_t>(bq.sb);
-      if (SCORES && (cg & 1) == 0) s_sb[b][r][cg >> 1] = static_cast<uint8_t>(bq.sb);
+      if ((cg & 1) == 0) s_sb[b][r][cg >> 1] = static_cast<uint8_t>(sb);
+    }
+    if (part_max != nullptr) {
+      if (SCORES) {
+#pragma unroll
+        for (int j = 0; j < 8; j += 2)
+          *reinterpret_cast<double2*>(&gsum[grp][8 * cg + j]) = make_double2(acc[j], acc[j + 1]);
+        *reinterpret_cast<uint4*>(&gmin[grp][8 * cg]) = make_uint4(mn[0], mn[1], mn[2], mn[3]);
+        *reinterpret_cast<uint4*>(&gmin[grp][8 * cg + 4]) = make_uint4(mn[4], mn[5], mn[6], mn[7]);
+      }
+      *reinterpret_cast<float4*>(&gmax[grp][8 * cg]) = make_float4(mx[0], mx[1], mx[2], mx[3]);
+      *reinterpret_cast<float4*>(&gmax[grp][8 * cg + 4]) = make_float4(mx[4], mx[5], mx[6], mx[7]);
+    }
+    __syncthreads();
+    // the tile's block scales leave from shared memory: one 512-byte atom
+    // (tiled layout: 32 threads x 16 bytes) or one 4-byte word per row
+    if (layout == 1) {
+      if (t < 32) {
+        const int64_t off = (tile * ((K + 63) / 64) + (col0 >> 6)) * 512 + 16 * t;
+        const uint32_t* sw = reinterpret_cast<const uint32_t*>(&s_sb[b][0][0]);
+        if (NV_IDX(off + 16 <= scale_extent(codes_rows, K, layout, kBlock)))
+          *reinterpret_cast<uint4*>(scales + off) = make_uint4(sw[t], sw[t + 32], sw[t + 64], sw[t + 96]);
+      }
+    } else if (t < kTileRows) {
+      const int64_t prow = tile * kTileRows + t;
+      const int64_t off = prow * (K / kBlock) + (col0 >> 4);
+      if (prow < codes_rows && NV_IDX(off + 4 <= scale_extent(codes_rows, K, layout, kBlock)))
+        *reinterpret_cast<uint32_t*>(scales + off) = *reinterpret_cast<const uint32_t*>(&s_sb[b][t][0]);
     }
     if (part_max == nullptr) continue;
-    if (SCORES) {
-#pragma unroll
-      for (int j = 0; j < 8; j += 2)
-        *reinterpret_cast<double2*>(&gsum[grp][8 * cg + j]) = make_double2(acc[j], acc[j + 1]);
-      *reinterpret_cast<uint4*>(&gmin[grp][8 * cg]) = make_uint4(mn[0], mn[1], mn[2], mn[3]);
-      *reinterpret_cast<uint4*>(&gmin[grp][8 * cg + 4]) = make_uint4(mn[4], mn[5], mn[6], mn[7]);
-    }
-    *reinterpret_cast<float4*>(&gmax[grp][8 * cg]) = make_float4(mx[0], mx[1], mx[2], mx[3]);
-    *reinterpret_cast<float4*>(&gmax[grp][8 * cg + 4]) = make_float4(mx[4], mx[5], mx[6], mx[7]);
-    __syncthreads();
     {
       const int c = t & (kQCols - 1), q4 = t >> 6;
       double sum = 0.0;
@@ -415,22 +554,8 @@ quant_score2_kernel(const uint16_t* __restrict__ x, int64_t K, int64_t ldx, RowG
     // is the prefetch two tiles ahead, issued after this point by every
     // thread), so 128 threads recompute the column's |dX| from it and the
     // tile's block-scale codes, and one thread adds them in row order.
-    if (SCORES && __syncthreads_or(wide)) {
-      for (int c = 0; c < kQCols; ++c) {
-        if (!s_wide[c]) continue;                  // uniform: every thread reads the same flag
-        if (t < kTileRows) {
-          const float xv = bf16_bits_to_f32(xbuf[b][t][c]);   // rows past the end were zero-filled
-          s_dxcol[t] = residual_abs_one(xv, s_sb[b][t][c >> 4], T);
-        }
-        __syncthreads();
-        if (t == 0) {
-          double chain = 0.0;
-          for (int r = 0; r < kTileRows; ++r) chain += static_cast<double>(s_dxcol[r]);
-          if (NV_IDX(tile < row_tiles && col0 + c < K)) part_sum[tile * K + col0 + c] = chain;
-        }
-        __syncthreads();
-      }
-    }
+    if (SCORES && __syncthreads_or(wide))
+      wide_columns(xbuf[b], s_sb[b], s_wide, s_dxcol, T, tile, row_tiles, col0, K, part_sum);
     if (strip_count == nullptr) continue;
     __syncthreads();
     const int64_t t0 = g.off == nullptr ? 0 : g.tile_start[ti.e];
@@ -443,54 +568,8 @@ quant_score2_kernel(const uint16_t* __restrict__ x, int64_t K, int64_t ldx, RowG
     }
     __syncthreads();
     if (!s_last) continue;
-    __threadfence();
-    double* ps = &gsum[0][0];                      // [32 tiles][64 cols]
-    float* pm = &gmax[0][0];
-    double total_s = 0.0;
-    float tmax = 0.0f;
-    for (int64_t c0 = t0; c0 < t1; c0 += kGroups) {
-      const int nt = static_cast<int>(t1 - c0 < kGroups ? t1 - c0 : kGroups);
-      __syncthreads();
-      for (int k = t; k < nt * kQCols; k += kQThreads) {
-        const int tt = k / kQCols, cc = k % kQCols;
-        if (SCORES) ps[k] = __ldcg(part_sum + (c0 + tt) * K + col0 + cc);
-        pm[k] = __ldcg(part_max + (c0 + tt) * K + col0 + cc);
-      }
-      __syncthreads();
-      if (t < kQCols) {
-        for (int tt = 0; tt < nt; ++tt) {          // chunk order
-          if (SCORES) total_s += ps[tt * kQCols + t];
-          tmax = fmaxf(tmax, pm[tt * kQCols + t]);
-        }
-      }
-    }
-    if (t < kQCols && NV_IDX(ti.e < g.E && col0 + t < K)) {
-      if (SCORES) score[static_cast<int64_t>(ti.e) * K + col0 + t] = total_s;
-      colamax[static_cast<int64_t>(ti.e) * K + col0 + t] = tmax;
-    }
-    if (t == 0) *counter = 0;                      // ready for the next call
-    __syncthreads();                               // staging buffers free before the next tile
-    if (SCORES && sel_out.n_sel >= 0) {
-      // the last strip to finish selects the channels; its scores were
-      // published like the partials (barrier, then one thread's fence before
-      // the counter moves)
-      if (t == 0) {
-        __threadfence();
-        s_last = atomicAdd(sel_out.strips_done, 1u) == static_cast<unsigned>(n_strips - 1);
-      }
-      __syncthreads();
-      if (s_last) {
-        __threadfence();
-        // keys in the (now idle) tile buffers and column maxima in the idle
-        // partial-sum buffer when they fit (K <= 4096), else read from L2
-        const bool fit = K * static_cast<int64_t>(sizeof(uint64_t)) <= 2 * kTileRows * kQCols * 2 &&
-                         K * static_cast<int64_t>(sizeof(float)) <= static_cast<int64_t>(sizeof(gsum));
-        topk_select(score, colamax, K, sel_out.n_sel, sel_out.mask, sel_out.sel, sel_out.s_t, 0,
-                    fit ? reinterpret_cast<uint64_t*>(q2_dyn) : nullptr,
-                    fit ? reinterpret_cast<float*>(&gsum[0][0]) : nullptr, true);
-        if (t == 0) *sel_out.strips_done = 0;
-      }
-    }
+    finish_strip<SCORES>(t0, t1, counter, &gsum[0][0], &gmax[0][0], part_sum, part_max, K, col0, score, colamax,
+                         ti.e, g.E, sel_out, n_strips, q2_dyn, &s_last);
   }
   cp_async_wait<0>();
 }
@@ -801,10 +880,10 @@ __device__ __forceinline__ uint32_t dup_e4m3_to_h2(uint32_t sb) { return e4m3x2_
 // MODE 0: W_sel from bf16 rows w; MODE 1: W_sel from the NVFP4 weight
 // (codes / scales / w_st); MODE 2: the residual dX_sel of dense activations:
 // rows of X (w, stride ldw) and of Q(X) (codes / scales / w_st = its tensor
-// scale) are staged side by side, each gathered element is x - DQ decoded
-// from the staged code nibble and scale byte (the product E2M1 E4M3 exact in
-// f16, then RN(p s_t) and RN(x - dq) in fp32, as the quantize pass forms dX),
-// and the passes of each CTA run from its last rows to its first.
+// scale) are staged side by side, the Q(X) rows are expanded once into the
+// exact f16 products p = E2M1dec E4M3dec, and each gathered element is
+// RN(x - RN(p s_t)) in fp32 (as the quantize pass forms dX); the passes of
+// each CTA run from its last rows to its first.
 struct RowsArgs {
   const uint16_t* w;
   int64_t ldw;
@@ -847,13 +926,17 @@ __device__ __forceinline__ void wsel_rows_body(const RowsArgs& A, uint8_t* ws_sm
   const int nblk = static_cast<int>(width / kBlock);
   const uint32_t R = static_cast<uint32_t>(g.R);
   // shared memory: [staged rows, 2 buffers (bf16) or 1 (NVFP4)][raw NVFP4 rows, 2 buffers]
-  // (residual: bf16 rows of X, 2 buffers, then the raw Q(X) rows, 2 buffers)
+  // (residual: bf16 rows of X, 2 buffers, then the raw Q(X) rows, 1 buffer,
+  // then their expansion into exact f16 products E2M1dec E4M3dec, 1 buffer)
   const uint32_t nbuf_rows = FP4 ? 1u : 2u;
   const uint32_t raw0 = nbuf_rows * R * g.rowbytes;
+  const uint32_t exp0 = raw0 + R * g.rawbytes;     // (residual only)
   // zero the tails (element K onwards) of every staged row once: copies and
-  // the expansion write only elements 0 .. K-1
-  for (uint32_t r = t; r < nbuf_rows * R; r += nthr)
-    *reinterpret_cast<uint4*>(ws_smem + r * g.rowbytes + 2u * Ku) = make_uint4(0u, 0u, 0u, 0u);
+  // the expansions write only elements 0 .. K-1
+  for (uint32_t r = t; r < (RES ? 3u : nbuf_rows) * R; r += nthr) {
+    const uint32_t ro = RES && r >= 2u * R ? exp0 + (r - 2u * R) * g.rowbytes : r * g.rowbytes;
+    *reinterpret_cast<uint4*>(ws_smem + ro + 2u * Ku) = make_uint4(0u, 0u, 0u, 0u);
+  }
   // this thread's blocks and row phase
   const bool shared_blocks = nblk <= nthr;
   const int phase = shared_blocks ? t / nblk : 0;
@@ -869,7 +952,7 @@ __device__ __forceinline__ void wsel_rows_body(const RowsArgs& A, uint8_t* ws_sm
     const int64_t r0 = p * R;
     const uint32_t nrows = static_cast<uint32_t>(rows - r0 < R ? rows - r0 : R);
     for (uint32_t r = 0; r < nrows; ++r) {
-      if (FP4 || RES) {
+      if (FP4) {
         const uint32_t ro = raw0 + (b * R + r) * g.rawbytes;
         const uint8_t* src = codes + (r0 + r) * static_cast<int64_t>(half);
         for (uint32_t q = t; q < half / 16u; q += nthr) cp_async16(ws_smem + ro + 16u * q, src + 16u * q);
@@ -881,6 +964,20 @@ __device__ __forceinline__ void wsel_rows_body(const RowsArgs& A, uint8_t* ws_sm
         const uint16_t* src = w + (r0 + r) * ldw;
         for (uint32_t q = t; q < Ku / 8u; q += nthr) cp_async16(ws_smem + ro + 16u * q, src + 8u * q);
       }
+    }
+    cp_async_commit();
+  };
+  // the raw Q(X) rows of a residual pass (one buffer: filled once the
+  // previous pass has expanded its rows)
+  auto stage_raw = [&](int64_t p) {
+    const int64_t r0 = p * R;
+    const uint32_t nrows = static_cast<uint32_t>(rows - r0 < R ? rows - r0 : R);
+    for (uint32_t r = 0; r < nrows; ++r) {
+      const uint32_t ro = raw0 + r * g.rawbytes;
+      const uint8_t* src = codes + (r0 + r) * static_cast<int64_t>(half);
+      for (uint32_t q = t; q < half / 16u; q += nthr) cp_async16(ws_smem + ro + 16u * q, src + 16u * q);
+      for (uint32_t q = t; q < Ku / 64u; q += nthr)
+        cp_async4(ws_smem + ro + half + 4u * q, scales + scale_offset(r0 + r, 4 * q, K, layout));
     }
     cp_async_commit();
   };
@@ -898,7 +995,10 @@ __device__ __forceinline__ void wsel_rows_body(const RowsArgs& A, uint8_t* ws_sm
   uint32_t cidx[16];
 #pragma unroll
   for (int u = 0; u < 16; ++u) cidx[u] = Ku;
-  if (p0 < p1) stage(pass_of(p0), 0u);
+  if (p0 < p1) {
+    stage(pass_of(p0), 0u);
+    if (RES) stage_raw(pass_of(p0));
+  }
   int cur_e = -1;
   float st_w = 0.0f;
   for (int64_t pi = p0; pi < p1; ++pi) {
@@ -962,6 +1062,27 @@ __device__ __forceinline__ void wsel_rows_body(const RowsArgs& A, uint8_t* ws_sm
       }
       __syncthreads();
     }
+    if (RES) {
+      // expand the raw Q(X) rows into exact f16 products (as above), then
+      // the raw buffer takes the next pass's rows
+      const uint32_t steps = half / 4u;
+      for (uint32_t r = 0; r < nrows; ++r) {
+        const uint32_t ro = raw0 + r * g.rawbytes;
+        uint8_t* dst = ws_smem + exp0 + r * g.rowbytes;
+        for (uint32_t q = t; q < steps; q += nthr) {
+          const uint32_t wd = *reinterpret_cast<const uint32_t*>(ws_smem + ro + 4u * q);
+          const uint32_t sv = dup_e4m3_to_h2(ws_smem[ro + half + (q >> 1)]);
+          uint4 o;
+          o.x = h2_mul(e2m1x2_to_h2(wd & 0xFFu), sv);
+          o.y = h2_mul(e2m1x2_to_h2((wd >> 8) & 0xFFu), sv);
+          o.z = h2_mul(e2m1x2_to_h2((wd >> 16) & 0xFFu), sv);
+          o.w = h2_mul(e2m1x2_to_h2(wd >> 24), sv);
+          *reinterpret_cast<uint4*>(dst + 16u * q) = o;
+        }
+      }
+      __syncthreads();
+      if (pi + 1 < p1) stage_raw(pass_of(pi + 1));
+    }
     if (active) {
       for (int i = 0; i < g.nob; ++i) {
         const int ob = ob0 + i * nthr;
@@ -971,7 +1092,7 @@ __device__ __forceinline__ void wsel_rows_body(const RowsArgs& A, uint8_t* ws_sm
           const uint32_t slot = static_cast<uint32_t>(phase + g.P * k);
           if (slot >= nrows) break;
           const uint8_t* rb = ws_smem + rows0 + slot * g.rowbytes;
-          const uint8_t* raw = ws_smem + raw0 + (b * R + slot) * g.rawbytes;
+          const uint8_t* eb = ws_smem + exp0 + slot * g.rowbytes;   // (residual)
           float v[16];
           float am = 0.0f;
 #pragma unroll
@@ -981,14 +1102,8 @@ __device__ __forceinline__ void wsel_rows_body(const RowsArgs& A, uint8_t* ws_sm
             if (FP4) {
               x = __fmul_rn(__half2float(__ushort_as_half(static_cast<unsigned short>(h))), st_w);
             } else if (RES) {
-              // padded channels read element K of the x row (zero) and a code
-              // and scale past the row's data; their product is discarded
-              const uint32_t c = cidx[u];
-              const bool real = c < Ku;
-              const uint32_t cb = real ? raw[c >> 1] : 0u;
-              const uint32_t sb = real ? raw[half + (c >> 4)] : 0u;
-              const uint32_t pr = h2_mul(e2m1x2_to_h2(cb), dup_e4m3_to_h2(sb));
-              const uint32_t ph = (c & 1u) ? (pr >> 16) : (pr & 0xFFFFu);
+              // padded channels read element K of both rows (zero): dX = 0
+              const uint32_t ph = *reinterpret_cast<const uint16_t*>(eb + 2u * cidx[u]);
               const float dq = __fmul_rn(__half2float(__ushort_as_half(static_cast<unsigned short>(ph))), st_w);
               x = __fsub_rn(__uint_as_float(h << 16), dq);
             } else {
@@ -1462,7 +1577,8 @@ struct WselPlan {
   bool ok;
 };
 // mode 0: bf16 weight rows; 1: NVFP4 weight rows; 2: the residual (bf16 X
-// rows and raw Q(X) rows, both double-buffered).
+// rows double-buffered, raw Q(X) rows and their f16 expansion one buffer
+// each).
 WselPlan wsel_plan(int64_t N, int64_t K, int32_t E, int64_t width, int mode) {
   const bool fp4 = mode == 1;
   // at most 54 KB of rows keeps four CTAs (the register limit) on an SM; the
@@ -1478,7 +1594,7 @@ WselPlan wsel_plan(int64_t N, int64_t K, int32_t E, int64_t width, int mode) {
   w.g.rowbytes = static_cast<uint32_t>(2 * K + 16);
   w.g.rawbytes = static_cast<uint32_t>((K / 2 + K / kBlock + 15) / 16 * 16);
   auto bytes = [&](int r) {
-    if (mode == 2) return static_cast<size_t>(2 * r) * (w.g.rowbytes + w.g.rawbytes);
+    if (mode == 2) return static_cast<size_t>(r) * (3 * w.g.rowbytes + w.g.rawbytes);
     return fp4 ? static_cast<size_t>(r) * (w.g.rowbytes + 2 * w.g.rawbytes)
                : static_cast<size_t>(2 * r) * w.g.rowbytes;
   };
