@@ -167,15 +167,15 @@ __device__ __forceinline__ float reduce_parts(const unsigned* parts, int n, uint
 //
 // The tile's rows are one 128-row chunk of the channel score, whose chunk sum
 // is defined as the fp64 sum of the chunk's |dX_ij| added one by one in row
-// order.  When the nonzero values of a column span at most 22 binades
-// (largest biased exponent minus smallest, a subnormal counted as exponent
-// 1), every partial sum of them is a multiple of the last bit of the
-// smallest and stays below 2^53 of those units, so every fp64 addition is
-// exact and any order of addition gives the row-order result: the tile then
-// adds the threads' 4-row sums through shared memory in two levels.  A
-// column whose values span more (a value far below the others; rare) is
-// summed again by one thread in row order, recomputing |dX| of each row from
-// X and the block's scale code with the same operations (so the same values).
+// order.  The threads write the tile's |dX| (fp32) to shared memory; then
+// four threads per column each take 32 rows.  When the nonzero values of a
+// column span at most 22 binades (largest biased exponent minus smallest, a
+// subnormal counted as exponent 1), every partial sum of them is a multiple
+// of the last bit of the smallest and stays below 2^53 of those units, so
+// every fp64 addition is exact and any order of addition gives the row-order
+// result: the four 32-row sums are added.  A column whose values span more
+// (a value far below the others; rare) is summed again by one thread over
+// the 128 rows in order.
 // ---------------------------------------------------------------------------
 constexpr int kSpanExact = 22;
 // tensor scales from 2^-55 up: every nonzero block decode scale
@@ -191,26 +191,6 @@ struct SelectOut {
   float* s_t;               // residual tensor scale
   unsigned* strips_done;    // zero on entry, left zero
 };
-
-// |dX| of one element x (fp32 value of its bf16) in a block with scale code
-// sb: the scalar form of the quantize pass's arithmetic (block_quotients,
-// the E2M1 conversion, DQ and the difference), rounded the same way.
-__device__ __noinline__ float residual_abs_one(float xv, uint32_t sb, const ScaleTable& T) {
-  const float sbv = T.sbv[sb], sdec = T.sdec[sb], y = T.rcp[sb];
-  float q;
-  if (sdec > 0.0f && y != 0.0f) {
-    const float q0 = __fmul_rn(xv, y);
-    const float r = __fmaf_rn(q0, -sdec, xv);
-    q = __fmaf_rn(r, y, q0);
-  } else {
-    q = sdec > 0.0f ? div_slow(fabsf(xv), sdec) : 0.0f;
-  }
-  q = __uint_as_float(__float_as_uint(q) | (__float_as_uint(xv) & 0x80000000u));
-  float v[8] = {q, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-  const uint32_t code = e2m1x8(v) & 15u;
-  const float p = __fmul_rn(e2m1_to_f32(code), sbv);
-  return fabsf(__fsub_rn(xv, __fmul_rn(p, T.s_t)));
-}
 
 // ---------------------------------------------------------------------------
 // The quantize + residual + score pass (persistent).  The grid is a few
@@ -228,32 +208,6 @@ __device__ __noinline__ float residual_abs_one(float xv, uint32_t sb, const Scal
 __device__ __forceinline__ void cp_async16_zfill(uint32_t dst, const void* src, bool valid) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0)
                : "memory");
-}
-
-// The row-order sums of the tile's wide columns (a column whose nonzero
-// |dX| span more than kSpanExact binades): the tile is still in its shared
-// buffer xt, so 128 threads recompute the column's |dX| from it and the
-// tile's block-scale codes sbt, and one thread adds them in row order.
-// Kept out of line like finish_strip (it never runs on most inputs).
-static __device__ __noinline__ void wide_columns(const uint16_t (*xt)[kQCols], const uint8_t (*sbt)[kQCols / kBlock],
-                                                 const uint8_t* s_wide, float* s_dxcol, const ScaleTable& T,
-                                                 int64_t tile, int64_t row_tiles, int64_t col0, int64_t K,
-                                                 double* part_sum) {
-  const int t = threadIdx.x;
-  for (int c = 0; c < kQCols; ++c) {
-    if (!s_wide[c]) continue;                      // uniform: every thread reads the same flag
-    if (t < kTileRows) {
-      const float xv = bf16_bits_to_f32(xt[t][c]);   // rows past the end were zero-filled
-      s_dxcol[t] = residual_abs_one(xv, sbt[t][c >> 4], T);
-    }
-    __syncthreads();
-    if (t == 0) {
-      double chain = 0.0;
-      for (int r = 0; r < kTileRows; ++r) chain += static_cast<double>(s_dxcol[r]);
-      if (NV_IDX(tile < row_tiles && col0 + c < K)) part_sum[tile * K + col0 + c] = chain;
-    }
-    __syncthreads();
-  }
 }
 
 // The last CTA to finish a column strip of a row group: the chunk-order
@@ -333,15 +287,16 @@ quant_score2_kernel(const uint16_t* __restrict__ x, int64_t K, int64_t ldx, RowG
   constexpr int kGroups = kTileRows / 4;
   extern __shared__ __align__(16) uint8_t q2_dyn[];                // 2 x 16 KB tile buffers
   uint16_t (*xbuf)[kTileRows][kQCols] = reinterpret_cast<uint16_t (*)[kTileRows][kQCols]>(q2_dyn);
-  __shared__ __align__(16) double gsum[kGroups][kQCols];          // also tail staging
-  __shared__ __align__(16) float gmax[kGroups][kQCols];
-  __shared__ __align__(16) uint32_t gmin[kGroups][kQCols];
+  // 32 KB: with scores the tile's |dX| (fp32 [128][64]); without, the
+  // per-thread column maxima [32][64]; after a strip the staging of its
+  // partials (finish_strip)
+  __shared__ __align__(16) uint8_t red[kTileRows * kQCols * 4];
+  float (*dxs)[kQCols] = reinterpret_cast<float (*)[kQCols]>(red);
+  float (*gmax)[kQCols] = reinterpret_cast<float (*)[kQCols]>(red);
   __shared__ __align__(16) double qsum[4][kQCols];
   __shared__ __align__(16) float qmax[4][kQCols];
   __shared__ __align__(16) uint32_t qmin[4][kQCols];
   __shared__ __align__(16) uint8_t s_sb[2][kTileRows][kQCols / kBlock];
-  __shared__ float s_dxcol[kTileRows];             // |dX| of one column for the row-order sum
-  __shared__ uint8_t s_wide[kQCols];
   __shared__ uint32_t wscratch[kQThreads / 32];
   __shared__ bool s_last;
   __shared__ ScaleTable T;
@@ -404,11 +359,9 @@ quant_score2_kernel(const uint16_t* __restrict__ x, int64_t K, int64_t ldx, RowG
     if (strip == 0 && t == 0 && (g.off == nullptr ? tile == 0 : tile == g.tile_start[ti.e]))
       tensor_scale[ti.e] = s_t;
     uint8_t* code_base = codes + tile * kTileRows * (K / 2) + col / 2;
-    double acc[8];
     float mx[8];
-    uint32_t mn[8];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) { acc[j] = 0.0; mx[j] = 0.0f; mn[j] = 0xFFFFFFFFu; }
+    for (int j = 0; j < 8; ++j) mx[j] = 0.0f;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const int r = 4 * grp + i;
@@ -455,6 +408,7 @@ quant_score2_kernel(const uint16_t* __restrict__ x, int64_t K, int64_t ldx, RowG
         sbv = bq.sbv;
       }
       const uint64_t sbv2 = f2_pack(sbv, sbv);
+      float dv[8];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         // dX = RN(x - RN(p s_t)) with p = E2M1dec E4M3dec exact (scalar
@@ -464,27 +418,24 @@ quant_score2_kernel(const uint16_t* __restrict__ x, int64_t K, int64_t ldx, RowG
         f2_unpack(x2[j], x0, x1);
         const float d0 = fabsf(__fsub_rn(x0, __fmul_rn(p0, s_t)));
         const float d1 = fabsf(__fsub_rn(x1, __fmul_rn(p1, s_t)));
-        if (SCORES) {
-          acc[2 * j] += static_cast<double>(d0);
-          acc[2 * j + 1] += static_cast<double>(d1);
-          mn[2 * j] = min(mn[2 * j], __float_as_uint(d0) - 1u);
-          mn[2 * j + 1] = min(mn[2 * j + 1], __float_as_uint(d1) - 1u);
+        dv[2 * j] = d0;
+        dv[2 * j + 1] = d1;
+        if (!SCORES) {
+          mx[2 * j] = fmaxf(mx[2 * j], d0);
+          mx[2 * j + 1] = fmaxf(mx[2 * j + 1], d1);
         }
-        mx[2 * j] = fmaxf(mx[2 * j], d0);
-        mx[2 * j + 1] = fmaxf(mx[2 * j + 1], d1);
+      }
+      if (SCORES) {
+        // columns 8 cg + 4 h + e sit at position 32 h + 4 cg + e of the row:
+        // each 16-byte store of 8 threads covers 128 contiguous bytes
+        *reinterpret_cast<float4*>(&dxs[r][4 * cg]) = make_float4(dv[0], dv[1], dv[2], dv[3]);
+        *reinterpret_cast<float4*>(&dxs[r][32 + 4 * cg]) = make_float4(dv[4], dv[5], dv[6], dv[7]);
       }
       if (prow < codes_rows && NV_IDX(col + 8 <= K))
         *reinterpret_cast<uint32_t*>(code_base + static_cast<uint32_t>(r) * static_cast<uint32_t>(K / 2)) = packed;
       if ((cg & 1) == 0) s_sb[b][r][cg >> 1] = static_cast<uint8_t>(sb);
     }
-    if (part_max != nullptr) {
-      if (SCORES) {
-#pragma unroll
-        for (int j = 0; j < 8; j += 2)
-          *reinterpret_cast<double2*>(&gsum[grp][8 * cg + j]) = make_double2(acc[j], acc[j + 1]);
-        *reinterpret_cast<uint4*>(&gmin[grp][8 * cg]) = make_uint4(mn[0], mn[1], mn[2], mn[3]);
-        *reinterpret_cast<uint4*>(&gmin[grp][8 * cg + 4]) = make_uint4(mn[4], mn[5], mn[6], mn[7]);
-      }
+    if (!SCORES && part_max != nullptr) {
       *reinterpret_cast<float4*>(&gmax[grp][8 * cg]) = make_float4(mx[0], mx[1], mx[2], mx[3]);
       *reinterpret_cast<float4*>(&gmax[grp][8 * cg + 4]) = make_float4(mx[4], mx[5], mx[6], mx[7]);
     }
@@ -506,17 +457,27 @@ quant_score2_kernel(const uint16_t* __restrict__ x, int64_t K, int64_t ldx, RowG
     }
     if (part_max == nullptr) continue;
     {
-      const int c = t & (kQCols - 1), q4 = t >> 6;
+      // column c, rows 32 q4 .. 32 q4 + 31 (scores: the fp64 sum, the
+      // smallest nonzero |dX| as bits - 1 and the maximum; else the maximum
+      // of the per-thread maxima)
+      int c = t & (kQCols - 1);
+      const int q4 = t >> 6;
       double sum = 0.0;
       float m = 0.0f;
       uint32_t lo = 0xFFFFFFFFu;
-#pragma unroll
-      for (int gi = 8 * q4; gi < 8 * q4 + 8; ++gi) {
-        if (SCORES) {
-          sum += gsum[gi][c];
-          lo = min(lo, gmin[gi][c]);
+      if (SCORES) {
+        const int pos = c;                         // this thread reads position pos of the rows
+        c = 8 * ((pos & 31) >> 2) + 4 * (pos >> 5) + (pos & 3);   // ... which holds column c
+#pragma unroll 8
+        for (int r = 32 * q4; r < 32 * q4 + 32; ++r) {
+          const float v = dxs[r][pos];
+          sum += static_cast<double>(v);
+          lo = min(lo, __float_as_uint(v) - 1u);
+          m = fmaxf(m, v);
         }
-        m = fmaxf(m, gmax[gi][c]);
+      } else {
+#pragma unroll
+        for (int gi = 8 * q4; gi < 8 * q4 + 8; ++gi) m = fmaxf(m, gmax[gi][c]);
       }
       if (SCORES) {
         qsum[q4][c] = sum;
@@ -543,19 +504,23 @@ quant_score2_kernel(const uint16_t* __restrict__ x, int64_t K, int64_t ldx, RowG
         const int e_lo = max(static_cast<int>((lo + 1u) >> 23), 1);
         wide = e_hi - e_lo > kSpanExact;
       }
-      if (SCORES) s_wide[t] = static_cast<uint8_t>(wide);
       if (NV_IDX(tile < row_tiles && col0 + t < K)) {
         if (SCORES && !wide) part_sum[tile * K + col0 + t] = part;
         part_max[tile * K + col0 + t] = m;
       }
     }
     // columns whose values span more than kSpanExact binades: the row-order
-    // sum itself.  The tile is still in this parity's buffer (its next use
-    // is the prefetch two tiles ahead, issued after this point by every
-    // thread), so 128 threads recompute the column's |dX| from it and the
-    // tile's block-scale codes, and one thread adds them in row order.
-    if (SCORES && __syncthreads_or(wide))
-      wide_columns(xbuf[b], s_sb[b], s_wide, s_dxcol, T, tile, row_tiles, col0, K, part_sum);
+    // sum itself, by the column's own thread from the |dX| tile (rows past
+    // the end hold 0), then a barrier before the next tile overwrites it
+    if (SCORES && __syncthreads_or(wide)) {
+      if (wide) {
+        const int pos = 32 * ((t >> 2) & 1) + 4 * (t >> 3) + (t & 3);   // column t's position
+        double chain = 0.0;
+        for (int r = 0; r < kTileRows; ++r) chain += static_cast<double>(dxs[r][pos]);
+        if (NV_IDX(tile < row_tiles && col0 + t < K)) part_sum[tile * K + col0 + t] = chain;
+      }
+      __syncthreads();
+    }
     if (strip_count == nullptr) continue;
     __syncthreads();
     const int64_t t0 = g.off == nullptr ? 0 : g.tile_start[ti.e];
@@ -568,8 +533,9 @@ quant_score2_kernel(const uint16_t* __restrict__ x, int64_t K, int64_t ldx, RowG
     }
     __syncthreads();
     if (!s_last) continue;
-    finish_strip<SCORES>(t0, t1, counter, &gsum[0][0], &gmax[0][0], part_sum, part_max, K, col0, score, colamax,
-                         ti.e, g.E, sel_out, n_strips, q2_dyn, &s_last);
+    finish_strip<SCORES>(t0, t1, counter, reinterpret_cast<double*>(red),
+                         reinterpret_cast<float*>(red + kGroups * kQCols * sizeof(double)), part_sum, part_max, K,
+                         col0, score, colamax, ti.e, g.E, sel_out, n_strips, q2_dyn, &s_last);
   }
   cp_async_wait<0>();
 }
