@@ -197,15 +197,20 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------- profile traffic
-KERNEL_SOURCES = ("common.cuh", "gemm.cu", "kernels.h", "quant.cu", "select.cu")
+KERNEL_SOURCES = ("common.cuh", "gemm.cu", "kernels.h", "quant.cu", "select.cu", "topk.cuh")
+# the files that hold each call's kernels and their launch code (a recorded
+# DRAM figure stays valid while these are unchanged)
+CALL_SOURCES = {"gemm": ("common.cuh", "gemm.cu", "kernels.h"),
+                "gemm_plain": ("common.cuh", "gemm.cu", "kernels.h")}
 
 
-def kernel_sources_hash():
-    """sha256 (first 16 hex digits) over the files that hold the kernels and
-    their launch code; the host-only ABI layer is not part of it."""
+def kernel_sources_hash(call=None):
+    """sha256 (first 16 hex digits) over the files that hold the kernels of
+    `call` (all kernel files when None) and their launch code; the host-only
+    ABI layer is not part of it."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "precision_rl_rollout_nvfp4_b200", "csrc")
-    for name in KERNEL_SOURCES:
+    for name in CALL_SOURCES.get(call, KERNEL_SOURCES):
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
@@ -217,7 +222,7 @@ def profiled_traffic(kernel, workload):
     path = os.path.join(ROOT, "profiles", "dram_traffic.md")
     if not os.path.exists(path):
         return None
-    src = kernel_sources_hash()
+    src = kernel_sources_hash(kernel)
     with open(path) as f:
         for line in f:
             cells = [c.strip() for c in line.strip().strip("|").split("|")]
@@ -631,7 +636,7 @@ def run_ours(args, rank, world, local_rank):
     dur = med[dominant] * 1e-3
     traffic = profiled_traffic(dominant, args.workload)
     traffic_source = (f"profiles/dram_traffic.md, ncu dram__bytes_read.sum + dram__bytes_write.sum per launch, "
-                      f"kernel sources sha256 {kernel_sources_hash()}") if traffic is not None else None
+                      f"kernel sources sha256 {kernel_sources_hash(dominant)}") if traffic is not None else None
     if d["bound"] == "tensor":
         achieved = d["flops"] / dur / 1e12
         roof = {"kernel": dominant, "bound": "tensor", "achieved": round(achieved, 1),
