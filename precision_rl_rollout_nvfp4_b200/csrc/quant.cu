@@ -178,6 +178,12 @@ __device__ __forceinline__ float reduce_parts(const unsigned* parts, int n, uint
 // the 128 rows in order.
 // ---------------------------------------------------------------------------
 constexpr int kSpanExact = 22;
+// strips one CTA may complete: the in-kernel strip totals serve dense X
+// (one group), whose strips all complete in the last row tile, where a CTA
+// takes at most ceil(K/64 / grid) <= 3 tiles (K <= 65472, grid >= min(work,
+// 3 SMs)); a completion beyond the list would be dropped, never written
+// out of bounds
+constexpr int kMaxDone = 64;
 // tensor scales from 2^-55 up: every nonzero block decode scale
 // RN(E4M3dec(sb) s_t) >= 2^-9 2^-55 = 2^-64, so its reciprocal table entry
 // serves the quotient (Markstein) and no division fallback is needed
@@ -299,6 +305,11 @@ quant_score2_kernel(const uint16_t* __restrict__ x, int64_t K, int64_t ldx, RowG
   __shared__ __align__(16) uint8_t s_sb[2][kTileRows][kQCols / kBlock];
   __shared__ uint32_t wscratch[kQThreads / 32];
   __shared__ bool s_last;
+  // (group, strip) of the strips this CTA completed: their chunk-order
+  // totals are formed after the tile loop (a call inside it would make the
+  // loop spill its live values around the call)
+  __shared__ int2 s_done[kMaxDone];
+  __shared__ int s_ndone;
   __shared__ ScaleTable T;
   __shared__ float4 T4[128];                       // {sbv, sdec, -rcp} per scale code
   const int t = threadIdx.x, cg = t & 7, grp = t >> 3;
@@ -331,6 +342,7 @@ quant_score2_kernel(const uint16_t* __restrict__ x, int64_t K, int64_t ldx, RowG
 
   int64_t idx = blockIdx.x;
   if (idx < total) prefetch(idx, 0);
+  if (t == 0) s_ndone = 0;                         // first read after the table build's barriers
   for (int it = 0; idx < total; ++it, idx += gridDim.x) {
     const int b = it & 1;
     const int64_t nidx = idx + gridDim.x;
@@ -529,13 +541,23 @@ quant_score2_kernel(const uint16_t* __restrict__ x, int64_t K, int64_t ldx, RowG
     if (t == 0) {
       __threadfence();
       const unsigned prev = atomicAdd(counter, 1u);
-      s_last = prev == static_cast<unsigned>(t1 - t0 - 1);
+      if (prev == static_cast<unsigned>(t1 - t0 - 1) && s_ndone < kMaxDone)
+        s_done[s_ndone++] = make_int2(ti.e, static_cast<int>(strip));
     }
-    __syncthreads();
-    if (!s_last) continue;
-    finish_strip<SCORES>(t0, t1, counter, reinterpret_cast<double*>(red),
+  }
+  // the strips this CTA completed, after its last tile (with a selection
+  // fused, the CTA that completes the last strip overall also selects)
+  __syncthreads();
+  const int nd = strip_count != nullptr ? s_ndone : 0;
+  for (int i = 0; i < nd; ++i) {
+    const int e = s_done[i].x;
+    const int64_t strip = s_done[i].y;
+    const int64_t t0 = g.off == nullptr ? 0 : g.tile_start[e];
+    const int64_t t1 = g.off == nullptr ? row_tiles : g.tile_start[e + 1];
+    finish_strip<SCORES>(t0, t1, strip_count + static_cast<int64_t>(e) * n_strips + strip,
+                         reinterpret_cast<double*>(red),
                          reinterpret_cast<float*>(red + kGroups * kQCols * sizeof(double)), part_sum, part_max, K,
-                         col0, score, colamax, ti.e, g.E, sel_out, n_strips, q2_dyn, &s_last);
+                         strip * kQCols, score, colamax, e, g.E, sel_out, n_strips, q2_dyn, &s_last);
   }
   cp_async_wait<0>();
 }
