@@ -811,7 +811,7 @@ __device__ __forceinline__ void gather_quant_body(const GatherArgs& A, GatherSme
 }
 
 template <int MODE>
-__global__ void __launch_bounds__(kGThreads) gather_quant_kernel(GatherArgs A) {
+__global__ void __launch_bounds__(kGThreads, 4) gather_quant_kernel(GatherArgs A) {
   pdl_wait();
   pdl_launch_dependents();
   __shared__ GatherSmem sm;
@@ -822,7 +822,7 @@ __global__ void __launch_bounds__(kGThreads) gather_quant_kernel(GatherArgs A) {
 // residual's tiles (MODE 1), the others the weight's (MODE 0, or 2 from the
 // NVFP4 weight).
 template <int WMODE>
-__global__ void __launch_bounds__(kGThreads) gather_pair_kernel(GatherArgs R, GatherArgs W, int n_res) {
+__global__ void __launch_bounds__(kGThreads, 4) gather_pair_kernel(GatherArgs R, GatherArgs W, int n_res) {
   pdl_wait();
   pdl_launch_dependents();
   __shared__ GatherSmem sm;
