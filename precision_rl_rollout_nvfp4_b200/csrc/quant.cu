@@ -1239,37 +1239,33 @@ __global__ void sel_tensor_scale_kernel(const float* __restrict__ colamax, int64
 // ---------------------------------------------------------------------------
 // weight fake quantization (W4A16 trainer side)
 // ---------------------------------------------------------------------------
-// CTA: 128 rows x 64 columns of one matrix; thread t: columns 8 (t & 7), rows
-// t/8 + 32 i, i = 0..3 (all four 16-byte loads issued first).
-// grid = (K/64, ceil(N/128), batch).
-__global__ void __launch_bounds__(kQThreads)
-weight_qdq_kernel(const uint16_t* w, int64_t N, int64_t K, int64_t ldw,
-                  const unsigned* __restrict__ amax_parts, int n_parts,
-                  uint16_t* w_out,   // w_out may alias w
-                  uint8_t* __restrict__ codes, uint8_t* __restrict__ scales, int layout,
-                  float* __restrict__ tensor_scale, unsigned* __restrict__ colamax_bits) {
-  pdl_wait();
-  pdl_launch_dependents();
-  const int64_t b = blockIdx.z;
-  const int t = threadIdx.x, cg = t & 7, rr = t >> 3;
-  const int64_t col = static_cast<int64_t>(blockIdx.x) * 64 + 8 * cg;
-  uint32_t cmax[4] = {0, 0, 0, 0};               // |bf16| bits of columns 2j, 2j+1
-  uint4 raw[4];
+// A tile is 128 rows x 64 columns of one matrix; thread t: columns 8 (t & 7),
+// rows t/8 + 32 i, i = 0..3.
+
+// The tile's four 16-byte rows of this thread (zero past row N).
+__device__ __forceinline__ void qdq_tile_load(const uint16_t* w, int64_t N, int64_t ldw, int64_t b, int64_t ty,
+                                              int64_t col, int rr, uint4* raw) {
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const int64_t n = static_cast<int64_t>(blockIdx.y) * 128 + rr + 32 * i;
+    const int64_t n = ty * 128 + rr + 32 * i;
     // coherent load: w may alias w_out
     raw[i] = n < N ? *reinterpret_cast<const uint4*>(w + (b * N + n) * ldw + col) : make_uint4(0, 0, 0, 0);
   }
-  __shared__ uint32_t wscratch[kQThreads / 32];
-  const float s_t = __fdiv_rn(reduce_parts(amax_parts + b * n_parts, n_parts, wscratch), kTensorScaleDiv);
-  if (tensor_scale && blockIdx.x == 0 && blockIdx.y == 0 && t == 0) tensor_scale[b] = s_t;
-  __shared__ ScaleTable T;
-  build_scale_table(T, s_t, t);
-  __syncthreads();                               // table ready
+}
+
+// W' = DQ(Q(W)) of the tile (and its codes, scales and column maxima) from
+// the loaded rows; every thread of the CTA calls it (one barrier inside when
+// column maxima are kept).
+__device__ __forceinline__ void qdq_tile_store(const uint4* raw, int64_t N, int64_t K, int64_t ldw, int64_t b,
+                                               int64_t ty, int64_t tx, float s_t, const ScaleTable& T,
+                                               uint16_t* w_out, uint8_t* codes, uint8_t* scales, int layout,
+                                               unsigned* colamax_bits, uint32_t (*cm)[65]) {
+  const int t = threadIdx.x, cg = t & 7, rr = t >> 3;
+  const int64_t col = tx * 64 + 8 * cg;
+  uint32_t cmax[4] = {0, 0, 0, 0};               // |bf16| bits of columns 2j, 2j+1
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const int64_t n = static_cast<int64_t>(blockIdx.y) * 128 + rr + 32 * i;
+    const int64_t n = ty * 128 + rr + 32 * i;
     const bool live = n < N;
     const int64_t off = (b * N + n) * ldw + col;
     const uint32_t wv[4] = {raw[i].x, raw[i].y, raw[i].z, raw[i].w};
@@ -1309,7 +1305,6 @@ weight_qdq_kernel(const uint16_t* w, int64_t N, int64_t K, int64_t ldw,
       scales[scale_offset(qrow, col / kBlock, K, layout)] = static_cast<uint8_t>(bs.sb);
   }
   if (colamax_bits == nullptr) return;
-  __shared__ uint32_t cm[32][65];
 #pragma unroll
   for (int j = 0; j < 4; ++j) {                  // |bf16| bits -> fp32 bits
     cm[rr][8 * cg + 2 * j] = (cmax[j] & 0xFFFFu) << 16;
@@ -1319,8 +1314,34 @@ weight_qdq_kernel(const uint16_t* w, int64_t N, int64_t K, int64_t ldw,
   if (t < 64) {
     uint32_t m = 0;
     for (int r = 0; r < 32; ++r) m = max(m, cm[r][t]);
-    if (m) atomicMax(colamax_bits + b * K + blockIdx.x * 64 + t, m);
+    if (m) atomicMax(colamax_bits + b * K + tx * 64 + t, m);
   }
+  __syncthreads();                               // cm is free again
+}
+
+// One tile per CTA, the tensor amax from amax_partial's partial maxima.
+// grid = (K/64, ceil(N/128), batch).
+__global__ void __launch_bounds__(kQThreads)
+weight_qdq_kernel(const uint16_t* w, int64_t N, int64_t K, int64_t ldw,
+                  const unsigned* __restrict__ amax_parts, int n_parts,
+                  uint16_t* w_out,   // w_out may alias w
+                  uint8_t* __restrict__ codes, uint8_t* __restrict__ scales, int layout,
+                  float* __restrict__ tensor_scale, unsigned* __restrict__ colamax_bits) {
+  pdl_wait();
+  pdl_launch_dependents();
+  const int64_t b = blockIdx.z;
+  const int t = threadIdx.x;
+  uint4 raw[4];
+  qdq_tile_load(w, N, ldw, b, blockIdx.y, static_cast<int64_t>(blockIdx.x) * 64 + 8 * (t & 7), t >> 3, raw);
+  __shared__ uint32_t wscratch[kQThreads / 32];
+  const float s_t = __fdiv_rn(reduce_parts(amax_parts + b * n_parts, n_parts, wscratch), kTensorScaleDiv);
+  if (tensor_scale && blockIdx.x == 0 && blockIdx.y == 0 && t == 0) tensor_scale[b] = s_t;
+  __shared__ ScaleTable T;
+  __shared__ uint32_t cm[32][65];
+  build_scale_table(T, s_t, t);
+  __syncthreads();                               // table ready
+  qdq_tile_store(raw, N, K, ldw, b, blockIdx.y, blockIdx.x, s_t, T, w_out, codes, scales, layout,
+                 colamax_bits, cm);
 }
 
 // ---------------------------------------------------------------------------

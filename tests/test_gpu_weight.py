@@ -12,17 +12,18 @@ from tests.layout import unpack_codes, untile_scales
 pytestmark = pytest.mark.gpu
 
 
-def _check_qdq(b, w, layout=1):
+def _check_qdq(b, w, layout=1, experts=None):
     wd = w.cuda()
     batch, N, K = (1, *w.shape) if w.dim() == 2 else w.shape
     w_out, qw, colamax = b.weight_qdq(wd, layout=layout)
     torch.cuda.synchronize()
+    assert b.stream_status() == 0
     wb = bits(w).reshape(batch, N, K)
     got_out = bits(w_out).reshape(batch, N, K)
     codes = unpack_codes(qw.codes.cpu().numpy())
     sc = qw.scales.cpu().numpy()
     scales = untile_scales(sc, batch * N, K) if layout == 1 else sc[: batch * N * K // 16].reshape(batch * N, K // 16)
-    for e in range(batch):
+    for e in (range(batch) if experts is None else experts):
         ref = oracle.weight_qdq(wb[e])
         assert np.array_equal(got_out[e], ref["w_out"])
         assert np.array_equal(codes[e * N:(e + 1) * N], ref["codes"])
@@ -41,6 +42,42 @@ def test_weight_qdq_batched_experts():
     b = need_gpu()
     _check_qdq(b, S.weights(256, 128, seed=3, batch=5))
     _check_qdq(b, S.weights(100, 64, seed=4, batch=3), layout=0)
+
+
+def test_weight_qdq_stacked_clusters():
+    """Stacks of several matrices (one launch pair for the whole stack):
+    ragged row counts, one and several column tiles, both scale layouts."""
+    b = need_gpu()
+    _check_qdq(b, S.weights(100, 64, seed=5, batch=12))
+    _check_qdq(b, S.weights(300, 320, seed=6, batch=9), layout=0)
+    _check_qdq(b, S.weights(128, 1024, seed=8, batch=40))
+
+
+def test_weight_qdq_stacked_clusters_in_place():
+    b = need_gpu()
+    w = S.weights(200, 256, seed=9, batch=10)
+    wb = bits(w).reshape(10, 200, 256)
+    wd = w.cuda()
+    b.weight_qdq(wd, want_q=False, want_colamax=False, out=wd)
+    torch.cuda.synchronize()
+    got = bits(wd).reshape(10, 200, 256)
+    for e in range(10):
+        assert np.array_equal(got[e], oracle.weight_qdq(wb[e])["w_out"])
+
+
+def test_weight_qdq_expert_stack_full_size():
+    """The prefill step's trainer-side QDQ shape, 64 experts x 1024 x 2048
+    (the two passes over the whole stack): four experts checked
+    against the oracle in full, every tensor scale against its amax."""
+    b = need_gpu()
+    w = S.weights(1024, 2048, seed=11, batch=64)
+    _check_qdq(b, w, experts=[0, 21, 42, 63])
+    _, qw, _ = b.weight_qdq(w.cuda())
+    torch.cuda.synchronize()
+    wf = w.float().numpy().reshape(64, 1024 * 2048)     # bf16 values, exact in fp32
+    st = qw.tensor_scale.cpu().numpy()
+    for e in range(64):
+        assert np.float32(st[e]) == oracle.nvfp4.tensor_scale(oracle.nvfp4.amax(wf[e]))
 
 
 def test_weight_qdq_in_place():
