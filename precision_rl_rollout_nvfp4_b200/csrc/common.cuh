@@ -335,6 +335,11 @@ struct Pow2Apply {
   __device__ __forceinline__ float operator()(float t) const { return __fmul_rn(__fmul_rn(t, p1), p2); }
 };
 
+// True when m 2^e (m in [0.25, 1)) is a normal fp32: then RN(t (m 2^e)) =
+// RN(RN(t m) 2^e) for every t whose result is normal (the power-of-two step
+// is exact there), so the output scale is one multiply.
+__device__ __forceinline__ bool scale_is_normal(int e) { return e >= -124 && e <= 127; }
+
 __device__ __forceinline__ Pow2Apply pow2_apply(int e) {
   Pow2Apply a;
   if (e > 127) {

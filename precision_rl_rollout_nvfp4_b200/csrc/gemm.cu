@@ -369,15 +369,25 @@ __device__ __forceinline__ void gemm1_body(const CUtensorMap& tmA0, const CUtens
       const int E = a0.m != 0.0f ? a0.e : a1.e;
       const float c0 = a0.m, c1 = a1.m != 0.0f ? ldexpf(a1.m, a1.e - E) : 0.0f;
       const Pow2Apply out = pow2_apply(E);
+      // with both segment scales normal the power-of-two step folds into
+      // them (exact scaling, the same roundings for normal results)
+      const bool one = scale_is_normal(E) && (a1.m == 0.0f || scale_is_normal(a1.e));
+      const float c0n = one ? ldexpf(c0, E) : 0.0f, c1n = one ? ldexpf(c1, E) : 0.0f;
 #pragma unroll
       for (int c = 0; c < BN / 32; ++c) {
         float v[32], u[32];
         tmem_ld32(trow + ACC0_COL + 32 * c, v);
         if (nseg > 1) tmem_ld32(trow + ACC1_COL + 32 * c, u);
         tmem_ld_wait();
-        if (nseg > 1) {
+        if (nseg > 1 && one) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = __fadd_rn(__fmul_rn(c0n, v[i]), __fmul_rn(c1n, u[i]));
+        } else if (nseg > 1) {
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] = out(__fadd_rn(__fmul_rn(c0, v[i]), __fmul_rn(c1, u[i])));
+        } else if (one) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(c0n, v[i]);
         } else {
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] = out(__fmul_rn(c0, v[i]));
@@ -841,6 +851,19 @@ __device__ __forceinline__ void gemm2_body(const CUtensorMap& tmA0, const CUtens
       const float ratio = (ap.m != 0.0f && ar.m != 0.0f) ? ldexpf(__fdiv_rn(ar.m, ap.m), ar.e - ap.e) : 0.0f;
       const float fin = ap.m;
       const Pow2Apply out = pow2_apply(ap.e);
+      // m 2^e as one fp32 multiplier when it is normal (see scale_is_normal)
+      const bool one = scale_is_normal(ap.e);
+      const float fin1 = one ? ldexpf(fin, ap.e) : 0.0f;
+      // Y of 32 accumulator values in place
+      auto scale32 = [&](float* v) {
+        if (one) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(fin1, v[i]);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = out(__fmul_rn(fin, v[i]));
+        }
+      };
       bool ok = true;
       if (has_res) {
         if (lane == 0) ok = mbar_wait(res_full, res_phase, p.err);
@@ -901,12 +924,11 @@ __device__ __forceinline__ void gemm2_body(const CUtensorMap& tmA0, const CUtens
             float v[32];
             tmem_ld32(trow + ACC2_COL + 128 * h + 32 * c, v);
             tmem_ld_wait();
+            scale32(v);
             uint32_t w[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const float lo = out(__fmul_rn(fin, v[2 * i])), hi = out(__fmul_rn(fin, v[2 * i + 1]));
-              asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(w[i]) : "f"(hi), "f"(lo));
-            }
+            for (int i = 0; i < 16; ++i)
+              asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(w[i]) : "f"(v[2 * i + 1]), "f"(v[2 * i]));
             if (h == 0) {
 #pragma unroll
               for (int i = 0; i < 16; i += 4)
@@ -936,11 +958,10 @@ __device__ __forceinline__ void gemm2_body(const CUtensorMap& tmA0, const CUtens
             float v[32];
             tmem_ld32(trow + ACC2_COL + 128 * h + 32 * c, v);
             tmem_ld_wait();
+            scale32(v);
 #pragma unroll
             for (int i = 0; i < 32; i += 4)
-              *reinterpret_cast<float4*>(stg_row + (32 * c + i) * 4) =
-                  make_float4(out(__fmul_rn(fin, v[i])), out(__fmul_rn(fin, v[i + 1])),
-                              out(__fmul_rn(fin, v[i + 2])), out(__fmul_rn(fin, v[i + 3])));
+              *reinterpret_cast<float4*>(stg_row + (32 * c + i) * 4) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
           }
           if (h == 1) {
             tc_fence_before();
