@@ -352,6 +352,12 @@ __device__ __forceinline__ void gemm1_body(const CUtensorMap& tmA0, const CUtens
     uint8_t* stg_warp = sOut + (32 * q) * STG_STRIDE;
     uint8_t* stg_row = stg_warp + lane * STG_STRIDE;
     uint32_t acc_phase = 0;
+    // the output scale factors depend on the row group only: formed when it
+    // changes (once for a dense product), not per tile
+    int cur_e = -1;
+    float c0 = 0.0f, c1 = 0.0f, c0n = 0.0f, c1n = 0.0f;
+    Pow2Apply out{1.0f, 1.0f};
+    bool one = true;
     for (int64_t tile = blockIdx.x; tile < total; tile += gridDim.x) {
       bool ok = true;
       if (lane == 0) ok = mbar_wait(tmem_full, acc_phase, p.err);
@@ -360,19 +366,24 @@ __device__ __forceinline__ void gemm1_body(const CUtensorMap& tmA0, const CUtens
       tc_fence_after();
       const int64_t mt = tile / p.n_tiles, nt = tile % p.n_tiles;
       const TileInfo ti = tile_info(p.g, mt);
-      // Y = a0 acc0 + a1 acc1 with a_s = s_tA,s s_tB,s = m_s 2^e_s: both
-      // segments in the units 2^E of the first nonzero one, then one
-      // power-of-two step (see Pow2Apply)
-      // (MXFP8 operands carry no tensor scale: the scale product is 1)
-      const ScaleProduct a0 = FP8 ? ScaleProduct{0.5f, 1} : scale_product(p.sta[0][ti.e], p.stb[0][ti.e]);
-      const ScaleProduct a1 = nseg > 1 ? scale_product(p.sta[1][ti.e], p.stb[1][ti.e]) : ScaleProduct{0.0f, 0};
-      const int E = a0.m != 0.0f ? a0.e : a1.e;
-      const float c0 = a0.m, c1 = a1.m != 0.0f ? ldexpf(a1.m, a1.e - E) : 0.0f;
-      const Pow2Apply out = pow2_apply(E);
-      // with both segment scales normal the power-of-two step folds into
-      // them (exact scaling, the same roundings for normal results)
-      const bool one = scale_is_normal(E) && (a1.m == 0.0f || scale_is_normal(a1.e));
-      const float c0n = one ? ldexpf(c0, E) : 0.0f, c1n = one ? ldexpf(c1, E) : 0.0f;
+      if (ti.e != cur_e) {
+        // Y = a0 acc0 + a1 acc1 with a_s = s_tA,s s_tB,s = m_s 2^e_s: both
+        // segments in the units 2^E of the first nonzero one, then one
+        // power-of-two step (see Pow2Apply)
+        // (MXFP8 operands carry no tensor scale: the scale product is 1)
+        const ScaleProduct a0 = FP8 ? ScaleProduct{0.5f, 1} : scale_product(p.sta[0][ti.e], p.stb[0][ti.e]);
+        const ScaleProduct a1 = nseg > 1 ? scale_product(p.sta[1][ti.e], p.stb[1][ti.e]) : ScaleProduct{0.0f, 0};
+        const int E = a0.m != 0.0f ? a0.e : a1.e;
+        c0 = a0.m;
+        c1 = a1.m != 0.0f ? ldexpf(a1.m, a1.e - E) : 0.0f;
+        out = pow2_apply(E);
+        // with both segment scales normal the power-of-two step folds into
+        // them (exact scaling, the same roundings for normal results)
+        one = scale_is_normal(E) && (a1.m == 0.0f || scale_is_normal(a1.e));
+        c0n = one ? ldexpf(c0, E) : 0.0f;
+        c1n = one ? ldexpf(c1, E) : 0.0f;
+        cur_e = ti.e;
+      }
 #pragma unroll
       for (int c = 0; c < BN / 32; ++c) {
         float v[32], u[32];
@@ -838,22 +849,31 @@ __device__ __forceinline__ void gemm2_body(const CUtensorMap& tmA0, const CUtens
     const uint32_t lead_tmem_empty = peer_addr(tmem_empty, 0);
     const uint32_t lead_res_done = peer_addr(res_done, 0);
     uint32_t acc_phase = 0, res_phase = 0;
+    // the output scale factors depend on the row group only: formed when it
+    // changes (once for a dense product), not per tile
+    int cur_e = -1;
+    float ratio = 0.0f, fin = 0.0f, fin1 = 0.0f;
+    Pow2Apply out{1.0f, 1.0f};
+    bool one = true;
     for (int tile = pair; tile < total; tile += npairs) {
       const int mt = tile / p.n_tiles, nt = tile % p.n_tiles;
       const PairRows pr = pair_rows(p, mt, rank);
-      // the residual is scaled to the plain segment's units (ratio =
-      // a_res / a_plain with a = s_tA s_tB = m 2^e), then Y = a_plain acc,
-      // applied as RN(acc m) and one power-of-two step (see Pow2Apply).  A
-      // zero plain scale means an all-zero X or W, whose residual and W_sel
-      // are zero as well: Y = 0.
-      const ScaleProduct ap = FP8 ? ScaleProduct{0.5f, 1} : scale_product(p.sta[1][pr.e], p.stb[1][pr.e]);
-      const ScaleProduct ar = has_res ? scale_product(p.sta[0][pr.e], p.stb[0][pr.e]) : ScaleProduct{0.0f, 0};
-      const float ratio = (ap.m != 0.0f && ar.m != 0.0f) ? ldexpf(__fdiv_rn(ar.m, ap.m), ar.e - ap.e) : 0.0f;
-      const float fin = ap.m;
-      const Pow2Apply out = pow2_apply(ap.e);
-      // m 2^e as one fp32 multiplier when it is normal (see scale_is_normal)
-      const bool one = scale_is_normal(ap.e);
-      const float fin1 = one ? ldexpf(fin, ap.e) : 0.0f;
+      if (pr.e != cur_e) {
+        // the residual is scaled to the plain segment's units (ratio =
+        // a_res / a_plain with a = s_tA s_tB = m 2^e), then Y = a_plain acc,
+        // applied as RN(acc m) and one power-of-two step (see Pow2Apply).  A
+        // zero plain scale means an all-zero X or W, whose residual and
+        // W_sel are zero as well: Y = 0.
+        const ScaleProduct ap = FP8 ? ScaleProduct{0.5f, 1} : scale_product(p.sta[1][pr.e], p.stb[1][pr.e]);
+        const ScaleProduct ar = has_res ? scale_product(p.sta[0][pr.e], p.stb[0][pr.e]) : ScaleProduct{0.0f, 0};
+        ratio = (ap.m != 0.0f && ar.m != 0.0f) ? ldexpf(__fdiv_rn(ar.m, ap.m), ar.e - ap.e) : 0.0f;
+        fin = ap.m;
+        out = pow2_apply(ap.e);
+        // m 2^e as one fp32 multiplier when it is normal (see scale_is_normal)
+        one = scale_is_normal(ap.e);
+        fin1 = one ? ldexpf(fin, ap.e) : 0.0f;
+        cur_e = pr.e;
+      }
       // Y of 32 accumulator values in place
       auto scale32 = [&](float* v) {
         if (one) {
