@@ -265,13 +265,11 @@ static __device__ __noinline__ void finish_strip(int64_t t0, int64_t t1, unsigne
     __syncthreads();
     if (*s_last) {
       __threadfence();
-      // keys in the (now idle) tile buffers and column maxima in the idle
-      // partial-sum buffer when they fit (K <= 4096), else read from L2
-      const bool fit = K * static_cast<int64_t>(sizeof(uint64_t)) <= 2 * kTileRows * kQCols * 2 &&
-                       K * static_cast<int64_t>(sizeof(float)) <= static_cast<int64_t>(kGroups * kQCols * sizeof(double));
-      topk_select(score, colamax, K, sel_out.n_sel, sel_out.mask, sel_out.sel, sel_out.s_t, 0,
-                  fit ? reinterpret_cast<uint64_t*>(keys) : nullptr,
-                  fit ? reinterpret_cast<float*>(ps) : nullptr, true);
+      // the (now idle) tile buffers and partial-sum buffer are its scratch
+      static_assert(2 * kTileRows * kQCols * 2 == kSelScratchBytes && kTileRows * kQCols * 4 == kSelScratchBytes,
+                    "selection scratch: two 32 KB buffers");
+      topk_select(score, colamax, K, sel_out.n_sel, sel_out.mask, sel_out.sel, sel_out.s_t, 0, keys,
+                  reinterpret_cast<uint8_t*>(ps));
       if (t == 0) *sel_out.strips_done = 0;
     }
   }

@@ -36,7 +36,7 @@ def main(argv=None):
     fns = {"prepare_weight": plan.prepare_weight, "quantize": plan.quantize, "select": plan.select,
            "weight_select": plan.weight_select, "gemm": plan.gemm, "gemm_plain": lambda: plan.gemm(plain=True),
            "quantize_plain": lambda: plan.quantize(scores=False), "quantize_select": plan.quantize_select,
-           "second_pass": plan.second_pass}
+           "second_pass": plan.second_pass, "select_channels": plan.select_channels}
     calls = [c for c in a.calls.split(",") if c]
     # the steps depend on each other: one full pass first
     plan.prepare_weight()

@@ -98,3 +98,92 @@ def test_plan_step_with_overlapped_gathers_matches_oracle():
     assert np.array_equal(plan.mask.cpu().numpy(), ref["mask"])
     from tests.gpu_common import REL_TOL, rel_err
     assert rel_err(plan.y.cpu().numpy()[rows], ref["y"]) < REL_TOL
+
+
+def _check_channels(b, score, k):
+    """rac_select_channels on given fp64 scores against oracle.select_channels
+    (mask, ascending sel, and s_tR = RN(max colamax over sel / 2688))."""
+    K = score.shape[0]
+    cm = np.random.default_rng(K).random(K).astype(np.float32)
+    mask, sel, n_sel, st = b.rac_select_channels(torch.from_numpy(score).cuda(), torch.from_numpy(cm).cuda(), k)
+    torch.cuda.synchronize()
+    n_ref = oracle.n_selected(k, K)
+    sel_ref, mask_ref = oracle.select_channels(score, n_ref)
+    assert n_sel == n_ref
+    assert np.array_equal(mask.cpu().numpy(), mask_ref)
+    assert np.array_equal(sel.cpu().numpy(), sel_ref)
+    want = np.float32(cm[sel_ref].max()) / np.float32(2688.0) if n_ref else np.float32(0.0)
+    assert np.float32(st.cpu().numpy()[0]) == want
+
+
+def _constructed_scores():
+    """Score vectors that steer the selection through each of its branches:
+    boundary bins taken whole, boundary bins ranked by bits below the 12-bit
+    digit (with exact ties), boundary bins of more than 1024 keys (equal or
+    merely close), many zero scores, and the two sides of the 16384-channel
+    digit limit."""
+    rng = np.random.default_rng(2024)
+    out = {}
+    # every key in its own 12-bit bin: 1 + j / 4096
+    out["whole_bins"] = 1.0 + rng.permutation(2048).astype(np.float64) / 4096.0
+    # four groups far apart, keys within a group differing only in the lowest
+    # 20 mantissa bits, some of them equal
+    g = rng.integers(0, 4, 2048).astype(np.float64)
+    lo = rng.integers(0, 1 << 20, 2048)
+    lo[rng.integers(0, 2048, 300)] = lo[0]
+    out["low_bits"] = 1.0 + g * 2.0 ** -8 + lo.astype(np.float64) * 2.0 ** -52
+    # 3000 equal keys straddling the boundary, distinct keys around them
+    v = np.concatenate([2.0 + rng.random(2500), np.full(3000, 1.5), 1.0 + 0.4 * rng.random(2692)])
+    out["big_equal_bin"] = v[rng.permutation(v.size)]
+    # 2000 distinct keys that share their leading 12 varying bits
+    c = np.concatenate([1.0 + rng.integers(0, 1 << 30, 2000).astype(np.float64) * 2.0 ** -52,
+                        8.0 + rng.random(1500), 0.25 * rng.random(596)])
+    out["big_close_bin"] = c[rng.permutation(c.size)]
+    # mostly zero scores
+    z = np.zeros(4096)
+    z[rng.choice(4096, 596, replace=False)] = rng.random(596) * 100.0
+    out["zeros"] = z
+    out["k16384"] = rng.random(16384) * rng.choice([1.0, 1e-3, 1e5], 16384)
+    out["k16448"] = rng.random(16448) * rng.choice([1.0, 1e-3, 1e5], 16448)
+    return out
+
+
+@pytest.mark.parametrize("name", ["whole_bins", "low_bits", "big_equal_bin", "big_close_bin", "zeros",
+                                  "k16384", "k16448"])
+def test_select_channels_constructed_scores(name):
+    b = need_gpu()
+    score = _constructed_scores()[name]
+    for k in (0.05, 12.5, 50.0, 99.96, 100.0, 0.0):
+        _check_channels(b, score, k)
+
+
+def test_select_channels_unaligned_buffers():
+    """Scores, colamax and mask at odd offsets (scores 8 bytes past a
+    16-byte boundary, colamax 4 bytes, the mask 1 byte) give the same
+    selection as the oracle."""
+    import ctypes
+    b = need_gpu()
+    K = 4096
+    rng = np.random.default_rng(7)
+    score = rng.random(K) * rng.choice([1.0, 1e-3, 1e5], K)
+    cm = rng.random(K).astype(np.float32)
+    sbuf = torch.zeros(K + 1, dtype=torch.float64, device="cuda")
+    cbuf = torch.zeros(K + 1, dtype=torch.float32, device="cuda")
+    mbuf = torch.zeros(K + 8, dtype=torch.uint8, device="cuda")
+    sbuf[1:] = torch.from_numpy(score).cuda()
+    cbuf[1:] = torch.from_numpy(cm).cuda()
+    for k in (12.5, 50.0, 99.96):
+        n_ref = oracle.n_selected(k, K)
+        sel = torch.zeros(max(n_ref, 1), dtype=torch.int32, device="cuda")
+        st = torch.zeros(1, dtype=torch.float32, device="cuda")
+        n_out = ctypes.c_int64(-1)
+        status = b._lib.rac_select_channels(ctypes.c_void_p(sbuf.data_ptr() + 8), ctypes.c_void_p(cbuf.data_ptr() + 4),
+                                            K, ctypes.c_float(k), ctypes.c_void_p(mbuf.data_ptr() + 1),
+                                            ctypes.c_void_p(sel.data_ptr()), ctypes.byref(n_out),
+                                            ctypes.c_void_p(st.data_ptr()), None)
+        torch.cuda.synchronize()
+        assert status == 0 and n_out.value == n_ref
+        sel_ref, mask_ref = oracle.select_channels(score, n_ref)
+        assert np.array_equal(mbuf[1:K + 1].cpu().numpy(), mask_ref)
+        assert np.array_equal(sel[:n_ref].cpu().numpy(), sel_ref)
+        assert np.float32(st.cpu().numpy()[0]) == np.float32(cm[sel_ref].max()) / np.float32(2688.0)
