@@ -1321,13 +1321,35 @@ __device__ __forceinline__ void qdq_tile_store(const uint4* raw, int64_t N, int6
     }
     float am = __uint_as_float(max(mbits & 0xFFFFu, mbits >> 16) << 16);
     am = fmaxf(am, __shfl_xor_sync(0xFFFFFFFFu, am, 1));
-    const BlockQ bs = block_q(am, T);
-    uint64_t q2[4];
-    block_quotients(x2, bs, q2);
-    const uint32_t q = e2m1x8_f2(q2);
+    uint32_t q, sb;
+    float sbv;
+    if (s_t >= kFastScale) {
+      // negated quotients, as in the quantize pass: every nonzero block
+      // decode scale is >= 2^-64, so its reciprocal table entry serves
+      const float q0 = __fmul_rn(am, T.rcp_d);
+      const float rr = __fmaf_rn(-q0, T.d, am);
+      sb = f32_to_e4m3(__fmaf_rn(rr, T.rcp_d, q0));
+      sbv = T.sbv[sb];
+      const float ny = -T.rcp[sb], sd = T.sdec[sb];
+      const uint64_t ny2 = f2_pack(ny, ny), sd2 = f2_pack(sd, sd);
+      uint64_t c2[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint64_t a = f2_mul(x2[j], ny2);
+        c2[j] = f2_fma(f2_fma(a, sd2, x2[j]), ny2, a);
+      }
+      q = e2m1x8_f2(c2) ^ 0x88888888u;
+    } else {
+      const BlockQ bs = block_q(am, T);
+      uint64_t q2[4];
+      block_quotients(x2, bs, q2);
+      q = e2m1x8_f2(q2);
+      sb = bs.sb;
+      sbv = bs.sbv;
+    }
     const int64_t qrow = b * N + n;
     if (live) {
-      const uint64_t sbv2 = f2_pack(bs.sbv, bs.sbv), st2 = f2_pack(s_t, s_t);
+      const uint64_t sbv2 = f2_pack(sbv, sbv), st2 = f2_pack(s_t, s_t);
       uint32_t o[4];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
@@ -1343,7 +1365,7 @@ __device__ __forceinline__ void qdq_tile_store(const uint4* raw, int64_t N, int6
     // rows past N belong to the next matrix: only live rows write (the caller
     // zero-fills the padding of a tiled scale buffer beforehand)
     if (scales && (cg & 1) == 0 && live)
-      scales[scale_offset(qrow, col / kBlock, K, layout)] = static_cast<uint8_t>(bs.sb);
+      scales[scale_offset(qrow, col / kBlock, K, layout)] = static_cast<uint8_t>(sb);
   }
   if (colamax_bits == nullptr) return;
 #pragma unroll

@@ -80,6 +80,17 @@ def test_weight_qdq_expert_stack_full_size():
         assert np.float32(st[e]) == oracle.nvfp4.tensor_scale(oracle.nvfp4.amax(wf[e]))
 
 
+def test_weight_qdq_tensor_scales_across_fast_bound():
+    """Stacked experts whose tensor scales lie on both sides of 2^-55 (the
+    bound above which the quotients take the reciprocal-table path), down to
+    a subnormal s_t: W4A16 outputs, codes, scales and colamax bit for bit."""
+    b = need_gpu()
+    w = S.weights(256, 192, seed=11, batch=7).float()
+    for e, k in enumerate((0, 40, 41, 44, 60, 100, 120)):
+        w[e] *= 2.0 ** -k
+    _check_qdq(b, w.to(torch.bfloat16))
+
+
 def test_weight_qdq_in_place():
     b = need_gpu()
     w = S.weights(256, 512, seed=7)
