@@ -1294,9 +1294,10 @@ __device__ __forceinline__ void qdq_tile_load(const uint16_t* w, int64_t N, int6
   }
 }
 
-// W' = DQ(Q(W)) of the tile (and its codes, scales and column maxima) from
-// the loaded rows; every thread of the CTA calls it (one barrier inside when
-// column maxima are kept).
+// W' = DQ(Q(W)) of the tile (and, with WQ, its codes and scales; with WCM,
+// its column maxima) from the loaded rows; every thread of the CTA calls it
+// (one barrier inside with WCM).
+template <bool WQ, bool WCM>
 __device__ __forceinline__ void qdq_tile_store(const uint4* raw, int64_t N, int64_t K, int64_t ldw, int64_t b,
                                                int64_t ty, int64_t tx, float s_t, const ScaleTable& T,
                                                uint16_t* w_out, uint8_t* codes, uint8_t* scales, int layout,
@@ -1317,7 +1318,7 @@ __device__ __forceinline__ void qdq_tile_store(const uint4* raw, int64_t N, int6
       x2[j] = bf16x2_to_f2(wv[j]);
       const uint32_t a = wv[j] & 0x7FFF7FFFu;
       mbits = __vmaxu2(mbits, a);
-      cmax[j] = __vmaxu2(cmax[j], a);            // columns 2j (low) and 2j+1 (high)
+      if (WCM) cmax[j] = __vmaxu2(cmax[j], a);   // columns 2j (low) and 2j+1 (high)
     }
     float am = __uint_as_float(max(mbits & 0xFFFFu, mbits >> 16) << 16);
     am = fmaxf(am, __shfl_xor_sync(0xFFFFFFFFu, am, 1));
@@ -1359,15 +1360,15 @@ __device__ __forceinline__ void qdq_tile_store(const uint4* raw, int64_t N, int6
       }
       if (NV_IDX(col + 8 <= K)) {
         *reinterpret_cast<uint4*>(w_out + off) = make_uint4(o[0], o[1], o[2], o[3]);
-        if (codes) *reinterpret_cast<uint32_t*>(codes + qrow * (K / 2) + col / 2) = q;
+        if (WQ) *reinterpret_cast<uint32_t*>(codes + qrow * (K / 2) + col / 2) = q;
       }
     }
     // rows past N belong to the next matrix: only live rows write (the caller
     // zero-fills the padding of a tiled scale buffer beforehand)
-    if (scales && (cg & 1) == 0 && live)
+    if (WQ && (cg & 1) == 0 && live)
       scales[scale_offset(qrow, col / kBlock, K, layout)] = static_cast<uint8_t>(sb);
   }
-  if (colamax_bits == nullptr) return;
+  if (!WCM) return;
 #pragma unroll
   for (int j = 0; j < 4; ++j) {                  // |bf16| bits -> fp32 bits
     cm[rr][8 * cg + 2 * j] = (cmax[j] & 0xFFFFu) << 16;
@@ -1383,7 +1384,9 @@ __device__ __forceinline__ void qdq_tile_store(const uint4* raw, int64_t N, int6
 }
 
 // One tile per CTA, the tensor amax from amax_partial's partial maxima.
-// grid = (K/64, ceil(N/128), batch).
+// grid = (K/64, ceil(N/128), batch).  WQ: codes and scales wanted; WCM:
+// column maxima wanted.
+template <bool WQ, bool WCM>
 __global__ void __launch_bounds__(kQThreads)
 weight_qdq_kernel(const uint16_t* w, int64_t N, int64_t K, int64_t ldw,
                   const unsigned* __restrict__ amax_parts, int n_parts,
@@ -1403,8 +1406,8 @@ weight_qdq_kernel(const uint16_t* w, int64_t N, int64_t K, int64_t ldw,
   __shared__ uint32_t cm[32][65];
   build_scale_table(T, s_t, t);
   __syncthreads();                               // table ready
-  qdq_tile_store(raw, N, K, ldw, b, blockIdx.y, blockIdx.x, s_t, T, w_out, codes, scales, layout,
-                 colamax_bits, cm);
+  qdq_tile_store<WQ, WCM>(raw, N, K, ldw, b, blockIdx.y, blockIdx.x, s_t, T, w_out, codes, scales, layout,
+                          colamax_bits, cm);
 }
 
 // ---------------------------------------------------------------------------
@@ -1817,7 +1820,9 @@ cudaError_t launch_weight_qdq(const uint16_t* w, int64_t N, int64_t K, int64_t l
   dim3 grid(static_cast<unsigned>(K / 64), static_cast<unsigned>((N + 127) / 128),
             static_cast<unsigned>(batch));
   {
-    const cudaError_t le = launch_k(weight_qdq_kernel, dim3(grid), dim3(kQThreads), 0, s, nullptr, 0,
+    auto kern = codes != nullptr ? (colamax_bits != nullptr ? weight_qdq_kernel<true, true> : weight_qdq_kernel<true, false>)
+                                 : (colamax_bits != nullptr ? weight_qdq_kernel<false, true> : weight_qdq_kernel<false, false>);
+    const cudaError_t le = launch_k(kern, dim3(grid), dim3(kQThreads), 0, s, nullptr, 0,
                                    w, N, K, ldw, amax_parts, n_parts, w_out, codes, scales, layout,
                                    tensor_scale, colamax_bits);
     if (le != cudaSuccess) return le;
