@@ -40,6 +40,14 @@
 // 256-column accumulator; the residual segment is computed first and scaled
 // in place by s_R s_Ws / (s_X s_W) (tcgen05.ld, multiply, tcgen05.st), then
 // the plain segment accumulates on top and Y = s_X s_W acc.
+//
+// Dense products with few 128 x 128 tiles (decode shapes) run the single-CTA
+// body split over K: a cluster of S = 2 or 4 CTAs per tile, CTA s taking the
+// K steps [T s / S, T (s + 1) / S) of the two segments.  Each CTA writes its
+// scaled fp32 partial over its idle pipeline stages; after a cluster
+// barrier, CTA s sums rows s 128/S .. of all S partials in CTA order through
+// distributed shared memory (ld.shared::cluster) and stores them; a second
+// barrier keeps every CTA until its partial has been read.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cstdlib>
@@ -67,6 +75,9 @@ struct Cfg {
   static constexpr int SMEM_BYTES = 1024 + STAGES * (A_STAGE + B_STAGE + 2 * SF_STAGE) + STG_BYTES + 256;
 };
 constexpr uint32_t TMEM_COLS = 512;
+// split-K partial tile: 128 fp32 rows of 128 columns, row stride padded by
+// 16 bytes (528 B), over the idle pipeline stages of A and B
+constexpr int kSplitStride = BN + 4;
 constexpr uint32_t ACC0_COL = 0, ACC1_COL = 128;   // two 128-column fp32 accumulators
 // block scales: per pipeline stage 32 columns (16 for A, 16 for B)
 constexpr uint32_t SF1_COL = 256, SF1_STAGE_COLS = 32;
@@ -94,6 +105,7 @@ struct KParams {
   int y_dtype;
   int64_t ldy, M;
   unsigned* err;
+  int split;                      // split-K kernel: CTAs (a cluster) per output tile
 };
 
 // ---- PTX wrappers ---------------------------------------------------------
@@ -174,19 +186,54 @@ __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Shared::cluster address of the same shared variable in CTA `rank`.
+__device__ __forceinline__ uint32_t peer_addr(const void* p, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+  return r;
+}
+
+// Shared::cluster address of shared-window address saddr in CTA `rank`.
+__device__ __forceinline__ uint32_t peer_addr_u32(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+
+// Distributed shared memory: a 16-byte load from the shared::cluster
+// address of another CTA of the cluster.
+__device__ __forceinline__ float4 ld_cluster_f4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr) : "memory");
+  return v;
+}
+
 // ---- the kernel -----------------------------------------------------------
 // The single-CTA kernel's body, for NVFP4 operands (FP8 = false: 256
 // elements per 128-byte K step, four kind::mxf4nvf4 MMAs of K = 64, one
 // 512-byte scale atom per MMA) or MXFP8 operands (FP8 = true: 128 elements
 // per K step, four kind::mxf8f6f4 MMAs of K = 32 reading the four bytes of
 // one scale atom, no residual segment).
-template <int YBYTES, bool FP8>
+template <int YBYTES, bool FP8, bool SPLIT = false>
 __device__ __forceinline__ void gemm1_body(const CUtensorMap& tmA0, const CUtensorMap& tmB0,
                                            const CUtensorMap& tmA1, const CUtensorMap& tmB1,
                                            const KParams& p) {
   constexpr int STAGES = Cfg<YBYTES>::STAGES;
   constexpr int SF_STEP = FP8 ? SF_ATOM : SF_STAGE;        // scale bytes per K step and operand
   constexpr int STG_STRIDE = Cfg<YBYTES>::STG_STRIDE;
+  static_assert(!SPLIT || BM * kSplitStride * 4 <= STAGES * (A_STAGE + B_STAGE),
+                "split-K partial tile fits over the A and B stages");
   extern __shared__ uint8_t smem_raw[];
   // 128-byte swizzled tiles need 1024-byte aligned shared addresses
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -234,6 +281,27 @@ __device__ __forceinline__ void gemm1_body(const CUtensorMap& tmA0, const CUtens
   const int64_t m_tiles = p.g.off ? p.g.tile_start[p.g.E] : p.m_tiles_dense;
   const int64_t total = m_tiles * p.n_tiles;
   const int nseg = p.kt[1] > 0 ? 2 : 1;
+  // split-K (dense only): the S CTAs of a cluster share one tile, CTA s
+  // taking K steps [T s / S, T (s + 1) / S) of the two segments in order;
+  // otherwise persistent over the tiles with the whole of K
+  const int S = SPLIT ? p.split : 1;
+  const int sidx = SPLIT ? static_cast<int>(blockIdx.x % static_cast<unsigned>(S)) : 0;
+  const int64_t tile_first = SPLIT ? blockIdx.x / S : blockIdx.x;
+  const int64_t tile_step = SPLIT ? total : gridDim.x;
+  const int T = p.kt[0] + (nseg > 1 ? p.kt[1] : 0);
+  const int k_lo = T * sidx / S, k_hi = T * (sidx + 1) / S;
+  auto kbeg = [&](int seg) { const int b = k_lo - (seg ? p.kt[0] : 0); return b > 0 ? b : 0; };
+  auto kend = [&](int seg) {
+    const int e = k_hi - (seg ? p.kt[0] : 0);
+    return e < p.kt[seg] ? e : p.kt[seg];
+  };
+  const bool has0 = kend(0) > kbeg(0), has1 = nseg > 1 && kend(1) > kbeg(1);
+  // the output scale factors depend on the row group only (dense: one
+  // group); formed by the epilogue warps, used again by the split-K reduction
+  int cur_e = -1;
+  float c0 = 0.0f, c1 = 0.0f, c0n = 0.0f, c1n = 0.0f;
+  Pow2Apply out{1.0f, 1.0f};
+  bool one = true;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -242,14 +310,14 @@ __device__ __forceinline__ void gemm1_body(const CUtensorMap& tmA0, const CUtens
       uint32_t phase = 0;
       uint32_t armed = 0, armed_phase = 0;     // per-stage: filled at least once / its parity
       bool ok = true;
-      for (int64_t tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+      for (int64_t tile = tile_first; tile < total && ok; tile += tile_step) {
         const int64_t mt = tile / p.n_tiles, nt = tile % p.n_tiles;
         const TileInfo ti = tile_info(p.g, mt);
         const int64_t b_row = static_cast<int64_t>(ti.e) * p.N + nt * BN;
         for (int seg = 0; seg < nseg && ok; ++seg) {
           const CUtensorMap* tA = seg ? &tmA1 : &tmA0;
           const CUtensorMap* tB = seg ? &tmB1 : &tmB0;
-          for (int kt = 0; kt < p.kt[seg]; ++kt) {
+          for (int kt = kbeg(seg); kt < kend(seg); ++kt) {
             if (!mbar_wait(&empty[stage], phase ^ 1, p.err)) { ok = false; break; }
             const int nkb = kt == p.kt[seg] - 1 ? p.kb_last[seg] : 4;
             const uint32_t sf_bytes = FP8 ? SF_ATOM : nkb * SF_ATOM;
@@ -281,12 +349,12 @@ __device__ __forceinline__ void gemm1_body(const CUtensorMap& tmA0, const CUtens
       int stage = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
-      for (int64_t tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+      for (int64_t tile = tile_first; tile < total && ok; tile += tile_step) {
         if (!mbar_wait(tmem_empty, acc_phase ^ 1, p.err)) break;
         tc_fence_after();
         for (int seg = 0; seg < nseg && ok; ++seg) {
           const uint32_t d = tmem + (seg ? ACC1_COL : ACC0_COL);
-          for (int kt = 0; kt < p.kt[seg]; ++kt) {
+          for (int kt = kbeg(seg); kt < kend(seg); ++kt) {
             if (!mbar_wait(&full[stage], phase, p.err) || !mbar_wait(&sf_ready[stage], phase, p.err)) {
               ok = false;
               break;
@@ -299,10 +367,10 @@ __device__ __forceinline__ void gemm1_body(const CUtensorMap& tmA0, const CUtens
               if (FP8)
                 mma_fp8(d, desc_sw128(a0 + 32 * j), desc_sw128(b0 + 32 * j),
                         IDESC8 | (static_cast<uint32_t>(j) << 29) | (static_cast<uint32_t>(j) << 4), sfa, sfb,
-                        (kt > 0 || j > 0) ? 1u : 0u);
+                        (kt > kbeg(seg) || j > 0) ? 1u : 0u);
               else
                 mma_fp4(d, desc_sw128(a0 + 32 * j), desc_sw128(b0 + 32 * j), sfa + 4 * j, sfb + 4 * j,
-                        (kt > 0 || j > 0) ? 1u : 0u);
+                        (kt > kbeg(seg) || j > 0) ? 1u : 0u);
             }
             umma_commit(&empty[stage]);
             if (++stage == STAGES) { stage = 0; phase ^= 1; }
@@ -322,9 +390,9 @@ __device__ __forceinline__ void gemm1_body(const CUtensorMap& tmA0, const CUtens
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (int64_t tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+      for (int64_t tile = tile_first; tile < total && ok; tile += tile_step) {
         for (int seg = 0; seg < nseg && ok; ++seg) {
-          for (int kt = 0; kt < p.kt[seg]; ++kt) {
+          for (int kt = kbeg(seg); kt < kend(seg); ++kt) {
             if (!mbar_wait(&full[stage], phase, p.err)) { ok = false; break; }
             tc_fence_after();
             const int nkb = kt == p.kt[seg] - 1 ? p.kb_last[seg] : 4;
@@ -352,13 +420,7 @@ __device__ __forceinline__ void gemm1_body(const CUtensorMap& tmA0, const CUtens
     uint8_t* stg_warp = sOut + (32 * q) * STG_STRIDE;
     uint8_t* stg_row = stg_warp + lane * STG_STRIDE;
     uint32_t acc_phase = 0;
-    // the output scale factors depend on the row group only: formed when it
-    // changes (once for a dense product), not per tile
-    int cur_e = -1;
-    float c0 = 0.0f, c1 = 0.0f, c0n = 0.0f, c1n = 0.0f;
-    Pow2Apply out{1.0f, 1.0f};
-    bool one = true;
-    for (int64_t tile = blockIdx.x; tile < total; tile += gridDim.x) {
+    for (int64_t tile = tile_first; tile < total; tile += tile_step) {
       bool ok = true;
       if (lane == 0) ok = mbar_wait(tmem_full, acc_phase, p.err);
       ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
@@ -383,6 +445,31 @@ __device__ __forceinline__ void gemm1_body(const CUtensorMap& tmA0, const CUtens
         c0n = one ? ldexpf(c0, E) : 0.0f;
         c1n = one ? ldexpf(c1, E) : 0.0f;
         cur_e = ti.e;
+      }
+      if (SPLIT) {
+        // this CTA's part of the tile, c0 acc0 + c1 acc1 over its K steps
+        // (with `one`, the power-of-two step folded in), as fp32 rows of the
+        // partial buffer over the idle pipeline stages
+        float* part = reinterpret_cast<float*>(sA);
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          float v[32], u[32];
+          if (has0) tmem_ld32(trow + ACC0_COL + 32 * c, v);
+          if (has1) tmem_ld32(trow + ACC1_COL + 32 * c, u);
+          tmem_ld_wait();
+          const float a0 = one ? c0n : c0, a1 = one ? c1n : c1;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float x0 = has0 ? __fmul_rn(a0, v[i]) : 0.0f, x1 = has1 ? __fmul_rn(a1, u[i]) : 0.0f;
+            v[i] = __fadd_rn(x0, x1);
+          }
+          float* dst = part + (32 * q + lane) * kSplitStride + 32 * c;
+#pragma unroll
+          for (int i = 0; i < 32; i += 4) *reinterpret_cast<float4*>(dst + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+        }
+        tc_fence_before();
+        acc_phase ^= 1;
+        continue;
       }
 #pragma unroll
       for (int c = 0; c < BN / 32; ++c) {
@@ -439,6 +526,48 @@ __device__ __forceinline__ void gemm1_body(const CUtensorMap& tmA0, const CUtens
   }
   tc_fence_before();
   __syncthreads();
+  if (SPLIT) {
+    // the tile's rows r0 .. r0 + 128/S - 1 of this CTA: the S partials in
+    // CTA order through distributed shared memory, then Y (the cluster
+    // barriers: every partial written before any is read, and no CTA leaves
+    // while its partial may still be read)
+    cluster_sync_all();
+    if (warp >= 2 && warp <= 5 && tile_first < total) {
+      const int64_t mt = tile_first / p.n_tiles, nt = tile_first % p.n_tiles;
+      const int rows = BM / S, r0 = sidx * rows;
+      const uint32_t pbase = smem_u32(sA);
+      for (int idx = threadIdx.x - 64; idx < rows * (BN / 4); idx += 128) {
+        const int row = r0 + idx / (BN / 4), c4 = idx % (BN / 4);
+        const uint32_t off = static_cast<uint32_t>((row * kSplitStride + 4 * c4) * 4);
+        float4 acc = ld_cluster_f4(peer_addr_u32(pbase + off, 0));
+        for (int sp = 1; sp < S; ++sp) {
+          const float4 t = ld_cluster_f4(peer_addr_u32(pbase + off, static_cast<uint32_t>(sp)));
+          acc.x = __fadd_rn(acc.x, t.x);
+          acc.y = __fadd_rn(acc.y, t.y);
+          acc.z = __fadd_rn(acc.z, t.z);
+          acc.w = __fadd_rn(acc.w, t.w);
+        }
+        if (!one) {
+          acc.x = out(acc.x);
+          acc.y = out(acc.y);
+          acc.z = out(acc.z);
+          acc.w = out(acc.w);
+        }
+        const int64_t grow = mt * BM + row, gcol = nt * BN + 4 * c4;
+        if (grow >= p.M || gcol + 4 > p.N || !NV_IDX(grow < p.M)) continue;
+        if (YBYTES == 4) {
+          *reinterpret_cast<float4*>(static_cast<float*>(p.y) + grow * p.ldy + gcol) = acc;
+        } else {
+          const uint32_t lo = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(acc.x))) |
+                              (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(acc.y))) << 16);
+          const uint32_t hi = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(acc.z))) |
+                              (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(acc.w))) << 16);
+          *reinterpret_cast<uint2*>(static_cast<uint16_t*>(p.y) + grow * p.ldy + gcol) = make_uint2(lo, hi);
+        }
+      }
+    }
+    cluster_sync_all();
+  }
   if (warp == 1) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(tmem), "r"(TMEM_COLS) : "memory");
@@ -451,6 +580,16 @@ w4a4_rac_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_cons
                      const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
                      const KParams p) {
   gemm1_body<YBYTES, false>(tmA0, tmB0, tmA1, tmB1, p);
+}
+
+// Split-K form (dense products with few tiles): a cluster of p.split CTAs
+// per output tile, the partials reduced through distributed shared memory.
+template <int YBYTES>
+__global__ void __launch_bounds__(THREADS1, 1)
+w4a4_rac_gemm_split_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
+                           const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
+                           const KParams p) {
+  gemm1_body<YBYTES, false, true>(tmA0, tmB0, tmA1, tmB1, p);
 }
 
 // MXFP8 x MXFP8 (the FP8 comparator): one K segment.
@@ -489,10 +628,27 @@ bool gemm_force_single_cta() {
   return v == 1;
 }
 
+// NVFP4_GEMM_NO_SPLIT=1 in the environment keeps the single-CTA kernel
+// persistent over whole tiles (no split over K; used to compare the two).
+bool gemm_no_split() {
+  static int v = -1;
+  if (v < 0) {
+    const char* e = getenv("NVFP4_GEMM_NO_SPLIT");
+    v = (e != nullptr && e[0] == '1') ? 1 : 0;
+  }
+  return v == 1;
+}
+
 template <int YBYTES>
 cudaError_t prepare_kernel() {
   static bool done[kMaxAttrDevices] = {};
   return set_max_smem(w4a4_rac_gemm_kernel<YBYTES>, Cfg<YBYTES>::SMEM_BYTES, done);
+}
+
+template <int YBYTES>
+cudaError_t prepare_split_kernel() {
+  static bool done[kMaxAttrDevices] = {};
+  return set_max_smem(w4a4_rac_gemm_split_kernel<YBYTES>, Cfg<YBYTES>::SMEM_BYTES, done);
 }
 
 template <int YBYTES>
@@ -580,23 +736,6 @@ __device__ __forceinline__ PairRows pair_rows(const KParams2& p, int64_t pt, uin
   r.local0 = local_tile * 128;
   r.out0 = p.g.off[lo];
   r.m = p.g.off[lo + 1] - p.g.off[lo];
-  return r;
-}
-
-__device__ __forceinline__ uint32_t cluster_rank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-
-__device__ __forceinline__ void cluster_sync_all() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-
-// Shared::cluster address of the same shared variable in CTA `rank`.
-__device__ __forceinline__ uint32_t peer_addr(const void* p, uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
   return r;
 }
 
@@ -1145,6 +1284,37 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s) {
   p.err = a.err;
   const int64_t tiles_bound = a.m_tiles * p.n_tiles;
   if (tiles_bound == 0) return cudaSuccess;
+  // dense products with few tiles: S CTAs per tile over K (S = 4 or 2, all
+  // tiles in one wave, at least three K steps per CTA: with two, the
+  // reduction cost more than the split saved), the partials reduced in a
+  // cluster of S
+  p.split = 1;
+  if (a.g.off == nullptr && !gemm_no_split()) {
+    const int64_t tiles = p.m_tiles_dense * p.n_tiles;
+    const int T = p.kt[0] + p.kt[1];
+    for (int c = 4; c >= 2; c /= 2)
+      if (tiles * c <= sm_count() && T >= 3 * c) {
+        p.split = c;
+        break;
+      }
+  }
+  if (p.split > 1) {
+    e = a.y_dtype == 0 ? prepare_split_kernel<4>() : prepare_split_kernel<2>();
+    if (e != cudaSuccess) return e;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = static_cast<unsigned>(p.split);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    const dim3 g(static_cast<unsigned>(p.m_tiles_dense * p.n_tiles * p.split));
+    const cudaError_t le =
+        a.y_dtype == 0 ? launch_k(w4a4_rac_gemm_split_kernel<4>, g, dim3(THREADS1), Cfg<4>::SMEM_BYTES, s, attr, 1,
+                                  maps[0], maps[1], maps[2], maps[3], p)
+                       : launch_k(w4a4_rac_gemm_split_kernel<2>, g, dim3(THREADS1), Cfg<2>::SMEM_BYTES, s, attr, 1,
+                                  maps[0], maps[1], maps[2], maps[3], p);
+    if (le != cudaSuccess) return le;
+    return cudaGetLastError();
+  }
   const int grid = static_cast<int>(tiles_bound < sm_count() ? tiles_bound : sm_count());
   if (a.y_dtype == 0)
     {
