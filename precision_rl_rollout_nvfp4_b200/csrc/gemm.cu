@@ -67,14 +67,15 @@ constexpr int SF_STAGE = 4 * SF_ATOM;            // 4 MMA K blocks per step
 // Per output type: pipeline depth and the epilogue staging tile (128 rows,
 // row stride padded by 16 bytes so 16-byte shared stores of 8 consecutive
 // rows hit distinct banks).
-template <int YBYTES>
+template <int YBYTES, bool SPLIT = false>
 struct Cfg {
-  static constexpr int STAGES = YBYTES == 2 ? 5 : 4;
+  // the split-K form keeps no epilogue staging tile (its partials go over
+  // the idle stages): one more stage
+  static constexpr int STAGES = SPLIT ? 6 : (YBYTES == 2 ? 5 : 4);
   static constexpr int STG_STRIDE = BN * YBYTES + 16;
-  static constexpr int STG_BYTES = BM * STG_STRIDE;
+  static constexpr int STG_BYTES = SPLIT ? 0 : BM * STG_STRIDE;
   static constexpr int SMEM_BYTES = 1024 + STAGES * (A_STAGE + B_STAGE + 2 * SF_STAGE) + STG_BYTES + 256;
-};
-constexpr uint32_t TMEM_COLS = 512;
+};constexpr uint32_t TMEM_COLS = 512;
 // split-K partial tile: 128 fp32 rows of 128 columns, row stride padded by
 // 16 bytes (528 B), over the idle pipeline stages of A and B
 constexpr int kSplitStride = BN + 4;
@@ -229,11 +230,12 @@ template <int YBYTES, bool FP8, bool SPLIT = false>
 __device__ __forceinline__ void gemm1_body(const CUtensorMap& tmA0, const CUtensorMap& tmB0,
                                            const CUtensorMap& tmA1, const CUtensorMap& tmB1,
                                            const KParams& p) {
-  constexpr int STAGES = Cfg<YBYTES>::STAGES;
+  constexpr int STAGES = Cfg<YBYTES, SPLIT>::STAGES;
   constexpr int SF_STEP = FP8 ? SF_ATOM : SF_STAGE;        // scale bytes per K step and operand
-  constexpr int STG_STRIDE = Cfg<YBYTES>::STG_STRIDE;
+  constexpr int STG_STRIDE = Cfg<YBYTES, SPLIT>::STG_STRIDE;
   static_assert(!SPLIT || BM * kSplitStride * 4 <= STAGES * (A_STAGE + B_STAGE),
                 "split-K partial tile fits over the A and B stages");
+  static_assert(Cfg<YBYTES, SPLIT>::SMEM_BYTES <= 227 * 1024, "shared memory of one CTA");
   extern __shared__ uint8_t smem_raw[];
   // 128-byte swizzled tiles need 1024-byte aligned shared addresses
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -242,7 +244,7 @@ __device__ __forceinline__ void gemm1_body(const CUtensorMap& tmA0, const CUtens
   uint8_t* sSFA = sB + STAGES * B_STAGE;
   uint8_t* sSFB = sSFA + STAGES * SF_STAGE;
   uint8_t* sOut = sSFB + STAGES * SF_STAGE;                     // epilogue staging
-  uint64_t* full = reinterpret_cast<uint64_t*>(sOut + Cfg<YBYTES>::STG_BYTES);
+  uint64_t* full = reinterpret_cast<uint64_t*>(sOut + Cfg<YBYTES, SPLIT>::STG_BYTES);
   uint64_t* empty = full + STAGES;
   uint64_t* sf_ready = empty + STAGES;       // the stage's scales are in TMEM
   uint64_t* tmem_full = sf_ready + STAGES;
@@ -648,7 +650,7 @@ cudaError_t prepare_kernel() {
 template <int YBYTES>
 cudaError_t prepare_split_kernel() {
   static bool done[kMaxAttrDevices] = {};
-  return set_max_smem(w4a4_rac_gemm_split_kernel<YBYTES>, Cfg<YBYTES>::SMEM_BYTES, done);
+  return set_max_smem(w4a4_rac_gemm_split_kernel<YBYTES>, Cfg<YBYTES, true>::SMEM_BYTES, done);
 }
 
 template <int YBYTES>
@@ -1284,16 +1286,18 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s) {
   p.err = a.err;
   const int64_t tiles_bound = a.m_tiles * p.n_tiles;
   if (tiles_bound == 0) return cudaSuccess;
-  // dense products with few tiles: S CTAs per tile over K (S = 4 or 2, all
-  // tiles in one wave, at least three K steps per CTA: with two, the
-  // reduction cost more than the split saved), the partials reduced in a
-  // cluster of S
+  // dense products with few tiles and a long K: S CTAs per tile over K
+  // (S = 4 or 2, all tiles in one wave, at least 16 K steps in all and 3 per
+  // CTA), the partials reduced in a cluster of S.  The split costs about
+  // 2 us (cluster barriers, partial stores, reduction): at 8 K steps of a
+  // 512 x 512 product it lost (10.4 -> 12.5 us), at 65 (decode down) it
+  // gains 34.6 -> 26 us.
   p.split = 1;
   if (a.g.off == nullptr && !gemm_no_split()) {
     const int64_t tiles = p.m_tiles_dense * p.n_tiles;
     const int T = p.kt[0] + p.kt[1];
     for (int c = 4; c >= 2; c /= 2)
-      if (tiles * c <= sm_count() && T >= 3 * c) {
+      if (tiles * c <= sm_count() && T >= 16 && T >= 3 * c) {
         p.split = c;
         break;
       }
@@ -1308,9 +1312,9 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s) {
     attr[0].val.clusterDim.z = 1;
     const dim3 g(static_cast<unsigned>(p.m_tiles_dense * p.n_tiles * p.split));
     const cudaError_t le =
-        a.y_dtype == 0 ? launch_k(w4a4_rac_gemm_split_kernel<4>, g, dim3(THREADS1), Cfg<4>::SMEM_BYTES, s, attr, 1,
+        a.y_dtype == 0 ? launch_k(w4a4_rac_gemm_split_kernel<4>, g, dim3(THREADS1), Cfg<4, true>::SMEM_BYTES, s, attr, 1,
                                   maps[0], maps[1], maps[2], maps[3], p)
-                       : launch_k(w4a4_rac_gemm_split_kernel<2>, g, dim3(THREADS1), Cfg<2>::SMEM_BYTES, s, attr, 1,
+                       : launch_k(w4a4_rac_gemm_split_kernel<2>, g, dim3(THREADS1), Cfg<2, true>::SMEM_BYTES, s, attr, 1,
                                   maps[0], maps[1], maps[2], maps[3], p);
     if (le != cudaSuccess) return le;
     return cudaGetLastError();

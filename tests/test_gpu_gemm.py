@@ -33,7 +33,12 @@ def _random_operand(b, rows, cols, rng, st):
                                      (512, 16, 64, 64),
                                      # CTA-pair kernel (256 x 256 tiles: enough tiles for its waves
                                      # to pay), ragged edges
-                                     (4000, 2000, 320, 64), (2560, 1040, 576, 448), (4096, 2048, 256, 0)])
+                                     (4000, 2000, 320, 64), (2560, 1040, 576, 448), (4096, 2048, 256, 0),
+                                     # split over K (few tiles, long K): 2 CTAs per tile; 4 per tile
+                                     # with ragged rows / columns and short last K steps; splits
+                                     # holding residual steps only
+                                     (256, 4096, 4096, 0), (200, 272, 4096, 448), (130, 400, 3904, 576),
+                                     (128, 128, 2048, 4096)])
 @pytest.mark.parametrize("out", ["f32", "bf16"])
 def test_gemm_on_random_operands(M, N, K, W, out):
     b = need_gpu()
