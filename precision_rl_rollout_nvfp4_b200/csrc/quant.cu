@@ -1019,6 +1019,7 @@ __device__ __forceinline__ void wsel_rows_body(const RowsArgs& A, uint8_t* ws_sm
   }
   int cur_e = -1;
   float st_w = 0.0f;
+  bool fastq = false;
   for (int64_t pi = p0; pi < p1; ++pi) {
     const int64_t p = pass_of(pi);
     const uint32_t b = static_cast<uint32_t>((pi - p0) & 1);
@@ -1053,6 +1054,7 @@ __device__ __forceinline__ void wsel_rows_body(const RowsArgs& A, uint8_t* ws_sm
       }
       __syncthreads();                             // the previous matrix's table is no longer read
       build_scale_table(T, st, t);
+      fastq = st >= kFastScale;
       if (FP4 || RES) st_w = w_st[e];
       cur_e = e;
     }
@@ -1142,12 +1144,34 @@ __device__ __forceinline__ void wsel_rows_body(const RowsArgs& A, uint8_t* ws_sm
             am = fmaxf(am, fabsf(x));
           }
           const int64_t row = r0 + slot;
-          const BlockQ bq = block_q(am, T);
-          const uint32_t lo = encode8_q(v, bq), hi = encode8_q(v + 8, bq);
+          uint32_t lo, hi, sb;
+          if (fastq) {
+            // negated quotients from the reciprocal table, as in the
+            // quantize pass (output tensor scale >= 2^-55)
+            const float q0 = __fmul_rn(am, T.rcp_d);
+            const float rr = __fmaf_rn(-q0, T.d, am);
+            sb = f32_to_e4m3(__fmaf_rn(rr, T.rcp_d, q0));
+            const float ny = -T.rcp[sb], sd = T.sdec[sb];
+            const uint64_t ny2 = f2_pack(ny, ny), sd2 = f2_pack(sd, sd);
+            uint64_t c2[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const uint64_t x2 = f2_pack(v[2 * j], v[2 * j + 1]);
+              const uint64_t a = f2_mul(x2, ny2);
+              c2[j] = f2_fma(f2_fma(a, sd2, x2), ny2, a);
+            }
+            lo = e2m1x8_f2(c2) ^ 0x88888888u;
+            hi = e2m1x8_f2(c2 + 4) ^ 0x88888888u;
+          } else {
+            const BlockQ bq = block_q(am, T);
+            lo = encode8_q(v, bq);
+            hi = encode8_q(v + 8, bq);
+            sb = bq.sb;
+          }
           if (NV_IDX(row < rows && (ob + 1) * kBlock <= width)) {
             *reinterpret_cast<uint2*>(out_codes + row * (width / 2) + static_cast<int64_t>(ob) * 8) =
                 make_uint2(lo, hi);
-            out_scales[scale_offset(row, ob, width, out_layout)] = static_cast<uint8_t>(bq.sb);
+            out_scales[scale_offset(row, ob, width, out_layout)] = static_cast<uint8_t>(sb);
           }
         }
       }
@@ -1724,6 +1748,30 @@ cudaError_t launch_residual_gather(const uint16_t* x, int64_t rows, int64_t K, i
       A.grp = g;
       A.prows = prows;
       const cudaError_t le = launch_k(wsel_rows_kernel<2>, dim3(grid), dim3(wp.threads), wp.smem, s, nullptr, 0, A);
+      if (le != cudaSuccess) return le;
+      return cudaGetLastError();
+    }
+  }
+  // dense activations with at least two passes per SM: the row-staged
+  // residual as in the fused second pass (it writes real rows only, so with
+  // a tiled scale layout the rows must fill whole 128-row blocks)
+  if (g.off == nullptr && (r_layout == 0 || prows % kTileRows == 0)) {
+    const WselPlan rp = wsel_plan(prows, K, 1, width, 2);
+    const int64_t sms = sm_count();
+    if (rp.ok && (prows + rp.g.R - 1) / rp.g.R >= 2 * sms) {
+      static bool done[kMaxAttrDevices] = {};
+      const cudaError_t ae = set_max_smem(wsel_rows_kernel<2>, 200 * 1024, done);
+      if (ae != cudaSuccess) return ae;
+      int per_sm = 0;
+      const cudaError_t oe =
+          cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, wsel_rows_kernel<2>, rp.threads, rp.smem);
+      if (oe != cudaSuccess) return oe;
+      const int64_t passes = (prows + rp.g.R - 1) / rp.g.R;
+      const int64_t cap = sms * (per_sm > 0 ? per_sm : 1);
+      const RowsArgs A{x, ldx, qx_codes, qx_scales, qx_layout, qx_st, prows, K, 1, sel, n_sel, width, nullptr, 0,
+                       const_cast<float*>(r_st), r_codes, r_scales, r_layout, rp.g};
+      const cudaError_t le = launch_k(wsel_rows_kernel<2>, dim3(static_cast<unsigned>(passes < cap ? passes : cap)),
+                                      dim3(rp.threads), rp.smem, s, nullptr, 0, A);
       if (le != cudaSuccess) return le;
       return cudaGetLastError();
     }
