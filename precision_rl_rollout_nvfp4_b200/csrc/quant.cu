@@ -189,6 +189,30 @@ constexpr int kMaxDone = 64;
 // serves the quotient (Markstein) and no division fallback is needed
 constexpr float kFastScale = 2.7755575615628914e-17f;   // 2^-55
 
+// E2M1 codes of 16 values with block amax am under a table of tensor scale
+// >= kFastScale: the block scale by Markstein's correction of am / d, then
+// the element quotients formed negated from the reciprocal table (c = -q,
+// see the quantize pass) and every code's sign bit flipped back.  Returns
+// the E4M3 block scale byte.
+__device__ __forceinline__ uint32_t encode16_fast(const float* v, float am, const ScaleTable& T, uint32_t& lo,
+                                                  uint32_t& hi) {
+  const float q0 = __fmul_rn(am, T.rcp_d);
+  const float rr = __fmaf_rn(-q0, T.d, am);
+  const uint32_t sb = f32_to_e4m3(__fmaf_rn(rr, T.rcp_d, q0));
+  const float ny = -T.rcp[sb], sd = T.sdec[sb];
+  const uint64_t ny2 = f2_pack(ny, ny), sd2 = f2_pack(sd, sd);
+  uint64_t c2[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const uint64_t x2 = f2_pack(v[2 * j], v[2 * j + 1]);
+    const uint64_t a = f2_mul(x2, ny2);
+    c2[j] = f2_fma(f2_fma(a, sd2, x2), ny2, a);
+  }
+  lo = e2m1x8_f2(c2) ^ 0x88888888u;
+  hi = e2m1x8_f2(c2 + 4) ^ 0x88888888u;
+  return sb;
+}
+
 // Optional top-k% selection fused into the quantize pass's tail.
 struct SelectOut {
   int64_t n_sel;            // < 0: no selection
@@ -797,12 +821,19 @@ __device__ __forceinline__ void gather_quant_body(const GatherArgs& A, GatherSme
         float am = 0.0f;
 #pragma unroll
         for (int u = 0; u < 16; ++u) am = fmaxf(am, fabsf(v[u]));
-        const BlockQ bq = block_q(am, T);
-        const uint32_t lo = encode8_q(v, bq), hi = encode8_q(v + 8, bq);
+        uint32_t lo, hi, sb;
+        if (st >= kFastScale) {
+          sb = encode16_fast(v, am, T, lo, hi);
+        } else {
+          const BlockQ bq = block_q(am, T);
+          lo = encode8_q(v, bq);
+          hi = encode8_q(v + 8, bq);
+          sb = bq.sb;
+        }
         if (in_rows && NV_IDX(blk * kBlock + 16 <= width))
           *reinterpret_cast<uint2*>(out_codes + prow * (width / 2) + blk * 8) = make_uint2(lo, hi);
         if (NV_IDX(scale_offset(prow, blk, width, out_layout) < scale_extent(grid_rows, width, out_layout, kBlock)))
-          out_scales[scale_offset(prow, blk, width, out_layout)] = static_cast<uint8_t>(bq.sb);
+          out_scales[scale_offset(prow, blk, width, out_layout)] = static_cast<uint8_t>(sb);
       }
     }
   }
@@ -1145,23 +1176,8 @@ __device__ __forceinline__ void wsel_rows_body(const RowsArgs& A, uint8_t* ws_sm
           }
           const int64_t row = r0 + slot;
           uint32_t lo, hi, sb;
-          if (fastq) {
-            // negated quotients from the reciprocal table, as in the
-            // quantize pass (output tensor scale >= 2^-55)
-            const float q0 = __fmul_rn(am, T.rcp_d);
-            const float rr = __fmaf_rn(-q0, T.d, am);
-            sb = f32_to_e4m3(__fmaf_rn(rr, T.rcp_d, q0));
-            const float ny = -T.rcp[sb], sd = T.sdec[sb];
-            const uint64_t ny2 = f2_pack(ny, ny), sd2 = f2_pack(sd, sd);
-            uint64_t c2[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              const uint64_t x2 = f2_pack(v[2 * j], v[2 * j + 1]);
-              const uint64_t a = f2_mul(x2, ny2);
-              c2[j] = f2_fma(f2_fma(a, sd2, x2), ny2, a);
-            }
-            lo = e2m1x8_f2(c2) ^ 0x88888888u;
-            hi = e2m1x8_f2(c2 + 4) ^ 0x88888888u;
+          if (fastq) {                             // output tensor scale >= 2^-55
+            sb = encode16_fast(v, am, T, lo, hi);
           } else {
             const BlockQ bq = block_q(am, T);
             lo = encode8_q(v, bq);
