@@ -301,10 +301,11 @@ static __device__ __noinline__ void topk_select(const double* __restrict__ score
                                                 int32_t* __restrict__ sel, float* __restrict__ s_t_out, int64_t e,
                                                 uint8_t* scr0, uint8_t* scr1) {
   const bool none = n_sel <= 0, all = n_sel >= K;
-  // (the 16-byte key loads below need K % 8 == 0 and 16-byte aligned
-  // scores; K is a multiple of 64 in every caller)
+  // (the classification below takes whole groups of 8 channels, so K % 8
+  // must be 0 for every n_sel; the 16-byte key loads also need 16-byte
+  // aligned scores.  K is a multiple of 64 in every caller.)
   const bool keys16 = (reinterpret_cast<uintptr_t>(score + e * K) & 15u) == 0;
-  if ((K > kSelDigitKeys || (K & 7) != 0 || !keys16) && !none && !all) {
+  if ((K & 7) != 0 || ((K > kSelDigitKeys || !keys16) && !none && !all)) {
     topk_select_radix(score, colamax, K, n_sel, mask, sel, s_t_out, e, nullptr, nullptr, true);
     return;
   }
